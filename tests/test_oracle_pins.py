@@ -1,0 +1,294 @@
+"""Pins for the CPU oracle: each test checks the oracle against something other than itself.
+
+- float decoders: numpy's binary16 and torch's bfloat16 conversions, over all 65536 bit patterns;
+- CRC-32: the published check value and zlib;
+- packing: the hand-derived golden blob of FORMAT.md's worked example, and a single-code bit-position sweep;
+- matvec: exact rational arithmetic on tiny shapes, closed forms on uniform widths, one-hot columns, and exact
+  power-of-two scale invariance.
+
+The method follows the VBQ paper ("Variable Bit-width Quantization", section 3.1, groups of 64 with a per-group
+scale and width from {1,2,4,8}; section 6, "Fused kernels over packed weights").
+"""
+import math
+import os
+import zlib
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import oracle as O
+import vbq_synth as S
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "format_n2_k64_r16.txt")
+
+
+def f16(bits):
+    return np.asarray(bits, np.uint16).view(np.float16).astype(np.float64)
+
+
+def bf16(bits):
+    t = torch.from_numpy(np.asarray(bits, np.uint16).astype(np.int16)).view(torch.bfloat16)
+    return t.to(torch.float64).numpy()
+
+
+# ------------------------------------------------------------------------------------------------ decoders
+def test_half_decoder_matches_numpy_all_patterns():
+    ref = f16(np.arange(65536, dtype=np.uint32).astype(np.uint16))
+    got = np.array([O.half_to_double(b) for b in range(65536)])
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan], ref[~nan])
+    assert np.array_equal(np.signbit(got[~nan]), np.signbit(ref[~nan]))
+
+
+def test_bf16_decoder_matches_torch_all_patterns():
+    ref = bf16(np.arange(65536, dtype=np.uint32).astype(np.uint16))
+    got = np.array([O.bf16_to_double(b) for b in range(65536)])
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan], ref[~nan])
+
+
+def test_crc32_check_value_and_zlib():
+    assert O.crc32(b"123456789") == 0xCBF43926
+    g = np.random.default_rng(1)
+    for n in (0, 1, 7, 64, 1000):
+        buf = g.integers(0, 256, n, dtype=np.uint8).tobytes()
+        assert O.crc32(buf) == zlib.crc32(buf)
+
+
+# ------------------------------------------------------------------------------------------------ packing
+def golden_example():
+    N, K, R = 2, 64, 16
+    widths = np.array([[1], [2]], np.uint8)
+    scales = np.array([[0x3C00], [0x3800]], np.uint16)
+    codes = np.zeros((2, 64), np.uint8)
+    codes[0] = np.arange(64) % 2
+    codes[1] = np.arange(64) % 4
+    return N, K, R, widths, scales, codes
+
+
+def parse_golden(path):
+    expect, crc_fields = {}, {}
+    for line in open(path):
+        line = line.split("#", 1)[0].strip() if line.lstrip().startswith("#") else line.strip()
+        if not line:
+            continue
+        parts = line.split()
+        off = int(parts[0])
+        if parts[1].startswith("CRC32_"):
+            crc_fields[parts[1]] = off
+            continue
+        for i, tok in enumerate(parts[1:]):
+            try:
+                b = int(tok, 16)
+            except ValueError:
+                break
+            if len(tok) != 2:
+                break
+            expect[off + i] = b
+    return expect, crc_fields
+
+
+def test_golden_blob_bytes():
+    N, K, R, w, s, c = golden_example()
+    blob = O.pack(N, K, R, w, s, c).tobytes()
+    expect, crc = parse_golden(GOLDEN)
+    assert len(blob) == 144
+    covered = set(expect) | {o + i for o in crc.values() for i in range(4)}
+    assert covered == set(range(144)), "golden file must describe every byte"
+    for off, b in expect.items():
+        assert blob[off] == b, f"byte {off}: got {blob[off]:#04x} want {b:#04x}"
+    assert int.from_bytes(blob[crc["CRC32_BODY"]:][:4], "little") == zlib.crc32(blob[64:144])
+    assert int.from_bytes(blob[crc["CRC32_HEADER"]:][:4], "little") == zlib.crc32(blob[0:60])
+
+
+@pytest.mark.parametrize("k", [1, 2, 4, 8])
+def test_single_code_bit_positions(k):
+    # One 1-bit... 8-bit group (N=1, K=64, R=16): header 64 + directory 16 = 80; record: counts+width word
+    # padded to 16, one scale padded to 16, then the group's 8k code bytes at record offset 32.
+    code_start = 80 + 32
+    for i in range(64):
+        for v in sorted({1, (1 << k) - 1, (0x5A % (1 << k)) or 1}):
+            codes = np.zeros((1, 64), np.uint8)
+            codes[0, i] = v
+            blob = O.pack(1, 64, 16, np.array([[k]], np.uint8), np.array([[0x3C00]], np.uint16), codes)
+            bits = np.unpackbits(blob[code_start:code_start + 8 * k], bitorder="little")
+            want = np.zeros(64 * k, np.uint8)
+            for b in range(k):
+                want[k * i + b] = (v >> b) & 1
+            assert np.array_equal(bits, want), (k, i, v)
+
+
+def random_logical(g, N, K, p=S.P_BASE):
+    w = S.widths_iid(N, K // 64, p, g)
+    s = S.scales_uniform(N, K // 64, g)
+    c = S.codes_uniform(w, g)
+    return w, s, c
+
+
+@pytest.mark.parametrize("N,K,R", [(1, 64, 16), (17, 128, 16), (100, 320, 32), (1000, 256, 1024),
+                                   (1030, 192, 512), (64, 64, 64)])
+def test_pack_unpack_round_trip(N, K, R):
+    g = np.random.default_rng(N * 1000 + K + R)
+    w, s, c = random_logical(g, N, K)
+    blob = O.pack(N, K, R, w, s, c)
+    assert blob.size % 16 == 0
+    assert O.packed_size(N, K, R, w) == blob.size
+    w2, s2, c2, R2 = O.unpack(blob)
+    assert R2 == R and np.array_equal(w, w2) and np.array_equal(s, s2) and np.array_equal(c, c2)
+    blob2 = O.pack(N, K, R, w2, s2, c2)
+    assert np.array_equal(blob, blob2)
+
+
+def test_unpack_rejects_corruption():
+    g = np.random.default_rng(7)
+    N, K, R = 40, 128, 16
+    w, s, c = random_logical(g, N, K)
+    blob = O.pack(N, K, R, w, s, c)
+
+    def refresh(b):
+        b = b.copy()
+        b[56:60] = np.frombuffer(zlib.crc32(b[64:].tobytes()).to_bytes(4, "little"), np.uint8)
+        b[60:64] = np.frombuffer(zlib.crc32(b[:60].tobytes()).to_bytes(4, "little"), np.uint8)
+        return b
+
+    assert O.unpack_status(blob[:63])[0] == O.ERR_BUFFER_TOO_SMALL
+    assert O.unpack_status(blob[:-16])[0] == O.ERR_BUFFER_TOO_SMALL
+    b = blob.copy(); b[0] ^= 1
+    assert O.unpack_status(b)[0] == O.ERR_BAD_MAGIC
+    b = blob.copy(); b[4] = 2
+    assert O.unpack_status(b)[0] == O.ERR_VERSION
+    b = blob.copy(); b[-1] ^= 0x10
+    assert O.unpack_status(b)[0] == O.ERR_CRC
+    b = blob.copy(); b[20] = 17
+    assert O.unpack_status(refresh(b))[0] == O.ERR_FORMAT
+    # first record: the width word region of a 16-row tile is exactly one word, so bytes 12..15 are padding
+    rec = 64 + ((4 * (3 * 2 + 1) + 15) // 16) * 16
+    b = blob.copy(); b[rec + 12] = 1
+    assert O.unpack_status(refresh(b))[0] == O.ERR_FORMAT
+    b = blob.copy(); b[rec] ^= 1   # count n1 no longer matches the width codes
+    assert O.unpack_status(refresh(b))[0] == O.ERR_FORMAT
+    assert O.unpack_status(refresh(blob))[0] == O.OK
+
+
+def test_pack_error_codes():
+    g = np.random.default_rng(3)
+    w, s, c = random_logical(g, 4, 128)
+    assert O.pack_status(4, 100, 16, w, s, c)[0] == O.ERR_SHAPE
+    assert O.pack_status(4, 128, 8, w, s, c)[0] == O.ERR_TILE
+    assert O.pack_status(4, 128, 24, w, s, c)[0] == O.ERR_TILE
+    bad = w.copy(); bad[1, 1] = 3
+    assert O.pack_status(4, 128, 16, bad, s, c)[0] == O.ERR_WIDTH
+    cc = c.copy(); r = int(np.argwhere(w[:, 0] == 1)[0][0]) if (w[:, 0] == 1).any() else None
+    if r is None:
+        w[0, 0] = 1; c[0, :64] &= 1; r = 0; cc = c.copy()
+    cc[r, 5] = 2
+    assert O.pack_status(4, 128, 16, w, s, cc)[0] == O.ERR_CODE_RANGE
+    size = O.packed_size(4, 128, 16, w)
+    assert O.pack_status(4, 128, 16, w, s, c, cap=size - 16)[0] == O.ERR_BUFFER_TOO_SMALL
+
+
+# ------------------------------------------------------------------------------------------------ matvec
+def exact_y(w, s, c, xbits):
+    """Exact rational y and bound, decoding with numpy/torch (not the oracle)."""
+    N, K = c.shape
+    sv = [[Fraction(float(v)) for v in row] for row in f16(s)]
+    xv = [Fraction(float(v)) for v in bf16(xbits)]
+    ys, bs = [], []
+    for r in range(N):
+        acc, a = Fraction(0), Fraction(0)
+        for i in range(K):
+            k = int(w[r, i // 64])
+            wt = sv[r][i // 64] * (int(c[r, i]) - Fraction((1 << k) - 1, 2))
+            acc += wt * xv[i]
+            a += abs(wt) * abs(xv[i])
+        ys.append(acc); bs.append(a)
+    return ys, bs
+
+
+def test_matvec_matches_exact_rationals_all_width_pairs():
+    # K=128 (2 groups): all 16 (width, width) pairs, one row each.
+    g = np.random.default_rng(11)
+    pairs = [(a, b) for a in (1, 2, 4, 8) for b in (1, 2, 4, 8)]
+    w = np.array(pairs, np.uint8)
+    s = S.scales_uniform(16, 2, g)
+    s[3, 1] = 0xB555   # a negative scale
+    s[5, 0] = 0x0003   # a subnormal scale
+    c = S.codes_uniform(w, g)
+    x = S.x_normal(1, 128, g)
+    x[0, 7] = 0x0001   # a subnormal activation
+    x[0, 9] = 0x7F00   # a large one
+    y, a = O.matvec(w, s, c, x)
+    ys, bs = exact_y(w, s, c, x[0])
+    for r in range(16):
+        assert abs(Fraction(y[0, r]) - ys[r]) <= Fraction(1, 2**50) * bs[r] + Fraction(1, 2**1000)
+        assert abs(Fraction(a[0, r]) - bs[r]) <= Fraction(1, 2**50) * bs[r]
+
+
+@pytest.mark.parametrize("N,K", [(1, 64), (3, 192), (5, 64)])
+def test_matvec_brute_force_small(N, K):
+    g = np.random.default_rng(N + K)
+    w, s, c = random_logical(g, N, K, p=(0.25, 0.25, 0.25, 0.25))
+    x = S.x_normal(2, K, g)
+    y, a = O.matvec(w, s, c, x)
+    for b in range(2):
+        ys, bs = exact_y(w, s, c, x[b])
+        for r in range(N):
+            assert abs(Fraction(y[b, r]) - ys[r]) <= Fraction(1, 2**50) * bs[r]
+
+
+@pytest.mark.parametrize("k", [1, 2, 4, 8])
+def test_closed_forms_uniform_width(k):
+    N, K = 6, 256
+    g = np.random.default_rng(100 + k)
+    x = S.x_normal(1, K, g)
+    xs = bf16(x[0])
+    s0 = 0x2E66  # fp16 0.1
+    s = np.full((N, K // 64), s0, np.uint16)
+    w = np.full((N, K // 64), k, np.uint8)
+    sv = float(f16(s0))
+    tot = math.fsum(xs)
+    top = np.full((N, K), (1 << k) - 1, np.uint8)
+    y, _ = O.matvec(w, s, top, x)
+    assert np.allclose(y[0], sv * ((1 << k) - 1) / 2 * tot, rtol=1e-13, atol=1e-13)
+    y, _ = O.matvec(w, s, np.zeros((N, K), np.uint8), x)
+    assert np.allclose(y[0], -sv * ((1 << k) - 1) / 2 * tot, rtol=1e-13, atol=1e-13)
+    if k == 1:
+        c = g.integers(0, 2, size=(N, K)).astype(np.uint8)
+        y, _ = O.matvec(w, s, c, x)
+        for r in range(N):
+            want = sv / 2 * (math.fsum(xs[c[r] == 1]) - math.fsum(xs[c[r] == 0]))
+            assert abs(y[0, r] - want) <= 1e-13 * (1 + abs(want))
+    if k == 8:  # code 255 -> +127.5 s, code 0 -> -127.5 s, checked on a one-hot activation
+        xe = np.zeros((1, K), np.uint16); xe[0, 3] = 0x3F80
+        y, _ = O.matvec(w, s, top, xe)
+        assert np.all(y[0] == 127.5 * sv)
+
+
+def test_one_hot_columns_are_dequantized_weights():
+    g = np.random.default_rng(5)
+    N, K = 9, 192
+    w, s, c = random_logical(g, N, K, p=(0.25, 0.25, 0.25, 0.25))
+    sv = f16(s)
+    for i in (0, 1, 63, 64, 100, 191):
+        x = np.zeros((1, K), np.uint16); x[0, i] = 0x3F80   # bf16 1.0
+        y, a = O.matvec(w, s, c, x)
+        for r in range(N):
+            k = int(w[r, i // 64])
+            want = sv[r, i // 64] * (int(c[r, i]) - ((1 << k) - 1) / 2)
+            assert y[0, r] == want and a[0, r] == abs(want)
+
+
+def test_power_of_two_scale_invariance():
+    g = np.random.default_rng(9)
+    N, K = 20, 320
+    w, s, c = random_logical(g, N, K)
+    x = S.x_normal(3, K, g)
+    y1, a1 = O.matvec(w, s, c, x)
+    s2 = (s.astype(np.uint32) + (1 << 10)).astype(np.uint16)   # exponent + 1: exact doubling for normal fp16
+    assert np.array_equal(f16(s2), 2 * f16(s))
+    y2, a2 = O.matvec(w, s2, c, x)
+    assert np.array_equal(y2, 2 * y1) and np.array_equal(a2, 2 * a1)
