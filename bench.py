@@ -1,0 +1,348 @@
+"""Benchmark of the VBQ mixed-bit GEMV on B200: achieved HBM GB/s against the measured copy peak.
+
+Default workload: the seven linears of one 9B-shaped decoder layer at batch 1 (q, k, v, o 4096x4096; gate, up
+4096->14336; down 14336->4096), with widths drawn from the VBQ paper's allocation (about 69% 1-bit groups,
+1.85 mean bits). One step runs all seven GEMVs. Four distinct seeded copies of the layer (about 260 MB, more
+than the 126 MB L2) are used in rotation, so every step streams its weights from HBM.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--batch B] [--impl vbq|reference]
+
+Under torchrun (N > 1) every rank runs an independent replica on its own GPU. The path has no cross-GPU
+exchange. Time is the max over ranks, and the value is the bytes of all ranks divided by that time.
+``--impl reference`` times the fp64 CPU oracle on a bounded sample of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import vbq_synth as S  # noqa: E402
+
+METRIC = "mixed-bit GEMV achieved HBM GB/s (% of B200 peak); decode-step µs at 1 GPU"
+UNIT = "GB/s"
+NAMES = ("q", "k", "v", "o", "gate", "up", "down")
+WORKLOAD = "9B-shaped decoder-layer linears (q,k,v,o 4096x4096; gate,up 4096->14336; down 14336->4096)"
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+# ----------------------------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, r in rows for i, v in enumerate(r) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------------------------------------------ setup
+def layer_matrices(copy: int):
+    return [S.make_matrix(4, n, *S.CFG4_SHAPES[n], layer=copy) for n in NAMES]
+
+
+def blob_bytes_of(m, R):
+    from decode_vbq_gemv_b200 import vbq
+    return vbq.vbq_packed_size(m.N, m.K, R, m.widths)
+
+
+def cpu_baseline(B: int, budget_s: float = 12.0, matrices=None):
+    """Times the fp64 oracle (as it stands) on a bounded sample of the workload: the first `rows` rows of each
+    of the seven linears, growing the sample until it takes about `budget_s` seconds or covers every row."""
+    from oracle import oracle as O
+    from decode_vbq_gemv_b200 import vbq
+    mats = matrices or layer_matrices(0)
+    threads = os.cpu_count() or 1
+    xs = [S.make_x(4, m.name, B, m.K) for m in mats]
+    full = [vbq.vbq_packed_size(m.N, m.K, 1024, m.widths) for m in mats]
+    rows = 64
+    while True:
+        t0 = time.perf_counter()
+        nbytes = 0.0
+        for m, x, fb in zip(mats, xs, full):
+            r = min(rows, m.N)
+            O.matvec(m.widths[:r], m.scales[:r], m.codes[:r], x, threads)
+            nbytes += fb * r / m.N + B * m.K * 2 + B * r * 4
+        dt = time.perf_counter() - t0
+        if dt > budget_s / 4 or rows >= max(m.N for m in mats):
+            break
+        rows *= 4
+    return {"value": nbytes / dt / 1e9, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"fp64 oracle on the first {rows} rows of each of the 7 linears, batch {B} "
+                      f"({dt:.2f} s); GB/s scaled from those rows' share of the packed bytes"}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def allreduce_max(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ------------------------------------------------------------------------------------------------ arms
+def run_reference(args):
+    world, rank, _ = dist_setup()
+    if rank != 0:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
+    from oracle import oracle as O
+    mats = layer_matrices(0)
+    xs = [S.make_x(4, m.name, args.batch, m.K) for m in mats]
+    full = [blob_bytes_of(m, 1024) for m in mats]
+    rows = args.ref_rows
+    threads = os.cpu_count() or 1
+
+    def step():
+        nb = 0.0
+        for m, x, fb in zip(mats, xs, full):
+            O.matvec(m.widths[:rows], m.scales[:rows], m.codes[:rows], x, threads)
+            nb += fb * rows / m.N + args.batch * m.K * 2 + args.batch * rows * 4
+        return nb
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    nb = sum(step() for _ in range(args.steps))
+    dt = time.perf_counter() - t0
+    val = nb / dt / 1e9
+    sample = f"fp64 oracle, first {rows} rows of each of the 7 linears per step, batch {args.batch}"
+    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": WORKLOAD + f", sampled rows ({rows} per linear)",
+                                            "batch": args.batch},
+            "cpu_baseline": {"value": val, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample},
+            "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def run_vbq(args):
+    import torch
+    from decode_vbq_gemv_b200 import vbq
+    world, rank, local = dist_setup()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    B, R = args.batch, args.tile_rows
+    stream = torch.cuda.current_stream()
+
+    layers = []   # per copy: list of (DeviceMatrix, x_dev, y_dev, x_host_pinned, y_host_pinned, bytes)
+    for cp in range(args.copies):
+        lin = []
+        for m in layer_matrices(cp):
+            blob, _ = vbq.vbq_pack(m.N, m.K, R, m.widths, m.scales, m.codes)
+            mat = vbq.DeviceMatrix(blob, dev, max_batch=B)
+            xb = S.make_x(4, m.name, B, m.K, layer=cp)
+            xh = torch.from_numpy(xb.astype(np.int16)).view(torch.bfloat16).pin_memory()
+            xd = xh.to(dev)
+            yd = torch.empty((B, m.N), dtype=torch.float32, device=dev)
+            yh = torch.empty((B, m.N), dtype=torch.float32).pin_memory()
+            nbytes = mat.nbytes + B * m.K * 2 + B * m.N * 4
+            lin.append((mat, xd, yd, xh, yh, nbytes, m.name))
+            del blob
+        layers.append(lin)
+    step_bytes = [sum(l[5] for l in lin) for lin in layers]
+
+    def launch(mat, xd, yd):
+        vbq.vbq_gemm_skinny(mat.desc, mat.blob, xd, B, yd, mat.workspaces[B], stream)
+
+    # ---- device-resident timing (value, roofline)
+    for i in range(args.warmup):
+        for mat, xd, yd, *_ in layers[i % args.copies]:
+            launch(mat, xd, yd)
+    torch.cuda.synchronize()
+    barrier(world)
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    ev = []
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    t_start.record(stream)
+    total_bytes = 0
+    for i in range(args.steps):
+        lin = layers[i % args.copies]
+        for mat, xd, yd, _, _, nb, name in lin:
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            launch(mat, xd, yd)
+            e1.record(stream)
+            ev.append((e0, e1, nb, name))
+        total_bytes += step_bytes[i % args.copies]
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks = sampler.stop()
+    ms = t_start.elapsed_time(t_end)
+    ms_max = allreduce_max(ms, world)
+    launch_ms = sum(e0.elapsed_time(e1) for e0, e1, _, _ in ev)
+    launch_bytes = sum(nb for _, _, nb, _ in ev)
+    per_shape = {}
+    for e0, e1, nb, name in ev:
+        d = per_shape.setdefault(name, [0.0, 0.0, 0])
+        d[0] += e0.elapsed_time(e1); d[1] += nb; d[2] += 1
+    value = total_bytes * world / (ms_max / 1e3) / 1e9
+
+    # ---- end to end through host buffers: pinned x -> device, GEMV, y -> pinned host, every step
+    h2d = sum(l[3].numel() * 2 for l in layers[0])
+    d2h = sum(l[4].numel() * 4 for l in layers[0])
+    for i in range(args.warmup):
+        for mat, xd, yd, xh, yh, *_ in layers[i % args.copies]:
+            xd.copy_(xh, non_blocking=True); launch(mat, xd, yd); yh.copy_(yd, non_blocking=True)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e0 = torch.cuda.Event(enable_timing=True)
+    e2e1 = torch.cuda.Event(enable_timing=True)
+    e2e0.record(stream)
+    for i in range(args.steps):
+        for mat, xd, yd, xh, yh, *_ in layers[i % args.copies]:
+            xd.copy_(xh, non_blocking=True)
+            launch(mat, xd, yd)
+            yh.copy_(yd, non_blocking=True)
+    e2e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = allreduce_max(e2e0.elapsed_time(e2e1), world)
+    e2e_val = total_bytes * world / (e2e_ms / 1e3) / 1e9
+
+    if rank == 0:
+        peak, peak_kind = peaks()
+        achieved = launch_bytes / (launch_ms / 1e3) / 1e9
+        cpu = cpu_baseline(B, args.cpu_budget) if (world == 1 and args.cpu_budget > 0) else None
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "fp32", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "batch": B, "tile_rows": R,
+                       "weights": "seeded synthetic VBQ groups: P(1,2,4,8 bit) = (0.69,0.16,0.09,0.06), fp16 "
+                                  "scales U(0.01,0.1), uniform codes; x ~ N(0,1) bf16",
+                       "l2": f"inputs larger than L2: {args.copies} distinct layer copies in rotation "
+                             f"({sum(step_bytes) / 1e6:.0f} MB of weights)",
+                       "parallelism": f"replicas x{world}"},
+            "pct_of_peak": 100.0 * value / world / peak,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": None, "peak_kind": peak_kind,
+                         "kernel": "vbq_kernel<1>",
+                         "algorithmic_bytes_per_launch": launch_bytes / len(ev)},
+            "per_linear": {k: {"us": v[0] / v[2] * 1e3, "GBps": v[1] / (v[0] / 1e3) / 1e9}
+                           for k, v in per_shape.items()},
+            "e2e": {"value": e2e_val, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": len(ev),
+            "clocks": clocks,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        barrier(world)
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--batch", type=int, default=1, choices=(1, 2, 4, 8, 16))
+    ap.add_argument("--impl", default="vbq", choices=("vbq", "reference"))
+    ap.add_argument("--copies", type=int, default=4)
+    ap.add_argument("--tile-rows", type=int, default=1024)
+    ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds for the CPU-oracle baseline (0: skip)")
+    ap.add_argument("--ref-rows", type=int, default=256, help="rows per linear per step for --impl reference")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_vbq(args)
+
+
+if __name__ == "__main__":
+    main()

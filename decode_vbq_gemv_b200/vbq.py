@@ -1,0 +1,245 @@
+"""Thin Python binding of libvbq (include/vbq.h): argument marshalling only.
+
+Each ``vbq_*`` function here calls the C entry point of the same name. Host arrays are numpy arrays. Device
+buffers and streams are torch CUDA tensors and streams, because PyTorch only provides device memory and streams.
+All work runs inside libvbq: the packer in C++ and the products in the sm_100a CUDA kernels. Nothing falls back to
+Python or to a CPU path. If the library is missing or fails to load, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+VBQ_OK = 0
+VBQ_ERR_NULL, VBQ_ERR_SHAPE, VBQ_ERR_WIDTH, VBQ_ERR_CODE_RANGE = -1, -2, -3, -4
+VBQ_ERR_BUFFER_TOO_SMALL, VBQ_ERR_BAD_MAGIC, VBQ_ERR_VERSION, VBQ_ERR_CRC = -5, -6, -7, -8
+VBQ_ERR_BATCH, VBQ_ERR_ALIGN, VBQ_ERR_CUDA, VBQ_ERR_TILE = -9, -10, -11, -12
+VBQ_ERR_FORMAT, VBQ_ERR_WORKSPACE = -13, -14
+BATCHES = (1, 2, 4, 8, 16)
+DEFAULT_TILE_ROWS = 1024
+
+
+class VbqError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {vbq_strerror(status)} (status {status})")
+        self.status = status
+
+
+class vbq_desc(ctypes.Structure):
+    _fields_ = [("version", ctypes.c_uint32), ("flags", ctypes.c_uint32), ("N", ctypes.c_int64),
+                ("K", ctypes.c_int64), ("G", ctypes.c_int64), ("R", ctypes.c_int64), ("T", ctypes.c_int64),
+                ("dir_offset", ctypes.c_uint64), ("rec_offset", ctypes.c_uint64),
+                ("total_bytes", ctypes.c_uint64)]
+
+
+_lib = None
+
+
+def library_path() -> str:
+    return _build.LIB
+
+
+def lib() -> ctypes.CDLL:
+    """Loads libvbq.so, building it first if the sources are newer. Raises if it cannot be built or loaded."""
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        if not os.path.exists(path):
+            raise RuntimeError(f"libvbq.so missing at {path}")
+        L = ctypes.CDLL(path)
+        vp, i64, u64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_uint64, ctypes.c_int
+        dp = ctypes.POINTER(vbq_desc)
+        sig = {
+            "vbq_strerror": (ctypes.c_char_p, [i32]),
+            "vbq_version": (ctypes.c_uint32, []),
+            "vbq_packed_size": (i32, [i64, i64, i64, vp, ctypes.POINTER(u64)]),
+            "vbq_pack": (i32, [i64, i64, i64, vp, vp, vp, vp, u64, dp]),
+            "vbq_describe": (i32, [vp, u64, dp]),
+            "vbq_unpack": (i32, [vp, u64, vp, vp, vp]),
+            "vbq_workspace_size": (i32, [dp, i32, ctypes.POINTER(u64)]),
+            "vbq_workspace_init": (i32, [vp, u64, vp]),
+            "vbq_gemv": (i32, [dp, vp, vp, vp, vp, u64, vp]),
+            "vbq_gemm_skinny": (i32, [dp, vp, vp, i32, vp, vp, u64, vp]),
+        }
+        for name, (res, args) in sig.items():
+            f = getattr(L, name)
+            f.restype, f.argtypes = res, args
+        _lib = L
+    return _lib
+
+
+def _np_ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _dev_ptr(t) -> int:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    return t.data_ptr()
+
+
+def _stream_ptr(stream) -> int | None:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    return getattr(stream, "cuda_stream", stream)
+
+
+def _check(st: int, where: str):
+    if st != VBQ_OK:
+        raise VbqError(st, where)
+
+
+def vbq_strerror(status: int) -> str:
+    return lib().vbq_strerror(status).decode()
+
+
+def vbq_version() -> int:
+    return int(lib().vbq_version())
+
+
+def vbq_packed_size(N: int, K: int, R: int, widths: np.ndarray) -> int:
+    w = np.ascontiguousarray(widths, np.uint8)
+    out = ctypes.c_uint64()
+    _check(lib().vbq_packed_size(N, K, R, _np_ptr(w), ctypes.byref(out)), "vbq_packed_size")
+    return int(out.value)
+
+
+def vbq_pack_status(N, K, R, widths, scales, codes, cap: int | None = None):
+    """Returns (status, blob[uint8] or None, vbq_desc)."""
+    w = np.ascontiguousarray(widths, np.uint8)
+    s = np.ascontiguousarray(scales, np.uint16)
+    c = np.ascontiguousarray(codes, np.uint8)
+    d = vbq_desc()
+    if cap is None:
+        out = ctypes.c_uint64()
+        st = lib().vbq_packed_size(N, K, R, _np_ptr(w), ctypes.byref(out))
+        if st != VBQ_OK:
+            return st, None, d
+        cap = int(out.value)
+    blob = np.zeros(max(cap, 1), np.uint8)
+    st = lib().vbq_pack(N, K, R, _np_ptr(w), _np_ptr(s), _np_ptr(c), _np_ptr(blob), cap, ctypes.byref(d))
+    return st, (blob[: d.total_bytes] if st == VBQ_OK else None), d
+
+
+def vbq_pack(N: int, K: int, R: int, widths, scales, codes):
+    """Packs a logical matrix. Returns (blob as uint8 numpy array, vbq_desc)."""
+    st, blob, d = vbq_pack_status(N, K, R, widths, scales, codes)
+    _check(st, "vbq_pack")
+    return blob, d
+
+
+def vbq_describe_status(blob: np.ndarray):
+    b = np.ascontiguousarray(blob, np.uint8)
+    d = vbq_desc()
+    return lib().vbq_describe(_np_ptr(b), b.size, ctypes.byref(d)), d
+
+
+def vbq_describe(blob: np.ndarray) -> vbq_desc:
+    st, d = vbq_describe_status(blob)
+    _check(st, "vbq_describe")
+    return d
+
+
+def vbq_unpack_status(blob: np.ndarray):
+    b = np.ascontiguousarray(blob, np.uint8)
+    st, d = vbq_describe_status(b)
+    if st != VBQ_OK:
+        return st, None
+    widths = np.zeros((d.N, d.G), np.uint8)
+    scales = np.zeros((d.N, d.G), np.uint16)
+    codes = np.zeros((d.N, d.K), np.uint8)
+    st = lib().vbq_unpack(_np_ptr(b), b.size, _np_ptr(widths), _np_ptr(scales), _np_ptr(codes))
+    return st, ((widths, scales, codes) if st == VBQ_OK else None)
+
+
+def vbq_unpack(blob: np.ndarray):
+    """Returns (widths[N,G], scales[N,G] fp16 bits, codes[N,K])."""
+    st, out = vbq_unpack_status(blob)
+    _check(st, "vbq_unpack")
+    return out
+
+
+def vbq_workspace_size(desc: vbq_desc, B: int) -> int:
+    out = ctypes.c_uint64()
+    _check(lib().vbq_workspace_size(ctypes.byref(desc), B, ctypes.byref(out)), "vbq_workspace_size")
+    return int(out.value)
+
+
+def vbq_workspace_init(workspace, stream=None) -> None:
+    if workspace is None or workspace.numel() == 0:
+        return
+    _check(lib().vbq_workspace_init(_dev_ptr(workspace), workspace.numel() * workspace.element_size(),
+                                    _stream_ptr(stream)), "vbq_workspace_init")
+
+
+def vbq_gemm_skinny_status(desc, blob_dev, x_bf16, B, y, workspace=None, stream=None) -> int:
+    ws_ptr = _dev_ptr(workspace) if workspace is not None and workspace.numel() > 0 else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    return lib().vbq_gemm_skinny(ctypes.byref(desc), _dev_ptr(blob_dev), _dev_ptr(x_bf16), B, _dev_ptr(y),
+                                 ws_ptr, ws_bytes, _stream_ptr(stream))
+
+
+def vbq_gemm_skinny(desc, blob_dev, x_bf16, B, y, workspace=None, stream=None) -> None:
+    """Y[B,N] = X[B,K] W^T on the device (asynchronous on `stream`, default: torch's current stream)."""
+    _check(vbq_gemm_skinny_status(desc, blob_dev, x_bf16, B, y, workspace, stream), "vbq_gemm_skinny")
+
+
+def vbq_gemv(desc, blob_dev, x_bf16, y, workspace=None, stream=None) -> None:
+    """y[N] = W x[K] on the device (batch 1)."""
+    ws_ptr = _dev_ptr(workspace) if workspace is not None and workspace.numel() > 0 else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(lib().vbq_gemv(ctypes.byref(desc), _dev_ptr(blob_dev), _dev_ptr(x_bf16), _dev_ptr(y), ws_ptr,
+                          ws_bytes, _stream_ptr(stream)), "vbq_gemv")
+
+
+class DeviceMatrix:
+    """A packed VBQ matrix resident on one CUDA device, plus a workspace sized for the largest batch used.
+
+    ``blob`` is a host numpy uint8 array (the canonical packed bytes). It is copied to the device once.
+    """
+
+    def __init__(self, blob: np.ndarray, device="cuda", max_batch: int = 16):
+        import torch
+        self.desc = vbq_describe(blob)
+        self.N, self.K = int(self.desc.N), int(self.desc.K)
+        self.device = torch.device(device)
+        host = torch.from_numpy(np.ascontiguousarray(blob, np.uint8))
+        self.blob = torch.empty(host.numel(), dtype=torch.uint8, device=self.device)
+        self.blob.copy_(host)
+        self.workspaces = {}
+        for B in BATCHES:
+            if B <= max_batch:
+                self.workspaces[B] = self._alloc_ws(B)
+
+    def _alloc_ws(self, B):
+        import torch
+        n = vbq_workspace_size(self.desc, B)
+        ws = torch.zeros(max((n + 15) // 16, 1) * 16, dtype=torch.uint8, device=self.device)
+        return ws
+
+    @property
+    def nbytes(self) -> int:
+        return int(self.desc.total_bytes)
+
+    def matmul(self, x_bf16, out=None, stream=None):
+        """x_bf16: torch.bfloat16 [B, K] (or [K]) on the device. Returns fp32 [B, N] (or [N])."""
+        import torch
+        squeeze = x_bf16.dim() == 1
+        x2 = x_bf16.reshape(-1, self.K)
+        B = x2.shape[0]
+        if out is None:
+            out = torch.empty((B, self.N), dtype=torch.float32, device=self.device)
+        ws = self.workspaces.get(B)
+        if ws is None:
+            ws = self.workspaces[B] = self._alloc_ws(B)
+        vbq_gemm_skinny(self.desc, self.blob, x2, B, out, ws, stream)
+        return out.reshape(self.N) if squeeze else out

@@ -1,0 +1,131 @@
+/*
+ * vbq.h: C ABI of the VBQ mixed-bit GEMV / skinny-GEMM library (libvbq.so).
+ *
+ * VBQ ("Variable Bit-width Quantization: Learning Per-Group Precision for 'Bigger-but-Smaller' Language
+ * Models") cuts each weight row into contiguous groups of 64 weights. Each group has its own scale and its
+ * own width from {1,2,4,8} bits (section 3.1). At decode time, fused kernels read the packed low-bit bytes of
+ * a group, expand them with the group scale in registers, and accumulate the matrix-vector product. The
+ * dense FP16 matrix is never built (section 6, paragraph "Fused kernels over packed weights").
+ *
+ * The dequantized weight is w = s * (q - (2^k - 1)/2), with q in [0, 2^k). The byte layout is "format v1" of
+ * FORMAT.md: row tiles, one record per (tile, group column), and per-width buckets inside each record.
+ *
+ * Conventions for every function:
+ *  - The return value is a status: VBQ_OK (0) or a negative VBQ_ERR_* code. No function aborts, exits or
+ *    prints.
+ *  - The caller owns and allocates every buffer. No function allocates or frees host or device memory.
+ *  - Logical host arrays are row-major: widths[N*G] (values 1,2,4,8), scales[N*G] (IEEE fp16 bit patterns),
+ *    codes[N*K] (one byte per weight, q < 2^width), with G = K/64.
+ *  - Device functions are asynchronous on the given CUDA stream (a cudaStream_t passed as void*; NULL is the
+ *    legacy default stream). They never synchronize. A launch failure is reported as VBQ_ERR_CUDA, read with
+ *    cudaPeekAtLastError (the sticky error state is not cleared).
+ */
+#ifndef VBQ_H_
+#define VBQ_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum vbq_status {
+  VBQ_OK = 0,
+  VBQ_ERR_NULL = -1,              /* a required pointer is NULL */
+  VBQ_ERR_SHAPE = -2,             /* N < 1, K < 64, K % 64 != 0, or N or K above 2^31 - 1 */
+  VBQ_ERR_WIDTH = -3,             /* a width is not 1, 2, 4 or 8 */
+  VBQ_ERR_CODE_RANGE = -4,        /* a code is >= 2^width */
+  VBQ_ERR_BUFFER_TOO_SMALL = -5,  /* output capacity or blob size too small */
+  VBQ_ERR_BAD_MAGIC = -6,         /* blob does not start with "VBQ1" */
+  VBQ_ERR_VERSION = -7,           /* unsupported format version */
+  VBQ_ERR_CRC = -8,               /* header or body CRC-32 mismatch */
+  VBQ_ERR_BATCH = -9,             /* batch B not in {1, 2, 4, 8, 16} */
+  VBQ_ERR_ALIGN = -10,            /* a device pointer breaks its alignment rule */
+  VBQ_ERR_CUDA = -11,             /* a CUDA runtime call or launch failed */
+  VBQ_ERR_TILE = -12,             /* tile rows R not a multiple of 16 in [16, 1024] */
+  VBQ_ERR_FORMAT = -13,           /* blob is not canonical format v1 (layout, padding, counts) */
+  VBQ_ERR_WORKSPACE = -14         /* workspace NULL, misaligned or smaller than vbq_workspace_size */
+} vbq_status;
+
+/* Host-side description of a packed blob. It is filled by vbq_pack or vbq_describe and passed by pointer to
+ * the device entry points, so the library never reads device memory from the host. */
+typedef struct vbq_desc {
+  uint32_t version;      /* format version (1) */
+  uint32_t flags;        /* 0 */
+  int64_t N;             /* output rows */
+  int64_t K;             /* input columns, multiple of 64 */
+  int64_t G;             /* K / 64 */
+  int64_t R;             /* rows per tile */
+  int64_t T;             /* ceil(N / R) tiles */
+  uint64_t dir_offset;   /* byte offset of the record directory */
+  uint64_t rec_offset;   /* byte offset of the first record */
+  uint64_t total_bytes;  /* blob size in bytes */
+} vbq_desc;
+
+/* Static English text for a status code; never NULL. */
+const char* vbq_strerror(int status);
+
+/* Library version as (major << 16 | minor); the packed format it reads and writes is version 1. */
+uint32_t vbq_version(void);
+
+/* ---------------------------------------------------------------------------------------------- host */
+
+/* Bytes of the canonical blob for this logical matrix (FORMAT.md, "Physical layout").
+ * widths: [N*G] in {1,2,4,8}. R: tile rows. Errors: NULL, SHAPE, TILE, WIDTH. Thread-safe, pure. */
+int vbq_packed_size(int64_t N, int64_t K, int64_t R, const uint8_t* widths, uint64_t* out_bytes);
+
+/* Pack a logical matrix into a canonical format-v1 blob written to out[0 .. *size). This is the export-time
+ * step of the VBQ paper's section 6 ("An export-time check validates this contract"): it validates every
+ * width and code first and writes nothing on error.
+ * Errors: NULL, SHAPE, TILE, WIDTH, CODE_RANGE, BUFFER_TOO_SMALL (out_cap < vbq_packed_size).
+ * out_desc may be NULL. Thread-safe, pure. */
+int vbq_pack(int64_t N, int64_t K, int64_t R, const uint8_t* widths, const uint16_t* scales,
+             const uint8_t* codes, void* out, uint64_t out_cap, vbq_desc* out_desc);
+
+/* Validate a host copy of a blob and fill *out_desc. Checks, in order: size >= 64 (BUFFER_TOO_SMALL), magic
+ * (BAD_MAGIC), version (VERSION), header CRC (CRC), header fields (FORMAT), total_bytes <= blob_bytes
+ * (BUFFER_TOO_SMALL), body CRC (CRC). It does not walk the records; vbq_unpack does. */
+int vbq_describe(const void* blob_host, uint64_t blob_bytes, vbq_desc* out_desc);
+
+/* Unpack a canonical blob (host memory) back into logical arrays sized from its header (N*G, N*G, N*K).
+ * Performs every vbq_describe check, then checks each record: counts agree with the width codes, and every
+ * padding byte and unused bit is zero (FORMAT). Any output pointer may be NULL to validate only. */
+int vbq_unpack(const void* blob_host, uint64_t blob_bytes, uint8_t* widths, uint16_t* scales,
+               uint8_t* codes);
+
+/* -------------------------------------------------------------------------------------------- device */
+
+/* Workspace bytes that vbq_gemv / vbq_gemm_skinny need for this matrix and batch on the CURRENT device (the
+ * launch shape depends on its SM count). The workspace holds per-CTA partial sums of split-K launches and one
+ * arrival counter per row tile. It may be 0 (then any pointer, including NULL, is accepted).
+ * Errors: NULL, BATCH, FORMAT (desc inconsistent), CUDA. */
+int vbq_workspace_size(const vbq_desc* d, int B, uint64_t* out_bytes);
+
+/* Zero a workspace before its first use (cudaMemsetAsync on `stream`). Every kernel call leaves the arrival
+ * counters at zero again, so one zeroing per workspace is enough. Errors: NULL, CUDA. */
+int vbq_workspace_init(void* workspace, uint64_t workspace_bytes, void* stream);
+
+/* y[N] = W x for one activation vector (batch 1): vbq_gemm_skinny with B = 1.
+ * blob_dev: byte-identical device copy of the packed blob, 16-byte aligned (ALIGN).
+ * x_bf16:   K bf16 values (device), 16-byte aligned (ALIGN).
+ * y:        N fp32 values (device), 4-byte aligned; fully overwritten.
+ * workspace: vbq_workspace_size(d, 1) device bytes, 16-byte aligned, zeroed once by vbq_workspace_init; it
+ *           must not be shared by calls that can run at the same time.
+ * Result per element: |y - y_exact| <= 1e-3 * sum_i |w_i||x_i| + 1e-6, with fp32 accumulation. Results are
+ * bitwise identical from run to run (no floating-point atomics). */
+int vbq_gemv(const vbq_desc* d, const void* blob_dev, const void* x_bf16, float* y, void* workspace,
+             uint64_t workspace_bytes, void* stream);
+
+/* Y[B][N] = X[B][K] W^T for B in {1, 2, 4, 8, 16} activation rows (skinny GEMM; decode with a small batch).
+ * x_bf16: B*K bf16 values, row-major (row b is activation b), 16-byte aligned. y: B*N fp32, row-major.
+ * B <= 4 runs on CUDA cores; B = 8 and 16 run the dequantized groups through tensor cores (bf16 operands
+ * that hold the exact odd integers 2q - (2^k - 1), fp32 accumulation, the group scale applied in fp32).
+ * Other arguments and guarantees as in vbq_gemv. Errors: NULL, BATCH, ALIGN, WORKSPACE, FORMAT, CUDA. */
+int vbq_gemm_skinny(const vbq_desc* d, const void* blob_dev, const void* x_bf16, int B, float* y,
+                    void* workspace, uint64_t workspace_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VBQ_H_ */

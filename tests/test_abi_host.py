@@ -1,0 +1,132 @@
+"""Host-side tests of the C ABI (no GPU needed): symbol exports, the packer against the oracle (byte-exact),
+unpack and validation error codes against the oracle's, and the argument checks of the device entry points
+that run before any CUDA call."""
+import ctypes
+import os
+import re
+import zlib
+
+import numpy as np
+import pytest
+
+import vbq_synth as S
+from decode_vbq_gemv_b200 import vbq
+from oracle import oracle as O
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def header_functions():
+    txt = open(os.path.join(ROOT, "include", "vbq.h")).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    return sorted(set(re.findall(r"\b(vbq_[a-z_0-9]+)\s*\(", txt)))
+
+
+def test_library_exports_every_declared_symbol():
+    names = header_functions()
+    assert "vbq_gemv" in names and "vbq_gemm_skinny" in names and "vbq_pack" in names
+    L = ctypes.CDLL(vbq.library_path() if os.path.exists(vbq.library_path()) else vbq.lib()._name)
+    for n in names:
+        assert hasattr(L, n), f"libvbq.so does not export {n}"
+
+
+def test_status_strings_and_version():
+    for st in range(-14, 1):
+        assert vbq.vbq_strerror(st) and "unknown" not in vbq.vbq_strerror(st)
+    assert vbq.vbq_strerror(-99) == "unknown status"
+    assert vbq.vbq_version() >> 16 == 1
+
+
+def logical(seed, N, K, p=S.P_BASE):
+    g = np.random.default_rng(seed)
+    w = S.widths_iid(N, K // 64, p, g)
+    return w, S.scales_uniform(N, K // 64, g), S.codes_uniform(w, g)
+
+
+SHAPES = [(1, 64, 16), (5, 128, 16), (31, 192, 32), (100, 768, 64), (1030, 256, 1024), (1024, 64, 1024),
+          (2049, 128, 512), (17, 320, 1024)]
+
+
+@pytest.mark.parametrize("N,K,R", SHAPES)
+@pytest.mark.parametrize("p", [S.P_BASE, (0.25, 0.25, 0.25, 0.25), (0, 0, 0, 1.0), (1.0, 0, 0, 0)])
+def test_pack_matches_oracle_bytes(N, K, R, p):
+    w, s, c = logical(N * 7 + K + R, N, K, p)
+    blob, d = vbq.vbq_pack(N, K, R, w, s, c)
+    ref = O.pack(N, K, R, w, s, c)
+    assert np.array_equal(blob, ref)
+    assert vbq.vbq_packed_size(N, K, R, w) == ref.size
+    assert (d.N, d.K, d.G, d.R, d.T, d.total_bytes) == (N, K, K // 64, R, (N + R - 1) // R, ref.size)
+    w2, s2, c2 = vbq.vbq_unpack(ref)
+    assert np.array_equal(w2, w) and np.array_equal(s2, s) and np.array_equal(c2, c)
+
+
+def test_pack_matches_oracle_on_workload_configs():
+    for m in S.cfg1() + S.cfg2()[:1] + [S.cfg3(256, 512)[4]]:
+        blob, _ = vbq.vbq_pack(m.N, m.K, 1024, m.widths, m.scales, m.codes)
+        assert np.array_equal(blob, O.pack(m.N, m.K, 1024, m.widths, m.scales, m.codes))
+
+
+def test_pack_error_codes_match_oracle():
+    w, s, c = logical(1, 6, 128)
+    cases = [(6, 100, 16, w, s, c), (6, 128, 8, w, s, c), (6, 128, 2048, w, s, c), (0, 128, 16, w, s, c)]
+    bad_w = w.copy(); bad_w[2, 1] = 5
+    cases.append((6, 128, 16, bad_w, s, c))
+    bad_c = c.copy(); r, g = np.argwhere(w < 8)[0]; bad_c[r, 64 * g + 3] = 1 << int(w[r, g])
+    cases.append((6, 128, 16, w, s, bad_c))
+    for args in cases:
+        st_lib = vbq.vbq_pack_status(*args)[0]
+        st_ora = O.pack_status(*args)[0]
+        assert st_lib == st_ora and st_lib < 0, (st_lib, st_ora)
+    size = vbq.vbq_packed_size(6, 128, 16, w)
+    assert vbq.vbq_pack_status(6, 128, 16, w, s, c, cap=size - 1)[0] == vbq.VBQ_ERR_BUFFER_TOO_SMALL
+
+
+def _refresh_crc(b):
+    b = b.copy()
+    b[56:60] = np.frombuffer(zlib.crc32(b[64:].tobytes()).to_bytes(4, "little"), np.uint8)
+    b[60:64] = np.frombuffer(zlib.crc32(b[:60].tobytes()).to_bytes(4, "little"), np.uint8)
+    return b
+
+
+def test_unpack_error_codes_match_oracle():
+    w, s, c = logical(2, 70, 192)
+    blob = O.pack(70, 192, 32, w, s, c)
+    rng = np.random.default_rng(0)
+    variants = [blob[:10], blob[:-16], blob.copy(), blob.copy(), blob.copy(), blob.copy()]
+    variants[2][0] ^= 0xFF
+    variants[3][4] = 9
+    variants[4][100] ^= 1
+    variants[5][-3] ^= 4
+    # single-byte corruptions anywhere, with the CRCs made consistent again so the layout checks decide
+    for _ in range(300):
+        b = blob.copy()
+        i = int(rng.integers(64, blob.size))
+        b[i] ^= np.uint8(1 << int(rng.integers(0, 8)))
+        variants.append(_refresh_crc(b))
+    for b in variants:
+        st_lib = vbq.vbq_unpack_status(b)[0]
+        st_ora = O.unpack_status(b)[0]
+        assert st_lib == st_ora, (st_lib, st_ora)
+        if st_lib == 0:   # a corruption that still decodes must decode identically
+            lw, ls, lc = vbq.vbq_unpack_status(b)[1]
+            ow, os_, oc, _ = O.unpack_status(b)[1]
+            assert np.array_equal(lw, ow) and np.array_equal(ls, os_) and np.array_equal(lc, oc)
+
+
+def test_device_entry_argument_checks_need_no_gpu():
+    w, s, c = logical(3, 40, 128)
+    _, d = vbq.vbq_pack(40, 128, 16, w, s, c)
+    L = vbq.lib()
+    dp = ctypes.byref(d)
+    assert L.vbq_gemv(dp, None, 16, 16, None, 0, None) == vbq.VBQ_ERR_NULL
+    assert L.vbq_gemm_skinny(dp, 16, 16, 3, 16, None, 0, None) == vbq.VBQ_ERR_BATCH
+    assert L.vbq_gemm_skinny(dp, 8, 16, 1, 16, None, 0, None) == vbq.VBQ_ERR_ALIGN
+    assert L.vbq_gemm_skinny(dp, 16, 18, 1, 16, None, 0, None) == vbq.VBQ_ERR_ALIGN
+    assert L.vbq_gemm_skinny(dp, 16, 16, 1, 18, None, 0, None) == vbq.VBQ_ERR_ALIGN
+    bad = vbq.vbq_desc.from_buffer_copy(d)
+    bad.K = 100
+    assert L.vbq_gemv(ctypes.byref(bad), 16, 16, 16, None, 0, None) == vbq.VBQ_ERR_FORMAT
+    out = ctypes.c_uint64()
+    assert L.vbq_workspace_size(dp, 3, ctypes.byref(out)) == vbq.VBQ_ERR_BATCH
+    assert L.vbq_workspace_size(dp, 16, ctypes.byref(out)) == vbq.VBQ_OK
+    assert L.vbq_workspace_init(None, 0, None) == vbq.VBQ_ERR_NULL

@@ -1,0 +1,187 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle, element by element.
+
+Bar: |y - y_ref| <= 1e-3 * sum_i |w_i||x_i| + 1e-6 per element (fp32 accumulation), bit-exact for one-hot
+activations, bitwise identical across runs. Full-size matrices are checked on sampled rows, which the oracle
+computes one by one.
+"""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import vbq_synth as S
+from decode_vbq_gemv_b200 import vbq
+from oracle import oracle as O
+
+pytestmark = pytest.mark.gpu
+NTH = os.cpu_count() or 1
+
+
+def dev():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    return torch.device("cuda:0")
+
+
+def to_dev_x(xbits: np.ndarray):
+    t = torch.from_numpy(xbits.astype(np.int16)).view(torch.bfloat16)
+    return t.to(dev()).contiguous()
+
+
+def gpu_y(m, xbits, R=1024, mat=None):
+    if mat is None:
+        blob, _ = vbq.vbq_pack(m.N, m.K, R, m.widths, m.scales, m.codes)
+        mat = vbq.DeviceMatrix(blob, dev())
+    y = mat.matmul(to_dev_x(xbits))
+    torch.cuda.synchronize()
+    return y.cpu().numpy().astype(np.float64), mat
+
+
+def check(y, yref, bound, what=""):
+    ok = O.within_tolerance(y, yref, bound)
+    if not ok.all():
+        i = np.argwhere(~ok)[0]
+        raise AssertionError(f"{what}: {int((~ok).sum())} elements out of tolerance; first {tuple(i)}: "
+                             f"got {y[tuple(i)]!r} want {yref[tuple(i)]!r} bound {bound[tuple(i)]!r}")
+
+
+def logical(seed, N, K, p):
+    g = np.random.default_rng(seed)
+    w = S.widths_iid(N, K // 64, p, g)
+    return S.Matrix("t", N, K, w, S.scales_uniform(N, K // 64, g), S.codes_uniform(w, g))
+
+
+SMALL = [(1, 64, 16), (31, 192, 16), (100, 768, 64), (1030, 256, 1024), (2100, 128, 512), (64, 1024, 32),
+         (777, 2048, 256)]
+DISTS = {"base": S.P_BASE, "flat": (0.25, 0.25, 0.25, 0.25), "all8": (0, 0, 0, 1.0), "all1": (1.0, 0, 0, 0)}
+
+
+@pytest.mark.parametrize("B", vbq.BATCHES)
+@pytest.mark.parametrize("shape", SMALL)
+@pytest.mark.parametrize("dist", list(DISTS))
+def test_small_shapes_all_batches(shape, dist, B):
+    N, K, R = shape
+    m = logical(N + K + R + B, N, K, DISTS[dist])
+    x = S.x_normal(B, K, np.random.default_rng(B + N))
+    y, _ = gpu_y(m, x, R)
+    yref, bound = O.matvec(m.widths, m.scales, m.codes, x, NTH)
+    check(y, yref, bound, f"{shape} {dist} B={B}")
+
+
+@pytest.mark.parametrize("B", vbq.BATCHES)
+def test_config1_single_linear(B):
+    m = S.cfg1()[0]
+    x = S.make_x(1, "single", B, m.K)
+    y, _ = gpu_y(m, x)
+    yref, bound = O.matvec(m.widths, m.scales, m.codes, x, NTH)
+    check(y, yref, bound, f"cfg1 B={B}")
+
+
+@pytest.mark.parametrize("B", [1, 4, 16])
+def test_config2_layer(B):
+    for m in S.cfg2():
+        x = S.make_x(2, m.name, B, m.K)
+        y, _ = gpu_y(m, x)
+        yref, bound = O.matvec(m.widths, m.scales, m.codes, x, NTH)
+        check(y, yref, bound, f"cfg2 {m.name} B={B}")
+
+
+@pytest.mark.parametrize("B", [1, 2, 8, 16])
+def test_config3_uniform_widths_full(B):
+    for m in S.cfg3():
+        x = S.make_x(3, "single", B, m.K)
+        y, _ = gpu_y(m, x)
+        yref, bound = O.matvec(m.widths, m.scales, m.codes, x, NTH)
+        check(y, yref, bound, f"cfg3 {m.name} B={B}")
+
+
+@pytest.mark.parametrize("k", [1, 2, 4, 8])
+@pytest.mark.parametrize("B", [1, 4, 16])
+def test_closed_form_all_max_codes(k, B):
+    N, K = 4096, 4096
+    m = S.Matrix("cf", N, K, np.full((N, K // 64), k, np.uint8), np.full((N, K // 64), 0x2E66, np.uint16),
+                 np.full((N, K), (1 << k) - 1, np.uint8))
+    x = S.x_normal(B, K, np.random.default_rng(k))
+    y, _ = gpu_y(m, x)
+    xs = torch.from_numpy(x.astype(np.int16)).view(torch.bfloat16).double().numpy()
+    s0 = float(np.uint16(0x2E66).view(np.float16))
+    want = (s0 * ((1 << k) - 1) / 2 * xs.sum(axis=1))[:, None] * np.ones((1, N))
+    bound = (s0 * ((1 << k) - 1) / 2 * np.abs(xs).sum(axis=1))[:, None] * np.ones((1, N))
+    check(y, want, bound, f"closed form k={k} B={B}")
+    assert np.all(y == y[:, :1]), "all rows are identical, so their outputs must be bitwise equal"
+
+
+@pytest.mark.parametrize("B", vbq.BATCHES)
+def test_config4_full_size_sampled_rows(B):
+    g = np.random.default_rng(B)
+    for m in S.cfg4(("q", "gate", "down")):
+        x = S.make_x(4, m.name, B, m.K)
+        y, _ = gpu_y(m, x)
+        rows = np.unique(np.concatenate([g.choice(m.N, 200, replace=False), [0, m.N - 1, 1023, 1024]]))
+        yref, bound = O.matvec(m.widths[rows], m.scales[rows], m.codes[rows], x, NTH)
+        check(y[:, rows], yref, bound, f"cfg4 {m.name} B={B}")
+
+
+@pytest.mark.parametrize("B", [1, 2, 8, 16])
+def test_lm_head_sampled_rows(B):
+    m = S.cfg5_head()
+    x = S.make_x(5, "head", B, m.K)
+    y, _ = gpu_y(m, x)
+    rows = np.unique(np.concatenate([np.arange(0, 3000, 7), np.random.default_rng(0).choice(m.N, 300), [m.N - 1]]))
+    yref, bound = O.matvec(m.widths[rows], m.scales[rows], m.codes[rows], x, NTH)
+    check(y[:, rows], yref, bound, f"head B={B}")
+
+
+@pytest.mark.parametrize("B", vbq.BATCHES)
+def test_one_hot_columns_bit_exact(B):
+    m = logical(5, 300, 256, (0.25, 0.25, 0.25, 0.25))
+    deq = O.dequant(m.widths, m.scales, m.codes)
+    cols = [0, 63, 64, 130, 255][:B] + [7] * max(0, B - 5)
+    x = np.zeros((B, m.K), np.uint16)
+    for b, i in enumerate(cols):
+        x[b, i] = 0x3F80
+    y, _ = gpu_y(m, x, R=64)
+    for b, i in enumerate(cols):
+        assert np.array_equal(y[b], deq[:, i]), f"B={B} column {i}"
+
+
+@pytest.mark.parametrize("B", vbq.BATCHES)
+def test_deterministic_across_runs(B):
+    m = S.cfg4(("gate",))[0]
+    x = S.make_x(4, "gate", B, m.K)
+    y1, mat = gpu_y(m, x)
+    y2, _ = gpu_y(m, x, mat=mat)
+    assert np.array_equal(y1, y2)
+
+
+def test_output_guard_regions_untouched():
+    m = logical(9, 1030, 512, S.P_BASE)
+    blob, _ = vbq.vbq_pack(m.N, m.K, 1024, m.widths, m.scales, m.codes)
+    mat = vbq.DeviceMatrix(blob, dev())
+    for B in vbq.BATCHES:
+        pad = 4096
+        buf = torch.full((B * m.N + 2 * pad,), 12345.0, dtype=torch.float32, device=dev())
+        y = buf[pad:pad + B * m.N].view(B, m.N)
+        x = to_dev_x(S.x_normal(B, m.K, np.random.default_rng(B)))
+        vbq.vbq_gemm_skinny(mat.desc, mat.blob, x, B, y, mat.workspaces[B])
+        torch.cuda.synchronize()
+        assert torch.all(buf[:pad] == 12345.0) and torch.all(buf[pad + B * m.N:] == 12345.0)
+        assert torch.isfinite(y).all()
+
+
+def test_abi_rejects_bad_device_arguments():
+    m = logical(11, 100, 256, S.P_BASE)
+    blob, _ = vbq.vbq_pack(m.N, m.K, 16, m.widths, m.scales, m.codes)
+    mat = vbq.DeviceMatrix(blob, dev())
+    x = torch.zeros(m.K + 8, dtype=torch.bfloat16, device=dev())
+    y = torch.zeros(m.N, dtype=torch.float32, device=dev())
+    st = vbq.vbq_gemm_skinny_status(mat.desc, mat.blob, x[1:1 + m.K], 1, y, mat.workspaces[1])
+    assert st == vbq.VBQ_ERR_ALIGN
+    need = vbq.vbq_workspace_size(mat.desc, 1)
+    if need > 0:
+        small = torch.zeros(need - 16, dtype=torch.uint8, device=dev())
+        st = vbq.vbq_gemm_skinny_status(mat.desc, mat.blob, x[:m.K], 1, y, small)
+        assert st == vbq.VBQ_ERR_WORKSPACE
+        assert vbq.vbq_gemm_skinny_status(mat.desc, mat.blob, x[:m.K], 1, y, None) == vbq.VBQ_ERR_WORKSPACE
+    torch.cuda.synchronize()
