@@ -209,7 +209,6 @@ def run_vbq(args):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     B, R = args.batch, args.tile_rows
-    stream = torch.cuda.current_stream()
 
     layers = []   # per copy: list of (DeviceMatrix, x_dev, y_dev, x_host_pinned, y_host_pinned, bytes)
     for cp in range(args.copies):
@@ -228,68 +227,89 @@ def run_vbq(args):
         layers.append(lin)
     step_bytes = [sum(l[5] for l in lin) for lin in layers]
 
-    def launch(mat, xd, yd):
-        vbq.vbq_gemm_skinny(mat.desc, mat.blob, xd, B, yd, mat.workspaces[B], stream)
+    def launch(mat, xd, yd, st):
+        vbq.vbq_gemm_skinny(mat.desc, mat.blob, xd, B, yd, mat.workspaces[B], st)
 
-    # ---- device-resident timing (value, roofline)
-    for i in range(args.warmup):
-        for mat, xd, yd, *_ in layers[i % args.copies]:
-            launch(mat, xd, yd)
+    # One CUDA graph per layer copy, so that the timed region has no host launch gaps: device-resident step
+    # (seven GEMVs) and end-to-end step (pinned x -> device, seven GEMVs, y -> pinned host).
+    stream = torch.cuda.Stream(dev)
+    graphs, graphs_e2e = [], []
+    with torch.cuda.stream(stream):
+        for lin in layers:
+            for mat, xd, yd, *_ in lin:
+                launch(mat, xd, yd, stream)
+        torch.cuda.synchronize()
+        for lin in layers:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for mat, xd, yd, *_ in lin:
+                    launch(mat, xd, yd, stream)
+            graphs.append(g)
+            g2 = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g2, stream=stream):
+                for mat, xd, yd, xh, yh, *_ in lin:
+                    xd.copy_(xh, non_blocking=True)
+                    launch(mat, xd, yd, stream)
+                    yh.copy_(yd, non_blocking=True)
+            graphs_e2e.append(g2)
     torch.cuda.synchronize()
-    barrier(world)
+    launches_per_step = len(NAMES)
+
+    def timed(gs):
+        for i in range(args.warmup):
+            gs[i % args.copies].replay()
+        torch.cuda.synchronize()
+        barrier(world)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for i in range(args.steps):
+                gs[i % args.copies].replay()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        return e0.elapsed_time(e1)
+
     sampler = ClockSampler(local)
     sampler.start()
     time.sleep(0.3)
-    ev = []
-    t_start = torch.cuda.Event(enable_timing=True)
-    t_end = torch.cuda.Event(enable_timing=True)
-    torch.cuda.synchronize()
-    t_start.record(stream)
-    total_bytes = 0
-    for i in range(args.steps):
-        lin = layers[i % args.copies]
-        for mat, xd, yd, _, _, nb, name in lin:
+    ms = timed(graphs)
+    clocks = sampler.stop()
+    total_bytes = sum(step_bytes[i % args.copies] for i in range(args.steps))
+    ms_max = allreduce_max(ms, world)
+    value = total_bytes * world / (ms_max / 1e3) / 1e9
+    launch_ms = ms / (args.steps * launches_per_step)
+    launch_bytes = total_bytes / (args.steps * launches_per_step)
+
+    # Per-linear kernel time: one graph of `reps` launches of that linear, timed alone (copy 0).
+    per_shape = {}
+    reps = 20
+    for k, (mat, xd, yd, *_rest) in enumerate(layers[0]):
+        name = NAMES[k]
+        with torch.cuda.stream(stream):
+            gl = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gl, stream=stream):
+                for _ in range(reps):
+                    launch(mat, xd, yd, stream)
+            gl.replay()
+            torch.cuda.synchronize()
             e0 = torch.cuda.Event(enable_timing=True)
             e1 = torch.cuda.Event(enable_timing=True)
             e0.record(stream)
-            launch(mat, xd, yd)
+            gl.replay()
             e1.record(stream)
-            ev.append((e0, e1, nb, name))
-        total_bytes += step_bytes[i % args.copies]
-    t_end.record(stream)
-    torch.cuda.synchronize()
-    barrier(world)
-    clocks = sampler.stop()
-    ms = t_start.elapsed_time(t_end)
-    ms_max = allreduce_max(ms, world)
-    launch_ms = sum(e0.elapsed_time(e1) for e0, e1, _, _ in ev)
-    launch_bytes = sum(nb for _, _, nb, _ in ev)
-    per_shape = {}
-    for e0, e1, nb, name in ev:
-        d = per_shape.setdefault(name, [0.0, 0.0, 0])
-        d[0] += e0.elapsed_time(e1); d[1] += nb; d[2] += 1
-    value = total_bytes * world / (ms_max / 1e3) / 1e9
+        torch.cuda.synchronize()
+        us = e0.elapsed_time(e1) * 1e3 / reps
+        nb = layers[0][k][5]
+        per_shape[name] = {"us": us, "GBps": nb / (us / 1e6) / 1e9, "note": "same matrix repeated (L2-warm)"}
 
-    # ---- end to end through host buffers: pinned x -> device, GEMV, y -> pinned host, every step
+    # End to end through host buffers.
     h2d = sum(l[3].numel() * 2 for l in layers[0])
     d2h = sum(l[4].numel() * 4 for l in layers[0])
-    for i in range(args.warmup):
-        for mat, xd, yd, xh, yh, *_ in layers[i % args.copies]:
-            xd.copy_(xh, non_blocking=True); launch(mat, xd, yd); yh.copy_(yd, non_blocking=True)
-    torch.cuda.synchronize()
-    barrier(world)
-    e2e0 = torch.cuda.Event(enable_timing=True)
-    e2e1 = torch.cuda.Event(enable_timing=True)
-    e2e0.record(stream)
-    for i in range(args.steps):
-        for mat, xd, yd, xh, yh, *_ in layers[i % args.copies]:
-            xd.copy_(xh, non_blocking=True)
-            launch(mat, xd, yd)
-            yh.copy_(yd, non_blocking=True)
-    e2e1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = allreduce_max(e2e0.elapsed_time(e2e1), world)
+    e2e_ms = allreduce_max(timed(graphs_e2e), world)
     e2e_val = total_bytes * world / (e2e_ms / 1e3) / 1e9
+    n_launches = args.steps * launches_per_step
 
     if rank == 0:
         peak, peak_kind = peaks()
@@ -308,12 +328,11 @@ def run_vbq(args):
             "pct_of_peak": 100.0 * value / world / peak,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": None, "peak_kind": peak_kind,
-                         "kernel": "vbq_kernel<1>",
-                         "algorithmic_bytes_per_launch": launch_bytes / len(ev)},
-            "per_linear": {k: {"us": v[0] / v[2] * 1e3, "GBps": v[1] / (v[0] / 1e3) / 1e9}
-                           for k, v in per_shape.items()},
+                         "kernel": f"vbq_kernel<{B}>",
+                         "algorithmic_bytes_per_launch": launch_bytes, "avg_launch_us": launch_ms * 1e3},
+            "per_linear": per_shape,
             "e2e": {"value": e2e_val, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-            "gpu_launches": len(ev),
+            "gpu_launches": n_launches,
             "clocks": clocks,
             "cpu_baseline": cpu,
         }

@@ -6,6 +6,7 @@
 // codes before writing anything, and writes only canonical blobs (zero padding), so the same logical matrix
 // always packs to the same bytes.
 #include <cstdint>
+#include <algorithm>
 #include <cstring>
 #include <vector>
 
@@ -107,7 +108,7 @@ int record_counts(const Geometry& geo, const uint8_t* widths, std::vector<uint32
   return VBQ_OK;
 }
 
-void fill_desc(const Geometry& geo, uint64_t total, vbq_desc* d) {
+void fill_desc(const Geometry& geo, uint64_t total, uint64_t max_rec, vbq_desc* d) {
   d->version = kVersion;
   d->flags = 0;
   d->N = geo.N;
@@ -118,6 +119,7 @@ void fill_desc(const Geometry& geo, uint64_t total, vbq_desc* d) {
   d->dir_offset = geo.dir_off;
   d->rec_offset = geo.rec_off;
   d->total_bytes = total;
+  d->max_record_bytes = max_rec;
 }
 
 // Writes one group's 64 k-bit codes as a little-endian bit string of 8k bytes (code i at bits [k*i, k*i+k)).
@@ -202,6 +204,8 @@ int vbq_pack(int64_t N, int64_t K, int64_t R, const uint8_t* widths, const uint1
       pos += RecordLayout(geo.tile_rows(t), &counts[size_t(t * geo.G + g) * 4]).bytes;
     }
   rec_start.back() = pos;
+  uint64_t max_rec = 0;
+  for (size_t i = 0; i + 1 < rec_start.size(); ++i) max_rec = std::max(max_rec, rec_start[i + 1] - rec_start[i]);
   const uint64_t total = geo.rec_off + pos;
   if (out_cap < total) return VBQ_ERR_BUFFER_TOO_SMALL;
 
@@ -248,7 +252,7 @@ int vbq_pack(int64_t N, int64_t K, int64_t R, const uint8_t* widths, const uint1
   st64(b + 48, total);
   st32(b + 56, crc32(b + kHeaderBytes, total - kHeaderBytes));
   st32(b + 60, crc32(b, 60));
-  if (out_desc) fill_desc(geo, total, out_desc);
+  if (out_desc) fill_desc(geo, total, max_rec, out_desc);
   return VBQ_OK;
 }
 
@@ -267,7 +271,19 @@ int vbq_describe(const void* blob_host, uint64_t blob_bytes, vbq_desc* out_desc)
   if (ld64(b + 32) != geo.dir_off || ld64(b + 40) != geo.rec_off || total < geo.rec_off) return VBQ_ERR_FORMAT;
   if (total > blob_bytes) return VBQ_ERR_BUFFER_TOO_SMALL;
   if (ld32(b + 56) != crc32(b + kHeaderBytes, total - kHeaderBytes)) return VBQ_ERR_CRC;
-  fill_desc(geo, total, out_desc);
+  // Directory: strictly increasing record starts that end exactly at total_bytes.
+  const uint64_t nrec = uint64_t(geo.T * geo.G);
+  if (geo.dir_off + 4 * (nrec + 1) > geo.rec_off) return VBQ_ERR_FORMAT;
+  uint64_t max_rec = 0, prev = ld32(b + geo.dir_off);
+  if (prev != 0) return VBQ_ERR_FORMAT;
+  for (uint64_t i = 1; i <= nrec; ++i) {
+    const uint64_t cur = ld32(b + geo.dir_off + 4 * i);
+    if (cur <= prev) return VBQ_ERR_FORMAT;
+    max_rec = std::max(max_rec, 16 * (cur - prev));
+    prev = cur;
+  }
+  if (geo.rec_off + 16 * prev != total) return VBQ_ERR_FORMAT;
+  fill_desc(geo, total, max_rec, out_desc);
   return VBQ_OK;
 }
 

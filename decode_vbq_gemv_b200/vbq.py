@@ -33,7 +33,7 @@ class vbq_desc(ctypes.Structure):
     _fields_ = [("version", ctypes.c_uint32), ("flags", ctypes.c_uint32), ("N", ctypes.c_int64),
                 ("K", ctypes.c_int64), ("G", ctypes.c_int64), ("R", ctypes.c_int64), ("T", ctypes.c_int64),
                 ("dir_offset", ctypes.c_uint64), ("rec_offset", ctypes.c_uint64),
-                ("total_bytes", ctypes.c_uint64)]
+                ("total_bytes", ctypes.c_uint64), ("max_record_bytes", ctypes.c_uint64)]
 
 
 _lib = None

@@ -60,6 +60,7 @@ typedef struct vbq_desc {
   uint64_t dir_offset;   /* byte offset of the record directory */
   uint64_t rec_offset;   /* byte offset of the first record */
   uint64_t total_bytes;  /* blob size in bytes */
+  uint64_t max_record_bytes; /* largest record; sets the shared-memory staging size of the kernels */
 } vbq_desc;
 
 /* Static English text for a status code; never NULL. */
@@ -96,9 +97,11 @@ int vbq_unpack(const void* blob_host, uint64_t blob_bytes, uint8_t* widths, uint
 /* -------------------------------------------------------------------------------------------- device */
 
 /* Workspace bytes that vbq_gemv / vbq_gemm_skinny need for this matrix and batch on the CURRENT device (the
- * launch shape depends on its SM count). The workspace holds per-CTA partial sums of split-K launches and one
- * arrival counter per row tile. It may be 0 (then any pointer, including NULL, is accepted).
- * Errors: NULL, BATCH, FORMAT (desc inconsistent), CUDA. */
+ * launch shape depends on its SM count). The workspace holds the partial sums of row tiles that several CTAs
+ * share, one arrival counter per row tile, and, in its 4 bytes at offset (size - 4), a device status word: 0 after every
+ * successful call; nonzero if a kernel gave up a bounded wait (bit 0) or met a record larger than the staging
+ * size its descriptor promised (bit 1), in which case the outputs of that call are not valid.
+ * Errors: NULL, BATCH, FORMAT (desc inconsistent). */
 int vbq_workspace_size(const vbq_desc* d, int B, uint64_t* out_bytes);
 
 /* Zero a workspace before its first use (cudaMemsetAsync on `stream`). Every kernel call leaves the arrival

@@ -33,8 +33,13 @@ def gpu_y(m, xbits, R=1024, mat=None):
     if mat is None:
         blob, _ = vbq.vbq_pack(m.N, m.K, R, m.widths, m.scales, m.codes)
         mat = vbq.DeviceMatrix(blob, dev())
-    y = mat.matmul(to_dev_x(xbits))
+    xd = to_dev_x(xbits)
+    y = mat.matmul(xd)
     torch.cuda.synchronize()
+    ws = mat.workspaces[xd.shape[0]]
+    need = vbq.vbq_workspace_size(mat.desc, xd.shape[0])
+    status = int(ws[need - 4:need].cpu().numpy().view(np.uint32)[0])
+    assert status == 0, f"device status word {status:#x}"
     return y.cpu().numpy().astype(np.float64), mat
 
 
