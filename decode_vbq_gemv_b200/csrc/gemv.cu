@@ -33,6 +33,8 @@
 #include <cuda_fp16.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "vbq.h"
 
 namespace vbq {
@@ -1029,3 +1031,49 @@ int vbq_gemv(const vbq_desc* d, const void* blob_dev, const void* x_bf16, float*
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------------------ allocation-free variant
+// Scratch for vbq_gemm_skinny_noalloc: one fixed buffer per device, created when the library is loaded on that
+// device and kept until the process exits. It replaces the caller-provided workspace of vbq_gemm_skinny.
+namespace vbq {
+constexpr uint64_t kStaticScratchBytes = 16ull << 20;  // 16 MiB
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+// Device address of g_static_scratch on the current device. In host code the array's name is only a host-side
+// stand-in, so the address is looked up once per device with cudaGetSymbolAddress (that device current).
+int static_scratch(void** out) {
+  static std::mutex mu;
+  static void* addr[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return VBQ_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_static_scratch) != cudaSuccess || !ptr) return VBQ_ERR_CUDA;
+    addr[dev] = ptr;
+  }
+  *out = addr[dev];
+  return VBQ_OK;
+}
+}  // namespace vbq
+
+extern "C" int vbq_gemm_skinny_noalloc(const vbq_desc* d, const void* blob_dev, const void* x_bf16, int B,
+                                       float* y, void* stream) {
+  if (!d || !blob_dev || !x_bf16 || !y) return VBQ_ERR_NULL;
+  if (B != 1 && B != 2 && B != 4 && B != 8 && B != 16) return VBQ_ERR_BATCH;
+  if (!vbq::desc_ok(d)) return VBQ_ERR_FORMAT;
+  uint64_t need = 0;
+  if (int st = vbq_workspace_size(d, B, &need)) return st;
+  if (need > vbq::kStaticScratchBytes) return VBQ_ERR_SCRATCH_LIMIT;
+  void* scratch = nullptr;
+  if (int st = vbq::static_scratch(&scratch)) return st;
+  // The buffer keeps the previous call's contents: clear the arrival counters and the status word, which the
+  // kernel needs at zero. The partial-sum area is always written before it is read.
+  vbq::Plan pl;
+  if (!vbq::make_plan(*d, B, vbq::num_sms(), pl)) return VBQ_ERR_FORMAT;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(static_cast<unsigned char*>(scratch) + pl.counters_off, 0,
+                      size_t(need - pl.counters_off), st) != cudaSuccess)
+    return VBQ_ERR_CUDA;
+  return vbq_gemm_skinny(d, blob_dev, x_bf16, B, y, scratch, need, stream);
+}

@@ -161,6 +161,7 @@ const char* vbq_strerror(int status) {
     case VBQ_ERR_TILE: return "tile rows must be a multiple of 16 in [16, 1024]";
     case VBQ_ERR_FORMAT: return "blob is not canonical VBQ format v1";
     case VBQ_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case VBQ_ERR_SCRATCH_LIMIT: return "problem needs more scratch than the 16 MiB fixed buffer of the allocation-free entry point";
     default: return "unknown status";
   }
 }

@@ -44,7 +44,8 @@ typedef enum vbq_status {
   VBQ_ERR_CUDA = -11,             /* a CUDA runtime call or launch failed */
   VBQ_ERR_TILE = -12,             /* tile rows R not a multiple of 16 in [16, 1024] */
   VBQ_ERR_FORMAT = -13,           /* blob is not canonical format v1 (layout, padding, counts) */
-  VBQ_ERR_WORKSPACE = -14         /* workspace NULL, misaligned or smaller than vbq_workspace_size */
+  VBQ_ERR_WORKSPACE = -14,        /* workspace NULL, misaligned or smaller than vbq_workspace_size */
+  VBQ_ERR_SCRATCH_LIMIT = -15     /* vbq_gemm_skinny_noalloc: problem needs more than its 16 MiB fixed buffer */
 } vbq_status;
 
 /* Host-side description of a packed blob. It is filled by vbq_pack or vbq_describe and passed by pointer to
@@ -126,6 +127,27 @@ int vbq_gemv(const vbq_desc* d, const void* blob_dev, const void* x_bf16, float*
  * Other arguments and guarantees as in vbq_gemv. Errors: NULL, BATCH, ALIGN, WORKSPACE, FORMAT, CUDA. */
 int vbq_gemm_skinny(const vbq_desc* d, const void* blob_dev, const void* x_bf16, int B, float* y,
                     void* workspace, uint64_t workspace_bytes, void* stream);
+
+/* Allocation-free variant of vbq_gemm_skinny (the VBQ paper has no counterpart; this is a deployment aid).
+ *
+ * Some callers cannot allocate device memory at all. Examples: plug-in hosts that give the library only pointers
+ * into their own pre-reserved pools, and serving loops that forbid cudaMalloc after start-up because it can
+ * synchronize the device and fragment their pools. Those callers can neither hold a workspace nor size one.
+ * This entry point takes the same inputs and outputs as vbq_gemm_skinny, but no workspace. Its scratch
+ * (split-K partial sums, arrival counters, status word) lives in one fixed 16 MiB device buffer inside the
+ * library. Every GPU that loads the library holds that buffer until the process exits.
+ *
+ * - Limit: problems whose vbq_workspace_size(d, B) exceeds 16 MiB are rejected with VBQ_ERR_SCRATCH_LIMIT, and
+ *   nothing is launched. With 1024-row tiles that covers any N at B <= 4, and N up to about 110K at B = 16.
+ * - First call per device: it looks up the buffer's device address (cudaGetSymbolAddress, with that device
+ *   current). Make this first call before any stream capture.
+ * - Each call clears the counters and the status word with one cudaMemsetAsync on `stream`, then launches the
+ *   same kernel as vbq_gemm_skinny. It allocates nothing and frees nothing.
+ * - All calls on a device share the one buffer, which keeps the last call's contents. Calls that can overlap
+ *   on the GPU (different streams, different host threads) race on it: serialize them.
+ * Errors: as vbq_gemm_skinny, plus SCRATCH_LIMIT; CUDA if the buffer's address cannot be obtained. */
+int vbq_gemm_skinny_noalloc(const vbq_desc* d, const void* blob_dev, const void* x_bf16, int B, float* y,
+                            void* stream);
 
 #ifdef __cplusplus
 }
