@@ -227,8 +227,10 @@ def run_vbq(args):
         layers.append(lin)
     step_bytes = [sum(l[5] for l in lin) for lin in layers]
 
+    flags = 0 if args.no_overlap else vbq.VBQ_LAUNCH_OVERLAP
+
     def launch(mat, xd, yd, st):
-        vbq.vbq_gemm_skinny(mat.desc, mat.blob, xd, B, yd, mat.workspaces[B], st)
+        vbq.vbq_gemm_skinny_ex(mat.desc, mat.blob, xd, B, yd, mat.workspaces[B], flags, st)
 
     # One CUDA graph per layer copy, so that the timed region has no host launch gaps: device-resident step
     # (seven GEMVs) and end-to-end step (pinned x -> device, seven GEMVs, y -> pinned host).
@@ -320,6 +322,7 @@ def run_vbq(args):
             "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "fp32", "data": "synthetic",
             "config": {"workload": WORKLOAD, "batch": B, "tile_rows": R,
+                       "launch": "plain" if args.no_overlap else "programmatic dependent launch (VBQ_LAUNCH_OVERLAP)",
                        "weights": "seeded synthetic VBQ groups: P(1,2,4,8 bit) = (0.69,0.16,0.09,0.06), fp16 "
                                   "scales U(0.01,0.1), uniform codes; x ~ N(0,1) bf16",
                        "l2": f"inputs larger than L2: {args.copies} distinct layer copies in rotation "
@@ -351,7 +354,9 @@ def main():
     ap.add_argument("--batch", type=int, default=1, choices=(1, 2, 4, 8, 16))
     ap.add_argument("--impl", default="vbq", choices=("vbq", "reference"))
     ap.add_argument("--copies", type=int, default=4)
-    ap.add_argument("--tile-rows", type=int, default=1024)
+    ap.add_argument("--tile-rows", type=int, default=256)
+    ap.add_argument("--no-overlap", action="store_true",
+                    help="plain launches instead of programmatic dependent launch between the linears")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds for the CPU-oracle baseline (0: skip)")
     ap.add_argument("--ref-rows", type=int, default=256, help="rows per linear per step for --impl reference")
     args = ap.parse_args()

@@ -4,30 +4,24 @@
 // "Fused kernels over packed weights"): y[b][r] = sum_g s[r][g] * sum_i (q[r][64g+i] - (2^k-1)/2) * x[b][64g+i].
 // The low-bit codes are expanded in registers. The dense matrix never exists in memory.
 //
-// Kernel structure (B200, sm_100a), one persistent CTA per SM:
+// Kernel structure (B200, sm_100a), one CTA per SM:
 //  - The blob is one record per (row tile, group column), stored tile-major. Inside a record, the tile's groups
-//    sit in four width buckets (1, 2, 4, 8 bits), each in ascending row order (FORMAT.md). CTA c owns the records
-//    whose start offsets fall in the c-th equal slice of the record bytes, so every CTA streams the same number
-//    of bytes.
-//  - Warp specialization. One producer warp streams whole records into a ring of shared-memory stages with
-//    cp.async.bulk (the TMA engine, no multicast). Completion is signaled through mbarrier transaction counts.
-//    For each landed record it rebuilds the item -> row map from the 2-bit width codes and stages the column's
-//    activations, then releases the stage to the consumer warps through a second mbarrier. Consumers hand the
-//    stage back through a third. Every wait is bounded by a timer. On timeout the kernel sets a status bit in
-//    the workspace and leaves.
-//  - Consumer warps take units of 32 items of one bucket, so every warp instruction runs a single width (the
-//    width-bucketed schedule). Units are dealt round-robin over the CTA's record sequence.
-//    Batch 1: each consumer warp accumulates into its own copy of the tile's outputs. No barrier is needed
-//    between records. Each lane owns one 64-weight group and holds the column's activations in registers.
-//    1-bit groups add the activations whose bit is set (predicated adds). 2/4-bit groups expand codes with a
-//    magic-number bit-to-float trick against pre-scaled activations. 8-bit groups use byte permutes.
-//    Batch 2/4 (CUDA cores) and 8/16 (mma.sync bf16 tensor cores): all consumer warps share one accumulator
-//    and synchronize once per record.
-//  - A row tile split across CTAs is reduced without floating-point atomics. Each owner CTA writes its partial
-//    sums to the workspace and counts itself in. Only the first and last tile of a CTA's range can be shared.
-//    At the end of the kernel, each owner waits (bounded) until all owners of the tile are in. It then adds all
-//    partials, in CTA order, for its own slice of the tile's rows. The launch is cooperative, so every CTA is
-//    resident while others wait for it. Results are bitwise deterministic.
+//    sit in four width buckets (1, 2, 4, 8 bits), each in ascending row order. CTA c owns the c-th equal share
+//    of the records (by count, computed without reading memory).
+//  - The CTA's warps form independent teams (one warp each when the CTA has many records, several warps each
+//    when it has few). A team owns a contiguous run of the CTA's records, streams them into its own ring of
+//    shared-memory stages with cp.async.bulk (the TMA engine, no multicast) and waits on mbarrier transaction
+//    counts, bounded by a timer; nothing waits on another team or another CTA.
+//  - Inside a team, warps take units of 32 items of one bucket, so every warp instruction runs a single width.
+//    Batch 1: each lane owns one 64-weight group and holds the column's activations in registers. 1-bit groups
+//    add the activations whose bit is set (predicated adds); 2/4-bit groups expand codes with a magic-number
+//    bit-to-float trick against pre-scaled activations; 8-bit groups use byte permutes. Results land in item
+//    order, and a row pass adds them to the tile's rows. Batch 2/4: CUDA cores. Batch 8/16: mma.sync bf16
+//    tensor cores on the exact integers 2q - (2^k - 1).
+//  - Row tiles that several owners share are reduced without floating-point atomics: teams of one CTA that
+//    share a tile are summed in shared memory in team order; CTAs that share a tile write partial sums to the
+//    workspace and count themselves in, and the last to arrive adds all partials in CTA order. Results are
+//    bitwise deterministic, and no CTA ever waits for another.
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -41,22 +35,19 @@ namespace vbq {
 
 constexpr int kMaxTileRows = 1024;
 constexpr int kAStride = 72;            // bf16 per staged A row for ldmatrix (64 + 8 pad: conflict-free rows)
-constexpr int kMaxStages = 4;
-constexpr int kSmemBudget = 227 * 1024;
+constexpr int kMaxTeams = 16;
+constexpr int kMaxStages = 2;
+constexpr int kSmemBudget = 227 * 1024 - 2048;  // dynamic shared memory; the rest is the static part
 constexpr unsigned long long kWaitNs = 2000000000ull;  // bounded mbarrier waits: 2 s
 constexpr unsigned kSuspendNs = 20000;                  // a waiting thread sleeps (no issue slots) up to 20 us per poll
-constexpr unsigned kStatusTimeout = 1u, kStatusOversize = 2u;
+constexpr unsigned kStatusTimeout = 1u, kStatusOversize = 2u, kStatusRecord = 4u;
 
 template <int B> struct Cfg {
-  // Batch 1: per-item results plus a lagged row pass, with no barrier between records. Other batches: the
-  // consumers add straight into the tile accumulators and synchronize once per record.
-  static constexpr bool kRowPass = (B == 1);
-  static constexpr int kConsumers = (B == 1) ? 14 : 8;  // consumer warps
-  static constexpr int kThreads = (kConsumers + 1) * 32;
-  static constexpr int kCThreads = kConsumers * 32;
-  // activations staged per record: B=1: raw, x*2^-shift for 2-bit, x*2^-shift for 4-bit (fp32);
-  // B=2,4: fp32 [64][B]; B=8,16: none (the tensor-core path reads the bf16 copy directly)
-  static constexpr int kXBytes = (B == 1) ? 3 * 64 * 4 : (B < 8 ? 64 * B * 4 : 0);
+  static constexpr int kWarps = (B == 1) ? 16 : (B < 8 ? 12 : 8);
+  static constexpr int kThreads = kWarps * 32;
+  // per-warp activation buffer: B=1: x, x*2^-shift for 2-bit codes, x*2^-shift for 4-bit codes (fp32);
+  // B=2,4: fp32 [64][B]; B=8,16: the bf16 A tile of the tensor-core path, [32][kAStride]
+  static constexpr int kXBytes = (B == 1) ? 3 * 64 * 4 : (B < 8 ? 64 * B * 4 : 32 * kAStride * 2);
 };
 
 struct Params {
@@ -66,36 +57,34 @@ struct Params {
   float* y;                // [B][N]
   float* partial;          // [nCTA + T][R][B] partial sums of shared row tiles
   unsigned* arrive;        // [T] owners that have published their partial sums; zero between calls
-  unsigned* depart;        // [T] owners done reducing; the last one resets both counters
   unsigned* status;        // device status word
   int N, K, G, R, T, nrec;
-  uint32_t units_total;    // dir[nrec]
+  uint32_t units_total;    // dir[nrec]: 16-byte units of all records
+  int NT, TW, S;           // teams per CTA, warps per team, stages per team
   int stage_bytes;         // record capacity of one stage (multiple of 128)
-  int stage_size;          // full stage size, record + row list + activations + meta
-  int NS;                  // stages
-  int ys_cap;              // floats of the tile-accumulator region (>= R*B and >= the CTA count)
+  int stage_size;          // stage: record, then the column's bf16 activations [B][64]
+  int team_bytes;          // per team: S stages | tile accumulators [R][B] f32 | item results (batch 1, 2 x R f32)
+  int acc_off, res_off;
+  int warps_off, warp_bytes;
 };
 
 __host__ __device__ constexpr int align16i(int v) { return (v + 15) & ~15; }
 __host__ __device__ constexpr int align128i(int v) { return (v + 127) & ~127; }
 
-// Stage layout: [record bytes | bf16 activations of the column ([B][64], landed by bulk copy) | expanded
-// activations | group sums (B f32) | width masks [4][32] u32 | item starts [4][32] i32 | item results (batch 1,
-// R f32) | meta (16 int)]
-struct StageOff {
-  int xraw, xv, sg, masks, pref, res, meta;
-  __host__ __device__ StageOff(int stage_bytes, int R, int xbytes, int B, bool rowpass) {
-    xraw = stage_bytes;
-    xv = xraw + 128 * B;
-    sg = xv + align16i(xbytes);
-    masks = sg + align16i(4 * B);
-    pref = masks + 512;
-    res = pref + 512;
-    meta = res + (rowpass ? 4 * R : 0);
+// Per-warp scratch: activations | group sums (B f32) | width masks [4][32] u32 | item starts [4][32] i32 |
+// width-code words of the record (up to 64 u32)
+struct WarpOff {
+  int x, sg, mk, pf, wd, sz;
+  __host__ __device__ WarpOff(int xbytes, int /*B*/) {
+    x = 0;
+    sg = align16i(xbytes);
+    mk = sg + 64;
+    pf = mk + 512;
+    wd = pf + 512;
+    sz = align128i(wd + 256);
   }
-  __host__ __device__ int size() const { return align128i(meta + 64); }
+  __host__ __device__ int size() const { return sz; }
 };
-enum Meta { M_T = 0, M_G, M_RT, M_N0, M_N1, M_N2, M_N3, M_UBASE, M_U };
 
 // ------------------------------------------------------------------------------------------ PTX helpers
 __device__ __forceinline__ uint32_t smem_u32(const void* p) { return uint32_t(__cvta_generic_to_shared(p)); }
@@ -147,6 +136,12 @@ __device__ __forceinline__ void mbar_drain(uint64_t* bar, unsigned parity) {
   const unsigned long long t0 = now_ns();
   while (!mbar_try_wait(bar, parity))
     if (now_ns() - t0 > kWaitNs) return;
+}
+// Atomic add with acquire-release semantics at GPU scope; returns the old value.
+__device__ __forceinline__ unsigned atom_add_acq_rel(unsigned* addr, unsigned v) {
+  unsigned old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(addr), "r"(v) : "memory");
+  return old;
 }
 // Bulk copy global -> shared through the TMA engine; completes `bytes` transactions on `bar`.
 __device__ __forceinline__ void tma_bulk_load(void* dst, const void* src, unsigned bytes, uint64_t* bar) {
@@ -298,6 +293,51 @@ __device__ __forceinline__ float dot_b8(const uint32_t (&w)[16], const float (&x
   return ((acc0.x + acc0.y) + (acc1.x + acc1.y)) + 0.5f * sg;
 }
 
+// Batch 1, one width bucket: the warp's units of 32 items each (local unit u for u = first, first + TW, ...).
+// Lane = item; the item's result s * dot goes to res[item] (byte addresses: codes, scales, res for item 0 of the
+// bucket). The activations this width needs are loaded into registers once, from xcopy.
+template <int KB>
+__device__ __forceinline__ void bucket_units(int n, int U, int first, int TW, int lane, uint32_t codes,
+                                             uint32_t scales, uint32_t res, float (&xr)[64], uint32_t xcopy,
+                                             float sg) {
+  if (first >= U) return;
+#pragma unroll
+  for (int q = 0; q < 16; ++q) {
+    const float4 f = lds128f(xcopy + 16 * q);
+    xr[4 * q] = f.x; xr[4 * q + 1] = f.y; xr[4 * q + 2] = f.z; xr[4 * q + 3] = f.w;
+  }
+  for (int u = first; u < U; u += TW) {
+    const int jj = 32 * u + lane;
+    if (jj >= n) continue;
+    float d;
+    if constexpr (KB == 1) {
+      d = dot_b1(lds64(codes + 8 * jj), xr, sg);
+    } else if constexpr (KB == 2) {
+      const uint4 a = lds128(codes + 16 * jj);
+      const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+      d = dot_magic<2>(w, xr, sg);
+    } else if constexpr (KB == 4) {
+      const uint4 a = lds128(codes + 32 * jj), b = lds128(codes + 32 * jj + 16);
+      const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+      d = dot_magic<4>(w, xr, sg);
+    } else {
+      uint32_t w[16];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint4 a = lds128(codes + 64 * jj + 16 * q);
+        w[4 * q] = a.x; w[4 * q + 1] = a.y; w[4 * q + 2] = a.z; w[4 * q + 3] = a.w;
+      }
+      d = dot_b8(w, xr, sg);
+    }
+    sts32f(res + 4 * jj, __half2float(__ushort_as_half((unsigned short)lds16(scales + 2 * jj))) * d);
+  }
+}
+// First local unit of a bucket for warp tw of TW, when the bucket's units follow `before` units of the record.
+__device__ __forceinline__ int first_unit(int tw, int before, int TW) {
+  const int r = (tw - before) % TW;
+  return r < 0 ? r + TW : r;
+}
+
 // q - 2^(k-1) of code i from a group's code words in shared memory (any width, runtime index).
 __device__ __forceinline__ float code_centered(const uint32_t* w, int k, int i) {
   const int bit = k * i;
@@ -352,17 +392,6 @@ struct Rec {
   }
 };
 
-// CTA c owns records [lo(c), lo(c+1)) with lo(c) = floor(c * nrec / nCTA): records of one matrix have similar
-// sizes, so equal record counts give nearly equal bytes. No memory is read to compute ownership.
-__device__ __forceinline__ int rec_lo(const Params& p, int c) {
-  return int((long long)c * p.nrec / int(gridDim.x));
-}
-// Owner of record j: the largest c with lo(c) <= j.
-__device__ __forceinline__ int owner(const Params& p, int j) {
-  const long long c = ((long long)(j + 1) * gridDim.x + p.nrec - 1) / p.nrec - 1;
-  return int(min(c, (long long)gridDim.x - 1));
-}
-
 // Gathers the even bits of a 64-bit word into 32 bits.
 __device__ __forceinline__ uint32_t even_bits(unsigned long long x) {
   x &= 0x5555555555555555ull;
@@ -374,517 +403,551 @@ __device__ __forceinline__ uint32_t even_bits(unsigned long long x) {
   return uint32_t(x);
 }
 
+// CTA c owns records [lo(c), lo(c+1)) with lo(c) = floor(c * nrec / nCTA): records of one matrix have similar
+// sizes, so equal record counts give nearly equal bytes. No memory is read to compute ownership.
+// 32-bit arithmetic when (nCTA + 1) * (nrec + 1) fits, which covers every realistic matrix; 64-bit otherwise.
+__device__ __forceinline__ bool small_ids(const Params& p) {
+  return (unsigned long long)(gridDim.x + 1) * unsigned(p.nrec + 1) < (1ull << 32);
+}
+__device__ __forceinline__ int rec_lo(const Params& p, int c) {
+  if (small_ids(p)) return int(unsigned(c) * unsigned(p.nrec) / gridDim.x);
+  return int((long long)c * p.nrec / int(gridDim.x));
+}
+// Owner of record j: the largest c with lo(c) <= j.
+__device__ __forceinline__ int owner(const Params& p, int j) {
+  const long long c = small_ids(p) ? (long long)((unsigned(j + 1) * gridDim.x + p.nrec - 1) / unsigned(p.nrec)) - 1
+                                   : ((long long)(j + 1) * gridDim.x + p.nrec - 1) / p.nrec - 1;
+  return int(min(c, (long long)gridDim.x - 1));
+}
+
+// Barrier of one team: the warp itself, or a named hardware barrier (ids 1..15, one per team) over its warps.
+__device__ __forceinline__ void team_sync(int team, int TW) {
+  if (TW == 1) {
+    __syncwarp();
+  } else {
+    asm volatile("bar.sync %0, %1;" ::"r"(team + 1), "r"(TW * 32) : "memory");
+  }
+}
+
+// Closed-form split of the CTA's records [L, H) among its NT teams. The records fall into segments, one per row
+// tile. Every team computes its own share; nothing is exchanged.
+//  - At most NT segments: each segment gets one team plus a share of the NT - nseg spare teams proportional to its
+//    records (cumulative rounding), and is cut evenly among its teams. A team then never leaves its tile, and a
+//    segment with several teams is summed in shared memory at the end.
+//  - More segments than teams: each team takes whole segments, spread evenly by count.
+struct TeamMap {
+  int L, H, G, NT, n, tL, nseg;
+  __device__ TeamMap(int L_, int H_, int G_, int NT_) : L(L_), H(H_), G(G_), NT(NT_), n(H_ - L_), tL(0), nseg(0) {
+    if (n > 0) {
+      tL = L / G;
+      nseg = (H - 1) / G - tL + 1;
+    }
+  }
+  __device__ bool split() const { return nseg <= NT; }
+  __device__ int seg_lo(int i) const { return max(L, (tL + i) * G); }
+  __device__ int seg_hi(int i) const { return min(H, (tL + i + 1) * G); }
+  // first team of segment i (split mode); seg_team0(nseg) == NT
+  __device__ int seg_team0(int i) const {
+    if (i >= nseg) return NT;
+    const unsigned num = unsigned(NT - nseg) * unsigned(seg_lo(i) - L);  // < 16 * n
+    return i + int(n < (1 << 27) ? num / unsigned(n) : (unsigned)((long long)(NT - nseg) * (seg_lo(i) - L) / n));
+  }
+  // records [lo, hi) of team k; seg = its segment when that segment has several teams, else -1
+  __device__ void team(int k, int& lo, int& hi, int& seg) const {
+    seg = -1;
+    if (n <= 0) { lo = hi = L; return; }
+    if (split()) {
+      int i = 0;
+      while (i + 1 < nseg && seg_team0(i + 1) <= k) ++i;
+      const int f = seg_team0(i), cnt = seg_team0(i + 1) - f;
+      const int s0 = seg_lo(i), len = seg_hi(i) - s0, q = k - f;
+      lo = s0 + q * len / cnt;
+      hi = s0 + (q + 1) * len / cnt;
+      if (cnt >= 2) seg = i;
+    } else {
+      const int a = int((long long)k * nseg / NT), b = int((long long)(k + 1) * nseg / NT);
+      lo = max(L, (tL + a) * G);
+      hi = min(H, (tL + b) * G);
+    }
+  }
+};
+
 // ------------------------------------------------------------------------------------------------ kernel
 template <int B>
 __global__ void __launch_bounds__(Cfg<B>::kThreads, 1) vbq_kernel(Params p) {
   using C = Cfg<B>;
-  constexpr int NW = C::kConsumers;
   extern __shared__ __align__(128) unsigned char smem[];
-  __shared__ uint64_t bar_full[kMaxStages], bar_ready[kMaxStages], bar_empty[kMaxStages], bar_done[kMaxStages];
-  __shared__ uint64_t bar_cons;
-  __shared__ int range[2];
-  __shared__ volatile int abort_flag;
-  __shared__ int pending[2], npending;  // shared tiles published by this CTA (at most its first and last)
+  __shared__ uint64_t bar_full[kMaxTeams * kMaxStages];
+  __shared__ int stage_bad[kMaxTeams * kMaxStages];
+  __shared__ volatile int team_abort[kMaxTeams];
+  __shared__ int team_live[kMaxTeams];  // team has records (its accumulators hold a partial sum)
+  __shared__ int cta_flags[2];
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int NS = p.NS;
-  const StageOff so(p.stage_bytes, p.R, C::kXBytes, B, C::kRowPass);
-  float* ys = reinterpret_cast<float*>(smem);                       // tile accumulators [R][B]
-  const int ys_floats = p.ys_cap;
-  unsigned char* astage = smem + align128i(ys_floats * 4);          // tensor-core A tiles (B >= 8)
-  unsigned char* stages = astage + (B >= 8 ? align128i(NW * 32 * kAStride * 2) : 0);
-
-  if (tid == 0) {
-    for (int s = 0; s < NS; ++s) {
-      mbar_init(&bar_full[s], 1);
-      mbar_init(&bar_ready[s], 32);
-      mbar_init(&bar_empty[s], NW);
-      mbar_init(&bar_done[s], NW);
-    }
-    mbar_init(&bar_cons, C::kCThreads);
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    abort_flag = 0;
-    npending = 0;
-    range[0] = rec_lo(p, blockIdx.x);
-    range[1] = rec_lo(p, blockIdx.x + 1);
-  }
-  for (int e = tid; e < ys_floats; e += C::kThreads) ys[e] = 0.f;
-  __syncthreads();
-  const int jbeg = range[0], jend = range[1], n = jend - jbeg;
-  if (n <= 0) return;
-  // Consumers fold record i's results into the tile accumulators one record later (lag 1), so that the row
-  // pass never waits; with a single stage there is nothing to overlap, and the lag is 0.
-  const int lag = (C::kRowPass && NS >= 2) ? 1 : 0;
-
-  if (warp == NW) {
-    // ================================================================ producer warp
-    // Directory entries of this CTA's records, 32 at a time in lanes (records are issued in order).
-    int win = 0;
-    uint32_t dlane = lane <= n ? __ldg(p.dir + jbeg + lane) : 0u;
-    auto dir_at = [&](int i) -> uint32_t {  // whole warp; i in [0, n]
-      if (i >= win + 32) {
-        win = i;
-        dlane = win + lane <= n ? __ldg(p.dir + jbeg + win + lane) : 0u;
-      }
-      return __shfl_sync(0xFFFFFFFFu, dlane, i - win);
-    };
-    // Issue record i: one bulk copy of the record and B bulk copies of the column's bf16 activations (128 B).
-    auto issue = [&](int i) {  // whole warp; lane 0 issues
-      const uint32_t a = dir_at(i);
-      const uint32_t b = i + 1 - win < 32 ? __shfl_sync(0xFFFFFFFFu, dlane, i + 1 - win) : __ldg(p.dir + jbeg + i + 1);
-      if (lane != 0) return;
-      const int j = jbeg + i, s = i % NS, g = j % p.G;
-      const unsigned bytes = 16u * (b - a);
-      unsigned char* dst = stages + s * p.stage_size;
-      if (bytes > unsigned(p.stage_bytes)) {  // descriptor promised a smaller record: flag and skip the copy
-        atomicOr(p.status, kStatusOversize);
-        mbar_arrive(&bar_full[s]);
-        return;
-      }
-      mbar_arrive_tx(&bar_full[s], bytes + 128u * B);
-      tma_bulk_load(dst, p.recs + 16ull * a, bytes, &bar_full[s]);
-#pragma unroll
-      for (int bb = 0; bb < B; ++bb)
-        tma_bulk_load(dst + so.xraw + 128 * bb, p.x + size_t(bb) * p.K + size_t(g) * 64, 128u, &bar_full[s]);
-    };
-    for (int i = 0; i < min(NS, n); ++i) issue(i);
-    __syncwarp();
-    int issued = min(NS, n);  // records whose bulk copy has been issued (warp-uniform)
-    int unit_base = 0;
-    for (int i = 0; i < n; ++i) {
-      const int s = i % NS;
-      unsigned char* st = stages + s * p.stage_size;
-      if (!mbar_wait(&bar_full[s], (i / NS) & 1, p.status, &abort_flag)) {
-        for (int r = i; r < issued; ++r) mbar_drain(&bar_full[r % NS], (r / NS) & 1);
-        break;
-      }
-      // -- width masks and item starts per 32-row word (lane = word)
-      const int j = jbeg + i, t = j / p.G, g = j - t * p.G;
-      const int Rt = min(p.R, p.N - t * p.R);
-      const uint2 cnt = *reinterpret_cast<const uint2*>(st);
-      const int n0 = cnt.x & 0xFFFF, n1 = cnt.x >> 16, n2 = cnt.y & 0xFFFF, n3 = cnt.y >> 16;
-      const int nvalid = max(0, min(32, Rt - 32 * lane));
-      unsigned long long v = 0;
-      if (nvalid > 0) v = *reinterpret_cast<const unsigned long long*>(st + 8 + 8 * lane);
-      const unsigned long long lo = v & 0x5555555555555555ull, hi = (v >> 1) & 0x5555555555555555ull;
-      const uint32_t valid = nvalid >= 32 ? 0xFFFFFFFFu : ((1u << nvalid) - 1u);
-      const uint32_t m0 = even_bits(~hi & ~lo) & valid, m1 = even_bits(~hi & lo) & valid;
-      const uint32_t m2 = even_bits(hi & ~lo) & valid, m3 = even_bits(hi & lo) & valid;
-      const unsigned long long mine = (unsigned long long)__popc(m0) | ((unsigned long long)__popc(m1) << 16) |
-                                      ((unsigned long long)__popc(m2) << 32) | ((unsigned long long)__popc(m3) << 48);
-      unsigned long long incl = mine;
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const unsigned long long u = __shfl_up_sync(0xFFFFFFFFu, incl, off);
-        if (lane >= off) incl += u;
-      }
-      const unsigned long long pre = incl - mine;
-      uint32_t* masks = reinterpret_cast<uint32_t*>(st + so.masks);
-      int* pref = reinterpret_cast<int*>(st + so.pref);
-      masks[lane] = m0; masks[32 + lane] = m1; masks[64 + lane] = m2; masks[96 + lane] = m3;
-      pref[lane] = int(pre & 0xFFFFull);
-      pref[32 + lane] = n0 + int((pre >> 16) & 0xFFFFull);
-      pref[64 + lane] = n0 + n1 + int((pre >> 32) & 0xFFFFull);
-      pref[96 + lane] = n0 + n1 + n2 + int(pre >> 48);
-      // -- expand the column's activations (and group sums for the CUDA-core paths)
-      const uint16_t* xg = reinterpret_cast<const uint16_t*>(st + so.xraw);  // [B][64] bf16, landed with the record
-      if constexpr (B == 1) {
-        float* xv = reinterpret_cast<float*>(st + so.xv);
-        const float x0 = __uint_as_float(uint32_t(xg[lane]) << 16);
-        const float x1 = __uint_as_float(uint32_t(xg[32 + lane]) << 16);
-        xv[lane] = x0;
-        xv[32 + lane] = x1;
-        xv[64 + lane] = x0 * __uint_as_float(uint32_t(127 - code_shift<2>(lane)) << 23);
-        xv[96 + lane] = x1 * __uint_as_float(uint32_t(127 - code_shift<2>(32 + lane)) << 23);
-        xv[128 + lane] = x0 * __uint_as_float(uint32_t(127 - code_shift<4>(lane)) << 23);
-        xv[160 + lane] = x1 * __uint_as_float(uint32_t(127 - code_shift<4>(32 + lane)) << 23);
-        float sgv = x0 + x1;
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) sgv += __shfl_xor_sync(0xFFFFFFFFu, sgv, off);
-        if (lane == 0) reinterpret_cast<float*>(st + so.sg)[0] = sgv;
-      } else if constexpr (B < 8) {
-        float* xv = reinterpret_cast<float*>(st + so.xv);
-#pragma unroll
-        for (int b = 0; b < B; ++b) {
-          const float x0 = __uint_as_float(uint32_t(xg[b * 64 + lane]) << 16);
-          const float x1 = __uint_as_float(uint32_t(xg[b * 64 + 32 + lane]) << 16);
-          xv[lane * B + b] = x0;
-          xv[(32 + lane) * B + b] = x1;
-          float sgv = x0 + x1;
-#pragma unroll
-          for (int off = 16; off > 0; off >>= 1) sgv += __shfl_xor_sync(0xFFFFFFFFu, sgv, off);
-          if (lane == 0) reinterpret_cast<float*>(st + so.sg)[b] = sgv;
-        }
-      }
-      const int U = ((n0 + 31) >> 5) + ((n1 + 31) >> 5) + ((n2 + 31) >> 5) + ((n3 + 31) >> 5);
-      if (lane == 0) {
-        int* meta = reinterpret_cast<int*>(st + so.meta);
-        meta[M_T] = t; meta[M_G] = g; meta[M_RT] = Rt;
-        meta[M_N0] = n0; meta[M_N1] = n1; meta[M_N2] = n2; meta[M_N3] = n3;
-        meta[M_UBASE] = unit_base; meta[M_U] = U;
-      }
-      unit_base += U;
-      __syncwarp();
-      mbar_arrive(&bar_ready[s]);
-      // -- refill a stage that the consumers release without needing a later record
-      const int rs = NS == 1 ? i : i - min(2, NS - 1), r = rs + NS;
-      if (rs >= 0 && r < n) {
-        if (!mbar_wait(&bar_empty[rs % NS], (rs / NS) & 1, p.status, &abort_flag)) {
-          for (int r2 = i + 1; r2 < issued; ++r2) mbar_drain(&bar_full[r2 % NS], (r2 / NS) & 1);
-          break;
-        }
-        issue(r);
-        ++issued;
-        __syncwarp();
-      }
-    }
-    return;
-  }
-
-  // ================================================================== consumer warps
-  const int ctid = tid;  // 0 .. kCThreads-1
-
-  // Bounded barrier of the consumer warps (an mbarrier with one arrival per consumer thread).
-  unsigned cons_phase = 0;
-  auto consumers_sync = [&]() -> bool {
-    mbar_arrive(&bar_cons);
-    const bool ok = mbar_wait(&bar_cons, cons_phase & 1u, p.status, &abort_flag);
-    ++cons_phase;
-    return ok;
-  };
+  const int NT = p.NT, TW = p.TW, S = p.S, G = p.G, R = p.R;
+  const int cta = blockIdx.x;
+  const int L = rec_lo(p, cta), H = rec_lo(p, cta + 1);
+  const TeamMap tm(L, H, G, NT);
+  // A kernel launched after this one with programmatic dependent launch may start its own prologue (which reads
+  // only its weights) as soon as SMs free up; it waits for this grid before touching activations or outputs.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   // Owners of tile t. With at least as many records as CTAs every CTA owns a contiguous, non-empty record range,
   // so the owners are first..last. With fewer records than CTAs each CTA owns at most one record, so the owners
   // are the owners of the tile's G records, one each.
   const bool dense = p.nrec >= int(gridDim.x);
   auto tile_owners = [&](int t, int& first) -> int {
-    first = owner(p, t * p.G);
-    return dense ? owner(p, t * p.G + p.G - 1) - first + 1 : p.G;
+    first = owner(p, t * G);
+    return dense ? owner(p, t * G + G - 1) - first + 1 : G;
   };
-  auto kth_owner = [&](int t, int first, int k) -> int { return dense ? first + k : owner(p, t * p.G + k); };
+  auto kth_owner = [&](int t, int first, int k) -> int { return dense ? first + k : owner(p, t * G + k); };
 
-  // Publishes the tile accumulators of tile t: straight into y when this CTA is the tile's only owner, otherwise
-  // into its partial slot (owner + tile indexes the slots without collision, since (owner, tile) pairs increase
-  // along the records) and counts itself in. Leaves the accumulators zeroed.
-  auto publish = [&](int t) -> bool {
-    if (!consumers_sync()) return false;
+  // Sum of all owners' partial slots of tile t, in CTA order, into y (threads gtid of gthreads). Each thread
+  // issues the loads of up to 8 owners at once, then adds them in owner order.
+  auto reduce_tile = [&](int t, int gtid, int gthreads) {
     int first;
     const int owners = tile_owners(t, first);
-    const int Rt = min(p.R, p.N - t * p.R);
-    const bool sole = owners == 1;
-    float* slot = p.partial + size_t(blockIdx.x + t) * p.R * B;
-    for (int e = ctid; e < Rt * B; e += C::kCThreads) {
-      const float v = ys[e];
-      ys[e] = 0.f;
-      if (sole) {
-        const int jj = e / B, b = e - jj * B;
-        p.y[size_t(b) * p.N + size_t(t) * p.R + jj] = v;
+    const int Rt = min(R, p.N - t * R);
+    for (int e = gtid; e < Rt * B; e += gthreads) {
+      float v = 0.f;
+      for (int k0 = 0; k0 < owners; k0 += 8) {
+        float part[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          part[q] = k0 + q < owners ? __ldcg(p.partial + size_t(kth_owner(t, first, k0 + q) + t) * R * B + e) : 0.f;
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          if (k0 + q < owners) v += part[q];
+      }
+      const int r = e / B, b = e - r * B;
+      p.y[size_t(b) * p.N + size_t(t) * R + r] = v;
+    }
+  };
+
+  const int team = warp / TW, tw = warp - team * TW;
+  int tb = L, te = L, tseg = -1;
+  if (team < NT) tm.team(team, tb, te, tseg);
+  if (team < NT && tw == 0 && lane == 0) {
+    team_abort[team] = 0;
+    team_live[team] = tb < te;
+  }
+  if (team < NT && tb < te) {
+    // ================================================================== one team: records [tb, te)
+    const int nt = te - tb;
+    volatile int* abort_flag = &team_abort[team];
+    unsigned char* tbase = smem + team * p.team_bytes;
+    float* acc = reinterpret_cast<float*>(tbase + p.acc_off);       // tile accumulators [R][B]
+    unsigned char* wbase = smem + p.warps_off + warp * p.warp_bytes;
+    const WarpOff wo(C::kXBytes, B);
+    uint32_t* mk = reinterpret_cast<uint32_t*>(wbase + wo.mk);      // [4][32] width masks per 32-row word
+    int* pf = reinterpret_cast<int*>(wbase + wo.pf);                // [4][32] item index of the word's first row
+    uint32_t* wd = reinterpret_cast<uint32_t*>(wbase + wo.wd);      // width-code words of the record
+    const int sl0 = tw * R / TW, sl1 = (tw + 1) * R / TW;           // this warp's rows in flushes and row passes
+    uint64_t* bars = bar_full + team * S;
+
+    // -- the team's first warp streams the records: directory entries 32 at a time in its lanes, loaded first
+    // (their latency is what the first copy waits for); lane 0 sets up the team's barriers and issues the copies
+    int issued = 0;
+    int win = 0;
+    uint32_t dlane = 0;
+    if (tw == 0) dlane = lane <= nt ? __ldg(p.dir + tb + lane) : 0u;
+    auto dir_at = [&](int i) -> uint32_t {  // whole warp; i in [0, nt], non-decreasing between calls
+      if (i >= win + 32) {
+        win = i;
+        dlane = win + lane <= nt ? __ldg(p.dir + tb + win + lane) : 0u;
+      }
+      return __shfl_sync(0xFFFFFFFFu, dlane, i - win);
+    };
+    // Record i's bulk copy into stage i % S (whole warp; lane 0 issues). The activations follow with issue_x.
+    auto issue_record = [&](int i) {
+      const uint32_t a = dir_at(i);
+      const uint32_t b = dir_at(i + 1);
+      if (lane != 0) return;
+      const int s = i % S;
+      unsigned char* dst = tbase + s * p.stage_size;
+      const unsigned bytes = 16u * (b - a);
+      if (b < a || b > p.units_total || bytes > unsigned(p.stage_bytes)) {  // not what the descriptor promised
+        stage_bad[team * S + s] = 1;
+        atomicOr(p.status, kStatusOversize);
+        mbar_arrive(&bars[s]);
       } else {
-        slot[e] = v;
+        stage_bad[team * S + s] = 0;
+        mbar_arrive_tx(&bars[s], bytes + 128u * B);
+        tma_bulk_load(dst, p.recs + 16ull * a, bytes, &bars[s]);
       }
-    }
-    if (!sole) {
-      __threadfence();
-      if (!consumers_sync()) return false;
-      if (ctid == 0) {
-        atomicAdd(&p.arrive[t], 1u);
-        pending[npending < 2 ? npending : 1] = t;
-        npending = min(npending + 1, 2);
-      }
-    }
-    return consumers_sync();
-  };
-
-  // Final step for a shared tile: wait (bounded) until every owner has published, then add all owners' slots
-  // in CTA order for this CTA's slice of the rows. All loads of a chunk are issued at once (one thread per
-  // (owner, element)) into the free accumulator space, then summed per element in owner order. The last owner
-  // to finish resets the tile's counters.
-  auto reduce_shared = [&](int t) -> bool {
-    int first;
-    const int owners = tile_owners(t, first);
-    if (ctid == 0) {
-      const volatile unsigned* arr = p.arrive + t;
-      const unsigned long long t0 = now_ns();
-      while (*arr < unsigned(owners)) {
-        if (abort_flag) break;
-        if (now_ns() - t0 > kWaitNs) {
-          abort_flag = 1;
-          atomicOr(p.status, kStatusTimeout);
-          break;
-        }
-        __nanosleep(32);
-      }
-    }
-    if (!consumers_sync()) return false;
-    __threadfence();
-    const int rank = dense ? int(blockIdx.x) - first : rec_lo(p, blockIdx.x) - t * p.G;
-    const int Rt = min(p.R, p.N - t * p.R);
-    const int e0 = int((long long)Rt * rank / owners) * B, e1 = int((long long)Rt * (rank + 1) / owners) * B;
-    const int chunk = max(1, ys_floats / owners);
-    for (int c0 = e0; c0 < e1; c0 += chunk) {
-      const int ne = min(chunk, e1 - c0);
-      for (int q = ctid; q < ne * owners; q += C::kCThreads) {
-        const int k = q / ne, e = q - k * ne;
-        ys[q] = __ldcg(p.partial + size_t(kth_owner(t, first, k) + t) * p.R * B + c0 + e);
-      }
-      if (!consumers_sync()) return false;
-      for (int e = ctid; e < ne; e += C::kCThreads) {
-        float v = 0.f;
-        for (int k = 0; k < owners; ++k) v += ys[k * ne + e];
-        const int ee = c0 + e, jj = ee / B, b = ee - jj * B;
-        p.y[size_t(b) * p.N + size_t(t) * p.R + jj] = v;
-      }
-      if (!consumers_sync()) return false;
-    }
-    for (int q = ctid; q < ys_floats; q += C::kCThreads) ys[q] = 0.f;
-    if (ctid == 0 && atomicAdd(&p.depart[t], 1u) == unsigned(owners - 1)) {
-      p.arrive[t] = 0u;
-      p.depart[t] = 0u;
-    }
-    return true;
-  };
-
-  int cur_t = -1;
-  // Publishes the current tile when record j (still resident) starts a new one.
-  auto tile_switch = [&](int j) -> bool {
-    const int t = reinterpret_cast<const int*>(stages + (j % NS) * p.stage_size + so.meta)[M_T];
-    if (t != cur_t) {
-      if (cur_t >= 0 && !publish(cur_t)) return false;
-      cur_t = t;
-    }
-    return true;
-  };
-
-  // Batch 1: folds record j's item results into the tile accumulators. Each warp owns a fixed slice of rows,
-  // so no two warps ever touch the same accumulator and every row sums its records in order. Row r's item is
-  // its bucket's item start for its 32-row word plus the rows of the same width before it in that word.
-  auto row_pass = [&](int j) -> bool {
-    const int s = j % NS;
-    const unsigned char* st = stages + s * p.stage_size;
-    if (!mbar_wait(&bar_done[s], (j / NS) & 1, p.status, &abort_flag)) return false;
-    if (!tile_switch(j)) return false;
-    const int Rt = reinterpret_cast<const int*>(st + so.meta)[M_RT];
-    const uint32_t sa = smem_u32(st);
-    const int r0 = warp * Rt / NW, r1 = (warp + 1) * Rt / NW;
-    for (int r = r0 + lane; r < r1; r += 32) {
-      const int c = int(lds8(sa + 8 + (r >> 2)) >> (2 * (r & 3))) & 3;
-      const int w = r >> 5;
-      const int item = int(lds32(sa + so.pref + 4 * (c * 32 + w))) +
-                       __popc(lds32(sa + so.masks + 4 * (c * 32 + w)) & ((1u << (r & 31)) - 1u));
-      ys[r] += lds32f(sa + so.res + 4 * item);
-    }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&bar_empty[s]);
-    return true;
-  };
-
-  int loaded_rec = -1, loaded_copy = -1;
-  float xr[B == 1 ? 64 : 1];
-  for (int i = 0; i < n; ++i) {
-    const int s = i % NS;
-    unsigned char* st = stages + s * p.stage_size;
-    if (!mbar_wait(&bar_ready[s], (i / NS) & 1, p.status, &abort_flag)) return;
-    const int* meta = reinterpret_cast<const int*>(st + so.meta);
-    const Rec rc(meta[M_RT], meta[M_N0], meta[M_N1], meta[M_N2], meta[M_N3]);
-    const int ubase = meta[M_UBASE];
-    const uint32_t* masks = reinterpret_cast<const uint32_t*>(st + so.masks);
-    const int* pref = reinterpret_cast<const int*>(st + so.pref);
-    const float* sgs = reinterpret_cast<const float*>(st + so.sg);
-    const int u_first = ((warp - ubase) % NW + NW) % NW;
-    if constexpr (!C::kRowPass) {
-      if (!tile_switch(i)) return;
-    }
-
-    if constexpr (B == 1) {
-      const float sg = sgs[0];
-      const uint32_t sa = smem_u32(st);
-      for (int u = u_first; u < rc.U; u += NW) {
-        int bk, j0, ibase, cbase, nb;
-        rc.unit(u, bk, j0, ibase, cbase, nb);
-        const int copy = bk == 1 ? 1 : (bk == 2 ? 2 : 0);
-        if (i != loaded_rec || copy != loaded_copy) {
-          const uint32_t src = sa + so.xv + 256 * copy;
+    };
+    auto issue_x = [&](int i) {  // lane 0
+      const int s = i % S, j = tb + i, g = j % G;
+      if (stage_bad[team * S + s]) return;
+      unsigned char* dst = tbase + s * p.stage_size + p.stage_bytes;
 #pragma unroll
-          for (int q = 0; q < 16; ++q) {
-            const float4 f = lds128f(src + 16 * q);
-            xr[4 * q] = f.x; xr[4 * q + 1] = f.y; xr[4 * q + 2] = f.z; xr[4 * q + 3] = f.w;
-          }
-          loaded_rec = i;
-          loaded_copy = copy;
-        }
-        const int j = j0 + lane;
-        if (j < nb) {
-          const uint32_t cp = sa + cbase;
-          float d;
-          if (bk == 0) {
-            d = dot_b1(lds64(cp + 8 * j), xr, sg);
-          } else if (bk == 1) {
-            const uint4 a = lds128(cp + 16 * j);
-            const uint32_t w[4] = {a.x, a.y, a.z, a.w};
-            d = dot_magic<2>(w, xr, sg);
-          } else if (bk == 2) {
-            const uint4 a = lds128(cp + 32 * j), b2 = lds128(cp + 32 * j + 16);
-            const uint32_t w[8] = {a.x, a.y, a.z, a.w, b2.x, b2.y, b2.z, b2.w};
-            d = dot_magic<4>(w, xr, sg);
-          } else {
-            uint32_t w[16];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const uint4 a = lds128(cp + 64 * j + 16 * q);
-              w[4 * q] = a.x; w[4 * q + 1] = a.y; w[4 * q + 2] = a.z; w[4 * q + 3] = a.w;
-            }
-            d = dot_b8(w, xr, sg);
-          }
-          const int item = ibase + j;
-          sts32f(sa + so.res + 4 * item, __half2float(__ushort_as_half((unsigned short)lds16(sa + rc.sc + 2 * item))) * d);
-        }
+      for (int bb = 0; bb < B; ++bb)
+        tma_bulk_load(dst + 128 * bb, p.x + size_t(bb) * p.K + size_t(g) * 64, 128u, &bars[s]);
+    };
+    if (tw == 0) {
+      if (lane == 0) {
+        for (int i = 0; i < S; ++i) mbar_init(&bars[i], 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bar_done[s]);
-      if (lag == 0) {
-        if (!row_pass(i)) return;
-      } else if (i >= 1) {
-        if (!row_pass(i - 1)) return;
+      issued = min(S, nt);
+      for (int i = 0; i < issued; ++i) issue_record(i);
+    }
+    team_sync(team, TW);  // the team's barriers are initialized
+    // The weights never depend on an earlier kernel; the activations, outputs and workspace may. Under
+    // programmatic dependent launch this waits for the previous kernel; otherwise it returns at once.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (tw == 0 && lane == 0)
+      for (int i = 0; i < issued; ++i) issue_x(i);
+
+    // -- flush of a finished tile: straight into y when this team covers the whole tile. A partial tile that no
+    // other team of the CTA shares goes to the CTA's partial slot, counted in at the end of the kernel; a
+    // partial tile shared inside the CTA stays here for the combine at the end.
+    auto flush = [&](int t) {
+      if (tseg >= 0) return;  // shared inside the CTA: the combine at the end writes it
+      const int Rt = min(R, p.N - t * R);
+      if (tb <= t * G && tb + nt >= (t + 1) * G) {
+        for (int r = sl0 + lane; r < min(sl1, Rt); r += 32)
+#pragma unroll
+          for (int b = 0; b < B; ++b) p.y[size_t(b) * p.N + size_t(t) * R + r] = acc[r * B + b];
+      } else {
+        float* slot = p.partial + size_t(cta + t) * R * B;
+        for (int e = sl0 * B + lane; e < min(sl1, Rt) * B; e += 32) slot[e] = acc[e];
       }
-      continue;
-    } else if constexpr (B < 8) {
-      // CUDA cores, B in {2, 4}: lane = group; activations of all batches broadcast from the stage.
-      const float* xc = reinterpret_cast<const float*>(st + so.xv);
-      for (int u = u_first; u < rc.U; u += NW) {
-        int bk, j0, ibase, cbase, nb;
-        rc.unit(u, bk, j0, ibase, cbase, nb);
-        const int j = j0 + lane;
-        if (j >= nb) continue;
-        const int k = 1 << bk;
-        const uint32_t* w = reinterpret_cast<const uint32_t*>(st + cbase + 8 * k * j);
-        float acc[B];
-#pragma unroll
-        for (int b = 0; b < B; ++b) acc[b] = 0.f;
-        if (bk == 0) {
-          const uint32_t w0 = w[0], w1 = w[1];
-#pragma unroll 8
-          for (int i2 = 0; i2 < 64; ++i2) {
-            if ((i2 < 32 ? w0 : w1) & (1u << (i2 & 31))) {
-#pragma unroll
-              for (int b = 0; b < B; ++b) acc[b] += xc[i2 * B + b];
-            }
-          }
-        } else {
-#pragma unroll 4
-          for (int i2 = 0; i2 < 64; ++i2) {
-            const float qv = code_centered(w, k, i2);
-#pragma unroll
-            for (int b = 0; b < B; ++b) acc[b] = fmaf(qv, xc[i2 * B + b], acc[b]);
-          }
-        }
-        const int item = ibase + j;
-        const float sc = __half2float(reinterpret_cast<const __half*>(st + rc.sc)[item]);
-        const int row = item_row(masks, pref, bk, item);
-        // sum (q - 2^(k-1)) x + 1/2 sum x == sum (q - (2^k-1)/2) x; for k = 1 the first sum is sum_{q=1} x - S.
-#pragma unroll
-        for (int b = 0; b < B; ++b) {
-          const float S = sgs[b];
-          const float d = (bk == 0) ? acc[b] - 0.5f * S : acc[b] + 0.5f * S;
-          ys[row * B + b] = fmaf(sc, d, ys[row * B + b]);
+    };
+
+    int cur_t = -1;
+    float xr[B == 1 ? 64 : 1];
+    for (int i = 0; i < nt; ++i) {
+      const int s = i % S;
+      const unsigned char* st = tbase + s * p.stage_size;
+      const uint32_t sa = smem_u32(st);
+      bool ok = mbar_wait(&bars[s], (i / S) & 1, p.status, abort_flag);
+      if (ok && stage_bad[team * S + s]) ok = false;
+      ok = __all_sync(0xFFFFFFFFu, ok);  // lanes can see an abort at different times; the warp decides as one
+      const int j = tb + i, t = j / G;
+      const int Rt = min(R, p.N - t * R);
+      if (t != cur_t) {
+        if (cur_t >= 0) flush(cur_t);
+        for (int e = sl0 * B + lane; e < sl1 * B; e += 32) acc[e] = 0.f;
+        if (B > 1) team_sync(team, TW);
+        cur_t = t;
+      }
+      int n0 = 0, n1 = 0, n2 = 0, n3 = 0;
+      if (ok) {
+        const uint2 cnt = lds64(sa);
+        n0 = cnt.x & 0xFFFF; n1 = cnt.x >> 16; n2 = cnt.y & 0xFFFF; n3 = cnt.y >> 16;
+        // a record whose counts disagree with its tile, or whose buckets overrun the stage, is not read
+        const Rec rc(Rt, n0, n1, n2, n3);
+        if (n0 + n1 + n2 + n3 != Rt || rc.c3 + 64 * n3 > p.stage_bytes) {
+          if (lane == 0) atomicOr(p.status, kStatusRecord);
+          ok = false;
         }
       }
-    } else {
-      // Tensor cores, B in {8, 16}: lane = group, dequantized to bf16 2q-(2^k-1) in this warp's A tile; two
-      // m16 tiles per unit through mma.sync m16n8k16 (bf16 in, fp32 accumulate), then s/2 per row.
-      constexpr int NT = B >= 8 ? B / 8 : 1;
-      __nv_bfloat16* As = reinterpret_cast<__nv_bfloat16*>(astage) + warp * 32 * kAStride;
-      const uint32_t* xb = reinterpret_cast<const uint32_t*>(st + so.xraw);
-      uint32_t bfr[4][NT][2];
-#pragma unroll
-      for (int ks = 0; ks < 4; ++ks)
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          const int nb2 = nt * 8 + (lane >> 2);
-          bfr[ks][nt][0] = xb[nb2 * 32 + 8 * ks + (lane & 3)];
-          bfr[ks][nt][1] = xb[nb2 * 32 + 8 * ks + 4 + (lane & 3)];
+      const Rec rc(Rt, n0, n1, n2, n3);
+      uint32_t m0 = 0, m1 = 0, m2 = 0, m3 = 0;
+      unsigned long long v = 0, pre = 0;
+      if (ok) {
+        // -- width masks and item starts per 32-row word (lane = word), and a copy of the width codes
+        const int nvalid = max(0, min(32, Rt - 32 * lane));
+        if (nvalid > 0) {
+          const uint2 v2 = lds64(sa + 8 + 8 * lane);
+          v = (unsigned long long)v2.x | ((unsigned long long)v2.y << 32);
         }
-      for (int u = u_first; u < rc.U; u += NW) {
-        int bk, j0, ibase, cbase, nb;
-        rc.unit(u, bk, j0, ibase, cbase, nb);
-        const int k = 1 << bk;
-        const int j = j0 + lane;
-        const bool valid = j < nb;
-        __nv_bfloat162* arow = reinterpret_cast<__nv_bfloat162*>(As + lane * kAStride);
-        if (valid) {
-          const uint32_t* w = reinterpret_cast<const uint32_t*>(st + cbase + 8 * k * j);
-          const float off = float((1 << k) - 1);
-          const uint32_t mask = (1u << k) - 1u;
-#pragma unroll 8
-          for (int i2 = 0; i2 < 64; i2 += 2) {
-            const int b0 = k * i2, b1 = k * (i2 + 1);
-            const uint32_t q0 = (w[b0 >> 5] >> (b0 & 31)) & mask;
-            const uint32_t q1 = (w[b1 >> 5] >> (b1 & 31)) & mask;
-            arow[i2 >> 1] = __floats2bfloat162_rn(2.f * float(q0) - off, 2.f * float(q1) - off);
-          }
-        } else {
+        const unsigned long long lo = v & 0x5555555555555555ull, hi = (v >> 1) & 0x5555555555555555ull;
+        const uint32_t valid = nvalid >= 32 ? 0xFFFFFFFFu : ((1u << nvalid) - 1u);
+        m0 = even_bits(~hi & ~lo) & valid;
+        m1 = even_bits(~hi & lo) & valid;
+        m2 = even_bits(hi & ~lo) & valid;
+        m3 = even_bits(hi & lo) & valid;
+        const unsigned long long mine = (unsigned long long)__popc(m0) | ((unsigned long long)__popc(m1) << 16) |
+                                        ((unsigned long long)__popc(m2) << 32) |
+                                        ((unsigned long long)__popc(m3) << 48);
+        unsigned long long incl = mine;
 #pragma unroll
-          for (int i2 = 0; i2 < 32; ++i2) arow[i2] = __floats2bfloat162_rn(0.f, 0.f);
+        for (int off = 1; off < 32; off <<= 1) {
+          const unsigned long long u = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+          if (lane >= off) incl += u;
+        }
+        pre = incl - mine;
+        // the width codes must agree with the bucket counts, or no item index derived from them is in range
+        const unsigned long long tot = __shfl_sync(0xFFFFFFFFu, incl, 31);
+        if (tot != ((unsigned long long)n0 | ((unsigned long long)n1 << 16) | ((unsigned long long)n2 << 32) |
+                    ((unsigned long long)n3 << 48))) {
+          if (lane == 0) atomicOr(p.status, kStatusRecord);
+          ok = false;
+        }
+      }
+      if (ok) {
+        mk[lane] = m0; mk[32 + lane] = m1; mk[64 + lane] = m2; mk[96 + lane] = m3;
+        pf[lane] = int(pre & 0xFFFFull);
+        pf[32 + lane] = n0 + int((pre >> 16) & 0xFFFFull);
+        pf[64 + lane] = n0 + n1 + int((pre >> 32) & 0xFFFFull);
+        pf[96 + lane] = n0 + n1 + n2 + int(pre >> 48);
+        wd[2 * lane] = uint32_t(v);
+        wd[2 * lane + 1] = uint32_t(v >> 32);
+        // -- the column's activations, from the bf16 copy that landed with the record
+        const uint16_t* xg = reinterpret_cast<const uint16_t*>(st + p.stage_bytes);  // [B][64]
+        float* xv = reinterpret_cast<float*>(wbase + wo.x);
+        float* sgv = reinterpret_cast<float*>(wbase + wo.sg);
+        if constexpr (B == 1) {
+          const float x0 = __uint_as_float(uint32_t(xg[lane]) << 16);
+          const float x1 = __uint_as_float(uint32_t(xg[32 + lane]) << 16);
+          xv[lane] = x0;
+          xv[32 + lane] = x1;
+          xv[64 + lane] = x0 * __uint_as_float(uint32_t(127 - code_shift<2>(lane)) << 23);
+          xv[96 + lane] = x1 * __uint_as_float(uint32_t(127 - code_shift<2>(32 + lane)) << 23);
+          xv[128 + lane] = x0 * __uint_as_float(uint32_t(127 - code_shift<4>(lane)) << 23);
+          xv[160 + lane] = x1 * __uint_as_float(uint32_t(127 - code_shift<4>(32 + lane)) << 23);
+          float sg = x0 + x1;
+#pragma unroll
+          for (int off = 16; off > 0; off >>= 1) sg += __shfl_xor_sync(0xFFFFFFFFu, sg, off);
+          if (lane == 0) sgv[0] = sg;
+        } else if constexpr (B < 8) {
+#pragma unroll
+          for (int b = 0; b < B; ++b) {
+            const float x0 = __uint_as_float(uint32_t(xg[b * 64 + lane]) << 16);
+            const float x1 = __uint_as_float(uint32_t(xg[b * 64 + 32 + lane]) << 16);
+            xv[lane * B + b] = x0;
+            xv[(32 + lane) * B + b] = x1;
+            float sg = x0 + x1;
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) sg += __shfl_xor_sync(0xFFFFFFFFu, sg, off);
+            if (lane == 0) sgv[b] = sg;
+          }
         }
         __syncwarp();
-        float scale_mine = 0.f;
-        int row_mine = 0;
-        if (valid) {
-          scale_mine = 0.5f * __half2float(reinterpret_cast<const __half*>(st + rc.sc)[ibase + j]);
-          row_mine = item_row(masks, pref, bk, ibase + j);
-        }
+
+        if constexpr (B == 1) {
+          // -- batch 1: item results s * dot into the team's result buffer (item order), one bucket at a time.
+          // Units are numbered across the buckets and dealt round-robin to the team's warps.
+          const float sg = sgv[0];
+          const uint32_t xa = smem_u32(xv);
+          const uint32_t ra = smem_u32(tbase + p.res_off) + (TW > 1 ? 4 * R * (i & 1) : 0);
+          const uint32_t sca = sa + rc.sc;
+          const int U0 = rc.u0, U1 = rc.u1 - rc.u0, U2 = rc.u2 - rc.u1, U3 = rc.U - rc.u2;
+          bucket_units<1>(n0, U0, first_unit(tw, 0, TW), TW, lane, sa + rc.c0, sca, ra, xr, xa, sg);
+          bucket_units<2>(n1, U1, first_unit(tw, rc.u0, TW), TW, lane, sa + rc.c1, sca + 2 * n0, ra + 4 * n0, xr,
+                          xa + 256, sg);
+          bucket_units<4>(n2, U2, first_unit(tw, rc.u1, TW), TW, lane, sa + rc.c2, sca + 2 * (n0 + n1),
+                          ra + 4 * (n0 + n1), xr, xa + 512, sg);
+          bucket_units<8>(n3, U3, first_unit(tw, rc.u2, TW), TW, lane, sa + rc.c3, sca + 2 * (n0 + n1 + n2),
+                          ra + 4 * (n0 + n1 + n2), xr, xa, sg);
+        } else if constexpr (B < 8) {
+          // -- CUDA cores, B in {2, 4}: lane = group; activations of all batches broadcast from shared memory
+          const float* xc = xv;
+          for (int u = tw; u < rc.U; u += TW) {
+            int bk, j0, ibase, cbase, nb;
+            rc.unit(u, bk, j0, ibase, cbase, nb);
+            const int jj = j0 + lane;
+            if (jj >= nb) continue;
+            const int k = 1 << bk;
+            const uint32_t* w = reinterpret_cast<const uint32_t*>(st + cbase + 8 * k * jj);
+            float a[B];
 #pragma unroll
-        for (int mt = 0; mt < 2; ++mt) {
-          float acc[NT][4];
+            for (int b = 0; b < B; ++b) a[b] = 0.f;
+            if (bk == 0) {
+              const uint32_t w0 = w[0], w1 = w[1];
+#pragma unroll 8
+              for (int i2 = 0; i2 < 64; ++i2) {
+                if ((i2 < 32 ? w0 : w1) & (1u << (i2 & 31))) {
 #pragma unroll
-          for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+                  for (int b = 0; b < B; ++b) a[b] += xc[i2 * B + b];
+                }
+              }
+            } else {
+#pragma unroll 4
+              for (int i2 = 0; i2 < 64; ++i2) {
+                const float qv = code_centered(w, k, i2);
 #pragma unroll
-          for (int ks = 0; ks < 4; ++ks) {
-            const int r = mt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-            const int kk = ks * 16 + (lane >> 4) * 8;
-            uint32_t a0, a1, a2, a3;
-            asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-                         : "=r"(a0), "=r"(a1), "=r"(a2), "=r"(a3) : "r"(smem_u32(As + r * kAStride + kk)));
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
-              asm volatile(
-                  "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-                  "{%0,%1,%2,%3};"
-                  : "+f"(acc[nt][0]), "+f"(acc[nt][1]), "+f"(acc[nt][2]), "+f"(acc[nt][3])
-                  : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(bfr[ks][nt][0]), "r"(bfr[ks][nt][1]));
-          }
-          // acc[nt][0..1]: tile row lane/4, batch nt*8 + 2(lane%4) + {0,1}; acc[nt][2..3]: tile row lane/4 + 8.
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int src = mt * 16 + (lane >> 2) + 8 * h;
-            const float sc = __shfl_sync(0xFFFFFFFFu, scale_mine, src);
-            const int row = __shfl_sync(0xFFFFFFFFu, row_mine, src);
-            if (j0 + src < nb) {
-#pragma unroll
-              for (int nt = 0; nt < NT; ++nt) {
-                const int b = nt * 8 + 2 * (lane & 3);
-                ys[row * B + b] = fmaf(sc, acc[nt][2 * h], ys[row * B + b]);
-                ys[row * B + b + 1] = fmaf(sc, acc[nt][2 * h + 1], ys[row * B + b + 1]);
+                for (int b = 0; b < B; ++b) a[b] = fmaf(qv, xc[i2 * B + b], a[b]);
               }
             }
+            const int item = ibase + jj;
+            const float sc = __half2float(reinterpret_cast<const __half*>(st + rc.sc)[item]);
+            const int row = item_row(mk, pf, bk, item);
+            // sum (q - 2^(k-1)) x + 1/2 sum x == sum (q - (2^k-1)/2) x; for k = 1 the first sum is sum_{q=1} x - S.
+#pragma unroll
+            for (int b = 0; b < B; ++b) {
+              const float Sb = sgv[b];
+              const float d = (bk == 0) ? a[b] - 0.5f * Sb : a[b] + 0.5f * Sb;
+              acc[row * B + b] = fmaf(sc, d, acc[row * B + b]);
+            }
+          }
+        } else {
+          // -- tensor cores, B in {8, 16}: lane = group, dequantized to bf16 2q-(2^k-1) in this warp's A tile;
+          // two m16 tiles per unit through mma.sync m16n8k16 (bf16 in, fp32 accumulate), then s/2 per row.
+          constexpr int NTL = B >= 8 ? B / 8 : 1;
+          __nv_bfloat16* As = reinterpret_cast<__nv_bfloat16*>(wbase + wo.x);
+          const uint32_t* xb = reinterpret_cast<const uint32_t*>(st + p.stage_bytes);
+          uint32_t bfr[4][NTL][2];
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks)
+#pragma unroll
+            for (int nt2 = 0; nt2 < NTL; ++nt2) {
+              const int nb2 = nt2 * 8 + (lane >> 2);
+              bfr[ks][nt2][0] = xb[nb2 * 32 + 8 * ks + (lane & 3)];
+              bfr[ks][nt2][1] = xb[nb2 * 32 + 8 * ks + 4 + (lane & 3)];
+            }
+          for (int u = tw; u < rc.U; u += TW) {
+            int bk, j0, ibase, cbase, nb;
+            rc.unit(u, bk, j0, ibase, cbase, nb);
+            const int k = 1 << bk;
+            const int jj = j0 + lane;
+            const bool valid = jj < nb;
+            __nv_bfloat162* arow = reinterpret_cast<__nv_bfloat162*>(As + lane * kAStride);
+            if (valid) {
+              const uint32_t* w = reinterpret_cast<const uint32_t*>(st + cbase + 8 * k * jj);
+              const float off = float((1 << k) - 1);
+              const uint32_t mask = (1u << k) - 1u;
+#pragma unroll 8
+              for (int i2 = 0; i2 < 64; i2 += 2) {
+                const int b0 = k * i2, b1 = k * (i2 + 1);
+                const uint32_t q0 = (w[b0 >> 5] >> (b0 & 31)) & mask;
+                const uint32_t q1 = (w[b1 >> 5] >> (b1 & 31)) & mask;
+                arow[i2 >> 1] = __floats2bfloat162_rn(2.f * float(q0) - off, 2.f * float(q1) - off);
+              }
+            } else {
+#pragma unroll
+              for (int i2 = 0; i2 < 32; ++i2) arow[i2] = __floats2bfloat162_rn(0.f, 0.f);
+            }
+            __syncwarp();
+            float scale_mine = 0.f;
+            int row_mine = 0;
+            if (valid) {
+              scale_mine = 0.5f * __half2float(reinterpret_cast<const __half*>(st + rc.sc)[ibase + jj]);
+              row_mine = item_row(mk, pf, bk, ibase + jj);
+            }
+#pragma unroll
+            for (int mt = 0; mt < 2; ++mt) {
+              float c4[NTL][4];
+#pragma unroll
+              for (int nt2 = 0; nt2 < NTL; ++nt2) c4[nt2][0] = c4[nt2][1] = c4[nt2][2] = c4[nt2][3] = 0.f;
+#pragma unroll
+              for (int ks = 0; ks < 4; ++ks) {
+                const int r = mt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+                const int kk = ks * 16 + (lane >> 4) * 8;
+                uint32_t a0, a1, a2, a3;
+                asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                             : "=r"(a0), "=r"(a1), "=r"(a2), "=r"(a3) : "r"(smem_u32(As + r * kAStride + kk)));
+#pragma unroll
+                for (int nt2 = 0; nt2 < NTL; ++nt2)
+                  asm volatile(
+                      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+                      "{%0,%1,%2,%3};"
+                      : "+f"(c4[nt2][0]), "+f"(c4[nt2][1]), "+f"(c4[nt2][2]), "+f"(c4[nt2][3])
+                      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(bfr[ks][nt2][0]), "r"(bfr[ks][nt2][1]));
+              }
+              // c4[nt][0..1]: tile row lane/4, batch nt*8 + 2(lane%4) + {0,1}; c4[nt][2..3]: tile row lane/4 + 8.
+#pragma unroll
+              for (int h = 0; h < 2; ++h) {
+                const int src = mt * 16 + (lane >> 2) + 8 * h;
+                const float sc = __shfl_sync(0xFFFFFFFFu, scale_mine, src);
+                const int row = __shfl_sync(0xFFFFFFFFu, row_mine, src);
+                if (j0 + src < nb) {
+#pragma unroll
+                  for (int nt2 = 0; nt2 < NTL; ++nt2) {
+                    const int b = nt2 * 8 + 2 * (lane & 3);
+                    acc[row * B + b] = fmaf(sc, c4[nt2][2 * h], acc[row * B + b]);
+                    acc[row * B + b + 1] = fmaf(sc, c4[nt2][2 * h + 1], acc[row * B + b + 1]);
+                  }
+                }
+              }
+            }
+            __syncwarp();
           }
         }
-        __syncwarp();
+      }
+      // every warp of the team is done with stage s (and, for batch 1, has written its item results)
+      team_sync(team, TW);
+      if (tw == 0 && i + S < nt) {
+        const int go = __shfl_sync(0xFFFFFFFFu, *abort_flag ? 0 : 1, 0);
+        if (go) {
+          if (lane == 0) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          issue_record(i + S);
+          if (lane == 0) issue_x(i + S);
+          ++issued;
+        }
+      }
+      if constexpr (B == 1) {
+        if (ok) {
+          // -- row pass: row r of this warp's slice takes the result of its item (bucket start for its 32-row
+          // word, plus the rows of the same width before it in that word)
+          const uint32_t ra = smem_u32(tbase + p.res_off) + (TW > 1 ? 4 * R * (i & 1) : 0);
+          for (int r = sl0 + lane; r < min(sl1, Rt); r += 32) {
+            const int cc = int(wd[r >> 4] >> (2 * (r & 15))) & 3;
+            const int w = r >> 5;
+            const int item = pf[cc * 32 + w] + __popc(mk[cc * 32 + w] & ((1u << (r & 31)) - 1u));
+            acc[r] += lds32f(ra + 4 * item);
+          }
+        }
       }
     }
-    // shared accumulators: every warp is done with this record before any warp starts the next one
-    if (!consumers_sync()) return;
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&bar_empty[s]);
+    if (cur_t >= 0) flush(cur_t);
+    // After an abort, wait (bounded) for this team's copies still in flight before the CTA can exit.
+    if (*abort_flag && tw == 0 && lane == 0)
+      for (int r = max(0, issued - S); r < issued; ++r) mbar_drain(&bars[r % S], (r / S) & 1);
   }
-  if (lag == 1 && !row_pass(n - 1)) return;
-  if (cur_t < 0 || !publish(cur_t)) return;
-  for (int k = 0; k < npending; ++k)
-    if (!reduce_shared(pending[k])) return;
+
+  // =================================================================== combine of tiles shared by teams
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // warps without records reach this point directly
+  __syncthreads();
+  for (int k = 0; k < NT; ++k)
+    if (team_abort[k]) return;  // a team gave up a wait: its outputs are not valid, publish nothing
+  if (tm.split()) {
+    for (int i = 0; i < tm.nseg; ++i) {
+      const int k0 = tm.seg_team0(i), m = tm.seg_team0(i + 1) - k0;
+      if (m < 2) continue;
+      const int s0 = tm.seg_lo(i), s1 = tm.seg_hi(i);
+      const int t = s0 / G, Rt = min(R, p.N - t * R);
+      const bool whole = s0 <= t * G && s1 >= (t + 1) * G;
+      float* slot = p.partial + size_t(cta + t) * R * B;
+      for (int e = tid; e < Rt * B; e += C::kThreads) {
+        float v = 0.f;
+        for (int q = 0; q < m; ++q)
+          if (team_live[k0 + q]) v += reinterpret_cast<const float*>(smem + (k0 + q) * p.team_bytes + p.acc_off)[e];
+        if (whole) {
+          const int r = e / B, b = e - r * B;
+          p.y[size_t(b) * p.N + size_t(t) * R + r] = v;
+        } else {
+          slot[e] = v;
+        }
+      }
+    }
+  }
+  // ================================================= tiles shared with other CTAs: only this CTA's first and last
+  // Every partial slot of this CTA is written. One thread makes them visible GPU-wide and counts the CTA in;
+  // the last owner of a tile to arrive adds all owners' slots in CTA order.
+  if (H <= L) return;
+  const int tfirst = L / G, tlast = (H - 1) / G;
+  const bool part0 = !(L <= tfirst * G && H >= (tfirst + 1) * G);
+  const bool part1 = tlast != tfirst && !(L <= tlast * G && H >= (tlast + 1) * G);
+  if (!part0 && !part1) return;
+  __syncthreads();
+  if (tid == 0) {
+    // acq_rel at GPU scope: the release publishes the CTA's slot writes (ordered before it by the barrier), the
+    // acquire makes the other owners' slots visible to the reduction that follows. Both counters at once.
+    int first;
+    const int own0 = part0 ? tile_owners(tfirst, first) : 0, own1 = part1 ? tile_owners(tlast, first) : 0;
+    const unsigned a0 = part0 ? atom_add_acq_rel(&p.arrive[tfirst], 1u) : 0u;
+    const unsigned a1 = part1 ? atom_add_acq_rel(&p.arrive[tlast], 1u) : 0u;
+    cta_flags[0] = part0 && a0 == unsigned(own0 - 1);
+    cta_flags[1] = part1 && a1 == unsigned(own1 - 1);
+  }
+  __syncthreads();
+  if (cta_flags[0]) {
+    reduce_tile(tfirst, tid, C::kThreads);
+    if (tid == 0) p.arrive[tfirst] = 0u;
+  }
+  if (cta_flags[1]) {
+    reduce_tile(tlast, tid, C::kThreads);
+    if (tid == 0) p.arrive[tlast] = 0u;
+  }
 }
 
 // ------------------------------------------------------------------------------------------ launch plan
 struct Plan {
-  int grid, threads, NS, stage_bytes, stage_size, smem, ys_cap;
+  int grid, threads, NT, TW, S, stage_bytes, stage_size, team_bytes, acc_off, res_off, warps_off, warp_bytes, smem;
   uint64_t ws_bytes, status_off, counters_off;
 };
 
@@ -894,25 +957,52 @@ inline int num_sms() {
   return sms;
 }
 
+// Teams per CTA, warps per team and stages per team. A team's record copies overlap its arithmetic when it has
+// two stages; with one, every record's load latency is exposed. The plan that fits in shared memory with the
+// fewest exposed load latencies (records per team / stages, rounded up) wins; ties go to more warps, then to
+// more teams.
 template <int B>
 inline bool make_plan_t(const vbq_desc& d, int sms, Plan& pl) {
   using C = Cfg<B>;
-  pl.grid = sms < 1024 ? sms : 1024;  // owner bitmaps cover 1024 CTAs
+  pl.grid = sms;
   pl.threads = C::kThreads;
-  pl.stage_bytes = align128i(int(d.max_record_bytes));
   const int R = int(d.R);
-  pl.stage_size = StageOff(pl.stage_bytes, R, C::kXBytes, B, C::kRowPass).size();
-  pl.ys_cap = R * B > pl.grid ? R * B : pl.grid;
-  const int fixed = align128i(pl.ys_cap * 4) +
-                    (B >= 8 ? align128i(C::kConsumers * 32 * kAStride * 2) : 0);
-  int ns = (kSmemBudget - fixed) / pl.stage_size;
-  if (ns > kMaxStages) ns = kMaxStages;
-  if (ns < 1) return false;
-  pl.NS = ns;
-  pl.smem = fixed + ns * pl.stage_size;
+  const long long nrec = d.T * d.G;
+  const int rpc = int((nrec + pl.grid - 1) / pl.grid);
+  pl.stage_bytes = align128i(int(d.max_record_bytes));
+  pl.stage_size = pl.stage_bytes + align128i(128 * B);
+  const int acc_bytes = align128i(R * B * 4);
+  pl.warp_bytes = WarpOff(C::kXBytes, B).size();
+  const int W = C::kWarps;
+  long long best_key = -1;
+  for (int NT = min(min(W, kMaxTeams), max(rpc, 1)); NT >= 1; --NT) {
+    const int TW = W / NT;
+    if (TW > 1 && NT > 15) continue;  // named barrier ids 1..15
+    const int rpt = (rpc + NT - 1) / NT;
+    // batch 1: item results, double-buffered when several warps share a record
+    const int res_bytes = B == 1 ? align128i((TW > 1 ? 2 : 1) * R * 4) : 0;
+    for (int S = min(max(rpt, 1), kMaxStages); S >= 1; --S) {
+      const int team_bytes = S * pl.stage_size + acc_bytes + res_bytes;
+      const long long smem = (long long)NT * team_bytes + (long long)NT * TW * pl.warp_bytes;
+      if (smem > kSmemBudget) continue;
+      const long long exposed = (rpt + S - 1) / S;
+      const long long key = (1000000 - exposed) * 10000 + (long long)NT * TW * 100 + NT;
+      if (key > best_key) {
+        best_key = key;
+        pl.NT = NT; pl.TW = TW; pl.S = S;
+        pl.team_bytes = team_bytes;
+        pl.acc_off = S * pl.stage_size;
+        pl.res_off = pl.acc_off + acc_bytes;
+        pl.warps_off = NT * team_bytes;
+        pl.smem = int(smem);
+      }
+      break;  // fewer stages only expose more latency
+    }
+  }
+  if (best_key < 0) return false;
   const uint64_t slots = uint64_t(pl.grid) + uint64_t(d.T);
   pl.counters_off = slots * uint64_t(R) * B * 4;
-  pl.ws_bytes = (pl.counters_off + uint64_t(d.T) * 8 + 4 + 15) / 16 * 16;
+  pl.ws_bytes = (pl.counters_off + uint64_t(d.T) * 4 + 4 + 15) / 16 * 16;
   pl.status_off = pl.ws_bytes - 4;
   return true;
 }
@@ -938,7 +1028,7 @@ inline bool desc_ok(const vbq_desc* d) {
 
 template <int B>
 int launch(const vbq_desc* d, const void* blob, const void* x, float* y, void* ws, uint64_t ws_bytes,
-           cudaStream_t stream) {
+           unsigned flags, cudaStream_t stream) {
   Plan pl;
   if (!make_plan_t<B>(*d, num_sms(), pl)) return VBQ_ERR_FORMAT;
   if (!ws || (reinterpret_cast<uintptr_t>(ws) & 15) || ws_bytes < pl.ws_bytes) return VBQ_ERR_WORKSPACE;
@@ -951,15 +1041,18 @@ int launch(const vbq_desc* d, const void* blob, const void* x, float* y, void* w
   uint8_t* w = static_cast<uint8_t*>(ws);
   p.partial = reinterpret_cast<float*>(w);
   p.arrive = reinterpret_cast<unsigned*>(w + pl.counters_off);
-  p.depart = p.arrive + d->T;
   p.status = reinterpret_cast<unsigned*>(w + pl.status_off);
   p.N = int(d->N); p.K = int(d->K); p.G = int(d->G); p.R = int(d->R); p.T = int(d->T);
   p.nrec = int(d->T * d->G);
   p.units_total = uint32_t((d->total_bytes - d->rec_offset) / 16);
+  p.NT = pl.NT; p.TW = pl.TW; p.S = pl.S;
   p.stage_bytes = pl.stage_bytes;
   p.stage_size = pl.stage_size;
-  p.NS = pl.NS;
-  p.ys_cap = pl.ys_cap;
+  p.team_bytes = pl.team_bytes;
+  p.acc_off = pl.acc_off;
+  p.res_off = pl.res_off;
+  p.warps_off = pl.warps_off;
+  p.warp_bytes = pl.warp_bytes;
   // Opt in to the dynamic shared memory once per device and size.
   static int opted[64] = {0};
   int dev = 0;
@@ -970,18 +1063,16 @@ int launch(const vbq_desc* d, const void* blob, const void* x, float* y, void* w
       return VBQ_ERR_CUDA;
     done = pl.smem;
   }
-  // Cooperative launch: all CTAs are co-resident, which the bounded cross-CTA wait of the split-K reduction
-  // relies on.
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(unsigned(pl.grid));
   cfg.blockDim = dim3(unsigned(pl.threads));
   cfg.dynamicSmemBytes = size_t(pl.smem);
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeCooperative;
-  attr[0].val.cooperative = 1;
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = (flags & VBQ_LAUNCH_OVERLAP) ? 1 : 0;
   if (cudaLaunchKernelEx(&cfg, vbq_kernel<B>, p) != cudaSuccess) return VBQ_ERR_CUDA;
   return cudaPeekAtLastError() == cudaSuccess ? VBQ_OK : VBQ_ERR_CUDA;
 }
@@ -1007,22 +1098,28 @@ int vbq_workspace_init(void* workspace, uint64_t workspace_bytes, void* stream) 
              ? VBQ_OK : VBQ_ERR_CUDA;
 }
 
-int vbq_gemm_skinny(const vbq_desc* d, const void* blob_dev, const void* x_bf16, int B, float* y,
-                    void* workspace, uint64_t workspace_bytes, void* stream) {
+int vbq_gemm_skinny_ex(const vbq_desc* d, const void* blob_dev, const void* x_bf16, int B, float* y,
+                       void* workspace, uint64_t workspace_bytes, unsigned flags, void* stream) {
   if (!d || !blob_dev || !x_bf16 || !y) return VBQ_ERR_NULL;
   if (B != 1 && B != 2 && B != 4 && B != 8 && B != 16) return VBQ_ERR_BATCH;
+  if (flags & ~unsigned(VBQ_LAUNCH_OVERLAP)) return VBQ_ERR_FLAGS;
   if (!vbq::desc_ok(d)) return VBQ_ERR_FORMAT;
   if ((reinterpret_cast<uintptr_t>(blob_dev) & 15) || (reinterpret_cast<uintptr_t>(x_bf16) & 15) ||
       (reinterpret_cast<uintptr_t>(y) & 3))
     return VBQ_ERR_ALIGN;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   switch (B) {
-    case 1: return vbq::launch<1>(d, blob_dev, x_bf16, y, workspace, workspace_bytes, st);
-    case 2: return vbq::launch<2>(d, blob_dev, x_bf16, y, workspace, workspace_bytes, st);
-    case 4: return vbq::launch<4>(d, blob_dev, x_bf16, y, workspace, workspace_bytes, st);
-    case 8: return vbq::launch<8>(d, blob_dev, x_bf16, y, workspace, workspace_bytes, st);
-    default: return vbq::launch<16>(d, blob_dev, x_bf16, y, workspace, workspace_bytes, st);
+    case 1: return vbq::launch<1>(d, blob_dev, x_bf16, y, workspace, workspace_bytes, flags, st);
+    case 2: return vbq::launch<2>(d, blob_dev, x_bf16, y, workspace, workspace_bytes, flags, st);
+    case 4: return vbq::launch<4>(d, blob_dev, x_bf16, y, workspace, workspace_bytes, flags, st);
+    case 8: return vbq::launch<8>(d, blob_dev, x_bf16, y, workspace, workspace_bytes, flags, st);
+    default: return vbq::launch<16>(d, blob_dev, x_bf16, y, workspace, workspace_bytes, flags, st);
   }
+}
+
+int vbq_gemm_skinny(const vbq_desc* d, const void* blob_dev, const void* x_bf16, int B, float* y,
+                    void* workspace, uint64_t workspace_bytes, void* stream) {
+  return vbq_gemm_skinny_ex(d, blob_dev, x_bf16, B, y, workspace, workspace_bytes, 0u, stream);
 }
 
 int vbq_gemv(const vbq_desc* d, const void* blob_dev, const void* x_bf16, float* y, void* workspace,

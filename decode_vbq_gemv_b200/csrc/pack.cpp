@@ -162,6 +162,7 @@ const char* vbq_strerror(int status) {
     case VBQ_ERR_FORMAT: return "blob is not canonical VBQ format v1";
     case VBQ_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
     case VBQ_ERR_SCRATCH_LIMIT: return "problem needs more scratch than the 16 MiB fixed buffer of the allocation-free entry point";
+    case VBQ_ERR_FLAGS: return "launch options word has bits outside VBQ_LAUNCH_OVERLAP";
     default: return "unknown status";
   }
 }

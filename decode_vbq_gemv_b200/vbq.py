@@ -18,9 +18,10 @@ VBQ_OK = 0
 VBQ_ERR_NULL, VBQ_ERR_SHAPE, VBQ_ERR_WIDTH, VBQ_ERR_CODE_RANGE = -1, -2, -3, -4
 VBQ_ERR_BUFFER_TOO_SMALL, VBQ_ERR_BAD_MAGIC, VBQ_ERR_VERSION, VBQ_ERR_CRC = -5, -6, -7, -8
 VBQ_ERR_BATCH, VBQ_ERR_ALIGN, VBQ_ERR_CUDA, VBQ_ERR_TILE = -9, -10, -11, -12
-VBQ_ERR_FORMAT, VBQ_ERR_WORKSPACE, VBQ_ERR_SCRATCH_LIMIT = -13, -14, -15
+VBQ_ERR_FORMAT, VBQ_ERR_WORKSPACE, VBQ_ERR_SCRATCH_LIMIT, VBQ_ERR_FLAGS = -13, -14, -15, -16
+VBQ_LAUNCH_OVERLAP = 1
 BATCHES = (1, 2, 4, 8, 16)
-DEFAULT_TILE_ROWS = 1024
+DEFAULT_TILE_ROWS = 256
 
 
 class VbqError(RuntimeError):
@@ -64,6 +65,7 @@ def lib() -> ctypes.CDLL:
             "vbq_workspace_init": (i32, [vp, u64, vp]),
             "vbq_gemv": (i32, [dp, vp, vp, vp, vp, u64, vp]),
             "vbq_gemm_skinny": (i32, [dp, vp, vp, i32, vp, vp, u64, vp]),
+            "vbq_gemm_skinny_ex": (i32, [dp, vp, vp, i32, vp, vp, u64, ctypes.c_uint, vp]),
             "vbq_gemm_skinny_noalloc": (i32, [dp, vp, vp, i32, vp, vp]),
         }
         for name, (res, args) in sig.items():
@@ -192,6 +194,18 @@ def vbq_gemm_skinny_status(desc, blob_dev, x_bf16, B, y, workspace=None, stream=
 def vbq_gemm_skinny(desc, blob_dev, x_bf16, B, y, workspace=None, stream=None) -> None:
     """Y[B,N] = X[B,K] W^T on the device (asynchronous on `stream`, default: torch's current stream)."""
     _check(vbq_gemm_skinny_status(desc, blob_dev, x_bf16, B, y, workspace, stream), "vbq_gemm_skinny")
+
+
+def vbq_gemm_skinny_ex_status(desc, blob_dev, x_bf16, B, y, workspace=None, flags=0, stream=None) -> int:
+    ws_ptr = _dev_ptr(workspace) if workspace is not None and workspace.numel() > 0 else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    return lib().vbq_gemm_skinny_ex(ctypes.byref(desc), _dev_ptr(blob_dev), _dev_ptr(x_bf16), B, _dev_ptr(y),
+                                    ws_ptr, ws_bytes, flags, _stream_ptr(stream))
+
+
+def vbq_gemm_skinny_ex(desc, blob_dev, x_bf16, B, y, workspace=None, flags=0, stream=None) -> None:
+    """vbq_gemm_skinny with launch options; flags=VBQ_LAUNCH_OVERLAP enables programmatic dependent launch."""
+    _check(vbq_gemm_skinny_ex_status(desc, blob_dev, x_bf16, B, y, workspace, flags, stream), "vbq_gemm_skinny_ex")
 
 
 def vbq_gemm_skinny_noalloc_status(desc, blob_dev, x_bf16, B, y, stream=None) -> int:

@@ -45,7 +45,8 @@ typedef enum vbq_status {
   VBQ_ERR_TILE = -12,             /* tile rows R not a multiple of 16 in [16, 1024] */
   VBQ_ERR_FORMAT = -13,           /* blob is not canonical format v1 (layout, padding, counts) */
   VBQ_ERR_WORKSPACE = -14,        /* workspace NULL, misaligned or smaller than vbq_workspace_size */
-  VBQ_ERR_SCRATCH_LIMIT = -15     /* vbq_gemm_skinny_noalloc: problem needs more than its 16 MiB fixed buffer */
+  VBQ_ERR_SCRATCH_LIMIT = -15,    /* vbq_gemm_skinny_noalloc: problem needs more than its 16 MiB fixed buffer */
+  VBQ_ERR_FLAGS = -16             /* vbq_gemm_skinny_ex: unknown bits in the launch-options word */
 } vbq_status;
 
 /* Host-side description of a packed blob. It is filled by vbq_pack or vbq_describe and passed by pointer to
@@ -100,8 +101,10 @@ int vbq_unpack(const void* blob_host, uint64_t blob_bytes, uint8_t* widths, uint
 /* Workspace bytes that vbq_gemv / vbq_gemm_skinny need for this matrix and batch on the CURRENT device (the
  * launch shape depends on its SM count). The workspace holds the partial sums of row tiles that several CTAs
  * share, one arrival counter per row tile, and, in its 4 bytes at offset (size - 4), a device status word: 0 after every
- * successful call; nonzero if a kernel gave up a bounded wait (bit 0) or met a record larger than the staging
- * size its descriptor promised (bit 1), in which case the outputs of that call are not valid.
+ * successful call; nonzero if a kernel gave up a bounded wait (bit 0), met a record larger than the staging
+ * size its descriptor promised or a directory entry past the end of the records (bit 1), or met a record whose
+ * bucket counts disagree with its tile or its width codes (bit 2). The outputs of such a call are not valid, and
+ * the workspace must be zeroed again (vbq_workspace_init) before its next use.
  * Errors: NULL, BATCH, FORMAT (desc inconsistent). */
 int vbq_workspace_size(const vbq_desc* d, int B, uint64_t* out_bytes);
 
@@ -127,6 +130,20 @@ int vbq_gemv(const vbq_desc* d, const void* blob_dev, const void* x_bf16, float*
  * Other arguments and guarantees as in vbq_gemv. Errors: NULL, BATCH, ALIGN, WORKSPACE, FORMAT, CUDA. */
 int vbq_gemm_skinny(const vbq_desc* d, const void* blob_dev, const void* x_bf16, int B, float* y,
                     void* workspace, uint64_t workspace_bytes, void* stream);
+
+/* Launch options of vbq_gemm_skinny_ex (bit flags). */
+#define VBQ_LAUNCH_OVERLAP 1u
+
+/* vbq_gemm_skinny with launch options (the VBQ paper has no counterpart; this is a deployment aid).
+ * VBQ_LAUNCH_OVERLAP: programmatic dependent launch. The kernel may begin while the kernel before it on `stream`
+ * is still running. Until that kernel has finished and its writes are visible, it reads only `blob_dev` (the
+ * directory and the records it streams into shared memory); it reads x and touches y and the workspace only
+ * afterwards. So a chain of launches (for example the projections of a decode step) overlaps each kernel's
+ * weight streaming with the tail of the one before. Do not set it when the kernel just before this call on
+ * `stream` writes the blob. Without the flag this is exactly vbq_gemm_skinny.
+ * Errors: as vbq_gemm_skinny, plus FLAGS (unknown bits). */
+int vbq_gemm_skinny_ex(const vbq_desc* d, const void* blob_dev, const void* x_bf16, int B, float* y,
+                       void* workspace, uint64_t workspace_bytes, unsigned flags, void* stream);
 
 /* Allocation-free variant of vbq_gemm_skinny (the VBQ paper has no counterpart; this is a deployment aid).
  *

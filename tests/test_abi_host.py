@@ -31,7 +31,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_status_strings_and_version():
-    for st in range(-14, 1):
+    for st in range(-16, 1):
         assert vbq.vbq_strerror(st) and "unknown" not in vbq.vbq_strerror(st)
     assert vbq.vbq_strerror(-99) == "unknown status"
     assert vbq.vbq_version() >> 16 == 1
@@ -130,3 +130,8 @@ def test_device_entry_argument_checks_need_no_gpu():
     assert L.vbq_workspace_size(dp, 3, ctypes.byref(out)) == vbq.VBQ_ERR_BATCH
     assert L.vbq_workspace_size(dp, 16, ctypes.byref(out)) == vbq.VBQ_OK
     assert L.vbq_workspace_init(None, 0, None) == vbq.VBQ_ERR_NULL
+    # the launch-options entry point: same checks, plus unknown option bits
+    assert L.vbq_gemm_skinny_ex(dp, 16, 16, 1, 16, None, 0, 2, None) == vbq.VBQ_ERR_FLAGS
+    assert L.vbq_gemm_skinny_ex(dp, 16, 16, 3, 16, None, 0, vbq.VBQ_LAUNCH_OVERLAP, None) == vbq.VBQ_ERR_BATCH
+    assert L.vbq_gemm_skinny_ex(dp, 8, 16, 1, 16, None, 0, vbq.VBQ_LAUNCH_OVERLAP, None) == vbq.VBQ_ERR_ALIGN
+    assert L.vbq_gemm_skinny_ex(dp, None, 16, 1, 16, None, 0, 0, None) == vbq.VBQ_ERR_NULL

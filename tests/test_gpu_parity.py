@@ -117,12 +117,13 @@ def test_closed_form_all_max_codes(k, B):
     assert np.all(y == y[:, :1]), "all rows are identical, so their outputs must be bitwise equal"
 
 
+@pytest.mark.parametrize("R", [256, 1024])
 @pytest.mark.parametrize("B", vbq.BATCHES)
-def test_config4_full_size_sampled_rows(B):
+def test_config4_full_size_sampled_rows(B, R):
     g = np.random.default_rng(B)
     for m in S.cfg4(("q", "gate", "down")):
         x = S.make_x(4, m.name, B, m.K)
-        y, _ = gpu_y(m, x)
+        y, _ = gpu_y(m, x, R)
         rows = np.unique(np.concatenate([g.choice(m.N, 200, replace=False), [0, m.N - 1, 1023, 1024]]))
         yref, bound = O.matvec(m.widths[rows], m.scales[rows], m.codes[rows], x, NTH)
         check(y[:, rows], yref, bound, f"cfg4 {m.name} B={B}")
@@ -190,3 +191,51 @@ def test_abi_rejects_bad_device_arguments():
         assert st == vbq.VBQ_ERR_WORKSPACE
         assert vbq.vbq_gemm_skinny_status(mat.desc, mat.blob, x[:m.K], 1, y, None) == vbq.VBQ_ERR_WORKSPACE
     torch.cuda.synchronize()
+
+
+def test_overlapped_launch_chain_matches_plain_launches():
+    """VBQ_LAUNCH_OVERLAP (programmatic dependent launch) on a chain of launches on one stream gives bitwise the
+    results of plain launches. The chain reuses one matrix, its workspace and its output twice in a row with
+    different activations, and feeds a launch with activations that a torch kernel writes just before it; the
+    same chain is also captured in a CUDA graph and replayed."""
+    import torch
+    q, gate = S.cfg4(("q",))[0], S.cfg4(("gate",))[0]
+    mq = vbq.DeviceMatrix(vbq.vbq_pack(q.N, q.K, 256, q.widths, q.scales, q.codes)[0], dev(), max_batch=1)
+    mg = vbq.DeviceMatrix(vbq.vbq_pack(gate.N, gate.K, 256, gate.widths, gate.scales, gate.codes)[0], dev(),
+                          max_batch=1)
+    xa, xb = (to_dev_x(S.x_normal(1, q.K, np.random.default_rng(s))) for s in (1, 2))
+    x_src = to_dev_x(S.x_normal(1, gate.K, np.random.default_rng(3)))
+
+    def chain(flags, x_c):
+        ys = [torch.full((1, m.N), np.nan, dtype=torch.float32, device=dev()) for m in (q, q, gate)]
+        vbq.vbq_gemm_skinny_ex(mq.desc, mq.blob, xa, 1, ys[0], mq.workspaces[1], flags)
+        vbq.vbq_gemm_skinny_ex(mq.desc, mq.blob, xb, 1, ys[1], mq.workspaces[1], flags)
+        x_c.copy_(x_src)  # a kernel writes the next launch's activations
+        vbq.vbq_gemm_skinny_ex(mg.desc, mg.blob, x_c, 1, ys[2], mg.workspaces[1], flags)
+        return ys
+
+    x_c = torch.zeros_like(x_src)
+    want = [y.cpu() for y in chain(0, x_c)]
+    torch.cuda.synchronize()
+    for rep in range(3):
+        x_c.zero_()
+        got = chain(vbq.VBQ_LAUNCH_OVERLAP, x_c)
+        torch.cuda.synchronize()
+        for k in range(3):
+            assert torch.equal(got[k].cpu(), want[k]), f"eager overlapped chain, rep {rep}, launch {k}"
+    s = torch.cuda.Stream()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        x_c.zero_()
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g, stream=s):
+            x_c.zero_()
+            ys = chain(vbq.VBQ_LAUNCH_OVERLAP, x_c)
+        for rep in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+    for k in range(3):
+        assert torch.equal(ys[k].cpu(), want[k]), f"graph-replayed overlapped chain, launch {k}"
+    for m in (mq, mg):
+        need = vbq.vbq_workspace_size(m.desc, 1)
+        assert int(m.workspaces[1][need - 4:need].cpu().numpy().view(np.uint32)[0]) == 0

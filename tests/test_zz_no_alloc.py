@@ -59,7 +59,7 @@ def test_noalloc_rejects_problems_above_its_fixed_buffer():
     w = np.ones((N, 1), np.uint8)
     s = np.full((N, 1), 0x3C00, np.uint16)
     c = np.zeros((N, K), np.uint8)
-    blob, desc = vbq.vbq_pack(N, K, vbq.DEFAULT_TILE_ROWS, w, s, c)
+    blob, desc = vbq.vbq_pack(N, K, 1024, w, s, c)
     assert vbq.vbq_workspace_size(desc, B) > 16 << 20
     blob_dev = torch.from_numpy(blob).to(dev())
     x = torch.zeros((B, K), dtype=torch.bfloat16, device=dev())
