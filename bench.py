@@ -32,6 +32,7 @@ import vbq_synth as S  # noqa: E402
 METRIC = "mixed-bit GEMV achieved HBM GB/s (% of B200 peak); decode-step µs at 1 GPU"
 UNIT = "GB/s"
 NAMES = ("q", "k", "v", "o", "gate", "up", "down")
+GROUPS = (("q", "k", "v"), ("o",), ("gate", "up"), ("down",))   # projections that share their input, fused
 WORKLOAD = "9B-shaped decoder-layer linears (q,k,v,o 4096x4096; gate,up 4096->14336; down 14336->4096)"
 
 
@@ -210,52 +211,70 @@ def run_vbq(args):
     torch.cuda.set_device(dev)
     B, R = args.batch, args.tile_rows
 
-    layers = []   # per copy: list of (DeviceMatrix, x_dev, y_dev, x_host_pinned, y_host_pinned, bytes)
-    for cp in range(args.copies):
-        lin = []
-        for m in layer_matrices(cp):
-            blob, _ = vbq.vbq_pack(m.N, m.K, R, m.widths, m.scales, m.codes)
-            mat = vbq.DeviceMatrix(blob, dev, max_batch=B)
-            xb = S.make_x(4, m.name, B, m.K, layer=cp)
-            xh = torch.from_numpy(xb.astype(np.int16)).view(torch.bfloat16).pin_memory()
-            xd = xh.to(dev)
-            yd = torch.empty((B, m.N), dtype=torch.float32, device=dev)
-            yh = torch.empty((B, m.N), dtype=torch.float32).pin_memory()
-            nbytes = mat.nbytes + B * m.K * 2 + B * m.N * 4
-            lin.append((mat, xd, yd, xh, yh, nbytes, m.name))
-            del blob
-        layers.append(lin)
-    step_bytes = [sum(l[5] for l in lin) for lin in layers]
-
+    # A step is one pass over the layer's seven linears, as launch groups. Fused (default): q/k/v share their
+    # input and run as one launch, so do gate/up; o and down run alone (4 launches). --no-fuse: 7 launches.
+    groups = [("q",), ("k",), ("v",), ("o",), ("gate",), ("up",), ("down",)] if args.no_fuse else GROUPS
     flags = 0 if args.no_overlap else vbq.VBQ_LAUNCH_OVERLAP
 
-    def launch(mat, xd, yd, st):
-        vbq.vbq_gemm_skinny_ex(mat.desc, mat.blob, xd, B, yd, mat.workspaces[B], flags, st)
+    class Group:
+        pass
+
+    layers = []   # per copy: list of Group
+    for cp in range(args.copies):
+        by_name = {m.name: m for m in layer_matrices(cp)}
+        lin = []
+        for names in groups:
+            g = Group()
+            g.name = "_".join(names)
+            ms = [by_name[n] for n in names]
+            g.mats = []
+            for m in ms:
+                blob, _ = vbq.vbq_pack(m.N, m.K, R, m.widths, m.scales, m.codes)
+                g.mats.append(vbq.DeviceMatrix(blob, dev, max_batch=B))
+                del blob
+            g.fused = vbq.FusedMatrices(g.mats, max_batch=B) if len(ms) > 1 else None
+            xb = S.make_x(4, names[0], B, ms[0].K, layer=cp)
+            g.xh = torch.from_numpy(xb.astype(np.int16)).view(torch.bfloat16).pin_memory()
+            g.xd = g.xh.to(dev)
+            g.yd = [torch.empty((B, m.N), dtype=torch.float32, device=dev) for m in ms]
+            g.yh = [torch.empty((B, m.N), dtype=torch.float32).pin_memory() for m in ms]
+            g.nbytes = sum(mt.nbytes for mt in g.mats) + B * ms[0].K * 2 + sum(B * m.N * 4 for m in ms)
+            lin.append(g)
+        layers.append(lin)
+    step_bytes = [sum(g.nbytes for g in lin) for lin in layers]
+
+    def launch(g, st):
+        if g.fused is not None:
+            g.fused.matmul(g.xd, g.yd, flags, st)
+        else:
+            mat = g.mats[0]
+            vbq.vbq_gemm_skinny_ex(mat.desc, mat.blob, g.xd, B, g.yd[0], mat.workspaces[B], flags, st)
 
     # One CUDA graph per layer copy, so that the timed region has no host launch gaps: device-resident step
-    # (seven GEMVs) and end-to-end step (pinned x -> device, seven GEMVs, y -> pinned host).
+    # and end-to-end step (pinned x -> device, the launches, y -> pinned host).
     stream = torch.cuda.Stream(dev)
     graphs, graphs_e2e = [], []
     with torch.cuda.stream(stream):
         for lin in layers:
-            for mat, xd, yd, *_ in lin:
-                launch(mat, xd, yd, stream)
+            for g in lin:
+                launch(g, stream)
         torch.cuda.synchronize()
         for lin in layers:
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=stream):
-                for mat, xd, yd, *_ in lin:
-                    launch(mat, xd, yd, stream)
-            graphs.append(g)
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr, stream=stream):
+                for g in lin:
+                    launch(g, stream)
+            graphs.append(gr)
             g2 = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g2, stream=stream):
-                for mat, xd, yd, xh, yh, *_ in lin:
-                    xd.copy_(xh, non_blocking=True)
-                    launch(mat, xd, yd, stream)
-                    yh.copy_(yd, non_blocking=True)
+                for g in lin:
+                    g.xd.copy_(g.xh, non_blocking=True)
+                    launch(g, stream)
+                    for yd, yh in zip(g.yd, g.yh):
+                        yh.copy_(yd, non_blocking=True)
             graphs_e2e.append(g2)
     torch.cuda.synchronize()
-    launches_per_step = len(NAMES)
+    launches_per_step = len(groups)
 
     def timed(gs):
         for i in range(args.warmup):
@@ -284,16 +303,15 @@ def run_vbq(args):
     launch_ms = ms / (args.steps * launches_per_step)
     launch_bytes = total_bytes / (args.steps * launches_per_step)
 
-    # Per-linear kernel time: one graph of `reps` launches of that linear, timed alone (copy 0).
+    # Per-launch-group kernel time: one graph of `reps` launches of that group, timed alone (copy 0).
     per_shape = {}
     reps = 20
-    for k, (mat, xd, yd, *_rest) in enumerate(layers[0]):
-        name = NAMES[k]
+    for g in layers[0]:
         with torch.cuda.stream(stream):
             gl = torch.cuda.CUDAGraph()
             with torch.cuda.graph(gl, stream=stream):
                 for _ in range(reps):
-                    launch(mat, xd, yd, stream)
+                    launch(g, stream)
             gl.replay()
             torch.cuda.synchronize()
             e0 = torch.cuda.Event(enable_timing=True)
@@ -303,12 +321,11 @@ def run_vbq(args):
             e1.record(stream)
         torch.cuda.synchronize()
         us = e0.elapsed_time(e1) * 1e3 / reps
-        nb = layers[0][k][5]
-        per_shape[name] = {"us": us, "GBps": nb / (us / 1e6) / 1e9, "note": "same matrix repeated (L2-warm)"}
+        per_shape[g.name] = {"us": us, "GBps": g.nbytes / (us / 1e6) / 1e9, "note": "same launch repeated (L2-warm)"}
 
     # End to end through host buffers.
-    h2d = sum(l[3].numel() * 2 for l in layers[0])
-    d2h = sum(l[4].numel() * 4 for l in layers[0])
+    h2d = sum(g.xh.numel() * 2 for g in layers[0])
+    d2h = sum(sum(y.numel() * 4 for y in g.yh) for g in layers[0])
     e2e_ms = allreduce_max(timed(graphs_e2e), world)
     e2e_val = total_bytes * world / (e2e_ms / 1e3) / 1e9
     n_launches = args.steps * launches_per_step
@@ -322,7 +339,9 @@ def run_vbq(args):
             "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "fp32", "data": "synthetic",
             "config": {"workload": WORKLOAD, "batch": B, "tile_rows": R,
-                       "launch": "plain" if args.no_overlap else "programmatic dependent launch (VBQ_LAUNCH_OVERLAP)",
+                       "launch": ("plain" if args.no_overlap else "programmatic dependent launch (VBQ_LAUNCH_OVERLAP)")
+                                 + ("; one launch per linear" if args.no_fuse
+                                    else "; q/k/v and gate/up fused (vbq_gemm_skinny_multi), 4 launches per layer"),
                        "weights": "seeded synthetic VBQ groups: P(1,2,4,8 bit) = (0.69,0.16,0.09,0.06), fp16 "
                                   "scales U(0.01,0.1), uniform codes; x ~ N(0,1) bf16",
                        "l2": f"inputs larger than L2: {args.copies} distinct layer copies in rotation "
@@ -333,7 +352,7 @@ def run_vbq(args):
                          "frac": achieved / peak, "traffic": None, "peak_kind": peak_kind,
                          "kernel": f"vbq_kernel<{B}>",
                          "algorithmic_bytes_per_launch": launch_bytes, "avg_launch_us": launch_ms * 1e3},
-            "per_linear": per_shape,
+            "per_launch_group": per_shape,
             "e2e": {"value": e2e_val, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": n_launches,
             "clocks": clocks,
@@ -355,6 +374,8 @@ def main():
     ap.add_argument("--impl", default="vbq", choices=("vbq", "reference"))
     ap.add_argument("--copies", type=int, default=4)
     ap.add_argument("--tile-rows", type=int, default=256)
+    ap.add_argument("--no-fuse", action="store_true",
+                    help="one launch per linear instead of fusing the projections that share their input")
     ap.add_argument("--no-overlap", action="store_true",
                     help="plain launches instead of programmatic dependent launch between the linears")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds for the CPU-oracle baseline (0: skip)")

@@ -50,16 +50,23 @@ template <int B> struct Cfg {
   static constexpr int kXBytes = (B == 1) ? 3 * 64 * 4 : (B < 8 ? 64 * B * 4 : 32 * kAStride * 2);
 };
 
+// Up to kMaxMats matrices with the same K and tile rows run as one sequence of records (and row tiles): matrix m
+// holds global records [rec_start[m], rec_start[m+1]) and tiles [tile_start[m], tile_start[m+1]).
+constexpr int kMaxMats = 4;
 struct Params {
-  const uint32_t* dir;     // record directory (16-byte units from recs), T*G+1 entries
-  const uint8_t* recs;     // first record
-  const uint16_t* x;       // bf16 bits, [B][K]
-  float* y;                // [B][N]
+  const uint32_t* dir[kMaxMats];   // record directory of matrix m (16-byte units from recs[m]), T_m*G+1 entries
+  const uint8_t* recs[kMaxMats];   // first record of matrix m
+  float* y[kMaxMats];              // output of matrix m, [B][N_m]
+  int N[kMaxMats];
+  uint32_t units_total[kMaxMats];  // dir[m][T_m*G]: 16-byte units of matrix m's records
+  int rec_start[kMaxMats + 1];
+  int tile_start[kMaxMats + 1];
+  int nmat;
+  const uint16_t* x;       // bf16 bits, [B][K], shared by all matrices
   float* partial;          // [nCTA + T][R][B] partial sums of shared row tiles
   unsigned* arrive;        // [T] owners that have published their partial sums; zero between calls
   unsigned* status;        // device status word
-  int N, K, G, R, T, nrec;
-  uint32_t units_total;    // dir[nrec]: 16-byte units of all records
+  int K, G, R, T, nrec;    // T, nrec: all matrices
   int NT, TW, S;           // teams per CTA, warps per team, stages per team
   int stage_bytes;         // record capacity of one stage (multiple of 128)
   int stage_size;          // stage: record, then the column's bf16 activations [B][64]
@@ -67,6 +74,33 @@ struct Params {
   int acc_off, res_off;
   int warps_off, warp_bytes;
 };
+
+// Element m of a kernel-parameter array through a select chain (a dynamic index would copy the array to local
+// memory).
+template <typename T>
+__device__ __forceinline__ T pick(const T (&a)[kMaxMats], int m) {
+  return m == 0 ? a[0] : m == 1 ? a[1] : m == 2 ? a[2] : a[3];
+}
+__device__ __forceinline__ int mat_of_tile(const Params& p, int t) {
+  return (p.nmat > 1 && t >= p.tile_start[1]) + (p.nmat > 2 && t >= p.tile_start[2]) +
+         (p.nmat > 3 && t >= p.tile_start[3]);
+}
+__device__ __forceinline__ int mat_of_rec(const Params& p, int j) {
+  return (p.nmat > 1 && j >= p.rec_start[1]) + (p.nmat > 2 && j >= p.rec_start[2]) +
+         (p.nmat > 3 && j >= p.rec_start[3]);
+}
+// Where tile t's outputs go: row r, batch b at y[b * ld + r]; Rt rows.
+struct TileOut {
+  float* y;
+  int ld, Rt;
+};
+__device__ __forceinline__ TileOut tile_out(const Params& p, int t) {
+  const int m = mat_of_tile(p, t);
+  const int tl = t - (m == 0 ? 0 : m == 1 ? p.tile_start[1] : m == 2 ? p.tile_start[2] : p.tile_start[3]);
+  const int N = pick(p.N, m);
+  return TileOut{pick(p.y, m) + size_t(tl) * p.R, N, min(p.R, N - tl * p.R)};
+}
+
 
 __host__ __device__ constexpr int align16i(int v) { return (v + 15) & ~15; }
 __host__ __device__ constexpr int align128i(int v) { return (v + 127) & ~127; }
@@ -507,7 +541,8 @@ __global__ void __launch_bounds__(Cfg<B>::kThreads, 1) vbq_kernel(Params p) {
   auto reduce_tile = [&](int t, int gtid, int gthreads) {
     int first;
     const int owners = tile_owners(t, first);
-    const int Rt = min(R, p.N - t * R);
+    const TileOut to = tile_out(p, t);
+    const int Rt = to.Rt;
     for (int e = gtid; e < Rt * B; e += gthreads) {
       float v = 0.f;
       for (int k0 = 0; k0 < owners; k0 += 8) {
@@ -520,7 +555,7 @@ __global__ void __launch_bounds__(Cfg<B>::kThreads, 1) vbq_kernel(Params p) {
           if (k0 + q < owners) v += part[q];
       }
       const int r = e / B, b = e - r * B;
-      p.y[size_t(b) * p.N + size_t(t) * R + r] = v;
+      to.y[size_t(b) * to.ld + r] = v;
     }
   };
 
@@ -549,31 +584,41 @@ __global__ void __launch_bounds__(Cfg<B>::kThreads, 1) vbq_kernel(Params p) {
     // (their latency is what the first copy waits for); lane 0 sets up the team's barriers and issues the copies
     int issued = 0;
     int win = 0;
-    uint32_t dlane = 0;
-    if (tw == 0) dlane = lane <= nt ? __ldg(p.dir + tb + lane) : 0u;
-    auto dir_at = [&](int i) -> uint32_t {  // whole warp; i in [0, nt], non-decreasing between calls
+    uint32_t d_lo = 0, d_hi = 0;  // directory entries (start, end) of record tb + win + lane
+    int d_m = 0;                  // its matrix
+    auto load_dir = [&]() {
+      const int j = tb + win + lane;
+      if (win + lane < nt) {
+        d_m = mat_of_rec(p, j);
+        const int jl = j - (d_m == 0 ? 0 : d_m == 1 ? p.rec_start[1] : d_m == 2 ? p.rec_start[2] : p.rec_start[3]);
+        const uint32_t* dir = pick(p.dir, d_m);
+        d_lo = __ldg(dir + jl);
+        d_hi = __ldg(dir + jl + 1);
+      }
+    };
+    if (tw == 0) load_dir();
+    // Record i's bulk copy into stage i % S (whole warp, i non-decreasing between calls; lane 0 issues). The
+    // activations follow with issue_x.
+    auto issue_record = [&](int i) {
       if (i >= win + 32) {
         win = i;
-        dlane = win + lane <= nt ? __ldg(p.dir + tb + win + lane) : 0u;
+        load_dir();
       }
-      return __shfl_sync(0xFFFFFFFFu, dlane, i - win);
-    };
-    // Record i's bulk copy into stage i % S (whole warp; lane 0 issues). The activations follow with issue_x.
-    auto issue_record = [&](int i) {
-      const uint32_t a = dir_at(i);
-      const uint32_t b = dir_at(i + 1);
+      const uint32_t a = __shfl_sync(0xFFFFFFFFu, d_lo, i - win);
+      const uint32_t b = __shfl_sync(0xFFFFFFFFu, d_hi, i - win);
+      const int m = __shfl_sync(0xFFFFFFFFu, d_m, i - win);
       if (lane != 0) return;
       const int s = i % S;
       unsigned char* dst = tbase + s * p.stage_size;
       const unsigned bytes = 16u * (b - a);
-      if (b < a || b > p.units_total || bytes > unsigned(p.stage_bytes)) {  // not what the descriptor promised
+      if (b < a || b > pick(p.units_total, m) || bytes > unsigned(p.stage_bytes)) {  // not what was promised
         stage_bad[team * S + s] = 1;
         atomicOr(p.status, kStatusOversize);
         mbar_arrive(&bars[s]);
       } else {
         stage_bad[team * S + s] = 0;
         mbar_arrive_tx(&bars[s], bytes + 128u * B);
-        tma_bulk_load(dst, p.recs + 16ull * a, bytes, &bars[s]);
+        tma_bulk_load(dst, pick(p.recs, m) + 16ull * a, bytes, &bars[s]);
       }
     };
     auto issue_x = [&](int i) {  // lane 0
@@ -605,11 +650,12 @@ __global__ void __launch_bounds__(Cfg<B>::kThreads, 1) vbq_kernel(Params p) {
     // partial tile shared inside the CTA stays here for the combine at the end.
     auto flush = [&](int t) {
       if (tseg >= 0) return;  // shared inside the CTA: the combine at the end writes it
-      const int Rt = min(R, p.N - t * R);
+      const TileOut to = tile_out(p, t);
+      const int Rt = to.Rt;
       if (tb <= t * G && tb + nt >= (t + 1) * G) {
         for (int r = sl0 + lane; r < min(sl1, Rt); r += 32)
 #pragma unroll
-          for (int b = 0; b < B; ++b) p.y[size_t(b) * p.N + size_t(t) * R + r] = acc[r * B + b];
+          for (int b = 0; b < B; ++b) to.y[size_t(b) * to.ld + r] = acc[r * B + b];
       } else {
         float* slot = p.partial + size_t(cta + t) * R * B;
         for (int e = sl0 * B + lane; e < min(sl1, Rt) * B; e += 32) slot[e] = acc[e];
@@ -626,7 +672,7 @@ __global__ void __launch_bounds__(Cfg<B>::kThreads, 1) vbq_kernel(Params p) {
       if (ok && stage_bad[team * S + s]) ok = false;
       ok = __all_sync(0xFFFFFFFFu, ok);  // lanes can see an abort at different times; the warp decides as one
       const int j = tb + i, t = j / G;
-      const int Rt = min(R, p.N - t * R);
+      const int Rt = tile_out(p, t).Rt;
       if (t != cur_t) {
         if (cur_t >= 0) flush(cur_t);
         for (int e = sl0 * B + lane; e < sl1 * B; e += 32) acc[e] = 0.f;
@@ -899,7 +945,9 @@ __global__ void __launch_bounds__(Cfg<B>::kThreads, 1) vbq_kernel(Params p) {
       const int k0 = tm.seg_team0(i), m = tm.seg_team0(i + 1) - k0;
       if (m < 2) continue;
       const int s0 = tm.seg_lo(i), s1 = tm.seg_hi(i);
-      const int t = s0 / G, Rt = min(R, p.N - t * R);
+      const int t = s0 / G;
+      const TileOut to = tile_out(p, t);
+      const int Rt = to.Rt;
       const bool whole = s0 <= t * G && s1 >= (t + 1) * G;
       float* slot = p.partial + size_t(cta + t) * R * B;
       for (int e = tid; e < Rt * B; e += C::kThreads) {
@@ -908,7 +956,7 @@ __global__ void __launch_bounds__(Cfg<B>::kThreads, 1) vbq_kernel(Params p) {
           if (team_live[k0 + q]) v += reinterpret_cast<const float*>(smem + (k0 + q) * p.team_bytes + p.acc_off)[e];
         if (whole) {
           const int r = e / B, b = e - r * B;
-          p.y[size_t(b) * p.N + size_t(t) * R + r] = v;
+          to.y[size_t(b) * to.ld + r] = v;
         } else {
           slot[e] = v;
         }
@@ -957,19 +1005,61 @@ inline int num_sms() {
   return sms;
 }
 
+// The matrices of one launch, seen as one record sequence.
+struct Problem {
+  int nmat;
+  const vbq_desc* d[kMaxMats];
+  int R, K, G;
+  long long T, nrec;
+  uint64_t max_record_bytes;
+};
+
+inline bool desc_ok(const vbq_desc* d) {
+  return d->version == 1 && d->N >= 1 && d->K >= 64 && d->K % 64 == 0 && d->G == d->K / 64 && d->R >= 16 &&
+         d->R <= kMaxTileRows && d->R % 16 == 0 && d->T == (d->N + d->R - 1) / d->R && d->N <= INT32_MAX &&
+         d->K <= INT32_MAX && d->dir_offset == 64 && d->rec_offset > d->dir_offset &&
+         d->total_bytes > d->rec_offset && d->max_record_bytes >= 32 &&
+         d->max_record_bytes <= d->total_bytes - d->rec_offset && d->max_record_bytes % 16 == 0 &&
+         (d->total_bytes - d->rec_offset) % 16 == 0 && (d->total_bytes - d->rec_offset) / 16 <= 0xFFFFFFFFull;
+}
+
+// Validates the descriptors of one launch: 1..kMaxMats consistent matrices with equal K (SHAPE) and equal tile
+// rows (TILE), and record and tile counts that fit the kernel's 32-bit indices (FORMAT).
+inline int make_problem(int nmat, const vbq_desc* const* d, Problem& pr) {
+  if (!d) return VBQ_ERR_NULL;
+  if (nmat < 1 || nmat > kMaxMats) return VBQ_ERR_SHAPE;
+  pr.nmat = nmat;
+  pr.T = pr.nrec = 0;
+  pr.max_record_bytes = 0;
+  for (int m = 0; m < nmat; ++m) {
+    if (!d[m]) return VBQ_ERR_NULL;
+    if (!desc_ok(d[m])) return VBQ_ERR_FORMAT;
+    if (d[m]->K != d[0]->K) return VBQ_ERR_SHAPE;
+    if (d[m]->R != d[0]->R) return VBQ_ERR_TILE;
+    pr.d[m] = d[m];
+    pr.T += d[m]->T;
+    pr.nrec += d[m]->T * d[m]->G;
+    if (d[m]->max_record_bytes > pr.max_record_bytes) pr.max_record_bytes = d[m]->max_record_bytes;
+  }
+  pr.R = int(d[0]->R);
+  pr.K = int(d[0]->K);
+  pr.G = int(d[0]->G);
+  if (pr.nrec >= (1ll << 30) || pr.max_record_bytes > (1ull << 30)) return VBQ_ERR_FORMAT;
+  return VBQ_OK;
+}
+
 // Teams per CTA, warps per team and stages per team. A team's record copies overlap its arithmetic when it has
 // two stages; with one, every record's load latency is exposed. The plan that fits in shared memory with the
 // fewest exposed load latencies (records per team / stages, rounded up) wins; ties go to more warps, then to
 // more teams.
 template <int B>
-inline bool make_plan_t(const vbq_desc& d, int sms, Plan& pl) {
+inline bool make_plan_t(const Problem& pr, int sms, Plan& pl) {
   using C = Cfg<B>;
   pl.grid = sms;
   pl.threads = C::kThreads;
-  const int R = int(d.R);
-  const long long nrec = d.T * d.G;
-  const int rpc = int((nrec + pl.grid - 1) / pl.grid);
-  pl.stage_bytes = align128i(int(d.max_record_bytes));
+  const int R = pr.R;
+  const int rpc = int((pr.nrec + pl.grid - 1) / pl.grid);
+  pl.stage_bytes = align128i(int(pr.max_record_bytes));
   pl.stage_size = pl.stage_bytes + align128i(128 * B);
   const int acc_bytes = align128i(R * B * 4);
   pl.warp_bytes = WarpOff(C::kXBytes, B).size();
@@ -1000,51 +1090,55 @@ inline bool make_plan_t(const vbq_desc& d, int sms, Plan& pl) {
     }
   }
   if (best_key < 0) return false;
-  const uint64_t slots = uint64_t(pl.grid) + uint64_t(d.T);
+  const uint64_t slots = uint64_t(pl.grid) + uint64_t(pr.T);
   pl.counters_off = slots * uint64_t(R) * B * 4;
-  pl.ws_bytes = (pl.counters_off + uint64_t(d.T) * 4 + 4 + 15) / 16 * 16;
+  pl.ws_bytes = (pl.counters_off + uint64_t(pr.T) * 4 + 4 + 15) / 16 * 16;
   pl.status_off = pl.ws_bytes - 4;
   return true;
 }
 
-inline bool make_plan(const vbq_desc& d, int B, int sms, Plan& pl) {
+inline bool make_plan(const Problem& pr, int B, int sms, Plan& pl) {
   switch (B) {
-    case 1: return make_plan_t<1>(d, sms, pl);
-    case 2: return make_plan_t<2>(d, sms, pl);
-    case 4: return make_plan_t<4>(d, sms, pl);
-    case 8: return make_plan_t<8>(d, sms, pl);
-    default: return make_plan_t<16>(d, sms, pl);
+    case 1: return make_plan_t<1>(pr, sms, pl);
+    case 2: return make_plan_t<2>(pr, sms, pl);
+    case 4: return make_plan_t<4>(pr, sms, pl);
+    case 8: return make_plan_t<8>(pr, sms, pl);
+    default: return make_plan_t<16>(pr, sms, pl);
   }
 }
 
-inline bool desc_ok(const vbq_desc* d) {
-  return d->version == 1 && d->N >= 1 && d->K >= 64 && d->K % 64 == 0 && d->G == d->K / 64 && d->R >= 16 &&
-         d->R <= kMaxTileRows && d->R % 16 == 0 && d->T == (d->N + d->R - 1) / d->R && d->N <= INT32_MAX &&
-         d->K <= INT32_MAX && d->dir_offset == 64 && d->rec_offset > d->dir_offset &&
-         d->total_bytes > d->rec_offset && d->max_record_bytes >= 32 &&
-         d->max_record_bytes <= d->total_bytes - d->rec_offset && d->max_record_bytes % 16 == 0 &&
-         (d->total_bytes - d->rec_offset) % 16 == 0 && (d->total_bytes - d->rec_offset) / 16 <= 0xFFFFFFFFull;
-}
-
 template <int B>
-int launch(const vbq_desc* d, const void* blob, const void* x, float* y, void* ws, uint64_t ws_bytes,
+int launch(const Problem& pr, const void* const* blobs, const void* x, float* const* ys, void* ws, uint64_t ws_bytes,
            unsigned flags, cudaStream_t stream) {
   Plan pl;
-  if (!make_plan_t<B>(*d, num_sms(), pl)) return VBQ_ERR_FORMAT;
+  if (!make_plan_t<B>(pr, num_sms(), pl)) return VBQ_ERR_FORMAT;
   if (!ws || (reinterpret_cast<uintptr_t>(ws) & 15) || ws_bytes < pl.ws_bytes) return VBQ_ERR_WORKSPACE;
-  Params p;
-  const uint8_t* base = static_cast<const uint8_t*>(blob);
-  p.dir = reinterpret_cast<const uint32_t*>(base + d->dir_offset);
-  p.recs = base + d->rec_offset;
+  Params p = {};
+  p.nmat = pr.nmat;
+  int tiles = 0, recs = 0;
+  for (int m = 0; m < kMaxMats; ++m) {
+    p.tile_start[m] = tiles;
+    p.rec_start[m] = recs;
+    if (m >= pr.nmat) continue;
+    const vbq_desc* d = pr.d[m];
+    const uint8_t* base = static_cast<const uint8_t*>(blobs[m]);
+    p.dir[m] = reinterpret_cast<const uint32_t*>(base + d->dir_offset);
+    p.recs[m] = base + d->rec_offset;
+    p.y[m] = ys[m];
+    p.N[m] = int(d->N);
+    p.units_total[m] = uint32_t((d->total_bytes - d->rec_offset) / 16);
+    tiles += int(d->T);
+    recs += int(d->T * d->G);
+  }
+  p.tile_start[kMaxMats] = tiles;
+  p.rec_start[kMaxMats] = recs;
   p.x = static_cast<const uint16_t*>(x);
-  p.y = y;
   uint8_t* w = static_cast<uint8_t*>(ws);
   p.partial = reinterpret_cast<float*>(w);
   p.arrive = reinterpret_cast<unsigned*>(w + pl.counters_off);
   p.status = reinterpret_cast<unsigned*>(w + pl.status_off);
-  p.N = int(d->N); p.K = int(d->K); p.G = int(d->G); p.R = int(d->R); p.T = int(d->T);
-  p.nrec = int(d->T * d->G);
-  p.units_total = uint32_t((d->total_bytes - d->rec_offset) / 16);
+  p.K = pr.K; p.G = pr.G; p.R = pr.R; p.T = tiles;
+  p.nrec = recs;
   p.NT = pl.NT; p.TW = pl.TW; p.S = pl.S;
   p.stage_bytes = pl.stage_bytes;
   p.stage_size = pl.stage_size;
@@ -1077,18 +1171,26 @@ int launch(const vbq_desc* d, const void* blob, const void* x, float* y, void* w
   return cudaPeekAtLastError() == cudaSuccess ? VBQ_OK : VBQ_ERR_CUDA;
 }
 
+inline bool batch_ok(int B) { return B == 1 || B == 2 || B == 4 || B == 8 || B == 16; }
+
 }  // namespace vbq
 
 extern "C" {
 
-int vbq_workspace_size(const vbq_desc* d, int B, uint64_t* out_bytes) {
+int vbq_workspace_size_multi(int nmat, const vbq_desc* const* d, int B, uint64_t* out_bytes) {
   if (!d || !out_bytes) return VBQ_ERR_NULL;
-  if (B != 1 && B != 2 && B != 4 && B != 8 && B != 16) return VBQ_ERR_BATCH;
-  if (!vbq::desc_ok(d)) return VBQ_ERR_FORMAT;
+  if (!vbq::batch_ok(B)) return VBQ_ERR_BATCH;
+  vbq::Problem pr;
+  if (int st = vbq::make_problem(nmat, d, pr)) return st;
   vbq::Plan pl;
-  if (!vbq::make_plan(*d, B, vbq::num_sms(), pl)) return VBQ_ERR_FORMAT;
+  if (!vbq::make_plan(pr, B, vbq::num_sms(), pl)) return VBQ_ERR_FORMAT;
   *out_bytes = pl.ws_bytes;
   return VBQ_OK;
+}
+
+int vbq_workspace_size(const vbq_desc* d, int B, uint64_t* out_bytes) {
+  if (!d) return VBQ_ERR_NULL;
+  return vbq_workspace_size_multi(1, &d, B, out_bytes);
 }
 
 int vbq_workspace_init(void* workspace, uint64_t workspace_bytes, void* stream) {
@@ -1098,23 +1200,34 @@ int vbq_workspace_init(void* workspace, uint64_t workspace_bytes, void* stream) 
              ? VBQ_OK : VBQ_ERR_CUDA;
 }
 
+int vbq_gemm_skinny_multi(int nmat, const vbq_desc* const* d, const void* const* blob_dev, const void* x_bf16,
+                          int B, float* const* y, void* workspace, uint64_t workspace_bytes, unsigned flags,
+                          void* stream) {
+  if (!d || !blob_dev || !x_bf16 || !y) return VBQ_ERR_NULL;
+  for (int m = 0; m < nmat && m < vbq::kMaxMats; ++m)
+    if (!d[m] || !blob_dev[m] || !y[m]) return VBQ_ERR_NULL;
+  if (!vbq::batch_ok(B)) return VBQ_ERR_BATCH;
+  if (flags & ~unsigned(VBQ_LAUNCH_OVERLAP)) return VBQ_ERR_FLAGS;
+  vbq::Problem pr;
+  if (int st = vbq::make_problem(nmat, d, pr)) return st;
+  if (reinterpret_cast<uintptr_t>(x_bf16) & 15) return VBQ_ERR_ALIGN;
+  for (int m = 0; m < nmat; ++m)
+    if ((reinterpret_cast<uintptr_t>(blob_dev[m]) & 15) || (reinterpret_cast<uintptr_t>(y[m]) & 3))
+      return VBQ_ERR_ALIGN;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  switch (B) {
+    case 1: return vbq::launch<1>(pr, blob_dev, x_bf16, y, workspace, workspace_bytes, flags, st);
+    case 2: return vbq::launch<2>(pr, blob_dev, x_bf16, y, workspace, workspace_bytes, flags, st);
+    case 4: return vbq::launch<4>(pr, blob_dev, x_bf16, y, workspace, workspace_bytes, flags, st);
+    case 8: return vbq::launch<8>(pr, blob_dev, x_bf16, y, workspace, workspace_bytes, flags, st);
+    default: return vbq::launch<16>(pr, blob_dev, x_bf16, y, workspace, workspace_bytes, flags, st);
+  }
+}
+
 int vbq_gemm_skinny_ex(const vbq_desc* d, const void* blob_dev, const void* x_bf16, int B, float* y,
                        void* workspace, uint64_t workspace_bytes, unsigned flags, void* stream) {
   if (!d || !blob_dev || !x_bf16 || !y) return VBQ_ERR_NULL;
-  if (B != 1 && B != 2 && B != 4 && B != 8 && B != 16) return VBQ_ERR_BATCH;
-  if (flags & ~unsigned(VBQ_LAUNCH_OVERLAP)) return VBQ_ERR_FLAGS;
-  if (!vbq::desc_ok(d)) return VBQ_ERR_FORMAT;
-  if ((reinterpret_cast<uintptr_t>(blob_dev) & 15) || (reinterpret_cast<uintptr_t>(x_bf16) & 15) ||
-      (reinterpret_cast<uintptr_t>(y) & 3))
-    return VBQ_ERR_ALIGN;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  switch (B) {
-    case 1: return vbq::launch<1>(d, blob_dev, x_bf16, y, workspace, workspace_bytes, flags, st);
-    case 2: return vbq::launch<2>(d, blob_dev, x_bf16, y, workspace, workspace_bytes, flags, st);
-    case 4: return vbq::launch<4>(d, blob_dev, x_bf16, y, workspace, workspace_bytes, flags, st);
-    case 8: return vbq::launch<8>(d, blob_dev, x_bf16, y, workspace, workspace_bytes, flags, st);
-    default: return vbq::launch<16>(d, blob_dev, x_bf16, y, workspace, workspace_bytes, flags, st);
-  }
+  return vbq_gemm_skinny_multi(1, &d, &blob_dev, x_bf16, B, &y, workspace, workspace_bytes, flags, stream);
 }
 
 int vbq_gemm_skinny(const vbq_desc* d, const void* blob_dev, const void* x_bf16, int B, float* y,
@@ -1157,7 +1270,7 @@ int static_scratch(void** out) {
 extern "C" int vbq_gemm_skinny_noalloc(const vbq_desc* d, const void* blob_dev, const void* x_bf16, int B,
                                        float* y, void* stream) {
   if (!d || !blob_dev || !x_bf16 || !y) return VBQ_ERR_NULL;
-  if (B != 1 && B != 2 && B != 4 && B != 8 && B != 16) return VBQ_ERR_BATCH;
+  if (!vbq::batch_ok(B)) return VBQ_ERR_BATCH;
   if (!vbq::desc_ok(d)) return VBQ_ERR_FORMAT;
   uint64_t need = 0;
   if (int st = vbq_workspace_size(d, B, &need)) return st;
@@ -1166,8 +1279,10 @@ extern "C" int vbq_gemm_skinny_noalloc(const vbq_desc* d, const void* blob_dev, 
   if (int st = vbq::static_scratch(&scratch)) return st;
   // The buffer keeps the previous call's contents: clear the arrival counters and the status word, which the
   // kernel needs at zero. The partial-sum area is always written before it is read.
+  vbq::Problem pr;
+  if (int st = vbq::make_problem(1, &d, pr)) return st;
   vbq::Plan pl;
-  if (!vbq::make_plan(*d, B, vbq::num_sms(), pl)) return VBQ_ERR_FORMAT;
+  if (!vbq::make_plan(pr, B, vbq::num_sms(), pl)) return VBQ_ERR_FORMAT;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(static_cast<unsigned char*>(scratch) + pl.counters_off, 0,
                       size_t(need - pl.counters_off), st) != cudaSuccess)

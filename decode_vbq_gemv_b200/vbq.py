@@ -66,6 +66,8 @@ def lib() -> ctypes.CDLL:
             "vbq_gemv": (i32, [dp, vp, vp, vp, vp, u64, vp]),
             "vbq_gemm_skinny": (i32, [dp, vp, vp, i32, vp, vp, u64, vp]),
             "vbq_gemm_skinny_ex": (i32, [dp, vp, vp, i32, vp, vp, u64, ctypes.c_uint, vp]),
+            "vbq_workspace_size_multi": (i32, [i32, vp, i32, ctypes.POINTER(u64)]),
+            "vbq_gemm_skinny_multi": (i32, [i32, vp, vp, vp, i32, vp, vp, u64, ctypes.c_uint, vp]),
             "vbq_gemm_skinny_noalloc": (i32, [dp, vp, vp, i32, vp, vp]),
         }
         for name, (res, args) in sig.items():
@@ -208,6 +210,36 @@ def vbq_gemm_skinny_ex(desc, blob_dev, x_bf16, B, y, workspace=None, flags=0, st
     _check(vbq_gemm_skinny_ex_status(desc, blob_dev, x_bf16, B, y, workspace, flags, stream), "vbq_gemm_skinny_ex")
 
 
+def _desc_array(descs):
+    arr = (ctypes.POINTER(vbq_desc) * max(1, len(descs)))()
+    for i, d in enumerate(descs):
+        arr[i] = ctypes.pointer(d)
+    return arr
+
+
+def vbq_workspace_size_multi(descs, B: int) -> int:
+    out = ctypes.c_uint64()
+    _check(lib().vbq_workspace_size_multi(len(descs), _desc_array(descs), B, ctypes.byref(out)),
+           "vbq_workspace_size_multi")
+    return int(out.value)
+
+
+def vbq_gemm_skinny_multi_status(descs, blobs_dev, x_bf16, B, ys, workspace=None, flags=0, stream=None) -> int:
+    n = len(descs)
+    blobs = (ctypes.c_void_p * max(1, n))(*[_dev_ptr(b) for b in blobs_dev])
+    yv = (ctypes.c_void_p * max(1, n))(*[_dev_ptr(y) for y in ys])
+    ws_ptr = _dev_ptr(workspace) if workspace is not None and workspace.numel() > 0 else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    return lib().vbq_gemm_skinny_multi(n, _desc_array(descs), blobs, _dev_ptr(x_bf16), B, yv, ws_ptr, ws_bytes,
+                                       flags, _stream_ptr(stream))
+
+
+def vbq_gemm_skinny_multi(descs, blobs_dev, x_bf16, B, ys, workspace=None, flags=0, stream=None) -> None:
+    """Fused launch over up to 4 matrices sharing x (same K and tile rows): ys[m][B, N_m] = X W_m^T."""
+    _check(vbq_gemm_skinny_multi_status(descs, blobs_dev, x_bf16, B, ys, workspace, flags, stream),
+           "vbq_gemm_skinny_multi")
+
+
 def vbq_gemm_skinny_noalloc_status(desc, blob_dev, x_bf16, B, y, stream=None) -> int:
     """Allocation-free variant: the library's fixed 16 MiB device buffer replaces the workspace."""
     return lib().vbq_gemm_skinny_noalloc(ctypes.byref(desc), _dev_ptr(blob_dev), _dev_ptr(x_bf16), B,
@@ -268,3 +300,35 @@ class DeviceMatrix:
             ws = self.workspaces[B] = self._alloc_ws(B)
         vbq_gemm_skinny(self.desc, self.blob, x2, B, out, ws, stream)
         return out.reshape(self.N) if squeeze else out
+
+
+class FusedMatrices:
+    """Up to 4 DeviceMatrix objects that share their input (same K and tile rows), run as one launch
+    (vbq_gemm_skinny_multi), plus a workspace per batch size for that launch."""
+
+    def __init__(self, mats, max_batch: int = 16):
+        import torch
+        self.mats = list(mats)
+        self.descs = [m.desc for m in self.mats]
+        self.K = self.mats[0].K
+        self.device = self.mats[0].device
+        self.workspaces = {}
+        for B in BATCHES:
+            if B <= max_batch:
+                n = vbq_workspace_size_multi(self.descs, B)
+                self.workspaces[B] = torch.zeros(max((n + 15) // 16, 1) * 16, dtype=torch.uint8, device=self.device)
+
+    @property
+    def nbytes(self) -> int:
+        return sum(m.nbytes for m in self.mats)
+
+    def matmul(self, x_bf16, outs=None, flags=0, stream=None):
+        """x_bf16: torch.bfloat16 [B, K] on the device. Returns the list of fp32 [B, N_m] outputs."""
+        import torch
+        x2 = x_bf16.reshape(-1, self.K)
+        B = x2.shape[0]
+        if outs is None:
+            outs = [torch.empty((B, m.N), dtype=torch.float32, device=self.device) for m in self.mats]
+        vbq_gemm_skinny_multi(self.descs, [m.blob for m in self.mats], x2, B, outs, self.workspaces[B], flags,
+                              stream)
+        return outs

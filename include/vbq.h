@@ -145,6 +145,26 @@ int vbq_gemm_skinny(const vbq_desc* d, const void* blob_dev, const void* x_bf16,
 int vbq_gemm_skinny_ex(const vbq_desc* d, const void* blob_dev, const void* x_bf16, int B, float* y,
                        void* workspace, uint64_t workspace_bytes, unsigned flags, void* stream);
 
+/* Several matrices that share their input, in one launch: fused projections such as q/k/v or gate/up, which the
+ * VBQ paper's deployment runs back to back on the same activation (the paper has no fused entry point; this
+ * one is a deployment aid). Up to 4 matrices, all with the same K (SHAPE otherwise) and the same tile rows R
+ * (TILE otherwise). Their records run as one sequence, so the launch's fixed costs are paid once and the
+ * small matrices share the SMs with the large ones.
+ * d[m], blob_dev[m]: descriptor and device blob of matrix m (blob 16-byte aligned).
+ * x_bf16: B*K bf16 values, row-major, 16-byte aligned, shared by all matrices.
+ * y[m]:   B*N_m fp32 values, row-major, 4-byte aligned; fully overwritten.
+ * workspace: vbq_workspace_size_multi(nmat, d, B) device bytes, 16-byte aligned, zeroed once by
+ *           vbq_workspace_init; not shared by calls that can run at the same time.
+ * flags: as vbq_gemm_skinny_ex.
+ * Each y[m] meets the tolerance of vbq_gemv and is bitwise identical from run to run. It need not be bitwise
+ * equal to a separate launch of matrix m, whose split among CTAs (and so whose summation order) differs.
+ * Errors: NULL, BATCH, FLAGS, SHAPE (nmat outside 1..4, or K differs), TILE (R differs), FORMAT, ALIGN,
+ * WORKSPACE, CUDA. */
+int vbq_workspace_size_multi(int nmat, const vbq_desc* const* d, int B, uint64_t* out_bytes);
+int vbq_gemm_skinny_multi(int nmat, const vbq_desc* const* d, const void* const* blob_dev, const void* x_bf16,
+                          int B, float* const* y, void* workspace, uint64_t workspace_bytes, unsigned flags,
+                          void* stream);
+
 /* Allocation-free variant of vbq_gemm_skinny (the VBQ paper has no counterpart; this is a deployment aid).
  *
  * Some callers cannot allocate device memory at all. Examples: plug-in hosts that give the library only pointers

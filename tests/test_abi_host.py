@@ -135,3 +135,31 @@ def test_device_entry_argument_checks_need_no_gpu():
     assert L.vbq_gemm_skinny_ex(dp, 16, 16, 3, 16, None, 0, vbq.VBQ_LAUNCH_OVERLAP, None) == vbq.VBQ_ERR_BATCH
     assert L.vbq_gemm_skinny_ex(dp, 8, 16, 1, 16, None, 0, vbq.VBQ_LAUNCH_OVERLAP, None) == vbq.VBQ_ERR_ALIGN
     assert L.vbq_gemm_skinny_ex(dp, None, 16, 1, 16, None, 0, 0, None) == vbq.VBQ_ERR_NULL
+
+
+def test_multi_entry_argument_checks_need_no_gpu():
+    """vbq_gemm_skinny_multi / vbq_workspace_size_multi reject bad matrix sets before any CUDA call."""
+    mk = lambda N, K, R, seed: vbq.vbq_pack(N, K, R, *logical(seed, N, K))[1]
+    a, b = mk(40, 128, 16, 1), mk(70, 128, 16, 2)
+    other_k, other_r = mk(40, 256, 16, 3), mk(40, 128, 32, 4)
+    size = vbq.lib().vbq_workspace_size_multi
+    out = ctypes.c_uint64()
+    arr = vbq._desc_array
+    assert size(2, arr([a, b]), 1, ctypes.byref(out)) == vbq.VBQ_OK
+    one = ctypes.c_uint64()
+    assert vbq.lib().vbq_workspace_size(ctypes.byref(a), 1, ctypes.byref(one)) == vbq.VBQ_OK
+    assert out.value >= one.value
+    assert size(0, arr([a]), 1, ctypes.byref(out)) == vbq.VBQ_ERR_SHAPE
+    assert size(5, arr([a, b, a, b, a]), 1, ctypes.byref(out)) == vbq.VBQ_ERR_SHAPE
+    assert size(2, arr([a, other_k]), 1, ctypes.byref(out)) == vbq.VBQ_ERR_SHAPE
+    assert size(2, arr([a, other_r]), 1, ctypes.byref(out)) == vbq.VBQ_ERR_TILE
+    assert size(2, arr([a, b]), 3, ctypes.byref(out)) == vbq.VBQ_ERR_BATCH
+    assert size(2, None, 1, ctypes.byref(out)) == vbq.VBQ_ERR_NULL
+    run = vbq.lib().vbq_gemm_skinny_multi
+    P = lambda *v: (ctypes.c_void_p * len(v))(*v)
+    assert run(2, arr([a, b]), P(16, 16), 16, 1, P(16, 16), None, 0, 0, None) == vbq.VBQ_ERR_WORKSPACE
+    assert run(2, arr([a, b]), P(16, None), 16, 1, P(16, 16), None, 0, 0, None) == vbq.VBQ_ERR_NULL
+    assert run(2, arr([a, b]), P(16, 16), 16, 1, P(16, 16), None, 0, 4, None) == vbq.VBQ_ERR_FLAGS
+    assert run(2, arr([a, b]), P(16, 24), 16, 1, P(16, 16), None, 0, 0, None) == vbq.VBQ_ERR_ALIGN
+    assert run(2, arr([a, b]), P(16, 16), 16, 1, P(16, 18), None, 0, 0, None) == vbq.VBQ_ERR_ALIGN
+    assert run(2, arr([a, other_r]), P(16, 16), 16, 1, P(16, 16), None, 0, 0, None) == vbq.VBQ_ERR_TILE

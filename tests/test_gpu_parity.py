@@ -239,3 +239,55 @@ def test_overlapped_launch_chain_matches_plain_launches():
     for m in (mq, mg):
         need = vbq.vbq_workspace_size(m.desc, 1)
         assert int(m.workspaces[1][need - 4:need].cpu().numpy().view(np.uint32)[0]) == 0
+
+
+def fused_status(fused, B):
+    ws = fused.workspaces[B]
+    need = vbq.vbq_workspace_size_multi(fused.descs, B)
+    return int(ws[need - 4:need].cpu().numpy().view(np.uint32)[0])
+
+
+@pytest.mark.parametrize("B", vbq.BATCHES)
+def test_fused_launch_ragged_matrices_all_batches(B):
+    """One vbq_gemm_skinny_multi launch over three matrices with the same K but different row counts (ragged
+    last tiles) and width mixes, element by element against the oracle."""
+    K = 256
+    spec = [(1030, "base"), (100, "flat"), (2100, "all8")]
+    ms = [logical(100 + i + B, N, K, DISTS[d]) for i, (N, d) in enumerate(spec)]
+    mats = [vbq.DeviceMatrix(vbq.vbq_pack(m.N, K, 64, m.widths, m.scales, m.codes)[0], dev(), max_batch=B)
+            for m in ms]
+    fused = vbq.FusedMatrices(mats, max_batch=B)
+    x = S.x_normal(B, K, np.random.default_rng(7 + B))
+    ys = fused.matmul(to_dev_x(x))
+    torch_sync()
+    assert fused_status(fused, B) == 0
+    for m, y in zip(ms, ys):
+        yref, bound = O.matvec(m.widths, m.scales, m.codes, x, NTH)
+        check(y.cpu().numpy().astype(np.float64), yref, bound, f"fused ragged N={m.N} B={B}")
+
+
+@pytest.mark.parametrize("B", [1, 4, 16])
+def test_fused_qkv_and_gate_up_full_size(B):
+    """The 9B-shaped fused projections (q/k/v share x; gate/up share x) in one launch each: sampled rows against
+    the oracle, and bitwise identical across two runs."""
+    g = np.random.default_rng(B)
+    for names in (("q", "k", "v"), ("gate", "up")):
+        ms = S.cfg4(names)
+        mats = [vbq.DeviceMatrix(vbq.vbq_pack(m.N, m.K, 256, m.widths, m.scales, m.codes)[0], dev(), max_batch=B)
+                for m in ms]
+        fused = vbq.FusedMatrices(mats, max_batch=B)
+        x = S.make_x(4, names[0], B, ms[0].K)
+        xd = to_dev_x(x)
+        y1 = [y.cpu().numpy().astype(np.float64) for y in fused.matmul(xd)]
+        y2 = [y.cpu().numpy().astype(np.float64) for y in fused.matmul(xd)]
+        assert fused_status(fused, B) == 0
+        for m, a, b in zip(ms, y1, y2):
+            assert np.array_equal(a, b), f"{m.name} B={B}: fused launch not deterministic"
+            rows = np.unique(np.concatenate([g.choice(m.N, 150, replace=False), [0, m.N - 1, 255, 256]]))
+            yref, bound = O.matvec(m.widths[rows], m.scales[rows], m.codes[rows], x, NTH)
+            check(a[:, rows], yref, bound, f"fused {'/'.join(names)}: {m.name} B={B}")
+
+
+def torch_sync():
+    import torch
+    torch.cuda.synchronize()
