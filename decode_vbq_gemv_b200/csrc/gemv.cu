@@ -329,16 +329,19 @@ __device__ __forceinline__ float dot_b8(const uint32_t (&w)[16], const float (&x
 
 // Batch 1, one width bucket: the warp's units of 32 items each (local unit u for u = first, first + TW, ...).
 // Lane = item; the item's result s * dot goes to res[item] (byte addresses: codes, scales, res for item 0 of the
-// bucket). The activations this width needs are loaded into registers once, from xcopy.
+// bucket). The activations this width needs are loaded into registers from xcopy, unless `load` is false
+// (they are already there).
 template <int KB>
 __device__ __forceinline__ void bucket_units(int n, int U, int first, int TW, int lane, uint32_t codes,
                                              uint32_t scales, uint32_t res, float (&xr)[64], uint32_t xcopy,
-                                             float sg) {
+                                             float sg, bool load) {
   if (first >= U) return;
+  if (load) {
 #pragma unroll
-  for (int q = 0; q < 16; ++q) {
-    const float4 f = lds128f(xcopy + 16 * q);
-    xr[4 * q] = f.x; xr[4 * q + 1] = f.y; xr[4 * q + 2] = f.z; xr[4 * q + 3] = f.w;
+    for (int q = 0; q < 16; ++q) {
+      const float4 f = lds128f(xcopy + 16 * q);
+      xr[4 * q] = f.x; xr[4 * q + 1] = f.y; xr[4 * q + 2] = f.z; xr[4 * q + 3] = f.w;
+    }
   }
   for (int u = first; u < U; u += TW) {
     const int jj = 32 * u + lane;
@@ -368,6 +371,7 @@ __device__ __forceinline__ void bucket_units(int n, int U, int first, int TW, in
 }
 // First local unit of a bucket for warp tw of TW, when the bucket's units follow `before` units of the record.
 __device__ __forceinline__ int first_unit(int tw, int before, int TW) {
+  if (TW == 1) return 0;
   const int r = (tw - before) % TW;
   return r < 0 ? r + TW : r;
 }
@@ -463,6 +467,18 @@ __device__ __forceinline__ void team_sync(int team, int TW) {
   }
 }
 
+// floor(a / b) for 0 <= a and 0 < b: through a float quotient when both are below 2^20 (then it is within one of
+// the exact quotient, and one correction step fixes it), else by integer division.
+__device__ __forceinline__ int div_floor(int a, int b) {
+  if ((a | b) < (1 << 20)) {
+    int q = __float2int_rz(__fdividef(float(a), float(b)));
+    if (q * b > a) --q;
+    else if ((q + 1) * b <= a) ++q;
+    return q;
+  }
+  return a / b;
+}
+
 // Closed-form split of the CTA's records [L, H) among its NT teams. The records fall into segments, one per row
 // tile. Every team computes its own share; nothing is exchanged.
 //  - At most NT segments: each segment gets one team plus a share of the NT - nseg spare teams proportional to its
@@ -473,8 +489,8 @@ struct TeamMap {
   int L, H, G, NT, n, tL, nseg;
   __device__ TeamMap(int L_, int H_, int G_, int NT_) : L(L_), H(H_), G(G_), NT(NT_), n(H_ - L_), tL(0), nseg(0) {
     if (n > 0) {
-      tL = L / G;
-      nseg = (H - 1) / G - tL + 1;
+      tL = div_floor(L, G);
+      nseg = div_floor(H - 1, G) - tL + 1;
     }
   }
   __device__ bool split() const { return nseg <= NT; }
@@ -484,7 +500,7 @@ struct TeamMap {
   __device__ int seg_team0(int i) const {
     if (i >= nseg) return NT;
     const unsigned num = unsigned(NT - nseg) * unsigned(seg_lo(i) - L);  // < 16 * n
-    return i + int(n < (1 << 27) ? num / unsigned(n) : (unsigned)((long long)(NT - nseg) * (seg_lo(i) - L) / n));
+    return i + (n < (1 << 27) ? div_floor(int(num), n) : int((long long)(NT - nseg) * (seg_lo(i) - L) / n));
   }
   // records [lo, hi) of team k; seg = its segment when that segment has several teams, else -1
   __device__ void team(int k, int& lo, int& hi, int& seg) const {
@@ -495,8 +511,8 @@ struct TeamMap {
       while (i + 1 < nseg && seg_team0(i + 1) <= k) ++i;
       const int f = seg_team0(i), cnt = seg_team0(i + 1) - f;
       const int s0 = seg_lo(i), len = seg_hi(i) - s0, q = k - f;
-      lo = s0 + q * len / cnt;
-      hi = s0 + (q + 1) * len / cnt;
+      lo = s0 + div_floor(q * len, cnt);
+      hi = s0 + div_floor((q + 1) * len, cnt);
       if (cnt >= 2) seg = i;
     } else {
       const int a = int((long long)k * nseg / NT), b = int((long long)(k + 1) * nseg / NT);
@@ -508,7 +524,7 @@ struct TeamMap {
 
 // ------------------------------------------------------------------------------------------------ kernel
 template <int B>
-__global__ void __launch_bounds__(Cfg<B>::kThreads, 1) vbq_kernel(Params p) {
+__global__ void __launch_bounds__(Cfg<B>::kThreads, 1) vbq_kernel(const __grid_constant__ Params params) {
   using C = Cfg<B>;
   extern __shared__ __align__(128) unsigned char smem[];
   __shared__ uint64_t bar_full[kMaxTeams * kMaxStages];
@@ -516,8 +532,16 @@ __global__ void __launch_bounds__(Cfg<B>::kThreads, 1) vbq_kernel(Params p) {
   __shared__ volatile int team_abort[kMaxTeams];
   __shared__ int team_live[kMaxTeams];  // team has records (its accumulators hold a partial sum)
   __shared__ int cta_flags[2];
+  __shared__ __align__(16) Params p;    // the launch parameters, read from here
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  // Copy the parameters to shared memory once, every word by its own thread: the first read of a parameter
+  // line misses the constant cache, and here those misses overlap instead of queuing up one after another
+  // wherever the parameters are first used.
+  static_assert(sizeof(Params) % 4 == 0 && sizeof(Params) / 4 <= Cfg<8>::kThreads, "parameter copy");
+  if (tid < int(sizeof(Params) / 4))
+    reinterpret_cast<uint32_t*>(&p)[tid] = reinterpret_cast<const uint32_t*>(&params)[tid];
+  __syncthreads();
   const int NT = p.NT, TW = p.TW, S = p.S, G = p.G, R = p.R;
   const int cta = blockIdx.x;
   const int L = rec_lo(p, cta), H = rec_lo(p, cta + 1);
@@ -536,25 +560,29 @@ __global__ void __launch_bounds__(Cfg<B>::kThreads, 1) vbq_kernel(Params p) {
   };
   auto kth_owner = [&](int t, int first, int k) -> int { return dense ? first + k : owner(p, t * G + k); };
 
-  // Sum of all owners' partial slots of tile t, in CTA order, into y (threads gtid of gthreads). Each thread
-  // issues the loads of up to 8 owners at once, then adds them in owner order.
-  auto reduce_tile = [&](int t, int gtid, int gthreads) {
-    int first;
-    const int owners = tile_owners(t, first);
-    const TileOut to = tile_out(p, t);
-    const int Rt = to.Rt;
-    for (int e = gtid; e < Rt * B; e += gthreads) {
+  // Sums of all owners' partial slots of the tiles in ts[0..nt), each in CTA order, into y (all threads; the
+  // elements of both tiles form one index space). Each thread has the loads of up to 16 owners in flight.
+  auto reduce_tiles = [&](int ta, int tb2, int ntiles) {  // tiles ta (and tb2 when ntiles == 2)
+    int fa, fb = 0;
+    const int oa = tile_owners(ta, fa), ob = ntiles > 1 ? tile_owners(tb2, fb) : 0;
+    const TileOut ya = tile_out(p, ta), yb = tile_out(p, ntiles > 1 ? tb2 : ta);
+    const int n0 = ya.Rt * B, ntot = n0 + (ntiles > 1 ? yb.Rt * B : 0);
+    for (int e2 = tid; e2 < ntot; e2 += C::kThreads) {
+      const bool second = e2 >= n0;
+      const int e = second ? e2 - n0 : e2, t = second ? tb2 : ta, first = second ? fb : fa;
+      const int owners = second ? ob : oa;
       float v = 0.f;
-      for (int k0 = 0; k0 < owners; k0 += 8) {
-        float part[8];
+      for (int o0 = 0; o0 < owners; o0 += 16) {
+        float part[16];
 #pragma unroll
-        for (int q = 0; q < 8; ++q)
-          part[q] = k0 + q < owners ? __ldcg(p.partial + size_t(kth_owner(t, first, k0 + q) + t) * R * B + e) : 0.f;
+        for (int q = 0; q < 16; ++q)
+          part[q] = o0 + q < owners ? __ldcg(p.partial + size_t(kth_owner(t, first, o0 + q) + t) * R * B + e) : 0.f;
 #pragma unroll
-        for (int q = 0; q < 8; ++q)
-          if (k0 + q < owners) v += part[q];
+        for (int q = 0; q < 16; ++q)
+          if (o0 + q < owners) v += part[q];
       }
       const int r = e / B, b = e - r * B;
+      const TileOut& to = second ? yb : ya;
       to.y[size_t(b) * to.ld + r] = v;
     }
   };
@@ -577,7 +605,7 @@ __global__ void __launch_bounds__(Cfg<B>::kThreads, 1) vbq_kernel(Params p) {
     uint32_t* mk = reinterpret_cast<uint32_t*>(wbase + wo.mk);      // [4][32] width masks per 32-row word
     int* pf = reinterpret_cast<int*>(wbase + wo.pf);                // [4][32] item index of the word's first row
     uint32_t* wd = reinterpret_cast<uint32_t*>(wbase + wo.wd);      // width-code words of the record
-    const int sl0 = tw * R / TW, sl1 = (tw + 1) * R / TW;           // this warp's rows in flushes and row passes
+    const int sl0 = div_floor(tw * R, TW), sl1 = div_floor((tw + 1) * R, TW);  // this warp's rows (flush, row pass)
     uint64_t* bars = bar_full + team * S;
 
     // -- the team's first warp streams the records: directory entries 32 at a time in its lanes, loaded first
@@ -772,13 +800,14 @@ __global__ void __launch_bounds__(Cfg<B>::kThreads, 1) vbq_kernel(Params p) {
           const uint32_t ra = smem_u32(tbase + p.res_off) + (TW > 1 ? 4 * R * (i & 1) : 0);
           const uint32_t sca = sa + rc.sc;
           const int U0 = rc.u0, U1 = rc.u1 - rc.u0, U2 = rc.u2 - rc.u1, U3 = rc.U - rc.u2;
-          bucket_units<1>(n0, U0, first_unit(tw, 0, TW), TW, lane, sa + rc.c0, sca, ra, xr, xa, sg);
-          bucket_units<2>(n1, U1, first_unit(tw, rc.u0, TW), TW, lane, sa + rc.c1, sca + 2 * n0, ra + 4 * n0, xr,
-                          xa + 256, sg);
-          bucket_units<4>(n2, U2, first_unit(tw, rc.u1, TW), TW, lane, sa + rc.c2, sca + 2 * (n0 + n1),
-                          ra + 4 * (n0 + n1), xr, xa + 512, sg);
+          // 1-bit and 8-bit units read the same (raw) activations, so they run back to back on one load.
+          bucket_units<1>(n0, U0, first_unit(tw, 0, TW), TW, lane, sa + rc.c0, sca, ra, xr, xa, sg, true);
           bucket_units<8>(n3, U3, first_unit(tw, rc.u2, TW), TW, lane, sa + rc.c3, sca + 2 * (n0 + n1 + n2),
-                          ra + 4 * (n0 + n1 + n2), xr, xa, sg);
+                          ra + 4 * (n0 + n1 + n2), xr, xa, sg, first_unit(tw, 0, TW) >= U0);
+          bucket_units<2>(n1, U1, first_unit(tw, rc.u0, TW), TW, lane, sa + rc.c1, sca + 2 * n0, ra + 4 * n0, xr,
+                          xa + 256, sg, true);
+          bucket_units<4>(n2, U2, first_unit(tw, rc.u1, TW), TW, lane, sa + rc.c2, sca + 2 * (n0 + n1),
+                          ra + 4 * (n0 + n1), xr, xa + 512, sg, true);
         } else if constexpr (B < 8) {
           // -- CUDA cores, B in {2, 4}: lane = group; activations of all batches broadcast from shared memory
           const float* xc = xv;
@@ -983,13 +1012,13 @@ __global__ void __launch_bounds__(Cfg<B>::kThreads, 1) vbq_kernel(Params p) {
     cta_flags[1] = part1 && a1 == unsigned(own1 - 1);
   }
   __syncthreads();
-  if (cta_flags[0]) {
-    reduce_tile(tfirst, tid, C::kThreads);
-    if (tid == 0) p.arrive[tfirst] = 0u;
-  }
-  if (cta_flags[1]) {
-    reduce_tile(tlast, tid, C::kThreads);
-    if (tid == 0) p.arrive[tlast] = 0u;
+  const int ntiles = cta_flags[0] + cta_flags[1];
+  if (ntiles == 0) return;
+  const int ta = cta_flags[0] ? tfirst : tlast;
+  reduce_tiles(ta, tlast, ntiles);
+  if (tid == 0) {
+    p.arrive[ta] = 0u;
+    if (ntiles > 1) p.arrive[tlast] = 0u;
   }
 }
 
