@@ -239,12 +239,24 @@ def run_vbq(args):
             g.yd = [torch.empty((B, m.N), dtype=torch.float32, device=dev) for m in ms]
             g.yh = [torch.empty((B, m.N), dtype=torch.float32).pin_memory() for m in ms]
             g.nbytes = sum(mt.nbytes for mt in g.mats) + B * ms[0].K * 2 + sum(B * m.N * 4 for m in ms)
+            g.h = None
+            g.x_from_device = False
             lin.append(g)
+        # The MLP runs as a chain: the fused gate/up launch writes h = silu(gate) * up (bf16) through its SwiGLU
+        # epilogue straight into the down projection's input.
+        names = [g.name for g in lin]
+        if not args.no_fuse and "gate_up" in names and "down" in names:
+            gu, dn = lin[names.index("gate_up")], lin[names.index("down")]
+            gu.h = dn.xd
+            gu.nbytes += dn.xd.numel() * 2
+            dn.x_from_device = True
         layers.append(lin)
     step_bytes = [sum(g.nbytes for g in lin) for lin in layers]
 
     def launch(g, st):
-        if g.fused is not None:
+        if g.h is not None:
+            g.fused.swiglu(g.xd, g.yd, g.h, flags, st)
+        elif g.fused is not None:
             g.fused.matmul(g.xd, g.yd, flags, st)
         else:
             mat = g.mats[0]
@@ -268,7 +280,8 @@ def run_vbq(args):
             g2 = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g2, stream=stream):
                 for g in lin:
-                    g.xd.copy_(g.xh, non_blocking=True)
+                    if not g.x_from_device:
+                        g.xd.copy_(g.xh, non_blocking=True)
                     launch(g, stream)
                     for yd, yh in zip(g.yd, g.yh):
                         yh.copy_(yd, non_blocking=True)
@@ -324,7 +337,7 @@ def run_vbq(args):
         per_shape[g.name] = {"us": us, "GBps": g.nbytes / (us / 1e6) / 1e9, "note": "same launch repeated (L2-warm)"}
 
     # End to end through host buffers.
-    h2d = sum(g.xh.numel() * 2 for g in layers[0])
+    h2d = sum(g.xh.numel() * 2 for g in layers[0] if not g.x_from_device)
     d2h = sum(sum(y.numel() * 4 for y in g.yh) for g in layers[0])
     e2e_ms = allreduce_max(timed(graphs_e2e), world)
     e2e_val = total_bytes * world / (e2e_ms / 1e3) / 1e9
@@ -341,7 +354,9 @@ def run_vbq(args):
             "config": {"workload": WORKLOAD, "batch": B, "tile_rows": R,
                        "launch": ("plain" if args.no_overlap else "programmatic dependent launch (VBQ_LAUNCH_OVERLAP)")
                                  + ("; one launch per linear" if args.no_fuse
-                                    else "; q/k/v and gate/up fused (vbq_gemm_skinny_multi), 4 launches per layer"),
+                                    else "; q/k/v fused (vbq_gemm_skinny_multi); gate/up fused with the SwiGLU "
+                                         "epilogue (vbq_gemm_swiglu) writing the down projection's input; "
+                                         "4 launches per layer"),
                        "weights": "seeded synthetic VBQ groups: P(1,2,4,8 bit) = (0.69,0.16,0.09,0.06), fp16 "
                                   "scales U(0.01,0.1), uniform codes; x ~ N(0,1) bf16",
                        "l2": f"inputs larger than L2: {args.copies} distinct layer copies in rotation "

@@ -5,10 +5,11 @@ The work runs in ``libvbq.so`` (C++ packer and hand-written sm_100a CUDA kernels
 """
 from .vbq import (BATCHES, DEFAULT_TILE_ROWS, VBQ_LAUNCH_OVERLAP, DeviceMatrix, FusedMatrices, VbqError, vbq_desc,
                   vbq_describe, vbq_gemm_skinny, vbq_gemm_skinny_ex, vbq_gemm_skinny_multi, vbq_gemm_skinny_noalloc,
+                  vbq_gemm_swiglu, vbq_workspace_size_swiglu,
                   vbq_gemv, vbq_pack, vbq_packed_size, vbq_strerror, vbq_unpack, vbq_version, vbq_workspace_init,
                   vbq_workspace_size, vbq_workspace_size_multi)
 
 __all__ = ["BATCHES", "DEFAULT_TILE_ROWS", "VBQ_LAUNCH_OVERLAP", "DeviceMatrix", "FusedMatrices", "VbqError",
            "vbq_desc", "vbq_describe", "vbq_gemm_skinny", "vbq_gemm_skinny_ex", "vbq_gemm_skinny_multi",
-           "vbq_gemm_skinny_noalloc", "vbq_gemv", "vbq_pack", "vbq_packed_size", "vbq_strerror", "vbq_unpack",
+           "vbq_gemm_skinny_noalloc", "vbq_gemm_swiglu", "vbq_workspace_size_swiglu", "vbq_gemv", "vbq_pack", "vbq_packed_size", "vbq_strerror", "vbq_unpack",
            "vbq_version", "vbq_workspace_init", "vbq_workspace_size", "vbq_workspace_size_multi"]

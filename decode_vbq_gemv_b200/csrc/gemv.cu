@@ -37,6 +37,7 @@ constexpr int kMaxTileRows = 1024;
 constexpr int kAStride = 72;            // bf16 per staged A row for ldmatrix (64 + 8 pad: conflict-free rows)
 constexpr int kMaxTeams = 16;
 constexpr int kMaxStages = 2;
+constexpr int kEpiChunk = 32;          // SwiGLU epilogue: tiles counted in per round
 constexpr int kSmemBudget = 227 * 1024 - 2048;  // dynamic shared memory; the rest is the static part
 constexpr unsigned long long kWaitNs = 2000000000ull;  // bounded mbarrier waits: 2 s
 constexpr unsigned kSuspendNs = 20000;                  // a waiting thread sleeps (no issue slots) up to 20 us per poll
@@ -62,6 +63,9 @@ struct Params {
   int rec_start[kMaxMats + 1];
   int tile_start[kMaxMats + 1];
   int nmat;
+  int swiglu;              // SwiGLU epilogue: matrices 0 (gate) and 1 (up) have the same rows; h = silu(y0) * y1
+  uint16_t* h;             // bf16 bits, [B][N_0] (SwiGLU only)
+  unsigned* pair;          // [T_0] row tiles of the gate/up pair already final; zero between calls (SwiGLU only)
   const uint16_t* x;       // bf16 bits, [B][K], shared by all matrices
   float* partial;          // [nCTA + T][R][B] partial sums of shared row tiles
   unsigned* arrive;        // [T] owners that have published their partial sums; zero between calls
@@ -532,6 +536,8 @@ __global__ void __launch_bounds__(Cfg<B>::kThreads, 1) vbq_kernel(const __grid_c
   __shared__ volatile int team_abort[kMaxTeams];
   __shared__ int team_live[kMaxTeams];  // team has records (its accumulators hold a partial sum)
   __shared__ int cta_flags[2];
+  __shared__ int epi_tiles[kEpiChunk];
+  __shared__ int epi_count;
   __shared__ __align__(16) Params p;    // the launch parameters, read from here
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -999,26 +1005,65 @@ __global__ void __launch_bounds__(Cfg<B>::kThreads, 1) vbq_kernel(const __grid_c
   const int tfirst = L / G, tlast = (H - 1) / G;
   const bool part0 = !(L <= tfirst * G && H >= (tfirst + 1) * G);
   const bool part1 = tlast != tfirst && !(L <= tlast * G && H >= (tlast + 1) * G);
-  if (!part0 && !part1) return;
-  __syncthreads();
-  if (tid == 0) {
-    // acq_rel at GPU scope: the release publishes the CTA's slot writes (ordered before it by the barrier), the
-    // acquire makes the other owners' slots visible to the reduction that follows. Both counters at once.
-    int first;
-    const int own0 = part0 ? tile_owners(tfirst, first) : 0, own1 = part1 ? tile_owners(tlast, first) : 0;
-    const unsigned a0 = part0 ? atom_add_acq_rel(&p.arrive[tfirst], 1u) : 0u;
-    const unsigned a1 = part1 ? atom_add_acq_rel(&p.arrive[tlast], 1u) : 0u;
-    cta_flags[0] = part0 && a0 == unsigned(own0 - 1);
-    cta_flags[1] = part1 && a1 == unsigned(own1 - 1);
+  if (part0 || part1) {
+    __syncthreads();
+    if (tid == 0) {
+      // acq_rel at GPU scope: the release publishes the CTA's slot writes (ordered before it by the barrier),
+      // the acquire makes the other owners' slots visible to the reduction that follows. Both counters at once.
+      int first;
+      const int own0 = part0 ? tile_owners(tfirst, first) : 0, own1 = part1 ? tile_owners(tlast, first) : 0;
+      const unsigned a0 = part0 ? atom_add_acq_rel(&p.arrive[tfirst], 1u) : 0u;
+      const unsigned a1 = part1 ? atom_add_acq_rel(&p.arrive[tlast], 1u) : 0u;
+      cta_flags[0] = part0 && a0 == unsigned(own0 - 1);
+      cta_flags[1] = part1 && a1 == unsigned(own1 - 1);
+    }
+    __syncthreads();
+    const int ntiles = cta_flags[0] + cta_flags[1];
+    if (ntiles > 0) {
+      const int ta = cta_flags[0] ? tfirst : tlast;
+      reduce_tiles(ta, tlast, ntiles);
+      if (tid == 0) {
+        p.arrive[ta] = 0u;
+        if (ntiles > 1) p.arrive[tlast] = 0u;
+      }
+    }
   }
-  __syncthreads();
-  const int ntiles = cta_flags[0] + cta_flags[1];
-  if (ntiles == 0) return;
-  const int ta = cta_flags[0] ? tfirst : tlast;
-  reduce_tiles(ta, tlast, ntiles);
-  if (tid == 0) {
-    p.arrive[ta] = 0u;
-    if (ntiles > 1) p.arrive[tlast] = 0u;
+  if (!p.swiglu) return;
+
+  // ================================================= SwiGLU epilogue: h = silu(gate) * up, bf16
+  // Matrix 0 is gate and matrix 1 is up, with the same rows and tiles, so gate tile tl and up tile tl cover the
+  // same rows. Whoever writes a tile's final y counts it in on the pair counter of tl; the second of the pair
+  // computes h for those rows from both (final) outputs. This CTA wrote the final y of its whole tiles and of
+  // the shared tiles it reduced.
+  const int tiles_here = tlast - tfirst + 1;
+  for (int c0 = 0; c0 < tiles_here; c0 += kEpiChunk) {
+    __syncthreads();  // this CTA's y writes (and the previous chunk's epilogue) are done
+    if (tid == 0) {
+      int n = 0;
+      for (int k = c0; k < min(tiles_here, c0 + kEpiChunk); ++k) {
+        const int t = tfirst + k;
+        const bool whole = L <= t * G && H >= (t + 1) * G;
+        const bool reduced = (t == tfirst && part0 && cta_flags[0]) || (t == tlast && part1 && cta_flags[1]);
+        if (!whole && !reduced) continue;
+        const int m = mat_of_tile(p, t), tl = m == 0 ? t : t - p.tile_start[1];
+        if (atom_add_acq_rel(&p.pair[tl], 1u) == 1u) epi_tiles[n++] = tl;
+      }
+      epi_count = n;
+    }
+    __syncthreads();
+    for (int k = 0; k < epi_count; ++k) {
+      const int tl = epi_tiles[k];
+      const int N = p.N[0], Rt = min(R, N - tl * R);
+      const size_t row0 = size_t(tl) * R;
+      for (int e = tid; e < Rt * B; e += C::kThreads) {
+        const int b = e / Rt, r = e - b * Rt;
+        const size_t at = size_t(b) * N + row0 + r;
+        const float g = __ldcg(p.y[0] + at), u = __ldcg(p.y[1] + at);
+        const float silu = g / (1.f + expf(-g));
+        p.h[at] = __bfloat16_as_ushort(__float2bfloat16_rn(silu * u));
+      }
+      if (tid == 0) p.pair[tl] = 0u;
+    }
   }
 }
 
@@ -1121,7 +1166,8 @@ inline bool make_plan_t(const Problem& pr, int sms, Plan& pl) {
   if (best_key < 0) return false;
   const uint64_t slots = uint64_t(pl.grid) + uint64_t(pr.T);
   pl.counters_off = slots * uint64_t(R) * B * 4;
-  pl.ws_bytes = (pl.counters_off + uint64_t(pr.T) * 4 + 4 + 15) / 16 * 16;
+  // counters: arrivals per tile, then SwiGLU pair counters per tile; then the status word
+  pl.ws_bytes = (pl.counters_off + uint64_t(pr.T) * 8 + 4 + 15) / 16 * 16;
   pl.status_off = pl.ws_bytes - 4;
   return true;
 }
@@ -1138,7 +1184,7 @@ inline bool make_plan(const Problem& pr, int B, int sms, Plan& pl) {
 
 template <int B>
 int launch(const Problem& pr, const void* const* blobs, const void* x, float* const* ys, void* ws, uint64_t ws_bytes,
-           unsigned flags, cudaStream_t stream) {
+           unsigned flags, cudaStream_t stream, uint16_t* h = nullptr) {
   Plan pl;
   if (!make_plan_t<B>(pr, num_sms(), pl)) return VBQ_ERR_FORMAT;
   if (!ws || (reinterpret_cast<uintptr_t>(ws) & 15) || ws_bytes < pl.ws_bytes) return VBQ_ERR_WORKSPACE;
@@ -1165,6 +1211,9 @@ int launch(const Problem& pr, const void* const* blobs, const void* x, float* co
   uint8_t* w = static_cast<uint8_t*>(ws);
   p.partial = reinterpret_cast<float*>(w);
   p.arrive = reinterpret_cast<unsigned*>(w + pl.counters_off);
+  p.pair = p.arrive + tiles;
+  p.swiglu = h != nullptr;
+  p.h = h;
   p.status = reinterpret_cast<unsigned*>(w + pl.status_off);
   p.K = pr.K; p.G = pr.G; p.R = pr.R; p.T = tiles;
   p.nrec = recs;
@@ -1250,6 +1299,39 @@ int vbq_gemm_skinny_multi(int nmat, const vbq_desc* const* d, const void* const*
     case 4: return vbq::launch<4>(pr, blob_dev, x_bf16, y, workspace, workspace_bytes, flags, st);
     case 8: return vbq::launch<8>(pr, blob_dev, x_bf16, y, workspace, workspace_bytes, flags, st);
     default: return vbq::launch<16>(pr, blob_dev, x_bf16, y, workspace, workspace_bytes, flags, st);
+  }
+}
+
+int vbq_workspace_size_swiglu(const vbq_desc* gate, const vbq_desc* up, int B, uint64_t* out_bytes) {
+  if (!gate || !up) return VBQ_ERR_NULL;
+  if (gate->N != up->N) return VBQ_ERR_SHAPE;
+  const vbq_desc* d[2] = {gate, up};
+  return vbq_workspace_size_multi(2, d, B, out_bytes);
+}
+
+int vbq_gemm_swiglu(const vbq_desc* gate, const vbq_desc* up, const void* blob_gate, const void* blob_up,
+                    const void* x_bf16, int B, float* y_gate, float* y_up, void* h_bf16, void* workspace,
+                    uint64_t workspace_bytes, unsigned flags, void* stream) {
+  if (!gate || !up || !blob_gate || !blob_up || !x_bf16 || !y_gate || !y_up || !h_bf16) return VBQ_ERR_NULL;
+  if (!vbq::batch_ok(B)) return VBQ_ERR_BATCH;
+  if (flags & ~unsigned(VBQ_LAUNCH_OVERLAP)) return VBQ_ERR_FLAGS;
+  const vbq_desc* d[2] = {gate, up};
+  vbq::Problem pr;
+  if (int st = vbq::make_problem(2, d, pr)) return st;
+  if (gate->N != up->N) return VBQ_ERR_SHAPE;
+  const void* blobs[2] = {blob_gate, blob_up};
+  float* ys[2] = {y_gate, y_up};
+  if ((reinterpret_cast<uintptr_t>(x_bf16) & 15) || (reinterpret_cast<uintptr_t>(h_bf16) & 1)) return VBQ_ERR_ALIGN;
+  for (int m = 0; m < 2; ++m)
+    if ((reinterpret_cast<uintptr_t>(blobs[m]) & 15) || (reinterpret_cast<uintptr_t>(ys[m]) & 3)) return VBQ_ERR_ALIGN;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint16_t* h = static_cast<uint16_t*>(h_bf16);
+  switch (B) {
+    case 1: return vbq::launch<1>(pr, blobs, x_bf16, ys, workspace, workspace_bytes, flags, st, h);
+    case 2: return vbq::launch<2>(pr, blobs, x_bf16, ys, workspace, workspace_bytes, flags, st, h);
+    case 4: return vbq::launch<4>(pr, blobs, x_bf16, ys, workspace, workspace_bytes, flags, st, h);
+    case 8: return vbq::launch<8>(pr, blobs, x_bf16, ys, workspace, workspace_bytes, flags, st, h);
+    default: return vbq::launch<16>(pr, blobs, x_bf16, ys, workspace, workspace_bytes, flags, st, h);
   }
 }
 

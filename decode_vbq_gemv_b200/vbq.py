@@ -68,6 +68,8 @@ def lib() -> ctypes.CDLL:
             "vbq_gemm_skinny_ex": (i32, [dp, vp, vp, i32, vp, vp, u64, ctypes.c_uint, vp]),
             "vbq_workspace_size_multi": (i32, [i32, vp, i32, ctypes.POINTER(u64)]),
             "vbq_gemm_skinny_multi": (i32, [i32, vp, vp, vp, i32, vp, vp, u64, ctypes.c_uint, vp]),
+            "vbq_workspace_size_swiglu": (i32, [dp, dp, i32, ctypes.POINTER(u64)]),
+            "vbq_gemm_swiglu": (i32, [dp, dp, vp, vp, vp, i32, vp, vp, vp, vp, u64, ctypes.c_uint, vp]),
             "vbq_gemm_skinny_noalloc": (i32, [dp, vp, vp, i32, vp, vp]),
         }
         for name, (res, args) in sig.items():
@@ -240,6 +242,29 @@ def vbq_gemm_skinny_multi(descs, blobs_dev, x_bf16, B, ys, workspace=None, flags
            "vbq_gemm_skinny_multi")
 
 
+def vbq_workspace_size_swiglu(gate: vbq_desc, up: vbq_desc, B: int) -> int:
+    out = ctypes.c_uint64()
+    _check(lib().vbq_workspace_size_swiglu(ctypes.byref(gate), ctypes.byref(up), B, ctypes.byref(out)),
+           "vbq_workspace_size_swiglu")
+    return int(out.value)
+
+
+def vbq_gemm_swiglu_status(gate, up, blob_gate, blob_up, x_bf16, B, y_gate, y_up, h_bf16, workspace=None,
+                           flags=0, stream=None) -> int:
+    ws_ptr = _dev_ptr(workspace) if workspace is not None and workspace.numel() > 0 else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    return lib().vbq_gemm_swiglu(ctypes.byref(gate), ctypes.byref(up), _dev_ptr(blob_gate), _dev_ptr(blob_up),
+                                 _dev_ptr(x_bf16), B, _dev_ptr(y_gate), _dev_ptr(y_up), _dev_ptr(h_bf16), ws_ptr,
+                                 ws_bytes, flags, _stream_ptr(stream))
+
+
+def vbq_gemm_swiglu(gate, up, blob_gate, blob_up, x_bf16, B, y_gate, y_up, h_bf16, workspace=None, flags=0,
+                    stream=None) -> None:
+    """Gate/up projections with the fused SwiGLU epilogue: h = silu(X W_gate^T) * (X W_up^T), bf16."""
+    _check(vbq_gemm_swiglu_status(gate, up, blob_gate, blob_up, x_bf16, B, y_gate, y_up, h_bf16, workspace,
+                                  flags, stream), "vbq_gemm_swiglu")
+
+
 def vbq_gemm_skinny_noalloc_status(desc, blob_dev, x_bf16, B, y, stream=None) -> int:
     """Allocation-free variant: the library's fixed 16 MiB device buffer replaces the workspace."""
     return lib().vbq_gemm_skinny_noalloc(ctypes.byref(desc), _dev_ptr(blob_dev), _dev_ptr(x_bf16), B,
@@ -321,6 +346,20 @@ class FusedMatrices:
     @property
     def nbytes(self) -> int:
         return sum(m.nbytes for m in self.mats)
+
+    def swiglu(self, x_bf16, outs=None, h=None, flags=0, stream=None):
+        """Two matrices (gate, up) with the fused SwiGLU epilogue. Returns (y_gate, y_up, h bf16 [B, N])."""
+        import torch
+        x2 = x_bf16.reshape(-1, self.K)
+        B = x2.shape[0]
+        gate, up = self.mats
+        if outs is None:
+            outs = [torch.empty((B, m.N), dtype=torch.float32, device=self.device) for m in self.mats]
+        if h is None:
+            h = torch.empty((B, gate.N), dtype=torch.bfloat16, device=self.device)
+        vbq_gemm_swiglu(gate.desc, up.desc, gate.blob, up.blob, x2, B, outs[0], outs[1], h, self.workspaces[B],
+                        flags, stream)
+        return outs[0], outs[1], h
 
     def matmul(self, x_bf16, outs=None, flags=0, stream=None):
         """x_bf16: torch.bfloat16 [B, K] on the device. Returns the list of fp32 [B, N_m] outputs."""

@@ -165,6 +165,21 @@ int vbq_gemm_skinny_multi(int nmat, const vbq_desc* const* d, const void* const*
                           int B, float* const* y, void* workspace, uint64_t workspace_bytes, unsigned flags,
                           void* stream);
 
+/* Gated MLP input projections with the SwiGLU epilogue fused in (VBQ paper, section 4: the models are
+ * LLaMA-style decoders with SwiGLU MLPs; the paper has no fused entry point, this is a deployment aid).
+ * One launch computes y_gate = X W_gate^T and y_up = X W_up^T as vbq_gemm_skinny_multi does, and
+ * h = silu(y_gate) * y_up with silu(g) = g / (1 + e^-g), rounded to bf16 (round to nearest even): the input
+ * of the down projection. gate and up must have the same N (SHAPE), K (SHAPE) and tile rows (TILE).
+ * h_bf16: B*N bf16 values, row-major, 2-byte aligned; y_gate, y_up as in vbq_gemm_skinny (also written).
+ * workspace: vbq_workspace_size_swiglu(gate, up, B) bytes, zeroed once by vbq_workspace_init.
+ * h meets |h - h_exact| <= 2^-8 |h_exact| + 1.1 |u| tol_g + |silu(g)| tol_u + tol_g tol_u + 1e-6, where
+ * tol_g, tol_u are the vbq_gemv tolerances of y_gate, y_up; every output is bitwise identical from run to run.
+ * Errors: as vbq_gemm_skinny_multi. */
+int vbq_workspace_size_swiglu(const vbq_desc* gate, const vbq_desc* up, int B, uint64_t* out_bytes);
+int vbq_gemm_swiglu(const vbq_desc* gate, const vbq_desc* up, const void* blob_gate, const void* blob_up,
+                    const void* x_bf16, int B, float* y_gate, float* y_up, void* h_bf16, void* workspace,
+                    uint64_t workspace_bytes, unsigned flags, void* stream);
+
 /* Allocation-free variant of vbq_gemm_skinny (the VBQ paper has no counterpart; this is a deployment aid).
  *
  * Some callers cannot allocate device memory at all. Examples: plug-in hosts that give the library only pointers

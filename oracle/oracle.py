@@ -180,3 +180,27 @@ def dequant(widths, scales, codes) -> np.ndarray:
 def within_tolerance(y_test: np.ndarray, y_ref: np.ndarray, bound: np.ndarray) -> np.ndarray:
     """Per-element parity bar of this project: |y - y_ref| <= 1e-3 * sum|w||x| + 1e-6."""
     return np.abs(np.asarray(y_test, np.float64) - y_ref) <= 1e-3 * bound + 1e-6
+
+
+def silu(g) -> np.ndarray:
+    """SiLU (swish) in fp64: g * logistic(g) = g / (1 + e^-g). The gate nonlinearity of the SwiGLU MLP that the
+    VBQ paper's decoders use (section 4); plain definition, written as g * e^g / (1 + e^g) for negative g so that
+    e^-g cannot overflow."""
+    g = np.asarray(g, np.float64)
+    e = np.exp(-np.abs(g))
+    return np.where(g >= 0, g / (1.0 + e), g * e / (1.0 + e))
+
+
+def swiglu(y_gate, y_up) -> np.ndarray:
+    """h = silu(gate) * up, elementwise, fp64."""
+    return silu(y_gate) * np.asarray(y_up, np.float64)
+
+
+def swiglu_bound(y_gate, y_up, bound_gate, bound_up) -> np.ndarray:
+    """Per-element bar for h computed from fp32 outputs that meet `within_tolerance` and rounded to bf16:
+    2^-8 |h| (bf16 rounding, with margin) + 1.1 |u| tol_g + |silu(g)| tol_u + tol_g tol_u + 1e-6, where
+    tol = 1e-3 * sum|w||x| + 1e-6 and 1.1 bounds |silu'|."""
+    g, u = np.asarray(y_gate, np.float64), np.asarray(y_up, np.float64)
+    tg, tu = 1e-3 * np.asarray(bound_gate) + 1e-6, 1e-3 * np.asarray(bound_up) + 1e-6
+    h = swiglu(g, u)
+    return 2.0 ** -8 * np.abs(h) + 1.1 * np.abs(u) * tg + np.abs(silu(g)) * tu + tg * tu + 1e-6

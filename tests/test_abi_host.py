@@ -163,3 +163,25 @@ def test_multi_entry_argument_checks_need_no_gpu():
     assert run(2, arr([a, b]), P(16, 24), 16, 1, P(16, 16), None, 0, 0, None) == vbq.VBQ_ERR_ALIGN
     assert run(2, arr([a, b]), P(16, 16), 16, 1, P(16, 18), None, 0, 0, None) == vbq.VBQ_ERR_ALIGN
     assert run(2, arr([a, other_r]), P(16, 16), 16, 1, P(16, 16), None, 0, 0, None) == vbq.VBQ_ERR_TILE
+
+
+def test_swiglu_entry_argument_checks_need_no_gpu():
+    """vbq_gemm_swiglu rejects mismatched gate/up shapes, odd h and unknown flags before any CUDA call."""
+    mk = lambda N, K, R, seed: vbq.vbq_pack(N, K, R, *logical(seed, N, K))[1]
+    g, u = mk(40, 128, 16, 1), mk(40, 128, 16, 2)
+    other_n, other_r = mk(48, 128, 16, 3), mk(40, 128, 32, 4)
+    L = vbq.lib()
+    r = ctypes.byref
+    out = ctypes.c_uint64()
+    assert L.vbq_workspace_size_swiglu(r(g), r(u), 1, r(out)) == vbq.VBQ_OK
+    assert out.value == vbq.vbq_workspace_size_multi([g, u], 1)
+    assert L.vbq_workspace_size_swiglu(r(g), r(other_n), 1, r(out)) == vbq.VBQ_ERR_SHAPE
+    assert L.vbq_workspace_size_swiglu(r(g), r(other_r), 1, r(out)) == vbq.VBQ_ERR_TILE
+    run = L.vbq_gemm_swiglu
+    assert run(r(g), r(u), 16, 16, 16, 1, 16, 16, None, None, 0, 0, None) == vbq.VBQ_ERR_NULL
+    assert run(r(g), r(u), 16, 16, 16, 3, 16, 16, 16, None, 0, 0, None) == vbq.VBQ_ERR_BATCH
+    assert run(r(g), r(u), 16, 16, 16, 1, 16, 16, 16, None, 0, 2, None) == vbq.VBQ_ERR_FLAGS
+    assert run(r(g), r(other_n), 16, 16, 16, 1, 16, 16, 16, None, 0, 0, None) == vbq.VBQ_ERR_SHAPE
+    assert run(r(g), r(other_r), 16, 16, 16, 1, 16, 16, 16, None, 0, 0, None) == vbq.VBQ_ERR_TILE
+    assert run(r(g), r(u), 16, 16, 16, 1, 16, 16, 17, None, 0, 0, None) == vbq.VBQ_ERR_ALIGN
+    assert run(r(g), r(u), 16, 16, 16, 1, 16, 16, 16, None, 0, 0, None) == vbq.VBQ_ERR_WORKSPACE

@@ -291,3 +291,101 @@ def test_fused_qkv_and_gate_up_full_size(B):
 def torch_sync():
     import torch
     torch.cuda.synchronize()
+
+
+def bf16_to_f64(t):
+    import torch
+    return t.float().cpu().numpy().astype(np.float64)
+
+
+def check_swiglu(h, g_ref, u_ref, bg, bu, what):
+    want = O.swiglu(g_ref, u_ref)
+    bar = O.swiglu_bound(g_ref, u_ref, bg, bu)
+    ok = np.abs(h - want) <= bar
+    if not ok.all():
+        i = tuple(np.argwhere(~ok)[0])
+        raise AssertionError(f"{what}: {int((~ok).sum())} of {ok.size} h out of bar; first {i}: got {h[i]!r} "
+                             f"want {want[i]!r} bar {bar[i]!r}")
+
+
+@pytest.mark.parametrize("B", vbq.BATCHES)
+def test_swiglu_epilogue_ragged_all_batches(B):
+    """vbq_gemm_swiglu on a ragged gate/up pair (1030 rows, 64-row tiles): y_gate and y_up against the oracle,
+    and the fused h = silu(y_gate) * y_up (bf16) against the oracle's fp64 h within its bar."""
+    N, K = 1030, 256
+    g_m = logical(200 + B, N, K, DISTS["base"])
+    u_m = logical(300 + B, N, K, DISTS["flat"])
+    mats = [vbq.DeviceMatrix(vbq.vbq_pack(m.N, K, 64, m.widths, m.scales, m.codes)[0], dev(), max_batch=B)
+            for m in (g_m, u_m)]
+    fused = vbq.FusedMatrices(mats, max_batch=B)
+    x = S.x_normal(B, K, np.random.default_rng(11 + B))
+    yg, yu, h = fused.swiglu(to_dev_x(x))
+    torch_sync()
+    assert fused_status(fused, B) == 0
+    g_ref, bg = O.matvec(g_m.widths, g_m.scales, g_m.codes, x, NTH)
+    u_ref, bu = O.matvec(u_m.widths, u_m.scales, u_m.codes, x, NTH)
+    check(yg.cpu().numpy().astype(np.float64), g_ref, bg, f"swiglu gate B={B}")
+    check(yu.cpu().numpy().astype(np.float64), u_ref, bu, f"swiglu up B={B}")
+    check_swiglu(bf16_to_f64(h), g_ref, u_ref, bg, bu, f"swiglu h B={B}")
+
+
+@pytest.mark.parametrize("B", [1, 4, 16])
+def test_swiglu_epilogue_full_size(B):
+    """The 9B-shaped gate/up pair (14336x4096 each) with the fused epilogue: sampled rows of y and h against the
+    oracle; h bitwise identical across runs and equal to silu(y_gate) * y_up from the same launch, rounded to
+    bf16."""
+    import torch
+    ms = S.cfg4(("gate", "up"))
+    mats = [vbq.DeviceMatrix(vbq.vbq_pack(m.N, m.K, 256, m.widths, m.scales, m.codes)[0], dev(), max_batch=B)
+            for m in ms]
+    fused = vbq.FusedMatrices(mats, max_batch=B)
+    x = S.make_x(4, "gate", B, ms[0].K)
+    xd = to_dev_x(x)
+    yg, yu, h1 = fused.swiglu(xd)
+    h1 = h1.clone()
+    _, _, h2 = fused.swiglu(xd)
+    torch_sync()
+    assert fused_status(fused, B) == 0
+    assert torch.equal(h1, h2), "SwiGLU output differs between runs"
+    # h is silu of this launch's own y_gate times its y_up, rounded once to bf16
+    g32, u32 = yg.double(), yu.double()
+    h_from_y = (g32 / (1 + torch.exp(-g32)) * u32).float().to(torch.bfloat16)
+    assert (h1.float() - h_from_y.float()).abs().max().item() <= 2 ** -7 * h_from_y.float().abs().max().item()
+    rows = np.unique(np.concatenate([np.random.default_rng(B).choice(ms[0].N, 150, replace=False),
+                                     [0, 255, 256, ms[0].N - 1]]))
+    g_m, u_m = ms
+    g_ref, bg = O.matvec(g_m.widths[rows], g_m.scales[rows], g_m.codes[rows], x, NTH)
+    u_ref, bu = O.matvec(u_m.widths[rows], u_m.scales[rows], u_m.codes[rows], x, NTH)
+    check_swiglu(bf16_to_f64(h1)[:, rows], g_ref, u_ref, bg, bu, f"swiglu full-size h B={B}")
+
+
+@pytest.mark.parametrize("B", [1, 4, 16])
+def test_recipe_workload_layers_and_head(B):
+    """The fixed-recipe workload (uniform width per projection; first-block MLP 4-bit, the rest 2-bit; tiered
+    head at 1.18 mean bits) through the fused launches: sampled rows against the oracle."""
+    g = np.random.default_rng(50 + B)
+
+    def sampled(m):
+        return np.unique(np.concatenate([g.choice(m.N, 100, replace=False), [0, 255, 256, m.N - 1]]))
+
+    for layer in (0, 1):
+        ms = {m.name: m for m in S.cfg6_recipe_layer(layer)}
+        for names in (("q", "k", "v"), ("gate", "up")):
+            group = [ms[n] for n in names]
+            mats = [vbq.DeviceMatrix(vbq.vbq_pack(m.N, m.K, 256, m.widths, m.scales, m.codes)[0], dev(),
+                                     max_batch=B) for m in group]
+            fused = vbq.FusedMatrices(mats, max_batch=B)
+            x = S.make_x(6, names[0], B, group[0].K, layer=layer)
+            ys = fused.matmul(to_dev_x(x))
+            torch_sync()
+            assert fused_status(fused, B) == 0
+            for m, y in zip(group, ys):
+                rows = sampled(m)
+                yref, bound = O.matvec(m.widths[rows], m.scales[rows], m.codes[rows], x, NTH)
+                check(y.cpu().numpy().astype(np.float64)[:, rows], yref, bound, f"recipe layer {layer} {m.name} B={B}")
+    head = S.cfg6_recipe_head()
+    x = S.make_x(6, "head", B, head.K)
+    y, _ = gpu_y(head, x, 256)
+    rows = np.unique(np.concatenate([np.arange(0, 4000, 9), g.choice(head.N, 200), [head.N - 1]]))
+    yref, bound = O.matvec(head.widths[rows], head.scales[rows], head.codes[rows], x, NTH)
+    check(y[:, rows], yref, bound, f"recipe head B={B}")

@@ -292,3 +292,41 @@ def test_power_of_two_scale_invariance():
     assert np.array_equal(f16(s2), 2 * f16(s))
     y2, a2 = O.matvec(w, s2, c, x)
     assert np.array_equal(y2, 2 * y1) and np.array_equal(a2, 2 * a1)
+
+
+def test_silu_pins_and_identities():
+    """SiLU, the gate nonlinearity of the SwiGLU epilogue, pinned to textbook values of the logistic function
+    sigma(t) = 1 / (1 + e^-t): sigma(1) = 0.7310585786300049, sigma(-1) = 0.2689414213699951."""
+    assert O.silu(0.0) == 0.0
+    assert abs(O.silu(1.0) - 0.7310585786300049) < 1e-15
+    assert abs(O.silu(-1.0) - (-0.2689414213699951)) < 1e-15
+    assert abs(O.silu(40.0) - 40.0) < 1e-12                      # sigma(40) = 1 - 4e-18
+    assert -1e-15 < O.silu(-40.0) < 0.0                           # -40 e^-40 / (1 + e^-40)
+    assert np.isfinite(O.silu(-1000.0)) and O.silu(-1000.0) <= 0.0   # no overflow for very negative inputs
+    t = np.linspace(-30, 30, 601)
+    assert np.allclose(O.silu(t) - O.silu(-t), t, rtol=0, atol=1e-12)   # sigma(t) + sigma(-t) = 1
+    assert np.array_equal(O.swiglu(t, 2 * np.ones_like(t)), 2 * O.silu(t))
+
+
+def test_swiglu_bound_covers_bf16_rounding():
+    """The h bar admits the bf16 rounding of an exact h (half an ulp is at most 2^-9 relative)."""
+    rng = np.random.default_rng(0)
+    g, u = rng.normal(0, 3, 1000), rng.normal(0, 3, 1000)
+    h = O.swiglu(g, u)
+    h_bf16 = (h.astype(np.float32).view(np.uint32) + 0x7FFF + ((h.astype(np.float32).view(np.uint32) >> 16) & 1)) \
+        & 0xFFFF0000
+    hq = h_bf16.astype(np.uint32).view(np.float32).astype(np.float64)
+    bound = O.swiglu_bound(g, u, np.zeros_like(g), np.zeros_like(u))
+    assert np.all(np.abs(hq - h) <= bound)
+
+
+def test_recipe_workload_shape():
+    """The fixed-recipe workload has the widths the recipe fixes: 2-bit projections, a 4-bit first-block MLP, and
+    a head whose tiers give 1.18 mean bits with rows in descending frequency order."""
+    l0, l1 = S.cfg6_recipe_layer(0), S.cfg6_recipe_layer(1)
+    assert all(np.all(m.widths == (4 if m.name in ("gate", "up", "down") else 2)) for m in l0)
+    assert all(np.all(m.widths == 2) for m in l1)
+    w = S.widths_head_tiered(32000, 64)
+    assert abs(w.mean() - 1.18) < 1e-3
+    assert np.all(np.diff(w[:, 0].astype(int)) <= 0)         # widths never increase down the frequency order
+    assert (w[:, 0] == 8).sum() == 160 and (w[:, 0] == 4).sum() == 480 and (w[:, 0] == 2).sum() == 3200

@@ -156,3 +156,37 @@ def cfg5_layer(layer: int):
 def cfg5_head(N: int = 32000, K: int = 4096):
     """LM head 4096 -> 32000 at about 1.09 mean bits."""
     return make_matrix(5, "head", N, K, widths=widths_head(N, K // 64, rng(5, 0, "head", "widths")))
+
+
+# Fixed deployment recipe (VBQ paper, section 3.4): one width per projection instead of per group. The first
+# block's MLP stays at 4 bits, every other projection is 2-bit, and the language-model head is tiered by token
+# frequency: the top 0.5% of rows (in descending frequency order) 8-bit, the next 1.5% 4-bit, the next 10%
+# 2-bit and the remaining 88% 1-bit (mean 0.005*8 + 0.015*4 + 0.10*2 + 0.88*1 = 1.18 bits).
+RECIPE_HEAD_TIERS = ((0.005, 8), (0.015, 4), (0.10, 2), (0.88, 1))
+
+
+def widths_head_tiered(N: int, G: int) -> np.ndarray:
+    """Recipe head widths: row tiers in descending token-frequency order (RECIPE_HEAD_TIERS)."""
+    w = np.ones((N, G), np.uint8)
+    start = 0
+    for frac, k in RECIPE_HEAD_TIERS[:-1]:
+        stop = min(N, start + int(round(frac * N)))
+        w[start:stop] = k
+        start = stop
+    return w
+
+
+def cfg6_recipe_layer(layer: int):
+    """One 9B-shaped layer under the fixed recipe: MLP (gate, up, down) 4-bit in layer 0, 2-bit elsewhere;
+    attention projections 2-bit."""
+    out = []
+    for n in ("q", "k", "v", "o", "gate", "up", "down"):
+        N, K = CFG4_SHAPES[n]
+        k = 4 if (layer == 0 and n in ("gate", "up", "down")) else 2
+        out.append(make_matrix(6, n, N, K, widths=widths_uniform(N, K // 64, k), layer=layer))
+    return out
+
+
+def cfg6_recipe_head(N: int = 32000, K: int = 4096):
+    """LM head 4096 -> 32000 under the recipe's frequency tiers (mean 1.18 bits)."""
+    return make_matrix(6, "head", N, K, widths=widths_head_tiered(N, K // 64))
