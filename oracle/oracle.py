@@ -24,7 +24,8 @@ _LIB_PATH = os.path.join(_BUILD, "libvbq_oracle.so")
 OK = 0
 ERR_NULL, ERR_SHAPE, ERR_WIDTH, ERR_CODE_RANGE, ERR_BUFFER_TOO_SMALL = -1, -2, -3, -4, -5
 ERR_BAD_MAGIC, ERR_VERSION, ERR_CRC, ERR_BATCH, ERR_ALIGN, ERR_CUDA = -6, -7, -8, -9, -10, -11
-ERR_TILE, ERR_FORMAT = -12, -13
+ERR_TILE, ERR_FORMAT, ERR_FLAGS, ERR_VALUE = -12, -13, -16, -17
+FLAG_GRID_SYMMETRIC = 1   # header flag bit 0: widths >= 2 on the paper's Eq. 1 integer grid
 
 
 class OracleError(RuntimeError):
@@ -59,13 +60,18 @@ def lib():
         L.vbqo_bf16_to_double.argtypes = [ctypes.c_uint16]
         L.vbqo_packed_size.argtypes = [i64, i64, i64, vp, ctypes.POINTER(u64)]
         L.vbqo_pack.argtypes = [i64, i64, i64, vp, vp, vp, vp, u64, ctypes.POINTER(u64)]
+        L.vbqo_pack_ex.argtypes = [i64, i64, i64, vp, vp, vp, ctypes.c_uint, vp, u64, ctypes.POINTER(u64)]
+        L.vbqo_read_header_ex.argtypes = [vp, u64, ctypes.POINTER(i64), ctypes.POINTER(i64), ctypes.POINTER(i64),
+                                          ctypes.POINTER(u64), ctypes.POINTER(ctypes.c_uint)]
+        L.vbqo_matvec_ex.argtypes = [i64, i64, i64, vp, vp, vp, vp, ctypes.c_uint, vp, vp, ctypes.c_int]
+        L.vbqo_dequant_ex.argtypes = [i64, i64, vp, vp, vp, ctypes.c_uint, vp]
         L.vbqo_read_header.argtypes = [vp, u64, ctypes.POINTER(i64), ctypes.POINTER(i64),
                                        ctypes.POINTER(i64), ctypes.POINTER(u64)]
         L.vbqo_unpack.argtypes = [vp, u64, vp, vp, vp]
         L.vbqo_matvec.argtypes = [i64, i64, i64, vp, vp, vp, vp, vp, vp, ctypes.c_int]
         L.vbqo_dequant.argtypes = [i64, i64, vp, vp, vp, vp]
         for f in ("vbqo_packed_size", "vbqo_pack", "vbqo_read_header", "vbqo_unpack", "vbqo_matvec",
-                  "vbqo_dequant"):
+                  "vbqo_dequant", "vbqo_pack_ex", "vbqo_read_header_ex", "vbqo_matvec_ex", "vbqo_dequant_ex"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -101,8 +107,8 @@ def packed_size(N: int, K: int, R: int, widths: np.ndarray) -> int:
     return int(out.value)
 
 
-def pack_status(N: int, K: int, R: int, widths, scales, codes, cap: int | None = None):
-    """Returns (status, blob or None)."""
+def pack_status(N: int, K: int, R: int, widths, scales, codes, cap: int | None = None, flags: int = 0):
+    """Returns (status, blob or None). flags: header flags (FLAG_GRID_SYMMETRIC selects Eq. 1's grid)."""
     w, s, c = _c(widths, np.uint8), _c(scales, np.uint16), _c(codes, np.uint8)
     if cap is None:
         try:
@@ -111,12 +117,12 @@ def pack_status(N: int, K: int, R: int, widths, scales, codes, cap: int | None =
             return e.status, None
     out = np.zeros(max(cap, 1), dtype=np.uint8)
     n = ctypes.c_uint64()
-    st = lib().vbqo_pack(N, K, R, _p(w), _p(s), _p(c), _p(out), cap, ctypes.byref(n))
+    st = lib().vbqo_pack_ex(N, K, R, _p(w), _p(s), _p(c), flags, _p(out), cap, ctypes.byref(n))
     return st, (out[: n.value] if st == OK else None)
 
 
-def pack(N: int, K: int, R: int, widths, scales, codes) -> np.ndarray:
-    st, blob = pack_status(N, K, R, widths, scales, codes)
+def pack(N: int, K: int, R: int, widths, scales, codes, flags: int = 0) -> np.ndarray:
+    st, blob = pack_status(N, K, R, widths, scales, codes, flags=flags)
     if st:
         raise OracleError(st, "pack")
     return blob
@@ -128,6 +134,15 @@ def read_header(blob: np.ndarray):
     st = lib().vbqo_read_header(_p(b), b.size, ctypes.byref(N), ctypes.byref(K), ctypes.byref(R),
                                 ctypes.byref(tot))
     return st, (N.value, K.value, R.value, tot.value)
+
+
+def header_flags(blob: np.ndarray) -> int:
+    b = _c(blob, np.uint8)
+    f = ctypes.c_uint()
+    st = lib().vbqo_read_header_ex(_p(b), b.size, None, None, None, None, ctypes.byref(f))
+    if st:
+        raise OracleError(st, "read_header")
+    return int(f.value)
 
 
 def unpack_status(blob: np.ndarray):
@@ -151,8 +166,9 @@ def unpack(blob: np.ndarray):
     return out
 
 
-def matvec(widths, scales, codes, x_bf16, nthreads: int | None = None):
-    """fp64 y[B,N] and bound A[B,N] = sum |w||x| for x_bf16[B,K] (bf16 bit patterns, uint16)."""
+def matvec(widths, scales, codes, x_bf16, nthreads: int | None = None, flags: int = 0):
+    """fp64 y[B,N] and bound A[B,N] = sum |w||x| for x_bf16[B,K] (bf16 bit patterns, uint16); flags selects the
+    value grid as in the blob header."""
     w, s, c = _c(widths, np.uint8), _c(scales, np.uint16), _c(codes, np.uint8)
     x = _c(x_bf16, np.uint16)
     if x.ndim == 1:
@@ -161,17 +177,17 @@ def matvec(widths, scales, codes, x_bf16, nthreads: int | None = None):
     B = x.shape[0]
     y = np.zeros((B, N), np.float64)
     a = np.zeros((B, N), np.float64)
-    st = lib().vbqo_matvec(N, K, B, _p(w), _p(s), _p(c), _p(x), _p(y), _p(a), int(nthreads or 1))
+    st = lib().vbqo_matvec_ex(N, K, B, _p(w), _p(s), _p(c), _p(x), flags, _p(y), _p(a), int(nthreads or 1))
     if st:
         raise OracleError(st, "matvec")
     return y, a
 
 
-def dequant(widths, scales, codes) -> np.ndarray:
+def dequant(widths, scales, codes, flags: int = 0) -> np.ndarray:
     w, s, c = _c(widths, np.uint8), _c(scales, np.uint16), _c(codes, np.uint8)
     N, K = c.shape
     out = np.zeros((N, K), np.float64)
-    st = lib().vbqo_dequant(N, K, _p(w), _p(s), _p(c), _p(out))
+    st = lib().vbqo_dequant_ex(N, K, _p(w), _p(s), _p(c), flags, _p(out))
     if st:
         raise OracleError(st, "dequant")
     return out
@@ -204,3 +220,62 @@ def swiglu_bound(y_gate, y_up, bound_gate, bound_up) -> np.ndarray:
     tg, tu = 1e-3 * np.asarray(bound_gate) + 1e-6, 1e-3 * np.asarray(bound_up) + 1e-6
     h = swiglu(g, u)
     return 2.0 ** -8 * np.abs(h) + 1.1 * np.abs(u) * tg + np.abs(silu(g)) * tu + tg * tu + 1e-6
+
+
+def fp16_bits(v) -> np.ndarray:
+    """fp16 bit patterns of fp64 values, round to nearest even (numpy's float64 -> float16 conversion)."""
+    with np.errstate(over="ignore"):   # values beyond fp16 become inf, which the callers check for
+        return np.asarray(v, np.float64).astype(np.float16).view(np.uint16)
+
+
+def round_half_away(v) -> np.ndarray:
+    """Nearest integer, ties away from zero (C's round()), exactly: integer part plus one step when the
+    fraction is at least one half."""
+    v = np.asarray(v, np.float64)
+    t = np.trunc(v)
+    return t + np.where(np.abs(v - t) >= 0.5, np.sign(v), 0.0)
+
+
+def quantize(w, widths, flags: int = 0):
+    """Quantize float32 weights w[N,K] to per-group codes for the given widths[N,G] (VBQ paper, section 3.1).
+
+    Per group of 64 weights (values in fp64):
+    - width 1: the scale is s = 2 * mean|w| (so that the two grid points +-s/2 are +-mean|w|: sign times the
+      mean magnitude), with the mean taken as the sum of |w| in index order divided by 64; code = 1 where w >= 0.
+    - width k >= 2, Eq. 1's symmetric grid (flags & FLAG_GRID_SYMMETRIC): L = 2^(k-1) - 1, s = max|w| / L,
+      q = clip(round(w / s), -L, L), code = q + L.
+    - width k >= 2, the default grid: c = (2^k - 1) / 2, s = max|w| / c, code = clip(round(w / s + c), 0,
+      2^k - 1).
+    The scale is rounded to fp16 (nearest even) first and the codes use that rounded scale; round() is to
+    nearest with ties away from zero. A group whose scale is 0 gets code L (symmetric) or 2^(k-1) (default),
+    i.e. the grid point nearest 0. Returns (status, scales[N,G] fp16 bits, codes[N,K]); status ERR_VALUE for a
+    non-finite weight or a scale that does not fit in fp16.
+    """
+    w = np.asarray(w, np.float32).astype(np.float64)
+    widths = np.asarray(widths, np.uint8)
+    N, K = w.shape
+    G = K // 64
+    if not np.all(np.isfinite(w)):
+        return ERR_VALUE, None, None
+    wg = w.reshape(N, G, 64)
+    a = np.abs(wg)
+    k = widths.astype(np.int64)
+    sym = bool(flags & FLAG_GRID_SYMMETRIC)
+    seq_sum = np.add.accumulate(a, axis=2)[:, :, -1]          # index-order sum of |w| over the group
+    amax = a.max(axis=2)
+    L = np.where(sym, (1 << (k - 1)) - 1, 0).astype(np.float64)
+    c = ((1 << k) - 1).astype(np.float64) / 2.0
+    ratio = np.where(k == 1, seq_sum / 32.0, np.where(sym, amax / np.maximum(L, 1.0), amax / c))
+    s16 = fp16_bits(ratio)
+    sd = s16.astype(np.uint16).view(np.float16).astype(np.float64)
+    if not np.all(np.isfinite(sd)):
+        return ERR_VALUE, None, None
+    sdx = sd[:, :, None]
+    kx, Lx, cx = k[:, :, None], L[:, :, None], c[:, :, None]
+    safe = np.where(sdx > 0, sdx, 1.0)
+    q1 = (wg >= 0).astype(np.float64)
+    qs = np.clip(round_half_away(wg / safe), -Lx, Lx) + Lx
+    qh = np.clip(round_half_away(wg / safe + cx), 0.0, (1 << kx) - 1.0)
+    zero_code = np.where(sym, Lx, (1 << (kx - 1)).astype(np.float64))
+    q = np.where(kx == 1, q1, np.where(sdx > 0, np.where(sym, qs, qh), zero_code))
+    return OK, s16.reshape(N, G), q.astype(np.uint8).reshape(N, K)

@@ -12,10 +12,11 @@
  * 64 weights, one scale and one width from {1,2,4,8} per group) and section 6,
  * paragraph "Fused kernels over packed weights" (the kernel dequantizes each
  * group with its scale and accumulates the matrix-vector product).
- * The value grid w = s*(q - (2^k-1)/2) with q in [0, 2^k) is this project's
- * reading: the paper's Eq. 1 uses a symmetric integer grid for k >= 2, which a
- * 2^k-level unsigned code cannot hold, while its 1-bit case (sign times a
- * per-group magnitude) is exactly +-s/2 here.
+ * The default value grid w = s*(q - (2^k-1)/2) with q in [0, 2^k) is this
+ * project's reading: the paper's Eq. 1 uses a symmetric integer grid for k >= 2,
+ * which a 2^k-level unsigned code cannot hold, while its 1-bit case (sign times a
+ * per-group magnitude) is exactly +-s/2 here. Header flag bit 0 selects Eq. 1's
+ * own grid for k >= 2 instead: w = s*(q - (2^(k-1)-1)), q in [0, 2^k - 2].
  *
  * Arithmetic is fp64. Every dequantized weight s*(q-c) is exact in fp64
  * (an 11-bit significand times a value with at most 9 significant bits), and
@@ -40,8 +41,22 @@
 enum {
   O_OK = 0, O_ERR_NULL = -1, O_ERR_SHAPE = -2, O_ERR_WIDTH = -3, O_ERR_CODE_RANGE = -4,
   O_ERR_BUFFER_TOO_SMALL = -5, O_ERR_BAD_MAGIC = -6, O_ERR_VERSION = -7, O_ERR_CRC = -8,
-  O_ERR_BATCH = -9, O_ERR_ALIGN = -10, O_ERR_CUDA = -11, O_ERR_TILE = -12, O_ERR_FORMAT = -13
+  O_ERR_BATCH = -9, O_ERR_ALIGN = -10, O_ERR_CUDA = -11, O_ERR_TILE = -12, O_ERR_FORMAT = -13,
+  O_ERR_FLAGS = -16
 };
+
+/* Header flag bit 0: widths >= 2 use the paper's symmetric integer grid (Eq. 1, section 3.1):
+ * w = s * (q - (2^(k-1) - 1)), q in [0, 2^k - 2]. 1-bit groups keep w = s * (q - 1/2) in both grids. */
+#define O_FLAG_SYM 1u
+
+/* Offset c of the value grid w = s * (q - c) for width k under header flags f. */
+static double grid_offset(int k, unsigned f) {
+  if ((f & O_FLAG_SYM) && k >= 2) return (double)((1 << (k - 1)) - 1);
+  return ((double)((1 << k) - 1)) / 2.0;
+}
+static unsigned max_code(int k, unsigned f) {
+  return ((f & O_FLAG_SYM) && k >= 2) ? (1u << k) - 2u : (1u << k) - 1u;
+}
 
 #define O_MAGIC 0x31514256u
 #define O_VERSION 1u
@@ -97,7 +112,7 @@ static int check_shape(int64_t N, int64_t K, int64_t R) {
   return O_OK;
 }
 
-static int check_logical(int64_t N, int64_t K, const uint8_t* widths, const uint8_t* codes) {
+static int check_logical(int64_t N, int64_t K, const uint8_t* widths, const uint8_t* codes, unsigned f) {
   int64_t G = K / 64;
   for (int64_t i = 0; i < N * G; ++i)
     if (width_code(widths[i]) < 0) return O_ERR_WIDTH;
@@ -105,7 +120,7 @@ static int check_logical(int64_t N, int64_t K, const uint8_t* widths, const uint
     for (int64_t r = 0; r < N; ++r)
       for (int64_t c = 0; c < K; ++c) {
         int k = widths[r * G + c / 64];
-        if (codes[r * K + c] >= (1u << k)) return O_ERR_CODE_RANGE;
+        if (codes[r * K + c] > max_code(k, f)) return O_ERR_CODE_RANGE;
       }
   }
   return O_OK;
@@ -130,7 +145,7 @@ int vbqo_packed_size(int64_t N, int64_t K, int64_t R, const uint8_t* widths, uin
   if (!widths || !out_bytes) return O_ERR_NULL;
   int st = check_shape(N, K, R);
   if (st) return st;
-  st = check_logical(N, K, widths, NULL);
+  st = check_logical(N, K, widths, NULL, 0);
   if (st) return st;
   int64_t G = K / 64, T = (N + R - 1) / R;
   uint64_t rec = 0;
@@ -149,12 +164,13 @@ int vbqo_packed_size(int64_t N, int64_t K, int64_t R, const uint8_t* widths, uin
 /* Pack logical (widths, scales, codes) into a canonical blob. Row-major logical
  * arrays: widths[N*G] in {1,2,4,8}, scales[N*G] fp16 bit patterns,
  * codes[N*K] with codes < 2^width. */
-int vbqo_pack(int64_t N, int64_t K, int64_t R, const uint8_t* widths, const uint16_t* scales,
-              const uint8_t* codes, uint8_t* out, uint64_t cap, uint64_t* written) {
+int vbqo_pack_ex(int64_t N, int64_t K, int64_t R, const uint8_t* widths, const uint16_t* scales,
+                 const uint8_t* codes, unsigned flags, uint8_t* out, uint64_t cap, uint64_t* written) {
   if (!widths || !scales || !codes || !out) return O_ERR_NULL;
+  if (flags & ~O_FLAG_SYM) return O_ERR_FLAGS;
   int st = check_shape(N, K, R);
   if (st) return st;
-  st = check_logical(N, K, widths, codes);
+  st = check_logical(N, K, widths, codes, flags);
   if (st) return st;
   uint64_t total;
   st = vbqo_packed_size(N, K, R, widths, &total);
@@ -211,7 +227,7 @@ int vbqo_pack(int64_t N, int64_t K, int64_t R, const uint8_t* widths, const uint
   uint8_t* h = out;
   put32(h + 0, O_MAGIC);
   put16(h + 4, O_VERSION);
-  put16(h + 6, 0);
+  put16(h + 6, (uint16_t)flags);
   put32(h + 8, (uint32_t)N);
   put32(h + 12, (uint32_t)K);
   put32(h + 16, (uint32_t)G);
@@ -227,10 +243,15 @@ int vbqo_pack(int64_t N, int64_t K, int64_t R, const uint8_t* widths, const uint
   return O_OK;
 }
 
+int vbqo_pack(int64_t N, int64_t K, int64_t R, const uint8_t* widths, const uint16_t* scales,
+              const uint8_t* codes, uint8_t* out, uint64_t cap, uint64_t* written) {
+  return vbqo_pack_ex(N, K, R, widths, scales, codes, 0u, out, cap, written);
+}
+
 /* Header check in the documented order: size, magic, version, header CRC,
  * field consistency, total size, body CRC. */
-int vbqo_read_header(const uint8_t* blob, uint64_t size, int64_t* N, int64_t* K, int64_t* R,
-                     uint64_t* total) {
+int vbqo_read_header_ex(const uint8_t* blob, uint64_t size, int64_t* N, int64_t* K, int64_t* R,
+                        uint64_t* total, unsigned* flags) {
   if (!blob) return O_ERR_NULL;
   if (size < 64) return O_ERR_BUFFER_TOO_SMALL;
   if (get32(blob) != O_MAGIC) return O_ERR_BAD_MAGIC;
@@ -238,7 +259,7 @@ int vbqo_read_header(const uint8_t* blob, uint64_t size, int64_t* N, int64_t* K,
   if (get32(blob + 60) != vbqo_crc32(blob, 60)) return O_ERR_CRC;
   int64_t n = get32(blob + 8), k = get32(blob + 12), g = get32(blob + 16), r = get32(blob + 20),
           t = get32(blob + 24);
-  if (get16(blob + 6) != 0 || get32(blob + 28) != 0) return O_ERR_FORMAT;
+  if ((get16(blob + 6) & ~O_FLAG_SYM) != 0 || get32(blob + 28) != 0) return O_ERR_FORMAT;
   if (check_shape(n, k, r) != O_OK) return O_ERR_FORMAT;
   if (g != k / 64 || t != (n + r - 1) / r) return O_ERR_FORMAT;
   uint64_t dir_off = get64(blob + 32), rec_off = get64(blob + 40), tot = get64(blob + 48);
@@ -250,7 +271,13 @@ int vbqo_read_header(const uint8_t* blob, uint64_t size, int64_t* N, int64_t* K,
   if (K) *K = k;
   if (R) *R = r;
   if (total) *total = tot;
+  if (flags) *flags = get16(blob + 6);
   return O_OK;
+}
+
+int vbqo_read_header(const uint8_t* blob, uint64_t size, int64_t* N, int64_t* K, int64_t* R,
+                     uint64_t* total) {
+  return vbqo_read_header_ex(blob, size, N, K, R, total, NULL);
 }
 
 /* Unpack a canonical blob to logical arrays; any non-canonical content is
@@ -258,7 +285,8 @@ int vbqo_read_header(const uint8_t* blob, uint64_t size, int64_t* N, int64_t* K,
 int vbqo_unpack(const uint8_t* blob, uint64_t size, uint8_t* widths, uint16_t* scales, uint8_t* codes) {
   int64_t N, K, R;
   uint64_t total;
-  int st = vbqo_read_header(blob, size, &N, &K, &R, &total);
+  unsigned flags;
+  int st = vbqo_read_header_ex(blob, size, &N, &K, &R, &total, &flags);
   if (st) return st;
   int64_t G = K / 64, T = (N + R - 1) / R;
   uint64_t dir_off = 64, rec_off = 64 + a16(4 * (uint64_t)(T * G + 1));
@@ -313,6 +341,7 @@ int vbqo_unpack(const uint8_t* blob, uint64_t size, uint8_t* widths, uint16_t* s
               uint64_t bit = (uint64_t)k * i + b;
               q |= (uint32_t)((rec[cpos + bit / 8] >> (bit % 8)) & 1u) << b;
             }
+            if (q > max_code(k, flags)) { free(used); free(wtmp); return O_ERR_FORMAT; }
             if (codes) codes[r * K + 64 * g + i] = (uint8_t)q;
           }
           for (int b = 0; b < 8 * k; ++b) used[cpos + b] = 0xFF;
@@ -338,12 +367,14 @@ int vbqo_unpack(const uint8_t* blob, uint64_t size, uint8_t* widths, uint16_t* s
 /* fp64 dequantize-then-matvec. x_bf16[B*K] row-major (batch b at row b),
  * y[B*N] and bound[B*N] row-major. y[b][r] = sum_i w[r][i] x[b][i] summed in
  * order i = 0..K-1; bound[b][r] = sum_i |w[r][i]| |x[b][i]|. */
-int vbqo_matvec(int64_t N, int64_t K, int64_t B, const uint8_t* widths, const uint16_t* scales,
-                const uint8_t* codes, const uint16_t* x_bf16, double* y, double* bound, int nthreads) {
+int vbqo_matvec_ex(int64_t N, int64_t K, int64_t B, const uint8_t* widths, const uint16_t* scales,
+                   const uint8_t* codes, const uint16_t* x_bf16, unsigned flags, double* y, double* bound,
+                   int nthreads) {
   if (!widths || !scales || !codes || !x_bf16 || !y) return O_ERR_NULL;
   if (N < 1 || K < 64 || K % 64 != 0) return O_ERR_SHAPE;
   if (B < 1) return O_ERR_BATCH;
-  int st = check_logical(N, K, widths, codes);
+  if (flags & ~O_FLAG_SYM) return O_ERR_FLAGS;
+  int st = check_logical(N, K, widths, codes, flags);
   if (st) return st;
   int64_t G = K / 64;
   double* xd = (double*)malloc(sizeof(double) * (size_t)(B * K));
@@ -360,7 +391,7 @@ int vbqo_matvec(int64_t N, int64_t K, int64_t B, const uint8_t* widths, const ui
         int64_t g = i / 64;
         int k = widths[r * G + g];
         double s = vbqo_half_to_double(scales[r * G + g]);
-        double c = ((double)((1 << k) - 1)) / 2.0;
+        double c = grid_offset(k, flags);
         double w = s * ((double)codes[r * K + i] - c);
         acc += w * xd[b * K + i];
         a += fabs(w) * fabs(xd[b * K + i]);
@@ -374,19 +405,30 @@ int vbqo_matvec(int64_t N, int64_t K, int64_t B, const uint8_t* widths, const ui
   return O_OK;
 }
 
+int vbqo_matvec(int64_t N, int64_t K, int64_t B, const uint8_t* widths, const uint16_t* scales,
+                const uint8_t* codes, const uint16_t* x_bf16, double* y, double* bound, int nthreads) {
+  return vbqo_matvec_ex(N, K, B, widths, scales, codes, x_bf16, 0u, y, bound, nthreads);
+}
+
 /* Dequantized dense matrix, w[N*K] in fp64 (same map as vbqo_matvec). */
-int vbqo_dequant(int64_t N, int64_t K, const uint8_t* widths, const uint16_t* scales,
-                 const uint8_t* codes, double* w) {
+int vbqo_dequant_ex(int64_t N, int64_t K, const uint8_t* widths, const uint16_t* scales,
+                    const uint8_t* codes, unsigned flags, double* w) {
   if (!widths || !scales || !codes || !w) return O_ERR_NULL;
   if (N < 1 || K < 64 || K % 64 != 0) return O_ERR_SHAPE;
-  int st = check_logical(N, K, widths, codes);
+  if (flags & ~O_FLAG_SYM) return O_ERR_FLAGS;
+  int st = check_logical(N, K, widths, codes, flags);
   if (st) return st;
   int64_t G = K / 64;
   for (int64_t r = 0; r < N; ++r)
     for (int64_t i = 0; i < K; ++i) {
       int k = widths[r * G + i / 64];
       double s = vbqo_half_to_double(scales[r * G + i / 64]);
-      w[r * K + i] = s * ((double)codes[r * K + i] - ((double)((1 << k) - 1)) / 2.0);
+      w[r * K + i] = s * ((double)codes[r * K + i] - grid_offset(k, flags));
     }
   return O_OK;
+}
+
+int vbqo_dequant(int64_t N, int64_t K, const uint8_t* widths, const uint16_t* scales,
+                 const uint8_t* codes, double* w) {
+  return vbqo_dequant_ex(N, K, widths, scales, codes, 0u, w);
 }

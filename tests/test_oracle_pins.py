@@ -330,3 +330,60 @@ def test_recipe_workload_shape():
     assert abs(w.mean() - 1.18) < 1e-3
     assert np.all(np.diff(w[:, 0].astype(int)) <= 0)         # widths never increase down the frequency order
     assert (w[:, 0] == 8).sum() == 160 and (w[:, 0] == 4).sum() == 480 and (w[:, 0] == 2).sum() == 3200
+
+
+def test_quantize_recovers_weights_on_either_grid_exactly():
+    """Weights that lie exactly on a grid (with an fp16-exact scale and an extreme point present) come back as
+    that scale and those codes: Eq. 1's symmetric grid (flag) and the default half-integer grid."""
+    rng = np.random.default_rng(3)
+    N, G = 6, 4
+    for k in (2, 4, 8):
+        Lk = (1 << (k - 1)) - 1
+        q = rng.integers(-Lk, Lk + 1, size=(N, G, 64))
+        q[:, :, 0] = Lk                                   # the extreme point fixes max|w| = L * s
+        s = 0.5
+        w = (s * q).reshape(N, G * 64).astype(np.float32)
+        st, s16, codes = O.quantize(w, np.full((N, G), k, np.uint8), O.FLAG_GRID_SYMMETRIC)
+        assert st == O.OK and np.all(s16 == 0x3800)
+        assert np.array_equal(codes.reshape(N, G, 64), (q + Lk).astype(np.uint8))
+        assert np.array_equal(O.dequant(np.full((N, G), k, np.uint8), s16, codes, flags=O.FLAG_GRID_SYMMETRIC), w)
+        qh = rng.integers(0, 1 << k, size=(N, G, 64))
+        qh[:, :, 0] = (1 << k) - 1
+        wh = (0.25 * (qh - ((1 << k) - 1) / 2)).reshape(N, G * 64).astype(np.float32)
+        st, s16, codes = O.quantize(wh, np.full((N, G), k, np.uint8))
+        assert st == O.OK and np.all(s16 == 0x3400)
+        assert np.array_equal(codes.reshape(N, G, 64), qh.astype(np.uint8))
+
+
+def test_quantize_one_bit_is_sign_times_mean_magnitude():
+    """1-bit groups: scale 2 * mean|w| (so the grid points are +-mean|w|), code 1 where w >= 0."""
+    w = np.tile(np.array([0.125, -0.375, 0.25, -0.25], np.float32), 16)[None, :]   # mean |w| = 0.25
+    st, s16, codes = O.quantize(w, np.ones((1, 1), np.uint8))
+    assert st == O.OK and s16[0, 0] == 0x3800                                      # 0.5 = 2 * 0.25
+    assert np.array_equal(codes[0], (w[0] >= 0).astype(np.uint8))
+    assert np.array_equal(O.dequant(np.ones((1, 1), np.uint8), s16, codes)[0], np.where(w[0] >= 0, 0.25, -0.25))
+
+
+def test_quantize_error_bound_zero_groups_and_bad_values():
+    """Every weight lands within half a grid step of its value (the scale's fp16 rounding can push the largest
+    one slightly out, by at most L * |s - s16|); all-zero groups decode to zero; non-finite weights and scales
+    beyond fp16 are refused."""
+    rng = np.random.default_rng(4)
+    N, G = 8, 6
+    w = rng.normal(0, 0.05, size=(N, G * 64)).astype(np.float32)
+    w[0, :64] = 0.0
+    widths = np.array([2, 4, 8, 2, 4, 8], np.uint8)[None, :].repeat(N, 0)
+    for flags in (0, O.FLAG_GRID_SYMMETRIC):
+        st, s16, codes = O.quantize(w, widths, flags)
+        assert st == O.OK
+        wq = O.dequant(widths, s16, codes, flags=flags)
+        sd = np.repeat(s16.view(np.float16).astype(np.float64), 64, axis=1)
+        kk = np.repeat(widths.astype(np.int64), 64, axis=1)
+        Lc = ((1 << (kk - 1)) - 1) if flags else ((1 << kk) - 1) / 2
+        amax = np.repeat(np.abs(w.astype(np.float64)).reshape(N, G, 64).max(axis=2), 64, axis=1)
+        assert np.all(np.abs(wq - w) <= sd / 2 + np.abs(amax - Lc * sd) + 1e-12)
+        assert np.all(wq[0, :64] == 0.0)
+    bad = w.copy()
+    bad[1, 5] = np.inf
+    assert O.quantize(bad, widths)[0] == O.ERR_VALUE
+    assert O.quantize(np.full((1, 64), 3e38, np.float32), np.full((1, 1), 2, np.uint8))[0] == O.ERR_VALUE
