@@ -228,8 +228,10 @@ def run_vbq(args):
             g.name = "_".join(names)
             ms = [by_name[n] for n in names]
             g.mats = []
+            g.R = R if R > 0 else vbq.suggest_tile_rows(sum(m.N for m in ms), ms[0].K,
+                                                         torch.cuda.get_device_properties(dev).multi_processor_count)
             for m in ms:
-                blob, _ = vbq.vbq_pack(m.N, m.K, R, m.widths, m.scales, m.codes)
+                blob, _ = vbq.vbq_pack(m.N, m.K, g.R, m.widths, m.scales, m.codes)
                 g.mats.append(vbq.DeviceMatrix(blob, dev, max_batch=B))
                 del blob
             g.fused = vbq.FusedMatrices(g.mats, max_batch=B) if len(ms) > 1 else None
@@ -351,7 +353,8 @@ def run_vbq(args):
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "fp32", "data": "synthetic",
-            "config": {"workload": WORKLOAD, "batch": B, "tile_rows": R,
+            "config": {"workload": WORKLOAD, "batch": B,
+                       "tile_rows": {g.name: g.R for g in layers[0]},
                        "launch": ("plain" if args.no_overlap else "programmatic dependent launch (VBQ_LAUNCH_OVERLAP)")
                                  + ("; one launch per linear" if args.no_fuse
                                     else "; q/k/v fused (vbq_gemm_skinny_multi); gate/up fused with the SwiGLU "
@@ -388,7 +391,8 @@ def main():
     ap.add_argument("--batch", type=int, default=1, choices=(1, 2, 4, 8, 16))
     ap.add_argument("--impl", default="vbq", choices=("vbq", "reference"))
     ap.add_argument("--copies", type=int, default=4)
-    ap.add_argument("--tile-rows", type=int, default=256)
+    ap.add_argument("--tile-rows", type=int, default=0,
+                    help="tile rows for packing; 0: per launch group, vbq.suggest_tile_rows")
     ap.add_argument("--no-fuse", action="store_true",
                     help="one launch per linear instead of fusing the projections that share their input")
     ap.add_argument("--no-overlap", action="store_true",

@@ -62,6 +62,7 @@ struct Params {
   uint32_t units_total[kMaxMats];  // dir[m][T_m*G]: 16-byte units of matrix m's records
   int rec_start[kMaxMats + 1];
   int tile_start[kMaxMats + 1];
+  int sym[kMaxMats];       // matrix m's widths >= 2 use Eq. 1's symmetric grid (format flag bit 0)
   int nmat;
   int swiglu;              // SwiGLU epilogue: matrices 0 (gate) and 1 (up) have the same rows; h = silu(y0) * y1
   uint16_t* h;             // bf16 bits, [B][N_0] (SwiGLU only)
@@ -292,8 +293,9 @@ __device__ __forceinline__ float dot_b1(uint2 w, const float (&xr)[64], float sg
 }
 
 // 2- and 4-bit: xr holds x_i * 2^-shift(i). v - 2^23 = q * 2^shift exactly, so (v - 2^23) * xr_i = q * x_i.
+// The grid offset is c = 2^(k-1) - corr: corr = 1/2 on the default grid, 1 on Eq. 1's symmetric grid.
 template <int KB>
-__device__ __forceinline__ float dot_magic(const uint32_t (&w)[2 * KB], const float (&xr)[64], float sg) {
+__device__ __forceinline__ float dot_magic(const uint32_t (&w)[2 * KB], const float (&xr)[64], float sg, float corr) {
   constexpr int CPW = 32 / KB;
   constexpr uint32_t M = (1u << KB) - 1u;
   const float2 neg = make_float2(-8388608.f, -8388608.f);
@@ -312,11 +314,12 @@ __device__ __forceinline__ float dot_magic(const uint32_t (&w)[2 * KB], const fl
     }
   }
   // sum q x - (2^(k-1) - 1/2) sum x
-  return ((acc0.x + acc0.y) + (acc1.x + acc1.y)) - (float(1 << (KB - 1)) - 0.5f) * sg;
+  return ((acc0.x + acc0.y) + (acc1.x + acc1.y)) - (float(1 << (KB - 1)) - corr) * sg;
 }
 
-// 8-bit: a byte permute places q in the low mantissa byte of 2^23; subtracting 2^23 + 128 gives q - 128 exactly.
-__device__ __forceinline__ float dot_b8(const uint32_t (&w)[16], const float (&xr)[64], float sg) {
+// 8-bit: a byte permute places q in the low mantissa byte of 2^23; subtracting 2^23 + 128 gives q - 128 exactly;
+// q - c = (q - 128) + corr with corr = 128 - c.
+__device__ __forceinline__ float dot_b8(const uint32_t (&w)[16], const float (&xr)[64], float sg, float corr) {
   const float2 neg = make_float2(-8388736.f, -8388736.f);
   float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
 #pragma unroll
@@ -328,7 +331,7 @@ __device__ __forceinline__ float dot_b8(const uint32_t (&w)[16], const float (&x
     acc0 = ffma2(q0, make_float2(xr[4 * m], xr[4 * m + 1]), acc0);
     acc1 = ffma2(q1, make_float2(xr[4 * m + 2], xr[4 * m + 3]), acc1);
   }
-  return ((acc0.x + acc0.y) + (acc1.x + acc1.y)) + 0.5f * sg;
+  return ((acc0.x + acc0.y) + (acc1.x + acc1.y)) + corr * sg;
 }
 
 // Batch 1, one width bucket: the warp's units of 32 items each (local unit u for u = first, first + TW, ...).
@@ -338,7 +341,7 @@ __device__ __forceinline__ float dot_b8(const uint32_t (&w)[16], const float (&x
 template <int KB>
 __device__ __forceinline__ void bucket_units(int n, int U, int first, int TW, int lane, uint32_t codes,
                                              uint32_t scales, uint32_t res, float (&xr)[64], uint32_t xcopy,
-                                             float sg, bool load) {
+                                             float sg, bool load, float corr) {
   if (first >= U) return;
   if (load) {
 #pragma unroll
@@ -356,11 +359,11 @@ __device__ __forceinline__ void bucket_units(int n, int U, int first, int TW, in
     } else if constexpr (KB == 2) {
       const uint4 a = lds128(codes + 16 * jj);
       const uint32_t w[4] = {a.x, a.y, a.z, a.w};
-      d = dot_magic<2>(w, xr, sg);
+      d = dot_magic<2>(w, xr, sg, corr);
     } else if constexpr (KB == 4) {
       const uint4 a = lds128(codes + 32 * jj), b = lds128(codes + 32 * jj + 16);
       const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-      d = dot_magic<4>(w, xr, sg);
+      d = dot_magic<4>(w, xr, sg, corr);
     } else {
       uint32_t w[16];
 #pragma unroll
@@ -368,7 +371,7 @@ __device__ __forceinline__ void bucket_units(int n, int U, int first, int TW, in
         const uint4 a = lds128(codes + 64 * jj + 16 * q);
         w[4 * q] = a.x; w[4 * q + 1] = a.y; w[4 * q + 2] = a.z; w[4 * q + 3] = a.w;
       }
-      d = dot_b8(w, xr, sg);
+      d = dot_b8(w, xr, sg, corr);
     }
     sts32f(res + 4 * jj, __half2float(__ushort_as_half((unsigned short)lds16(scales + 2 * jj))) * d);
   }
@@ -707,6 +710,8 @@ __global__ void __launch_bounds__(Cfg<B>::kThreads, 1) vbq_kernel(const __grid_c
       ok = __all_sync(0xFFFFFFFFu, ok);  // lanes can see an abort at different times; the warp decides as one
       const int j = tb + i, t = j / G;
       const int Rt = tile_out(p, t).Rt;
+      const bool grid_sym = pick(p.sym, mat_of_tile(p, t)) != 0;
+      const float corr = grid_sym ? 1.f : 0.5f;  // (q - c) = (q - 2^(k-1)) + corr for k >= 2
       if (t != cur_t) {
         if (cur_t >= 0) flush(cur_t);
         for (int e = sl0 * B + lane; e < sl1 * B; e += 32) acc[e] = 0.f;
@@ -807,13 +812,13 @@ __global__ void __launch_bounds__(Cfg<B>::kThreads, 1) vbq_kernel(const __grid_c
           const uint32_t sca = sa + rc.sc;
           const int U0 = rc.u0, U1 = rc.u1 - rc.u0, U2 = rc.u2 - rc.u1, U3 = rc.U - rc.u2;
           // 1-bit and 8-bit units read the same (raw) activations, so they run back to back on one load.
-          bucket_units<1>(n0, U0, first_unit(tw, 0, TW), TW, lane, sa + rc.c0, sca, ra, xr, xa, sg, true);
+          bucket_units<1>(n0, U0, first_unit(tw, 0, TW), TW, lane, sa + rc.c0, sca, ra, xr, xa, sg, true, 0.5f);
           bucket_units<8>(n3, U3, first_unit(tw, rc.u2, TW), TW, lane, sa + rc.c3, sca + 2 * (n0 + n1 + n2),
-                          ra + 4 * (n0 + n1 + n2), xr, xa, sg, first_unit(tw, 0, TW) >= U0);
+                          ra + 4 * (n0 + n1 + n2), xr, xa, sg, first_unit(tw, 0, TW) >= U0, corr);
           bucket_units<2>(n1, U1, first_unit(tw, rc.u0, TW), TW, lane, sa + rc.c1, sca + 2 * n0, ra + 4 * n0, xr,
-                          xa + 256, sg, true);
+                          xa + 256, sg, true, corr);
           bucket_units<4>(n2, U2, first_unit(tw, rc.u1, TW), TW, lane, sa + rc.c2, sca + 2 * (n0 + n1),
-                          ra + 4 * (n0 + n1), xr, xa + 512, sg, true);
+                          ra + 4 * (n0 + n1), xr, xa + 512, sg, true, corr);
         } else if constexpr (B < 8) {
           // -- CUDA cores, B in {2, 4}: lane = group; activations of all batches broadcast from shared memory
           const float* xc = xv;
@@ -847,16 +852,18 @@ __global__ void __launch_bounds__(Cfg<B>::kThreads, 1) vbq_kernel(const __grid_c
             const int item = ibase + jj;
             const float sc = __half2float(reinterpret_cast<const __half*>(st + rc.sc)[item]);
             const int row = item_row(mk, pf, bk, item);
-            // sum (q - 2^(k-1)) x + 1/2 sum x == sum (q - (2^k-1)/2) x; for k = 1 the first sum is sum_{q=1} x - S.
+            // sum (q - 2^(k-1)) x + corr sum x == sum (q - c) x (corr = 1/2 default grid, 1 symmetric grid);
+            // for k = 1 the first sum is sum_{q=1} x - S, and c = 1/2 on both grids.
 #pragma unroll
             for (int b = 0; b < B; ++b) {
               const float Sb = sgv[b];
-              const float d = (bk == 0) ? a[b] - 0.5f * Sb : a[b] + 0.5f * Sb;
+              const float d = (bk == 0) ? a[b] - 0.5f * Sb : a[b] + corr * Sb;
               acc[row * B + b] = fmaf(sc, d, acc[row * B + b]);
             }
           }
         } else {
-          // -- tensor cores, B in {8, 16}: lane = group, dequantized to bf16 2q-(2^k-1) in this warp's A tile;
+          // -- tensor cores, B in {8, 16}: lane = group, dequantized to bf16 2(q - c) (2q-(2^k-1) on the default grid,
+          // 2q-(2^k-2) on the symmetric one; both exact) in this warp's A tile;
           // two m16 tiles per unit through mma.sync m16n8k16 (bf16 in, fp32 accumulate), then s/2 per row.
           constexpr int NTL = B >= 8 ? B / 8 : 1;
           __nv_bfloat16* As = reinterpret_cast<__nv_bfloat16*>(wbase + wo.x);
@@ -879,7 +886,7 @@ __global__ void __launch_bounds__(Cfg<B>::kThreads, 1) vbq_kernel(const __grid_c
             __nv_bfloat162* arow = reinterpret_cast<__nv_bfloat162*>(As + lane * kAStride);
             if (valid) {
               const uint32_t* w = reinterpret_cast<const uint32_t*>(st + cbase + 8 * k * jj);
-              const float off = float((1 << k) - 1);
+              const float off = float((1 << k) - 1 - ((grid_sym && k >= 2) ? 1 : 0));  // 2c: A = 2(q - c)
               const uint32_t mask = (1u << k) - 1u;
 #pragma unroll 8
               for (int i2 = 0; i2 < 64; i2 += 2) {
@@ -1089,7 +1096,7 @@ struct Problem {
 };
 
 inline bool desc_ok(const vbq_desc* d) {
-  return d->version == 1 && d->N >= 1 && d->K >= 64 && d->K % 64 == 0 && d->G == d->K / 64 && d->R >= 16 &&
+  return d->version == 1 && (d->flags & ~unsigned(VBQ_FLAG_GRID_SYMMETRIC)) == 0 && d->N >= 1 && d->K >= 64 && d->K % 64 == 0 && d->G == d->K / 64 && d->R >= 16 &&
          d->R <= kMaxTileRows && d->R % 16 == 0 && d->T == (d->N + d->R - 1) / d->R && d->N <= INT32_MAX &&
          d->K <= INT32_MAX && d->dir_offset == 64 && d->rec_offset > d->dir_offset &&
          d->total_bytes > d->rec_offset && d->max_record_bytes >= 32 &&
@@ -1201,6 +1208,7 @@ int launch(const Problem& pr, const void* const* blobs, const void* x, float* co
     p.recs[m] = base + d->rec_offset;
     p.y[m] = ys[m];
     p.N[m] = int(d->N);
+    p.sym[m] = (d->flags & VBQ_FLAG_GRID_SYMMETRIC) ? 1 : 0;
     p.units_total[m] = uint32_t((d->total_bytes - d->rec_offset) / 16);
     tiles += int(d->T);
     recs += int(d->T * d->G);

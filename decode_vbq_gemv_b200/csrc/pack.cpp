@@ -8,6 +8,7 @@
 #include <cstdint>
 #include <algorithm>
 #include <cstring>
+#include <cmath>
 #include <vector>
 
 #include "vbq.h"
@@ -108,9 +109,9 @@ int record_counts(const Geometry& geo, const uint8_t* widths, std::vector<uint32
   return VBQ_OK;
 }
 
-void fill_desc(const Geometry& geo, uint64_t total, uint64_t max_rec, vbq_desc* d) {
+void fill_desc(const Geometry& geo, uint64_t total, uint64_t max_rec, unsigned flags, vbq_desc* d) {
   d->version = kVersion;
-  d->flags = 0;
+  d->flags = flags;
   d->N = geo.N;
   d->K = geo.K;
   d->G = geo.G;
@@ -140,6 +141,37 @@ void get_group_codes(const uint8_t* src, uint8_t* q, int k) {
   }
 }
 
+// Largest code of a k-bit group: 2^k - 1, or 2^k - 2 on the symmetric grid (header flag bit 0, k >= 2).
+inline unsigned max_code(int k, unsigned flags) {
+  return ((flags & VBQ_FLAG_GRID_SYMMETRIC) && k >= 2) ? (1u << k) - 2u : (1u << k) - 1u;
+}
+
+// IEEE binary16 bit pattern of a finite v >= 0, rounded to nearest, ties to even (values from 65520 up become
+// infinity). The significand is scaled by a power of two (exact) and rounded with nearbyint, whose default
+// rounding mode is to nearest even.
+uint16_t half_bits_rne(double v) {
+  if (v == 0.0) return 0;
+  int e;
+  std::frexp(v, &e);  // v = m * 2^e, m in [0.5, 1)
+  if (e <= -14) {     // below 2^-14: subnormal step 2^-24 (a result of 1024 is the smallest normal)
+    return uint16_t(std::nearbyint(std::ldexp(v, 24)));
+  }
+  double r = std::nearbyint(std::ldexp(v, 11 - e));  // 11 significant bits: r in [1024, 2048]
+  int E = e - 1 + 15;
+  if (r >= 2048.0) {
+    r = 1024.0;
+    ++E;
+  }
+  if (E >= 31) return 0x7C00u;
+  return uint16_t((unsigned(E) << 10) | (unsigned(r) - 1024u));
+}
+
+double half_value(uint16_t h) {
+  const int E = (h >> 10) & 31, M = h & 1023;
+  const double mag = E == 0 ? std::ldexp(double(M), -24) : std::ldexp(double(M + 1024), E - 25);
+  return (h & 0x8000u) ? -mag : mag;
+}
+
 }  // namespace
 
 extern "C" {
@@ -162,7 +194,8 @@ const char* vbq_strerror(int status) {
     case VBQ_ERR_FORMAT: return "blob is not canonical VBQ format v1";
     case VBQ_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
     case VBQ_ERR_SCRATCH_LIMIT: return "problem needs more scratch than the 16 MiB fixed buffer of the allocation-free entry point";
-    case VBQ_ERR_FLAGS: return "launch options word has bits outside VBQ_LAUNCH_OVERLAP";
+    case VBQ_ERR_FLAGS: return "flags word has bits this entry point does not define";
+    case VBQ_ERR_VALUE: return "a weight is not finite, or a group scale does not fit in fp16";
     default: return "unknown status";
   }
 }
@@ -182,9 +215,10 @@ int vbq_packed_size(int64_t N, int64_t K, int64_t R, const uint8_t* widths, uint
   return VBQ_OK;
 }
 
-int vbq_pack(int64_t N, int64_t K, int64_t R, const uint8_t* widths, const uint16_t* scales,
-             const uint8_t* codes, void* out, uint64_t out_cap, vbq_desc* out_desc) {
+int vbq_pack_ex(int64_t N, int64_t K, int64_t R, const uint8_t* widths, const uint16_t* scales,
+                const uint8_t* codes, unsigned format_flags, void* out, uint64_t out_cap, vbq_desc* out_desc) {
   if (!widths || !scales || !codes || !out) return VBQ_ERR_NULL;
+  if (format_flags & ~unsigned(VBQ_FLAG_GRID_SYMMETRIC)) return VBQ_ERR_FLAGS;
   if (int st = shape_status(N, K, R)) return st;
   Geometry geo(N, K, R);
   std::vector<uint32_t> counts;
@@ -192,11 +226,10 @@ int vbq_pack(int64_t N, int64_t K, int64_t R, const uint8_t* widths, const uint1
   // Code range check, row by row.
   for (int64_t r = 0; r < N; ++r)
     for (int64_t g = 0; g < geo.G; ++g) {
-      const uint8_t lim = uint8_t((1u << widths[r * geo.G + g]) - 1u);
+      const unsigned lim = max_code(widths[r * geo.G + g], format_flags);
       const uint8_t* q = codes + r * K + 64 * g;
-      uint8_t bad = 0;
-      for (int i = 0; i < 64; ++i) bad |= uint8_t(q[i] & ~lim);
-      if (bad) return VBQ_ERR_CODE_RANGE;
+      for (int i = 0; i < 64; ++i)
+        if (q[i] > lim) return VBQ_ERR_CODE_RANGE;
     }
   std::vector<uint64_t> rec_start(size_t(geo.T * geo.G) + 1);
   uint64_t pos = 0;
@@ -242,7 +275,7 @@ int vbq_pack(int64_t N, int64_t K, int64_t R, const uint8_t* widths, const uint1
   }
   st32(b + 0, kMagic);
   st16(b + 4, kVersion);
-  st16(b + 6, 0);
+  st16(b + 6, format_flags);
   st32(b + 8, uint32_t(N));
   st32(b + 12, uint32_t(K));
   st32(b + 16, uint32_t(geo.G));
@@ -254,8 +287,13 @@ int vbq_pack(int64_t N, int64_t K, int64_t R, const uint8_t* widths, const uint1
   st64(b + 48, total);
   st32(b + 56, crc32(b + kHeaderBytes, total - kHeaderBytes));
   st32(b + 60, crc32(b, 60));
-  if (out_desc) fill_desc(geo, total, max_rec, out_desc);
+  if (out_desc) fill_desc(geo, total, max_rec, format_flags, out_desc);
   return VBQ_OK;
+}
+
+int vbq_pack(int64_t N, int64_t K, int64_t R, const uint8_t* widths, const uint16_t* scales,
+             const uint8_t* codes, void* out, uint64_t out_cap, vbq_desc* out_desc) {
+  return vbq_pack_ex(N, K, R, widths, scales, codes, 0u, out, out_cap, out_desc);
 }
 
 int vbq_describe(const void* blob_host, uint64_t blob_bytes, vbq_desc* out_desc) {
@@ -266,7 +304,9 @@ int vbq_describe(const void* blob_host, uint64_t blob_bytes, vbq_desc* out_desc)
   if (ld16(b + 4) != kVersion) return VBQ_ERR_VERSION;
   if (ld32(b + 60) != crc32(b, 60)) return VBQ_ERR_CRC;
   const int64_t N = ld32(b + 8), K = ld32(b + 12), G = ld32(b + 16), R = ld32(b + 20), T = ld32(b + 24);
-  if (ld16(b + 6) != 0 || ld32(b + 28) != 0 || shape_status(N, K, R) != VBQ_OK) return VBQ_ERR_FORMAT;
+  const unsigned flags = ld16(b + 6);
+  if ((flags & ~unsigned(VBQ_FLAG_GRID_SYMMETRIC)) || ld32(b + 28) != 0 || shape_status(N, K, R) != VBQ_OK)
+    return VBQ_ERR_FORMAT;
   const Geometry geo(N, K, R);
   if (G != geo.G || T != geo.T) return VBQ_ERR_FORMAT;
   const uint64_t total = ld64(b + 48);
@@ -285,7 +325,7 @@ int vbq_describe(const void* blob_host, uint64_t blob_bytes, vbq_desc* out_desc)
     prev = cur;
   }
   if (geo.rec_off + 16 * prev != total) return VBQ_ERR_FORMAT;
-  fill_desc(geo, total, max_rec, out_desc);
+  fill_desc(geo, total, max_rec, flags, out_desc);
   return VBQ_OK;
 }
 
@@ -333,10 +373,11 @@ int vbq_unpack(const void* blob_host, uint64_t blob_bytes, uint8_t* widths, uint
           std::memset(&mask[size_t(co)], 0xFF, size_t(8u << c));
           if (widths) widths[r * geo.G + g] = uint8_t(1u << c);
           if (scales) scales[r * geo.G + g] = uint16_t(ld16(rec + so));
-          if (codes) {
-            get_group_codes(rec + co, q, 1 << c);
-            std::memcpy(codes + r * geo.K + 64 * g, q, 64);
-          }
+          get_group_codes(rec + co, q, 1 << c);
+          const unsigned lim = max_code(1 << c, d.flags);
+          for (int i = 0; i < 64; ++i)
+            if (q[i] > lim) return VBQ_ERR_FORMAT;
+          if (codes) std::memcpy(codes + r * geo.K + 64 * g, q, 64);
         }
       }
       for (uint64_t i = 0; i < L.bytes; ++i)
@@ -345,6 +386,51 @@ int vbq_unpack(const void* blob_host, uint64_t blob_bytes, uint8_t* widths, uint
     }
   }
   if (geo.rec_off + expect != d.total_bytes) return VBQ_ERR_FORMAT;
+  return VBQ_OK;
+}
+
+int vbq_quantize(int64_t N, int64_t K, const float* w, const uint8_t* widths, unsigned format_flags,
+                 uint16_t* scales, uint8_t* codes) {
+  if (!w || !widths || !scales || !codes) return VBQ_ERR_NULL;
+  if (N < 1 || K < 64 || K % 64 != 0 || N > INT32_MAX || K > INT32_MAX) return VBQ_ERR_SHAPE;
+  if (format_flags & ~unsigned(VBQ_FLAG_GRID_SYMMETRIC)) return VBQ_ERR_FLAGS;
+  const bool sym = format_flags & VBQ_FLAG_GRID_SYMMETRIC;
+  const int64_t G = K / 64;
+  for (int64_t i = 0; i < N * G; ++i)
+    if (wcode(widths[i]) < 0) return VBQ_ERR_WIDTH;
+  for (int64_t i = 0; i < N * K; ++i)
+    if (!std::isfinite(w[i])) return VBQ_ERR_VALUE;
+  for (int64_t r = 0; r < N; ++r)
+    for (int64_t g = 0; g < G; ++g) {
+      const int k = widths[r * G + g];
+      const float* wg = w + r * K + 64 * g;
+      uint8_t* q = codes + r * K + 64 * g;
+      double sum = 0.0, amax = 0.0;
+      for (int i = 0; i < 64; ++i) {
+        const double a = std::fabs(double(wg[i]));
+        sum += a;
+        amax = std::max(amax, a);
+      }
+      const double L = double((1 << (k - 1)) - 1), c = double((1 << k) - 1) / 2.0;
+      const double ratio = k == 1 ? sum / 32.0 : (sym ? amax / L : amax / c);
+      const uint16_t s16 = half_bits_rne(ratio);
+      if (s16 == 0x7C00u) return VBQ_ERR_VALUE;
+      scales[r * G + g] = s16;
+      const double sd = half_value(s16);
+      for (int i = 0; i < 64; ++i) {
+        double v;
+        if (k == 1) {
+          v = wg[i] >= 0.f ? 1.0 : 0.0;
+        } else if (sd == 0.0) {
+          v = sym ? L : double(1 << (k - 1));
+        } else if (sym) {
+          v = std::min(std::max(std::round(double(wg[i]) / sd), -L), L) + L;
+        } else {
+          v = std::min(std::max(std::round(double(wg[i]) / sd + c), 0.0), double((1 << k) - 1));
+        }
+        q[i] = uint8_t(v);
+      }
+    }
   return VBQ_OK;
 }
 

@@ -46,7 +46,8 @@ typedef enum vbq_status {
   VBQ_ERR_FORMAT = -13,           /* blob is not canonical format v1 (layout, padding, counts) */
   VBQ_ERR_WORKSPACE = -14,        /* workspace NULL, misaligned or smaller than vbq_workspace_size */
   VBQ_ERR_SCRATCH_LIMIT = -15,    /* vbq_gemm_skinny_noalloc: problem needs more than its 16 MiB fixed buffer */
-  VBQ_ERR_FLAGS = -16             /* vbq_gemm_skinny_ex: unknown bits in the launch-options word */
+  VBQ_ERR_FLAGS = -16,            /* unknown bits in a flags word (launch options or format flags) */
+  VBQ_ERR_VALUE = -17             /* vbq_quantize: non-finite weight, or a group scale beyond fp16 */
 } vbq_status;
 
 /* Host-side description of a packed blob. It is filled by vbq_pack or vbq_describe and passed by pointer to
@@ -84,6 +85,30 @@ int vbq_packed_size(int64_t N, int64_t K, int64_t R, const uint8_t* widths, uint
  * out_desc may be NULL. Thread-safe, pure. */
 int vbq_pack(int64_t N, int64_t K, int64_t R, const uint8_t* widths, const uint16_t* scales,
              const uint8_t* codes, void* out, uint64_t out_cap, vbq_desc* out_desc);
+
+/* Format flags of a blob (header field `flags`, vbq_desc.flags). */
+#define VBQ_FLAG_GRID_SYMMETRIC 1u  /* widths >= 2 on the VBQ paper's Eq. 1 integer grid (section 3.1):
+                                       w = s*(q - (2^(k-1)-1)), q in [0, 2^k - 2]; 1-bit groups unchanged */
+
+/* vbq_pack with format flags (0 or VBQ_FLAG_GRID_SYMMETRIC); the codes are checked against the flagged grid
+ * (CODE_RANGE). Errors: as vbq_pack, plus FLAGS. */
+int vbq_pack_ex(int64_t N, int64_t K, int64_t R, const uint8_t* widths, const uint16_t* scales,
+                const uint8_t* codes, unsigned format_flags, void* out, uint64_t out_cap, vbq_desc* out_desc);
+
+/* Quantize float32 weights w[N*K] (row-major) to the logical arrays for given widths[N*G] (VBQ paper,
+ * section 3.1), group by group (64 weights):
+ *  - width 1: scale s = 2 * mean|w| (the grid points +-s/2 are +-mean|w|: sign times the mean magnitude), the
+ *    mean being the index-order sum of |w| in fp64 divided by 64; code 1 where w >= 0, else 0.
+ *  - width k >= 2 with VBQ_FLAG_GRID_SYMMETRIC (Eq. 1): L = 2^(k-1) - 1, s = max|w| / L,
+ *    code = clamp(round(w / s), -L, L) + L.
+ *  - width k >= 2 without it (the default grid): c = (2^k - 1)/2, s = max|w| / c,
+ *    code = clamp(round(w / s + c), 0, 2^k - 1).
+ * The scale is computed in fp64, rounded to fp16 (nearest even), and that rounded value is the s the codes
+ * use; round() is to nearest, ties away from zero. A group whose rounded scale is 0 gets the code of the grid
+ * point nearest 0 (L, or 2^(k-1)). Pack the result with vbq_pack_ex and the same flags.
+ * Errors: NULL, SHAPE, WIDTH, FLAGS, VALUE (a non-finite weight, or a scale that rounds past fp16). Pure. */
+int vbq_quantize(int64_t N, int64_t K, const float* w, const uint8_t* widths, unsigned format_flags,
+                 uint16_t* scales, uint8_t* codes);
 
 /* Validate a host copy of a blob and fill *out_desc. Checks, in order: size >= 64 (BUFFER_TOO_SMALL), magic
  * (BAD_MAGIC), version (VERSION), header CRC (CRC), header fields (FORMAT), total_bytes <= blob_bytes

@@ -31,7 +31,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_status_strings_and_version():
-    for st in range(-16, 1):
+    for st in range(-17, 1):
         assert vbq.vbq_strerror(st) and "unknown" not in vbq.vbq_strerror(st)
     assert vbq.vbq_strerror(-99) == "unknown status"
     assert vbq.vbq_version() >> 16 == 1
@@ -185,3 +185,63 @@ def test_swiglu_entry_argument_checks_need_no_gpu():
     assert run(r(g), r(other_r), 16, 16, 16, 1, 16, 16, 16, None, 0, 0, None) == vbq.VBQ_ERR_TILE
     assert run(r(g), r(u), 16, 16, 16, 1, 16, 16, 17, None, 0, 0, None) == vbq.VBQ_ERR_ALIGN
     assert run(r(g), r(u), 16, 16, 16, 1, 16, 16, 16, None, 0, 0, None) == vbq.VBQ_ERR_WORKSPACE
+
+
+def test_quantize_matches_oracle_bitwise_on_both_grids():
+    """vbq_quantize (C++) and the oracle's quantize (numpy) give the same scales and codes, bit for bit: random
+    weights over many magnitudes (fp16-subnormal scales included), every width, both grids, plus crafted
+    groups whose scale ratio lies exactly halfway between two fp16 values and weights exactly halfway between
+    two grid points."""
+    rng = np.random.default_rng(21)
+    N, G = 24, 8
+    K = 64 * G
+    w = (rng.normal(0, 1, size=(N, K)) * np.exp(rng.uniform(-14, 3, size=(N, 1)))).astype(np.float32)
+    # ratio exactly halfway between fp16 1.0 and 1.0009765625 (k = 2 symmetric: L = 1, ratio = max|w|)
+    w[0, :64] = 0.0
+    w[0, 0] = np.float32(1.0 + 2.0 ** -11)
+    # weights at x.5 steps of a power-of-two scale (ties for round())
+    w[1, :64] = np.float32(0.5) * (np.arange(64) - 31.5).astype(np.float32) / np.float32(31.5) * np.float32(3.5)
+    w[2, :64] = -w[1, :64]
+    widths = rng.choice(np.array([1, 2, 4, 8], np.uint8), size=(N, G))
+    widths[0, 0] = 2
+    widths[1, 0] = widths[2, 0] = 8
+    for flags in (0, vbq.VBQ_FLAG_GRID_SYMMETRIC):
+        st_o, s_o, c_o = O.quantize(w, widths, flags)
+        st_l, s_l, c_l = vbq.vbq_quantize_status(w, widths, flags)
+        assert st_o == st_l == 0
+        assert np.array_equal(s_o, s_l), np.argwhere(s_o != s_l)[:5]
+        assert np.array_equal(c_o, c_l), np.argwhere(c_o != c_l)[:5]
+
+
+def test_symmetric_grid_pack_unpack_and_errors():
+    """Format flag bit 0 (Eq. 1's grid): the library's blob equals the oracle's byte for byte, carries the flag
+    in its header and descriptor, and unpacks back; a code 2^k - 1 (outside the symmetric range) is refused by
+    pack and, planted into a blob, by unpack; unknown format bits and bad weights are refused."""
+    rng = np.random.default_rng(22)
+    N, K = 70, 256
+    widths = rng.choice(np.array([1, 2, 4, 8], np.uint8), size=(N, K // 64))
+    w = rng.normal(0, 0.05, size=(N, K)).astype(np.float32)
+    sym = vbq.VBQ_FLAG_GRID_SYMMETRIC
+    scales, codes = vbq.vbq_quantize(w, widths, sym)
+    blob, d = vbq.vbq_pack(N, K, 32, widths, scales, codes, format_flags=sym)
+    assert d.flags == sym and vbq.vbq_describe(blob).flags == sym
+    assert np.array_equal(blob, O.pack(N, K, 32, widths, scales, codes, flags=sym))
+    assert O.header_flags(blob) == sym
+    uw, us, uc = vbq.vbq_unpack(blob)
+    assert np.array_equal(uw, widths) and np.array_equal(us, scales) and np.array_equal(uc, codes)
+    r, g = np.argwhere(widths >= 2)[0]
+    bad = codes.copy()
+    bad[r, 64 * g] = (1 << int(widths[r, g])) - 1
+    assert vbq.vbq_pack_status(N, K, 32, widths, scales, bad, format_flags=sym)[0] == vbq.VBQ_ERR_CODE_RANGE
+    assert vbq.vbq_pack_status(N, K, 32, widths, scales, bad)[0] == vbq.VBQ_OK   # fine on the default grid
+    plain, _ = vbq.vbq_pack(N, K, 32, widths, scales, bad)
+    flagged = plain.copy()
+    flagged[6] = sym                                            # claim the symmetric grid for that blob
+    flagged = _refresh_crc(flagged)
+    assert vbq.vbq_unpack_status(flagged)[0] == vbq.VBQ_ERR_FORMAT == O.unpack_status(flagged)[0]
+    assert vbq.vbq_pack_status(N, K, 32, widths, scales, codes, format_flags=2)[0] == vbq.VBQ_ERR_FLAGS
+    nan = w.copy()
+    nan[3, 7] = np.nan
+    assert vbq.vbq_quantize_status(nan, widths, 0)[0] == vbq.VBQ_ERR_VALUE
+    assert vbq.vbq_quantize_status(np.full((1, 64), 1e38, np.float32), np.full((1, 1), 2, np.uint8), 0)[0] \
+        == vbq.VBQ_ERR_VALUE

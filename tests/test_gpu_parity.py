@@ -389,3 +389,63 @@ def test_recipe_workload_layers_and_head(B):
     rows = np.unique(np.concatenate([np.arange(0, 4000, 9), g.choice(head.N, 200), [head.N - 1]]))
     yref, bound = O.matvec(head.widths[rows], head.scales[rows], head.codes[rows], x, NTH)
     check(y[:, rows], yref, bound, f"recipe head B={B}")
+
+
+def sym_matrix(seed, N, K, p):
+    """Random widths, scales and codes on Eq. 1's symmetric grid (codes in [0, 2^k - 2] for k >= 2)."""
+    g = np.random.default_rng(seed)
+    w = S.widths_iid(N, K // 64, p, g)
+    codes = S.codes_uniform(w, g)
+    top = np.repeat(np.where(w >= 2, (1 << w.astype(np.int64)) - 2, 1), 64, axis=1)
+    codes = np.minimum(codes, top).astype(np.uint8)
+    return S.Matrix("sym", N, K, w, S.scales_uniform(N, K // 64, g), codes)
+
+
+@pytest.mark.parametrize("B", vbq.BATCHES)
+def test_symmetric_grid_all_batches(B):
+    """Blobs flagged with Eq. 1's symmetric grid (VBQ_FLAG_GRID_SYMMETRIC) through every batch path (CUDA cores
+    at B <= 4, tensor cores at B = 8, 16) against the oracle's flag-aware matvec; and one fused launch mixing a
+    flagged and an unflagged matrix."""
+    sym = vbq.VBQ_FLAG_GRID_SYMMETRIC
+    for (N, K, R, dist) in ((1030, 256, 64, "flat"), (777, 2048, 256, "base"), (300, 512, 1024, "all8")):
+        m = sym_matrix(N + K + B, N, K, DISTS[dist])
+        blob, d = vbq.vbq_pack(m.N, m.K, R, m.widths, m.scales, m.codes, format_flags=sym)
+        assert d.flags == sym
+        mat = vbq.DeviceMatrix(blob, dev(), max_batch=B)
+        x = S.x_normal(B, K, np.random.default_rng(B + N))
+        y, _ = gpu_y(m, x, mat=mat)
+        yref, bound = O.matvec(m.widths, m.scales, m.codes, x, NTH, flags=sym)
+        check(y, yref, bound, f"symmetric grid {N}x{K} R={R} B={B}")
+    a = sym_matrix(7 + B, 500, 256, DISTS["flat"])
+    b = logical(8 + B, 900, 256, DISTS["flat"])
+    ma = vbq.DeviceMatrix(vbq.vbq_pack(a.N, a.K, 64, a.widths, a.scales, a.codes, format_flags=sym)[0], dev(),
+                          max_batch=B)
+    mb = vbq.DeviceMatrix(vbq.vbq_pack(b.N, b.K, 64, b.widths, b.scales, b.codes)[0], dev(), max_batch=B)
+    fused = vbq.FusedMatrices([ma, mb], max_batch=B)
+    x = S.x_normal(B, 256, np.random.default_rng(99 + B))
+    ya, yb = fused.matmul(to_dev_x(x))
+    torch_sync()
+    assert fused_status(fused, B) == 0
+    ra, ba = O.matvec(a.widths, a.scales, a.codes, x, NTH, flags=sym)
+    rb, bb = O.matvec(b.widths, b.scales, b.codes, x, NTH)
+    check(ya.cpu().numpy().astype(np.float64), ra, ba, f"fused symmetric+default: symmetric B={B}")
+    check(yb.cpu().numpy().astype(np.float64), rb, bb, f"fused symmetric+default: default B={B}")
+
+
+@pytest.mark.parametrize("B", [1, 16])
+def test_quantize_pack_gemv_pipeline(B):
+    """Float weights -> vbq_quantize (Eq. 1 grid, and the default grid) -> vbq_pack_ex -> device GEMV, against the
+    oracle's matvec on the same codes."""
+    rng = np.random.default_rng(30 + B)
+    N, K = 1100, 1024
+    w = rng.normal(0, 0.02, size=(N, K)).astype(np.float32)
+    widths = S.widths_iid(N, K // 64, S.P_BASE, rng)
+    x = S.x_normal(B, K, rng)
+    for flags in (vbq.VBQ_FLAG_GRID_SYMMETRIC, 0):
+        scales, codes = vbq.vbq_quantize(w, widths, flags)
+        blob, _ = vbq.vbq_pack(N, K, 256, widths, scales, codes, format_flags=flags)
+        mat = vbq.DeviceMatrix(blob, dev(), max_batch=B)
+        m = S.Matrix("q", N, K, widths, scales, codes)
+        y, _ = gpu_y(m, x, mat=mat)
+        yref, bound = O.matvec(widths, scales, codes, x, NTH, flags=flags)
+        check(y, yref, bound, f"quantize pipeline flags={flags} B={B}")
