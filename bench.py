@@ -1,11 +1,14 @@
-"""Benchmark of the VBQ mixed-bit GEMV on B200: achieved HBM GB/s against the measured copy peak.
+"""Benchmark of the VBQ mixed-bit GEMV on B200: achieved HBM GB/s against the measured copy peak, and the
+decode-step time.
 
-Default workload: the seven linears of one 9B-shaped decoder layer at batch 1 (q, k, v, o 4096x4096; gate, up
-4096->14336; down 14336->4096), with widths drawn from the VBQ paper's allocation (about 69% 1-bit groups,
-1.85 mean bits). One step runs all seven GEMVs. Four distinct seeded copies of the layer (about 260 MB, more
-than the 126 MB L2) are used in rotation, so every step streams its weights from HBM.
+Default workload: every linear of one batch-1 decode step of a 9B-shaped decoder (32 layers of q, k, v, o
+4096x4096, gate, up 4096->14336 and down 14336->4096, then the LM head 4096->32000), with seeded synthetic
+weights drawn from the VBQ paper's allocation (about 69% 1-bit groups and 1.85 mean bits in the layers, the
+first block's MLP at 2.5 bits, the head at about 1.09 bits). The 2.1 GB of packed weights are about 17 times
+the 126 MB L2, so every step streams them from HBM. One step is one token: 129 launches (per layer q/k/v
+fused, o, gate/up fused with the SwiGLU epilogue feeding down's input, down; then the head).
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--batch B] [--impl vbq|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--batch B] [--layers L] [--impl vbq|reference]
 
 Under torchrun (N > 1) every rank runs an independent replica on its own GPU. The path has no cross-GPU
 exchange. Time is the max over ranks, and the value is the bytes of all ranks divided by that time.
@@ -33,7 +36,26 @@ METRIC = "mixed-bit GEMV achieved HBM GB/s (% of B200 peak); decode-step µs at 
 UNIT = "GB/s"
 NAMES = ("q", "k", "v", "o", "gate", "up", "down")
 GROUPS = (("q", "k", "v"), ("o",), ("gate", "up"), ("down",))   # projections that share their input, fused
-WORKLOAD = "9B-shaped decoder-layer linears (q,k,v,o 4096x4096; gate,up 4096->14336; down 14336->4096)"
+WORKLOAD = ("9B-shaped decode step: 32 layers of q,k,v,o 4096x4096, gate,up 4096->14336, down 14336->4096, "
+            "plus the LM head 4096->32000")
+SYNTH_CFG = 5   # seed family of the full decode-step stack in vbq_synth
+
+# DRAM traffic of the kernel from one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum, cold L2) of the
+# first five launches of `python bench.py --layers 1 --steps 3 --warmup 3 --cpu-budget 0`: layer 0's four launch
+# groups and the LM head at batch 1, fused, with the tile rows below. The line reports it per launch, scaled to
+# this step's algorithmic bytes per launch (traffic grows in proportion: the five launches span 4.5 to 41 MB, each
+# at 0.999 to 1.019 times its algorithmic bytes), and only while the kernel source and the tile rows are the
+# captured ones.
+NCU_TRAFFIC = {"kernel_source_sha256": "2c3dd4e2525fd0eaf6a70ee76e2fea95a04a6b70d546c0374438288f0e54478d",
+               "tile_rows": {"q_k_v": 224, "o": 512, "gate_up": 224, "down": 224, "head": 224},
+               "dram_bytes": 102596864, "algorithmic_bytes": 102422912, "launches": 5,
+               "summary": "profiles/vbq_kernel_b1_decode_step_9b_launches.md"}
+
+
+def kernel_source_sha256() -> str:
+    import hashlib
+    with open(os.path.join(ROOT, "decode_vbq_gemv_b200", "csrc", "gemv.cu"), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()
 
 
 def peaks():
@@ -96,8 +118,14 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------------------------------------ setup
-def layer_matrices(copy: int):
-    return [S.make_matrix(4, n, *S.CFG4_SHAPES[n], layer=copy) for n in NAMES]
+def step_matrices(layer: int):
+    """The seven linears of decoder layer `layer` (layer 0's MLP at the first-block mix)."""
+    return S.cfg5_layer(layer)
+
+
+def sample_matrices(with_head: bool = True):
+    """What the CPU oracle samples: layer 0's seven linears and the LM head."""
+    return step_matrices(0) + ([S.cfg5_head()] if with_head else [])
 
 
 def blob_bytes_of(m, R):
@@ -107,12 +135,12 @@ def blob_bytes_of(m, R):
 
 def cpu_baseline(B: int, budget_s: float = 12.0, matrices=None):
     """Times the fp64 oracle (as it stands) on a bounded sample of the workload: the first `rows` rows of each
-    of the seven linears, growing the sample until it takes about `budget_s` seconds or covers every row."""
+    sampled linear, growing the sample until it takes about `budget_s` seconds or covers every row."""
     from oracle import oracle as O
     from decode_vbq_gemv_b200 import vbq
-    mats = matrices or layer_matrices(0)
+    mats = matrices or sample_matrices()
     threads = os.cpu_count() or 1
-    xs = [S.make_x(4, m.name, B, m.K) for m in mats]
+    xs = [S.make_x(SYNTH_CFG, m.name, B, m.K) for m in mats]
     full = [vbq.vbq_packed_size(m.N, m.K, 1024, m.widths) for m in mats]
     rows = 64
     while True:
@@ -127,8 +155,8 @@ def cpu_baseline(B: int, budget_s: float = 12.0, matrices=None):
             break
         rows *= 4
     return {"value": nbytes / dt / 1e9, "unit": UNIT, "cores": threads, "kind": "oracle",
-            "sample": f"fp64 oracle on the first {rows} rows of each of the 7 linears, batch {B} "
-                      f"({dt:.2f} s); GB/s scaled from those rows' share of the packed bytes"}
+            "sample": f"fp64 oracle on the first {rows} rows of each of layer 0's 7 linears and the LM head, "
+                      f"batch {B} ({dt:.2f} s); GB/s scaled from those rows' share of the packed bytes"}
 
 
 def dist_setup():
@@ -163,15 +191,13 @@ def barrier(world: int):
 
 # ------------------------------------------------------------------------------------------------ arms
 def run_reference(args):
-    world, rank, _ = dist_setup()
-    if rank != 0:
-        if world > 1:
-            import torch.distributed as dist
-            dist.destroy_process_group()
+    # The oracle arm runs on rank 0's host cores alone and needs no process group: the other ranks exit at once.
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if int(os.environ.get("RANK", "0")) != 0:
         return
     from oracle import oracle as O
-    mats = layer_matrices(0)
-    xs = [S.make_x(4, m.name, args.batch, m.K) for m in mats]
+    mats = sample_matrices()
+    xs = [S.make_x(SYNTH_CFG, m.name, args.batch, m.K) for m in mats]
     full = [blob_bytes_of(m, 1024) for m in mats]
     rows = args.ref_rows
     threads = os.cpu_count() or 1
@@ -189,71 +215,90 @@ def run_reference(args):
     nb = sum(step() for _ in range(args.steps))
     dt = time.perf_counter() - t0
     val = nb / dt / 1e9
-    sample = f"fp64 oracle, first {rows} rows of each of the 7 linears per step, batch {args.batch}"
+    sample = (f"fp64 oracle, first {rows} rows of each of layer 0's 7 linears and the LM head per step, "
+              f"batch {args.batch}")
     line = {"impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": WORKLOAD + f", sampled rows ({rows} per linear)",
+            "data": "synthetic", "config": {"workload": WORKLOAD + f"; sampled rows ({rows} per linear)",
                                             "batch": args.batch},
             "cpu_baseline": {"value": val, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample},
             "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
-    if world > 1:
-        import torch.distributed as dist
-        dist.destroy_process_group()
 
 
 def run_vbq(args):
+    import concurrent.futures as cf
     import torch
     from decode_vbq_gemv_b200 import vbq
     world, rank, local = dist_setup()
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     B, R = args.batch, args.tile_rows
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
 
-    # A step is one pass over the layer's seven linears, as launch groups. Fused (default): q/k/v share their
-    # input and run as one launch, so do gate/up; o and down run alone (4 launches). --no-fuse: 7 launches.
+    # A step is one token: per layer the seven linears as launch groups, then the LM head. Fused (default): q/k/v
+    # share their input and run as one launch, so do gate/up; o and down run alone (4 launches per layer).
+    # --no-fuse: 7 launches per layer.
     groups = [("q",), ("k",), ("v",), ("o",), ("gate",), ("up",), ("down",)] if args.no_fuse else GROUPS
-    flags = 0 if args.no_overlap else vbq.VBQ_LAUNCH_OVERLAP
+
+    def tile_rows(ms):
+        return R if R > 0 else vbq.suggest_tile_rows(sum(m.N for m in ms), ms[0].K, sms)
+
+    def prepare(layer):
+        """Host side of one layer (or the head, layer -1): seeded matrices, packed; logical arrays dropped."""
+        mats = [S.cfg5_head()] if layer < 0 else step_matrices(layer)
+        by_name = {m.name: m for m in mats}
+        out = []
+        for names in ([("head",)] if layer < 0 else groups):
+            ms = [by_name[n] for n in names]
+            rt = tile_rows(ms)
+            blobs = [vbq.vbq_pack(m.N, m.K, rt, m.widths, m.scales, m.codes)[0] for m in ms]
+            x = S.make_x(SYNTH_CFG, names[0], B, ms[0].K, layer=max(layer, 0))
+            out.append((names, rt, [(m.N, m.K) for m in ms], blobs, x))
+        return layer, out
 
     class Group:
         pass
 
-    layers = []   # per copy: list of Group
-    for cp in range(args.copies):
-        by_name = {m.name: m for m in layer_matrices(cp)}
+    def upload(layer, prepared):
         lin = []
-        for names in groups:
+        for names, rt, shapes, blobs, xb in prepared:
             g = Group()
-            g.name = "_".join(names)
-            ms = [by_name[n] for n in names]
-            g.mats = []
-            g.R = R if R > 0 else vbq.suggest_tile_rows(sum(m.N for m in ms), ms[0].K,
-                                                         torch.cuda.get_device_properties(dev).multi_processor_count)
-            for m in ms:
-                blob, _ = vbq.vbq_pack(m.N, m.K, g.R, m.widths, m.scales, m.codes)
-                g.mats.append(vbq.DeviceMatrix(blob, dev, max_batch=B))
-                del blob
-            g.fused = vbq.FusedMatrices(g.mats, max_batch=B) if len(ms) > 1 else None
-            xb = S.make_x(4, names[0], B, ms[0].K, layer=cp)
+            g.name = ("head" if layer < 0 else f"L{layer}.") + ("" if layer < 0 else "_".join(names))
+            g.R = rt
+            g.shapes = shapes
+            g.mats = [vbq.DeviceMatrix(bl, dev, max_batch=B) for bl in blobs]
+            g.fused = vbq.FusedMatrices(g.mats, max_batch=B) if len(g.mats) > 1 else None
             g.xh = torch.from_numpy(xb.astype(np.int16)).view(torch.bfloat16).pin_memory()
             g.xd = g.xh.to(dev)
-            g.yd = [torch.empty((B, m.N), dtype=torch.float32, device=dev) for m in ms]
-            g.yh = [torch.empty((B, m.N), dtype=torch.float32).pin_memory() for m in ms]
-            g.nbytes = sum(mt.nbytes for mt in g.mats) + B * ms[0].K * 2 + sum(B * m.N * 4 for m in ms)
+            g.yd = [torch.empty((B, N), dtype=torch.float32, device=dev) for N, _ in shapes]
+            g.yh = [torch.empty((B, N), dtype=torch.float32).pin_memory() for N, _ in shapes]
+            g.nbytes = sum(mt.nbytes for mt in g.mats) + B * shapes[0][1] * 2 + sum(B * N * 4 for N, _ in shapes)
             g.h = None
             g.x_from_device = False
             lin.append(g)
         # The MLP runs as a chain: the fused gate/up launch writes h = silu(gate) * up (bf16) through its SwiGLU
         # epilogue straight into the down projection's input.
-        names = [g.name for g in lin]
-        if not args.no_fuse and "gate_up" in names and "down" in names:
+        names = [g.name.split(".")[-1] for g in lin]
+        if "gate_up" in names and "down" in names:
             gu, dn = lin[names.index("gate_up")], lin[names.index("down")]
             gu.h = dn.xd
             gu.nbytes += dn.xd.numel() * 2
             dn.x_from_device = True
-        layers.append(lin)
-    step_bytes = [sum(g.nbytes for g in lin) for lin in layers]
+        return lin
+
+    # Host preparation runs on a few threads (the packer and most of the generator release the GIL); device
+    # uploads stay on this thread, in layer order.
+    order = list(range(args.layers)) + ([-1] if not args.no_head else [])
+    step = []
+    t_setup = time.perf_counter()
+    with cf.ThreadPoolExecutor(max_workers=min(4, os.cpu_count() or 1)) as pool:
+        for layer, prepared in pool.map(prepare, order):
+            step.extend(upload(layer, prepared))
+    t_setup = time.perf_counter() - t_setup
+    step_bytes = sum(g.nbytes for g in step)
+    flags = 0 if args.no_overlap else vbq.VBQ_LAUNCH_OVERLAP
 
     def launch(g, st):
         if g.h is not None:
@@ -264,44 +309,40 @@ def run_vbq(args):
             mat = g.mats[0]
             vbq.vbq_gemm_skinny_ex(mat.desc, mat.blob, g.xd, B, g.yd[0], mat.workspaces[B], flags, st)
 
-    # One CUDA graph per layer copy, so that the timed region has no host launch gaps: device-resident step
-    # and end-to-end step (pinned x -> device, the launches, y -> pinned host).
+    # One CUDA graph per step, so that the timed region has no host launch gaps: the device-resident step and
+    # the end-to-end step (each linear's x from pinned host memory to the device, the launches, every y back).
     stream = torch.cuda.Stream(dev)
-    graphs, graphs_e2e = [], []
     with torch.cuda.stream(stream):
-        for lin in layers:
-            for g in lin:
-                launch(g, stream)
+        for g in step:
+            launch(g, stream)
         torch.cuda.synchronize()
-        for lin in layers:
-            gr = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(gr, stream=stream):
-                for g in lin:
-                    launch(g, stream)
-            graphs.append(gr)
-            g2 = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g2, stream=stream):
-                for g in lin:
-                    if not g.x_from_device:
-                        g.xd.copy_(g.xh, non_blocking=True)
-                    launch(g, stream)
-                    for yd, yh in zip(g.yd, g.yh):
-                        yh.copy_(yd, non_blocking=True)
-            graphs_e2e.append(g2)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream):
+            for g in step:
+                launch(g, stream)
+        graph_e2e = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph_e2e, stream=stream):
+            for g in step:
+                if not g.x_from_device:
+                    g.xd.copy_(g.xh, non_blocking=True)
+                launch(g, stream)
+                for yd, yh in zip(g.yd, g.yh):
+                    yh.copy_(yd, non_blocking=True)
     torch.cuda.synchronize()
-    launches_per_step = len(groups)
+    launches_per_step = len(step)
 
-    def timed(gs):
-        for i in range(args.warmup):
-            gs[i % args.copies].replay()
+    def timed(gr):
+        with torch.cuda.stream(stream):
+            for _ in range(args.warmup):
+                gr.replay()
         torch.cuda.synchronize()
         barrier(world)
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         with torch.cuda.stream(stream):
             e0.record(stream)
-            for i in range(args.steps):
-                gs[i % args.copies].replay()
+            for _ in range(args.steps):
+                gr.replay()
             e1.record(stream)
         torch.cuda.synchronize()
         barrier(world)
@@ -310,18 +351,21 @@ def run_vbq(args):
     sampler = ClockSampler(local)
     sampler.start()
     time.sleep(0.3)
-    ms = timed(graphs)
+    ms = timed(graph)
     clocks = sampler.stop()
-    total_bytes = sum(step_bytes[i % args.copies] for i in range(args.steps))
     ms_max = allreduce_max(ms, world)
-    value = total_bytes * world / (ms_max / 1e3) / 1e9
+    value = step_bytes * args.steps * world / (ms_max / 1e3) / 1e9
     launch_ms = ms / (args.steps * launches_per_step)
-    launch_bytes = total_bytes / (args.steps * launches_per_step)
+    launch_bytes = step_bytes / launches_per_step
 
-    # Per-launch-group kernel time: one graph of `reps` launches of that group, timed alone (copy 0).
+    # Per launch group of one representative layer (layer 1 when there is one: layer 0's MLP uses the first-block
+    # mix) and the head: one graph of `reps` launches of that group alone, L2-warm.
+    rep_layer = "L1." if args.layers > 1 else "L0."
     per_shape = {}
     reps = 20
-    for g in layers[0]:
+    for g in step:
+        if not (g.name.startswith(rep_layer) or g.name == "head"):
+            continue
         with torch.cuda.stream(stream):
             gl = torch.cuda.CUDAGraph()
             with torch.cuda.graph(gl, stream=stream):
@@ -339,44 +383,88 @@ def run_vbq(args):
         per_shape[g.name] = {"us": us, "GBps": g.nbytes / (us / 1e6) / 1e9, "note": "same launch repeated (L2-warm)"}
 
     # End to end through host buffers.
-    h2d = sum(g.xh.numel() * 2 for g in layers[0] if not g.x_from_device)
-    d2h = sum(sum(y.numel() * 4 for y in g.yh) for g in layers[0])
-    e2e_ms = allreduce_max(timed(graphs_e2e), world)
-    e2e_val = total_bytes * world / (e2e_ms / 1e3) / 1e9
+    h2d = sum(g.xh.numel() * 2 for g in step if not g.x_from_device)
+    d2h = sum(sum(y.numel() * 4 for y in g.yh) for g in step)
+    e2e_ms = allreduce_max(timed(graph_e2e), world)
+    e2e_val = step_bytes * args.steps * world / (e2e_ms / 1e3) / 1e9
     n_launches = args.steps * launches_per_step
+
+    # Reference point: the same linears as dense FP16 weights through cuBLAS (torch.matmul, one launch per linear),
+    # captured in one CUDA graph per step and timed the same way. Weights and activations are random on the device.
+    fp16 = None
+    if not args.no_fp16_ref:
+        shapes = [sh for g in step for sh in g.shapes]
+        Ws = [torch.empty((N, K), dtype=torch.float16, device=dev).normal_(0.0, 0.02) for N, K in shapes]
+        xs = [torch.randn((B, K), dtype=torch.float16, device=dev) for _, K in shapes]
+        ys = [torch.empty((B, N), dtype=torch.float16, device=dev) for N, _ in shapes]
+        with torch.cuda.stream(stream):
+            for W, xx, yy in zip(Ws, xs, ys):
+                torch.matmul(xx, W.t(), out=yy)
+            torch.cuda.synchronize()
+            g16 = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g16, stream=stream):
+                for W, xx, yy in zip(Ws, xs, ys):
+                    torch.matmul(xx, W.t(), out=yy)
+        torch.cuda.synchronize()
+        ms16 = allreduce_max(timed(g16), world)
+        b16 = sum(N * K * 2 + B * K * 2 + B * N * 2 for N, K in shapes)
+        fp16 = {"value": b16 * args.steps * world / (ms16 / 1e3) / 1e9, "unit": UNIT,
+                "us_per_token": 1e3 * ms16 / args.steps, "weight_bytes_per_step": sum(N * K * 2 for N, K in shapes),
+                "launch": f"torch.matmul (cuBLAS), {len(shapes)} launches per step in one CUDA graph",
+                "vbq_speedup": ms16 / ms_max}
+        del g16, Ws, xs, ys
+        torch.cuda.empty_cache()
+
+    traffic = None
+    if (B == 1 and not args.no_fuse and {g.name.split(".")[-1]: g.R for g in step} == NCU_TRAFFIC["tile_rows"]
+            and kernel_source_sha256() == NCU_TRAFFIC["kernel_source_sha256"]):
+        traffic = launch_bytes * NCU_TRAFFIC["dram_bytes"] / NCU_TRAFFIC["algorithmic_bytes"]
 
     if rank == 0:
         peak, peak_kind = peaks()
         achieved = launch_bytes / (launch_ms / 1e3) / 1e9
         cpu = cpu_baseline(B, args.cpu_budget) if (world == 1 and args.cpu_budget > 0) else None
+        l2_bytes = 126e6
+        workload = WORKLOAD if (args.layers == 32 and not args.no_head) else (
+            f"{args.layers} of the 32 layers of the 9B-shaped decode step" + ("" if args.no_head else " plus the LM head"))
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "fp32", "data": "synthetic",
-            "config": {"workload": WORKLOAD, "batch": B,
-                       "tile_rows": {g.name: g.R for g in layers[0]},
+            "config": {"workload": workload, "batch": B, "layers": args.layers, "lm_head": not args.no_head,
+                       "us_per_token": 1e3 * ms_max / args.steps,
+                       "weight_bytes_per_step": sum(sum(mt.nbytes for mt in g.mats) for g in step),
+                       "tile_rows": {g.name.split(".")[-1]: g.R for g in step},
                        "launch": ("plain" if args.no_overlap else "programmatic dependent launch (VBQ_LAUNCH_OVERLAP)")
                                  + ("; one launch per linear" if args.no_fuse
                                     else "; q/k/v fused (vbq_gemm_skinny_multi); gate/up fused with the SwiGLU "
                                          "epilogue (vbq_gemm_swiglu) writing the down projection's input; "
-                                         "4 launches per layer"),
-                       "weights": "seeded synthetic VBQ groups: P(1,2,4,8 bit) = (0.69,0.16,0.09,0.06), fp16 "
-                                  "scales U(0.01,0.1), uniform codes; x ~ N(0,1) bf16",
-                       "l2": f"inputs larger than L2: {args.copies} distinct layer copies in rotation "
-                             f"({sum(step_bytes) / 1e6:.0f} MB of weights)",
+                                         f"{launches_per_step} launches per step"),
+                       "weights": "seeded synthetic VBQ groups: P(1,2,4,8 bit) = (0.69,0.16,0.09,0.06), layer 0's "
+                                  "MLP (0.40,0.35,0.15,0.10), LM head tiered to ~1.09 bits; fp16 scales "
+                                  "U(0.01,0.1), uniform codes; x ~ N(0,1) bf16, one seeded x per linear",
+                       "l2": (f"inputs larger than L2: {step_bytes / 1e6:.0f} MB of distinct weights streamed once per "
+                              "step" if step_bytes > 2 * l2_bytes else
+                              f"inputs NOT larger than L2 ({step_bytes / 1e6:.0f} MB): L2-warm, not an HBM figure"),
+                       "setup_s": round(t_setup, 1),
                        "parallelism": f"replicas x{world}"},
             "pct_of_peak": 100.0 * value / world / peak,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak, "traffic": None, "peak_kind": peak_kind,
+                         "frac": achieved / peak, "traffic": traffic, "peak_kind": peak_kind,
+                         "traffic_source": (f"ncu capture of {NCU_TRAFFIC['launches']} launches (layer 0 and the LM "
+                                            "head), scaled to this step's bytes per launch; "
+                                            + NCU_TRAFFIC["summary"]) if traffic is not None else None,
                          "kernel": f"vbq_kernel<{B}>",
                          "algorithmic_bytes_per_launch": launch_bytes, "avg_launch_us": launch_ms * 1e3},
             "per_launch_group": per_shape,
             "e2e": {"value": e2e_val, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "fp16_cublas_reference": fp16,
             "gpu_launches": n_launches,
             "clocks": clocks,
             "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
+    del graph, graph_e2e
     if world > 1:
         import torch.distributed as dist
         barrier(world)
@@ -386,11 +474,14 @@ def run_vbq(args):
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--batch", type=int, default=1, choices=(1, 2, 4, 8, 16))
     ap.add_argument("--impl", default="vbq", choices=("vbq", "reference"))
-    ap.add_argument("--copies", type=int, default=4)
+    ap.add_argument("--layers", type=int, default=32, help="decoder layers in the step (1..32)")
+    ap.add_argument("--no-head", action="store_true", help="leave the LM head out of the step")
+    ap.add_argument("--no-fp16-ref", action="store_true",
+                    help="skip the dense FP16 cuBLAS reference point (same shapes, same timing)")
     ap.add_argument("--tile-rows", type=int, default=0,
                     help="tile rows for packing; 0: per launch group, vbq.suggest_tile_rows")
     ap.add_argument("--no-fuse", action="store_true",
@@ -402,6 +493,8 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
+    if not 1 <= args.layers <= 32:
+        ap.error("--layers must be in 1..32")
     if args.impl == "reference":
         run_reference(args)
     else:

@@ -739,12 +739,13 @@ __global__ void __launch_bounds__(Cfg<B>::kThreads, 1) vbq_kernel(const __grid_c
           const uint2 v2 = lds64(sa + 8 + 8 * lane);
           v = (unsigned long long)v2.x | ((unsigned long long)v2.y << 32);
         }
-        const unsigned long long lo = v & 0x5555555555555555ull, hi = (v >> 1) & 0x5555555555555555ull;
+        // bit r of lo / hi: the low / high bit of row r's width code
+        const uint32_t lo = even_bits(v), hi = even_bits(v >> 1);
         const uint32_t valid = nvalid >= 32 ? 0xFFFFFFFFu : ((1u << nvalid) - 1u);
-        m0 = even_bits(~hi & ~lo) & valid;
-        m1 = even_bits(~hi & lo) & valid;
-        m2 = even_bits(hi & ~lo) & valid;
-        m3 = even_bits(hi & lo) & valid;
+        m0 = ~hi & ~lo & valid;
+        m1 = ~hi & lo & valid;
+        m2 = hi & ~lo & valid;
+        m3 = hi & lo & valid;
         const unsigned long long mine = (unsigned long long)__popc(m0) | ((unsigned long long)__popc(m1) << 16) |
                                         ((unsigned long long)__popc(m2) << 32) |
                                         ((unsigned long long)__popc(m3) << 48);

@@ -27,10 +27,15 @@ DEFAULT_TILE_ROWS = 256
 
 def suggest_tile_rows(rows: int, K: int, sms: int = 148) -> int:
     """Tile rows for packing a matrix (or the matrices of one fused launch, `rows` in total) on a GPU with `sms`
-    SMs: 256 unless that leaves fewer than 10 records per SM, then 512 (on B200, 512-row tiles run a 4096x4096
-    GEMV in 17.9 us against 20.5 us, while 256-row tiles win for the 14336-row and K=14336 projections)."""
+    SMs, for batch 1: 224 unless 256-row tiles would leave fewer than 10 records per SM, then 512.
+
+    From a sweep of 128..512-row tiles over the 9B-shaped launch groups on B200 (graph-timed, batch 1):
+    224-row tiles ran fused q/k/v in 21.1 us (256: 21.2), fused gate/up with the SwiGLU epilogue in 37.2 us
+    (38.5), down in 21.4 us (21.8) and the 32000-row LM head in 42.6 us (43.8); 512-row tiles ran the lone
+    4096x4096 projection in 15.3 us (256: 17.5). At 224 rows, sixteen single-warp teams with two record stages
+    each fit in shared memory for these width mixes; at 256 only fifteen do."""
     records = -(-rows // 256) * (K // 64)
-    return 512 if records < 10 * sms else 256
+    return 512 if records < 10 * sms else 224
 
 
 class VbqError(RuntimeError):

@@ -245,3 +245,16 @@ def test_symmetric_grid_pack_unpack_and_errors():
     assert vbq.vbq_quantize_status(nan, widths, 0)[0] == vbq.VBQ_ERR_VALUE
     assert vbq.vbq_quantize_status(np.full((1, 64), 1e38, np.float32), np.full((1, 1), 2, np.uint8), 0)[0] \
         == vbq.VBQ_ERR_VALUE
+
+
+def test_suggest_tile_rows_rule():
+    # 512-row tiles when 256-row tiles would leave fewer than 10 records per SM, else 224
+    assert vbq.suggest_tile_rows(4096, 4096, 148) == 512
+    assert vbq.suggest_tile_rows(3 * 4096, 4096, 148) == 224
+    assert vbq.suggest_tile_rows(2 * 14336, 4096, 148) == 224
+    assert vbq.suggest_tile_rows(4096, 14336, 148) == 224
+    assert vbq.suggest_tile_rows(32000, 4096, 148) == 224
+    assert vbq.suggest_tile_rows(768, 768, 148) == 512
+    for rows, K in ((1, 64), (4096, 4096), (32000, 4096)):
+        R = vbq.suggest_tile_rows(rows, K, 148)
+        assert 16 <= R <= 1024 and R % 16 == 0

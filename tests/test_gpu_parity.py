@@ -58,7 +58,7 @@ def logical(seed, N, K, p):
 
 
 SMALL = [(1, 64, 16), (31, 192, 16), (100, 768, 64), (1030, 256, 1024), (2100, 128, 512), (64, 1024, 32),
-         (777, 2048, 256)]
+         (777, 2048, 256), (1000, 512, 208), (3000, 1024, 224)]
 DISTS = {"base": S.P_BASE, "flat": (0.25, 0.25, 0.25, 0.25), "all8": (0, 0, 0, 1.0), "all1": (1.0, 0, 0, 0)}
 
 
