@@ -174,13 +174,20 @@ def dist_setup():
 
 
 def allreduce_max(v: float, world: int) -> float:
+    """The largest v over the ranks (the job's time is its slowest rank's)."""
     if world == 1:
         return v
     import torch
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    t = torch.tensor([v], dtype=torch.float64, device="cuda" if dist.get_backend() == "nccl" else "cpu")
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_gbps(bytes_per_step: float, steps: int, world: int, ms_max: float) -> float:
+    """Aggregate throughput of `world` replicas that each move `bytes_per_step` per step for `steps` steps, over
+    the slowest rank's time."""
+    return bytes_per_step * steps * world / (ms_max / 1e3) / 1e9
 
 
 def barrier(world: int):
@@ -354,7 +361,7 @@ def run_vbq(args):
     ms = timed(graph)
     clocks = sampler.stop()
     ms_max = allreduce_max(ms, world)
-    value = step_bytes * args.steps * world / (ms_max / 1e3) / 1e9
+    value = whole_job_gbps(step_bytes, args.steps, world, ms_max)
     launch_ms = ms / (args.steps * launches_per_step)
     launch_bytes = step_bytes / launches_per_step
 
@@ -386,7 +393,7 @@ def run_vbq(args):
     h2d = sum(g.xh.numel() * 2 for g in step if not g.x_from_device)
     d2h = sum(sum(y.numel() * 4 for y in g.yh) for g in step)
     e2e_ms = allreduce_max(timed(graph_e2e), world)
-    e2e_val = step_bytes * args.steps * world / (e2e_ms / 1e3) / 1e9
+    e2e_val = whole_job_gbps(step_bytes, args.steps, world, e2e_ms)
     n_launches = args.steps * launches_per_step
 
     # Reference point: the same linears as dense FP16 weights through cuBLAS (torch.matmul, one launch per linear),
@@ -408,7 +415,7 @@ def run_vbq(args):
         torch.cuda.synchronize()
         ms16 = allreduce_max(timed(g16), world)
         b16 = sum(N * K * 2 + B * K * 2 + B * N * 2 for N, K in shapes)
-        fp16 = {"value": b16 * args.steps * world / (ms16 / 1e3) / 1e9, "unit": UNIT,
+        fp16 = {"value": whole_job_gbps(b16, args.steps, world, ms16), "unit": UNIT,
                 "us_per_token": 1e3 * ms16 / args.steps, "weight_bytes_per_step": sum(N * K * 2 for N, K in shapes),
                 "launch": f"torch.matmul (cuBLAS), {len(shapes)} launches per step in one CUDA graph",
                 "vbq_speedup": ms16 / ms_max}

@@ -42,3 +42,36 @@ def test_argument_checks():
     for bad in (["--warmup", "2"], ["--layers", "0"], ["--layers", "33"], ["--batch", "3"]):
         r = _run(bad, timeout=120)
         assert r.returncode == 2, (bad, r.stderr)
+
+
+def _replica_rank(rank, world, port, times, out):
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import bench
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world)
+    try:
+        bench.barrier(world)
+        ms_max = bench.allreduce_max(times[rank], world)
+        out[rank] = (ms_max, bench.whole_job_gbps(1e9, 10, world, ms_max))
+        bench.barrier(world)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_replica_timing_is_the_slowest_rank_over_gloo():
+    """The N > 1 host logic on CPU (gloo, 2 ranks): every rank sees the slowest rank's time, and the whole-job
+    value counts both ranks' bytes over that time."""
+    import socket
+    import torch.multiprocessing as mp
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    times = [120.0, 200.0]
+    with mp.Manager() as mgr:
+        out = mgr.dict()
+        mp.start_processes(_replica_rank, args=(2, port, times, out), nprocs=2, join=True, start_method="spawn")
+        res = dict(out)
+    for rank in (0, 1):
+        ms_max, gbps = res[rank]
+        assert ms_max == 200.0
+        assert abs(gbps - 1e9 * 10 * 2 / 0.2 / 1e9) < 1e-9

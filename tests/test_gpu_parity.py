@@ -449,3 +449,107 @@ def test_quantize_pack_gemv_pipeline(B):
         y, _ = gpu_y(m, x, mat=mat)
         yref, bound = O.matvec(widths, scales, codes, x, NTH, flags=flags)
         check(y, yref, bound, f"quantize pipeline flags={flags} B={B}")
+
+
+def test_decode_step_in_the_bench_launch_configuration():
+    """Two layers of the 9B-shaped decode step (layer 0 at the first-block MLP mix, layer 1 at the base mix) and
+    the LM head, packed with vbq.suggest_tile_rows and launched as the bench times them: fused q/k/v, o, fused
+    gate/up whose SwiGLU epilogue writes down's input, down, then the head, chained by programmatic dependent
+    launch inside one CUDA graph at batch 1. Sampled rows of every output against the oracle. Down reads the
+    epilogue's bf16 h, so its bar adds the propagated h bar: with E = sum |w| bar_h and A = sum |w||h_ref|,
+    |y - y_ref| <= 1e-3 (A + E) + 1e-6 + E. A second replay must reproduce every output bit for bit."""
+    import torch
+    d = dev()
+    sms = torch.cuda.get_device_properties(d).multi_processor_count
+    B, flags = 1, vbq.VBQ_LAUNCH_OVERLAP
+    rng = np.random.default_rng(5)
+    launches, checks = [], []
+
+    def rows_of(N, R):
+        extra = [r for r in (0, R - 1, R, N - 1) if 0 <= r < N]
+        return np.unique(np.concatenate([rng.choice(N, 120, replace=False), extra]))
+
+    def add_group(ms, x_bits, h=None, x_dev=None):
+        R = vbq.suggest_tile_rows(sum(m.N for m in ms), ms[0].K, sms)
+        mats = [vbq.DeviceMatrix(vbq.vbq_pack(m.N, m.K, R, m.widths, m.scales, m.codes)[0], d, max_batch=B)
+                for m in ms]
+        fused = vbq.FusedMatrices(mats, max_batch=B) if len(mats) > 1 else None
+        xd = x_dev if x_dev is not None else to_dev_x(x_bits)
+        ys = [torch.empty((B, m.N), dtype=torch.float32, device=d) for m in ms]
+
+        def run(st):
+            if h is not None:
+                fused.swiglu(xd, ys, h, flags, st)
+            elif fused is not None:
+                fused.matmul(xd, ys, flags, st)
+            else:
+                vbq.vbq_gemm_skinny_ex(mats[0].desc, mats[0].blob, xd, B, ys[0], mats[0].workspaces[B], flags, st)
+
+        def status():
+            if fused is not None:
+                return fused_status(fused, B)
+            ws, need = mats[0].workspaces[B], vbq.vbq_workspace_size(mats[0].desc, B)
+            return int(ws[need - 4:need].cpu().numpy().view(np.uint32)[0])
+
+        launches.append((run, status))
+        return R, ys
+
+    for layer in (0, 1):
+        ms = {m.name: m for m in S.cfg5_layer(layer)}
+        for names in (("q", "k", "v"), ("o",)):
+            x = S.make_x(5, names[0], B, 4096, layer=layer)
+            R, ys = add_group([ms[n] for n in names], x)
+            checks += [("plain", ms[n], x, R, y, f"layer {layer} {n}") for n, y in zip(names, ys)]
+        h = torch.empty((B, ms["down"].K), dtype=torch.bfloat16, device=d)
+        x = S.make_x(5, "gate", B, 4096, layer=layer)
+        R, (yg, yu) = add_group([ms["gate"], ms["up"]], x, h=h)
+        checks += [("plain", ms["gate"], x, R, yg, f"layer {layer} gate"),
+                   ("plain", ms["up"], x, R, yu, f"layer {layer} up"),
+                   ("down", (ms["gate"], ms["up"], ms["down"]), x, None, h, f"layer {layer} h and down")]
+        R, (yd,) = add_group([ms["down"]], None, x_dev=h)
+        checks[-1] = checks[-1][:3] + (R, (h, yd), checks[-1][5])
+    head = S.cfg5_head()
+    x = S.make_x(5, "head", B, 4096)
+    R, (yh,) = add_group([head], x)
+    checks.append(("plain", head, x, R, yh, "LM head"))
+
+    st = torch.cuda.Stream(d)
+    with torch.cuda.stream(st):
+        for run, _ in launches:
+            run(st)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=st):
+            for run, _ in launches:
+                run(st)
+        g.replay()
+        torch.cuda.synchronize()
+        first = [c[4].clone() if c[0] == "plain" else (c[4][0].clone(), c[4][1].clone()) for c in checks]
+        g.replay()
+    torch.cuda.synchronize()
+    for (_, status) in launches:
+        assert status() == 0
+    for c, f in zip(checks, first):
+        if c[0] == "plain":
+            assert torch.equal(c[4], f), f"{c[5]}: second replay differs"
+        else:
+            assert torch.equal(c[4][0], f[0]) and torch.equal(c[4][1], f[1]), f"{c[5]}: second replay differs"
+
+    for kind, m, x, R, out, what in checks:
+        if kind == "plain":
+            rows = rows_of(m.N, R)
+            yref, bound = O.matvec(m.widths[rows], m.scales[rows], m.codes[rows], x, NTH)
+            check(out.cpu().numpy().astype(np.float64)[:, rows], yref, bound, what)
+            continue
+        g_m, u_m, d_m = m
+        h, yd = out
+        g_ref, bg = O.matvec(g_m.widths, g_m.scales, g_m.codes, x, NTH)
+        u_ref, bu = O.matvec(u_m.widths, u_m.scales, u_m.codes, x, NTH)
+        check_swiglu(bf16_to_f64(h), g_ref, u_ref, bg, bu, what + " (h)")
+        h_ref, bar_h = O.swiglu(g_ref, u_ref)[0], O.swiglu_bound(g_ref, u_ref, bg, bu)[0]
+        rows = rows_of(d_m.N, R)
+        W = O.dequant(d_m.widths[rows], d_m.scales[rows], d_m.codes[rows])
+        y_ref, A, E = W @ h_ref, np.abs(W) @ np.abs(h_ref), np.abs(W) @ bar_h
+        got = yd.cpu().numpy().astype(np.float64)[0, rows]
+        bad = np.abs(got - y_ref) > 1e-3 * (A + E) + 1e-6 + E
+        assert not bad.any(), f"{what} (down): {int(bad.sum())} rows out of bar; first row {rows[bad][0]}"
