@@ -46,9 +46,9 @@ SYNTH_CFG = 5   # seed family of the full decode-step stack in vbq_synth
 # this step's algorithmic bytes per launch (traffic grows in proportion: the five launches span 4.5 to 41 MB, each
 # at 0.999 to 1.019 times its algorithmic bytes), and only while the kernel source and the tile rows are the
 # captured ones.
-NCU_TRAFFIC = {"kernel_source_sha256": "2c3dd4e2525fd0eaf6a70ee76e2fea95a04a6b70d546c0374438288f0e54478d",
+NCU_TRAFFIC = {"kernel_source_sha256": "317a63a4cb9a58463de9a0201e351eefe7d512cb85c8aa762cac2f6451f45a36",
                "tile_rows": {"q_k_v": 224, "o": 512, "gate_up": 224, "down": 224, "head": 224},
-               "dram_bytes": 102596864, "algorithmic_bytes": 102422912, "launches": 5,
+               "dram_bytes": 102602752, "algorithmic_bytes": 102422912, "launches": 5,
                "summary": "profiles/vbq_kernel_b1_decode_step_9b_launches.md"}
 
 

@@ -46,9 +46,9 @@ constexpr unsigned kStatusTimeout = 1u, kStatusOversize = 2u, kStatusRecord = 4u
 template <int B> struct Cfg {
   static constexpr int kWarps = (B == 1) ? 16 : (B < 8 ? 12 : 8);
   static constexpr int kThreads = kWarps * 32;
-  // per-warp activation buffer: B=1: x, x*2^-shift for 2-bit codes, x*2^-shift for 4-bit codes (fp32);
-  // B=2,4: fp32 [64][B]; B=8,16: the bf16 A tile of the tensor-core path, [32][kAStride]
-  static constexpr int kXBytes = (B == 1) ? 3 * 64 * 4 : (B < 8 ? 64 * B * 4 : 32 * kAStride * 2);
+  // per-warp activation buffer: B <= 4: three fp32 tables [3][B][64]: x, x*2^-shift for 2-bit codes,
+  // x*2^-shift for 4-bit codes; B=8,16: the bf16 A tile of the tensor-core path, [32][kAStride]
+  static constexpr int kXBytes = (B <= 4) ? 3 * B * 64 * 4 : 32 * kAStride * 2;
 };
 
 // Up to kMaxMats matrices with the same K and tile rows run as one sequence of records (and row tiles): matrix m
@@ -334,16 +334,20 @@ __device__ __forceinline__ float dot_b8(const uint32_t (&w)[16], const float (&x
   return ((acc0.x + acc0.y) + (acc1.x + acc1.y)) + corr * sg;
 }
 
-// Batch 1, one width bucket: the warp's units of 32 items each (local unit u for u = first, first + TW, ...).
-// Lane = item; the item's result s * dot goes to res[item] (byte addresses: codes, scales, res for item 0 of the
-// bucket). The activations this width needs are loaded into registers from xcopy, unless `load` is false
-// (they are already there).
-template <int KB>
+// Batch B <= 4, one width bucket: the warp's units (local unit u for u = first, first + TW, ...) of 32 / B items
+// each. Lane = item * B + b: the lane computes the dot of its item's group with batch row b of the activations,
+// whose 64 values it holds in registers. The result s * dot goes to res[item][b] (byte addresses: codes, scales
+// and res for item 0 of the bucket; xtab is the activation table this width reads, [B][64] fp32). The
+// activations are loaded into registers unless `load` is false (they are already there). sg = sum of x of row b.
+template <int KB, int B>
 __device__ __forceinline__ void bucket_units(int n, int U, int first, int TW, int lane, uint32_t codes,
-                                             uint32_t scales, uint32_t res, float (&xr)[64], uint32_t xcopy,
+                                             uint32_t scales, uint32_t res, float (&xr)[64], uint32_t xtab,
                                              float sg, bool load, float corr) {
+  constexpr int IPU = 32 / B;  // items per unit
   if (first >= U) return;
+  const int sub = lane / B, b = lane - sub * B;
   if (load) {
+    const uint32_t xcopy = xtab + 256 * b;
 #pragma unroll
     for (int q = 0; q < 16; ++q) {
       const float4 f = lds128f(xcopy + 16 * q);
@@ -351,7 +355,7 @@ __device__ __forceinline__ void bucket_units(int n, int U, int first, int TW, in
     }
   }
   for (int u = first; u < U; u += TW) {
-    const int jj = 32 * u + lane;
+    const int jj = IPU * u + sub;
     if (jj >= n) continue;
     float d;
     if constexpr (KB == 1) {
@@ -361,8 +365,8 @@ __device__ __forceinline__ void bucket_units(int n, int U, int first, int TW, in
       const uint32_t w[4] = {a.x, a.y, a.z, a.w};
       d = dot_magic<2>(w, xr, sg, corr);
     } else if constexpr (KB == 4) {
-      const uint4 a = lds128(codes + 32 * jj), b = lds128(codes + 32 * jj + 16);
-      const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+      const uint4 a = lds128(codes + 32 * jj), c = lds128(codes + 32 * jj + 16);
+      const uint32_t w[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
       d = dot_magic<4>(w, xr, sg, corr);
     } else {
       uint32_t w[16];
@@ -373,7 +377,7 @@ __device__ __forceinline__ void bucket_units(int n, int U, int first, int TW, in
       }
       d = dot_b8(w, xr, sg, corr);
     }
-    sts32f(res + 4 * jj, __half2float(__ushort_as_half((unsigned short)lds16(scales + 2 * jj))) * d);
+    sts32f(res + 4 * (jj * B + b), __half2float(__ushort_as_half((unsigned short)lds16(scales + 2 * jj))) * d);
   }
 }
 // First local unit of a bucket for warp tw of TW, when the bucket's units follow `before` units of the record.
@@ -381,13 +385,6 @@ __device__ __forceinline__ int first_unit(int tw, int before, int TW) {
   if (TW == 1) return 0;
   const int r = (tw - before) % TW;
   return r < 0 ? r + TW : r;
-}
-
-// q - 2^(k-1) of code i from a group's code words in shared memory (any width, runtime index).
-__device__ __forceinline__ float code_centered(const uint32_t* w, int k, int i) {
-  const int bit = k * i;
-  const uint32_t q = (w[bit >> 5] >> (bit & 31)) & ((1u << k) - 1u);
-  return float(int(q) - (1 << (k - 1)));
 }
 
 // Row (within the tile) of item `item` of bucket c. masks[c][w] marks the rows of 32-row word w whose width code
@@ -700,7 +697,7 @@ __global__ void __launch_bounds__(Cfg<B>::kThreads, 1) vbq_kernel(const __grid_c
     };
 
     int cur_t = -1;
-    float xr[B == 1 ? 64 : 1];
+    float xr[B <= 4 ? 64 : 1];
     for (int i = 0; i < nt; ++i) {
       const int s = i % S;
       const unsigned char* st = tbase + s * p.stage_size;
@@ -715,7 +712,7 @@ __global__ void __launch_bounds__(Cfg<B>::kThreads, 1) vbq_kernel(const __grid_c
       if (t != cur_t) {
         if (cur_t >= 0) flush(cur_t);
         for (int e = sl0 * B + lane; e < sl1 * B; e += 32) acc[e] = 0.f;
-        if (B > 1) team_sync(team, TW);
+        if (B >= 8) team_sync(team, TW);  // the tensor-core path accumulates any row of the tile
         cur_t = t;
       }
       int n0 = 0, n1 = 0, n2 = 0, n3 = 0;
@@ -776,26 +773,22 @@ __global__ void __launch_bounds__(Cfg<B>::kThreads, 1) vbq_kernel(const __grid_c
         const uint16_t* xg = reinterpret_cast<const uint16_t*>(st + p.stage_bytes);  // [B][64]
         float* xv = reinterpret_cast<float*>(wbase + wo.x);
         float* sgv = reinterpret_cast<float*>(wbase + wo.sg);
-        if constexpr (B == 1) {
-          const float x0 = __uint_as_float(uint32_t(xg[lane]) << 16);
-          const float x1 = __uint_as_float(uint32_t(xg[32 + lane]) << 16);
-          xv[lane] = x0;
-          xv[32 + lane] = x1;
-          xv[64 + lane] = x0 * __uint_as_float(uint32_t(127 - code_shift<2>(lane)) << 23);
-          xv[96 + lane] = x1 * __uint_as_float(uint32_t(127 - code_shift<2>(32 + lane)) << 23);
-          xv[128 + lane] = x0 * __uint_as_float(uint32_t(127 - code_shift<4>(lane)) << 23);
-          xv[160 + lane] = x1 * __uint_as_float(uint32_t(127 - code_shift<4>(32 + lane)) << 23);
-          float sg = x0 + x1;
-#pragma unroll
-          for (int off = 16; off > 0; off >>= 1) sg += __shfl_xor_sync(0xFFFFFFFFu, sg, off);
-          if (lane == 0) sgv[0] = sg;
-        } else if constexpr (B < 8) {
+        if constexpr (B <= 4) {
+          // tables [3][B][64]: x, x * 2^-shift for 2-bit codes, x * 2^-shift for 4-bit codes; row b's group sum
+          const float s2a = __uint_as_float(uint32_t(127 - code_shift<2>(lane)) << 23);
+          const float s2b = __uint_as_float(uint32_t(127 - code_shift<2>(32 + lane)) << 23);
+          const float s4a = __uint_as_float(uint32_t(127 - code_shift<4>(lane)) << 23);
+          const float s4b = __uint_as_float(uint32_t(127 - code_shift<4>(32 + lane)) << 23);
 #pragma unroll
           for (int b = 0; b < B; ++b) {
             const float x0 = __uint_as_float(uint32_t(xg[b * 64 + lane]) << 16);
             const float x1 = __uint_as_float(uint32_t(xg[b * 64 + 32 + lane]) << 16);
-            xv[lane * B + b] = x0;
-            xv[(32 + lane) * B + b] = x1;
+            xv[b * 64 + lane] = x0;
+            xv[b * 64 + 32 + lane] = x1;
+            xv[(B + b) * 64 + lane] = x0 * s2a;
+            xv[(B + b) * 64 + 32 + lane] = x1 * s2b;
+            xv[(2 * B + b) * 64 + lane] = x0 * s4a;
+            xv[(2 * B + b) * 64 + 32 + lane] = x1 * s4b;
             float sg = x0 + x1;
 #pragma unroll
             for (int off = 16; off > 0; off >>= 1) sg += __shfl_xor_sync(0xFFFFFFFFu, sg, off);
@@ -804,64 +797,25 @@ __global__ void __launch_bounds__(Cfg<B>::kThreads, 1) vbq_kernel(const __grid_c
         }
         __syncwarp();
 
-        if constexpr (B == 1) {
-          // -- batch 1: item results s * dot into the team's result buffer (item order), one bucket at a time.
-          // Units are numbered across the buckets and dealt round-robin to the team's warps.
-          const float sg = sgv[0];
+        if constexpr (B <= 4) {
+          // -- CUDA cores, B <= 4: item results s * dot into the team's result buffer ([item][B], item order),
+          // one bucket at a time; lane = item * B + b. Units of 32 / B items are numbered across the buckets and
+          // dealt round-robin to the team's warps.
+          constexpr int IPU = 32 / B;
+          const float sg = sgv[lane % B];
           const uint32_t xa = smem_u32(xv);
-          const uint32_t ra = smem_u32(tbase + p.res_off) + (TW > 1 ? 4 * R * (i & 1) : 0);
+          const uint32_t ra = smem_u32(tbase + p.res_off) + (TW > 1 ? 4 * R * B * (i & 1) : 0);
           const uint32_t sca = sa + rc.sc;
-          const int U0 = rc.u0, U1 = rc.u1 - rc.u0, U2 = rc.u2 - rc.u1, U3 = rc.U - rc.u2;
+          const int c0 = (n0 + IPU - 1) / IPU, c1 = c0 + (n1 + IPU - 1) / IPU, c2 = c1 + (n2 + IPU - 1) / IPU,
+                    cU = c2 + (n3 + IPU - 1) / IPU;
           // 1-bit and 8-bit units read the same (raw) activations, so they run back to back on one load.
-          bucket_units<1>(n0, U0, first_unit(tw, 0, TW), TW, lane, sa + rc.c0, sca, ra, xr, xa, sg, true, 0.5f);
-          bucket_units<8>(n3, U3, first_unit(tw, rc.u2, TW), TW, lane, sa + rc.c3, sca + 2 * (n0 + n1 + n2),
-                          ra + 4 * (n0 + n1 + n2), xr, xa, sg, first_unit(tw, 0, TW) >= U0, corr);
-          bucket_units<2>(n1, U1, first_unit(tw, rc.u0, TW), TW, lane, sa + rc.c1, sca + 2 * n0, ra + 4 * n0, xr,
-                          xa + 256, sg, true, corr);
-          bucket_units<4>(n2, U2, first_unit(tw, rc.u1, TW), TW, lane, sa + rc.c2, sca + 2 * (n0 + n1),
-                          ra + 4 * (n0 + n1), xr, xa + 512, sg, true, corr);
-        } else if constexpr (B < 8) {
-          // -- CUDA cores, B in {2, 4}: lane = group; activations of all batches broadcast from shared memory
-          const float* xc = xv;
-          for (int u = tw; u < rc.U; u += TW) {
-            int bk, j0, ibase, cbase, nb;
-            rc.unit(u, bk, j0, ibase, cbase, nb);
-            const int jj = j0 + lane;
-            if (jj >= nb) continue;
-            const int k = 1 << bk;
-            const uint32_t* w = reinterpret_cast<const uint32_t*>(st + cbase + 8 * k * jj);
-            float a[B];
-#pragma unroll
-            for (int b = 0; b < B; ++b) a[b] = 0.f;
-            if (bk == 0) {
-              const uint32_t w0 = w[0], w1 = w[1];
-#pragma unroll 8
-              for (int i2 = 0; i2 < 64; ++i2) {
-                if ((i2 < 32 ? w0 : w1) & (1u << (i2 & 31))) {
-#pragma unroll
-                  for (int b = 0; b < B; ++b) a[b] += xc[i2 * B + b];
-                }
-              }
-            } else {
-#pragma unroll 4
-              for (int i2 = 0; i2 < 64; ++i2) {
-                const float qv = code_centered(w, k, i2);
-#pragma unroll
-                for (int b = 0; b < B; ++b) a[b] = fmaf(qv, xc[i2 * B + b], a[b]);
-              }
-            }
-            const int item = ibase + jj;
-            const float sc = __half2float(reinterpret_cast<const __half*>(st + rc.sc)[item]);
-            const int row = item_row(mk, pf, bk, item);
-            // sum (q - 2^(k-1)) x + corr sum x == sum (q - c) x (corr = 1/2 default grid, 1 symmetric grid);
-            // for k = 1 the first sum is sum_{q=1} x - S, and c = 1/2 on both grids.
-#pragma unroll
-            for (int b = 0; b < B; ++b) {
-              const float Sb = sgv[b];
-              const float d = (bk == 0) ? a[b] - 0.5f * Sb : a[b] + corr * Sb;
-              acc[row * B + b] = fmaf(sc, d, acc[row * B + b]);
-            }
-          }
+          bucket_units<1, B>(n0, c0, first_unit(tw, 0, TW), TW, lane, sa + rc.c0, sca, ra, xr, xa, sg, true, 0.5f);
+          bucket_units<8, B>(n3, cU - c2, first_unit(tw, c2, TW), TW, lane, sa + rc.c3, sca + 2 * (n0 + n1 + n2),
+                             ra + 4 * B * (n0 + n1 + n2), xr, xa, sg, first_unit(tw, 0, TW) >= c0, corr);
+          bucket_units<2, B>(n1, c1 - c0, first_unit(tw, c0, TW), TW, lane, sa + rc.c1, sca + 2 * n0,
+                             ra + 4 * B * n0, xr, xa + 256 * B, sg, true, corr);
+          bucket_units<4, B>(n2, c2 - c1, first_unit(tw, c1, TW), TW, lane, sa + rc.c2, sca + 2 * (n0 + n1),
+                             ra + 4 * B * (n0 + n1), xr, xa + 512 * B, sg, true, corr);
         } else {
           // -- tensor cores, B in {8, 16}: lane = group, dequantized to bf16 2(q - c) (2q-(2^k-1) on the default grid,
           // 2q-(2^k-2) on the symmetric one; both exact) in this warp's A tile;
@@ -958,16 +912,17 @@ __global__ void __launch_bounds__(Cfg<B>::kThreads, 1) vbq_kernel(const __grid_c
           ++issued;
         }
       }
-      if constexpr (B == 1) {
+      if constexpr (B <= 4) {
         if (ok) {
-          // -- row pass: row r of this warp's slice takes the result of its item (bucket start for its 32-row
+          // -- row pass: row r of this warp's slice takes the results of its item (bucket start for its 32-row
           // word, plus the rows of the same width before it in that word)
-          const uint32_t ra = smem_u32(tbase + p.res_off) + (TW > 1 ? 4 * R * (i & 1) : 0);
+          const uint32_t ra = smem_u32(tbase + p.res_off) + (TW > 1 ? 4 * R * B * (i & 1) : 0);
           for (int r = sl0 + lane; r < min(sl1, Rt); r += 32) {
             const int cc = int(wd[r >> 4] >> (2 * (r & 15))) & 3;
             const int w = r >> 5;
             const int item = pf[cc * 32 + w] + __popc(mk[cc * 32 + w] & ((1u << (r & 31)) - 1u));
-            acc[r] += lds32f(ra + 4 * item);
+#pragma unroll
+            for (int b = 0; b < B; ++b) acc[r * B + b] += lds32f(ra + 4 * (item * B + b));
           }
         }
       }
@@ -1151,8 +1106,8 @@ inline bool make_plan_t(const Problem& pr, int sms, Plan& pl) {
     const int TW = W / NT;
     if (TW > 1 && NT > 15) continue;  // named barrier ids 1..15
     const int rpt = (rpc + NT - 1) / NT;
-    // batch 1: item results, double-buffered when several warps share a record
-    const int res_bytes = B == 1 ? align128i((TW > 1 ? 2 : 1) * R * 4) : 0;
+    // batch <= 4: item results, double-buffered when several warps share a record
+    const int res_bytes = B <= 4 ? align128i((TW > 1 ? 2 : 1) * R * B * 4) : 0;
     for (int S = min(max(rpt, 1), kMaxStages); S >= 1; --S) {
       const int team_bytes = S * pl.stage_size + acc_bytes + res_bytes;
       const long long smem = (long long)NT * team_bytes + (long long)NT * TW * pl.warp_bytes;
