@@ -46,16 +46,23 @@ SYNTH_CFG = 5   # seed family of the full decode-step stack in vbq_synth
 # this step's algorithmic bytes per launch (traffic grows in proportion: the five launches span 4.5 to 41 MB, each
 # at 0.999 to 1.019 times its algorithmic bytes), and only while the kernel source and the tile rows are the
 # captured ones.
-NCU_TRAFFIC = {"kernel_source_sha256": "317a63a4cb9a58463de9a0201e351eefe7d512cb85c8aa762cac2f6451f45a36",
+NCU_TRAFFIC = {"kernel_source_sha256": "ab72677274a3d1929df24d6f3ee06d44a9ba7e8e192c3bacc0b2db331c08f2b3",
                "tile_rows": {"q_k_v": 224, "o": 512, "gate_up": 224, "down": 224, "head": 224},
                "dram_bytes": 102602752, "algorithmic_bytes": 102422912, "launches": 5,
                "summary": "profiles/vbq_kernel_b1_decode_step_9b_launches.md"}
 
 
 def kernel_source_sha256() -> str:
+    """SHA-256 of the kernel source's code: comments and blank lines removed, so that a comment edit does not
+    void a capture. (A // or /* inside a string literal would be cut too; the kernel source has none.)"""
     import hashlib
-    with open(os.path.join(ROOT, "decode_vbq_gemv_b200", "csrc", "gemv.cu"), "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()
+    import re
+    with open(os.path.join(ROOT, "decode_vbq_gemv_b200", "csrc", "gemv.cu")) as f:
+        src = f.read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", "", src)
+    code = "\n".join(ln.rstrip() for ln in src.splitlines() if ln.strip())
+    return hashlib.sha256(code.encode()).hexdigest()
 
 
 def peaks():

@@ -12,12 +12,12 @@
 //    when it has few). A team owns a contiguous run of the CTA's records, streams them into its own ring of
 //    shared-memory stages with cp.async.bulk (the TMA engine, no multicast) and waits on mbarrier transaction
 //    counts, bounded by a timer; nothing waits on another team or another CTA.
-//  - Inside a team, warps take units of 32 items of one bucket, so every warp instruction runs a single width.
-//    Batch 1: each lane owns one 64-weight group and holds the column's activations in registers. 1-bit groups
-//    add the activations whose bit is set (predicated adds); 2/4-bit groups expand codes with a magic-number
-//    bit-to-float trick against pre-scaled activations; 8-bit groups use byte permutes. Results land in item
-//    order, and a row pass adds them to the tile's rows. Batch 2/4: CUDA cores. Batch 8/16: mma.sync bf16
-//    tensor cores on the exact integers 2q - (2^k - 1).
+//  - Inside a team, warps take units of items of one bucket, so every warp instruction runs a single width.
+//    Batch 1, 2, 4 (CUDA cores): each lane owns one 64-weight group and one batch row (32/B groups per unit) and
+//    holds that row's activations in registers. 1-bit groups add the activations whose bit is set (predicated
+//    adds); 2/4-bit groups expand codes with a magic-number bit-to-float trick against pre-scaled activations;
+//    8-bit groups use byte permutes. Results land in item order, and a row pass adds them to the tile's rows.
+//    Batch 8/16: mma.sync bf16 tensor cores on the exact integers 2(q - c), units of 32 groups.
 //  - Row tiles that several owners share are reduced without floating-point atomics: teams of one CTA that
 //    share a tile are summed in shared memory in team order; CTAs that share a tile write partial sums to the
 //    workspace and count themselves in, and the last to arrive adds all partials in CTA order. Results are
@@ -75,7 +75,7 @@ struct Params {
   int NT, TW, S;           // teams per CTA, warps per team, stages per team
   int stage_bytes;         // record capacity of one stage (multiple of 128)
   int stage_size;          // stage: record, then the column's bf16 activations [B][64]
-  int team_bytes;          // per team: S stages | tile accumulators [R][B] f32 | item results (batch 1, 2 x R f32)
+  int team_bytes;          // per team: S stages | tile accumulators [R][B] f32 | item results (B <= 4, 1-2 x R x B f32)
   int acc_off, res_off;
   int warps_off, warp_bytes;
 };
@@ -901,7 +901,7 @@ __global__ void __launch_bounds__(Cfg<B>::kThreads, 1) vbq_kernel(const __grid_c
           }
         }
       }
-      // every warp of the team is done with stage s (and, for batch 1, has written its item results)
+      // every warp of the team is done with stage s (and, for B <= 4, has written its item results)
       team_sync(team, TW);
       if (tw == 0 && i + S < nt) {
         const int go = __shfl_sync(0xFFFFFFFFu, *abort_flag ? 0 : 1, 0);
