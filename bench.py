@@ -46,9 +46,9 @@ SYNTH_CFG = 5   # seed family of the full decode-step stack in vbq_synth
 # this step's algorithmic bytes per launch (traffic grows in proportion: the five launches span 4.5 to 41 MB, each
 # at 0.999 to 1.019 times its algorithmic bytes), and only while the kernel source and the tile rows are the
 # captured ones.
-NCU_TRAFFIC = {"kernel_source_sha256": "ab72677274a3d1929df24d6f3ee06d44a9ba7e8e192c3bacc0b2db331c08f2b3",
+NCU_TRAFFIC = {"kernel_source_sha256": "d6593dba6f9e3797de02ec23fbc0e6694a6afe2bb7ff84544ee57261af5ffeb1",
                "tile_rows": {"q_k_v": 224, "o": 512, "gate_up": 224, "down": 224, "head": 224},
-               "dram_bytes": 102602752, "algorithmic_bytes": 102422912, "launches": 5,
+               "dram_bytes": 102591232, "algorithmic_bytes": 102422912, "launches": 5,
                "summary": "profiles/vbq_kernel_b1_decode_step_9b_launches.md"}
 
 

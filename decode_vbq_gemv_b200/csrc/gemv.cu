@@ -228,6 +228,10 @@ __device__ __forceinline__ uint32_t lds8(uint32_t a) {
 __device__ __forceinline__ void sts32f(uint32_t a, float v) {
   asm volatile("st.shared.f32 [%0], %1;" ::"r"(a), "f"(v) : "memory");
 }
+__device__ __forceinline__ void sts128(uint32_t a, const uint32_t (&v)[4]) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3])
+               : "memory");
+}
 
 // d = a * b + c on two fp32 lanes at once (sm_100 packed FMA).
 __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
@@ -253,6 +257,7 @@ __device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
 // read from (word >> HI) instead of word.
 template <int KB> struct Magic;
 template <> struct Magic<2> { static constexpr int HI = 10; };
+template <> struct Magic<1> { static constexpr int HI = 9; };
 template <> struct Magic<4> { static constexpr int HI = 12; };
 template <int KB> __host__ __device__ constexpr bool magic_hi(int t) { return KB * t + KB > 23; }
 template <int KB> __host__ __device__ constexpr int magic_shift(int t) {
@@ -332,6 +337,64 @@ __device__ __forceinline__ float dot_b8(const uint32_t (&w)[16], const float (&x
     acc1 = ffma2(q1, make_float2(xr[4 * m + 2], xr[4 * m + 3]), acc1);
   }
   return ((acc0.x + acc0.y) + (acc1.x + acc1.y)) + corr * sg;
+}
+
+// 2^e for a small integer e, exact in fp32.
+__host__ __device__ constexpr float pow2f(int e) { return e >= 0 ? float(1u << e) : 1.0f / float(1u << -e); }
+
+__device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// Tensor-core A row of one KB-bit group: its 64 values 2(q_i - c) as bf16 at byte address arow, from the group's
+// code words at byte address codes; off = 2c. Every value is an integer of magnitude at most 255, so every step
+// is exact: the magic-number expansion gives q * 2^shift (as in the batch-1 loops), one packed FMA scales it by
+// 2^(1 - shift) and subtracts 2c, and bf16 holds the result. 8-bit codes use the byte-permute form.
+template <int KB>
+__device__ __forceinline__ void dequant_a_row(uint32_t codes, uint32_t arow, float off) {
+  uint32_t w[2 * KB];
+  if constexpr (KB == 1) {
+    const uint2 a = lds64(codes);
+    w[0] = a.x; w[1] = a.y;
+  } else {
+#pragma unroll
+    for (int q = 0; q < KB / 2; ++q) {
+      const uint4 a = lds128(codes + 16 * q);
+      w[4 * q] = a.x; w[4 * q + 1] = a.y; w[4 * q + 2] = a.z; w[4 * q + 3] = a.w;
+    }
+  }
+  uint32_t out[4];
+  if constexpr (KB == 8) {
+    const float2 neg = make_float2(-8388736.f, -8388736.f);  // -(2^23 + 128)
+    const float2 two = make_float2(2.f, 2.f), c = make_float2(256.f - off, 256.f - off);
+#pragma unroll
+    for (int m = 0; m < 16; ++m) {
+      const float2 q0 = fadd2(make_float2(__uint_as_float(__byte_perm(w[m], 0x4B000000u, 0x7440u)),
+                                          __uint_as_float(__byte_perm(w[m], 0x4B000000u, 0x7441u))), neg);
+      const float2 q1 = fadd2(make_float2(__uint_as_float(__byte_perm(w[m], 0x4B000000u, 0x7442u)),
+                                          __uint_as_float(__byte_perm(w[m], 0x4B000000u, 0x7443u))), neg);
+      const float2 a0 = ffma2(q0, two, c), a1 = ffma2(q1, two, c);  // 2(q - 128) + 256 - 2c
+      out[(2 * m) & 3] = bf16x2_bits(a0.x, a0.y);
+      out[(2 * m + 1) & 3] = bf16x2_bits(a1.x, a1.y);
+      if (m & 1) sts128(arow + 16 * (m >> 1), out);
+    }
+  } else {
+    constexpr int CPW = 32 / KB;
+    constexpr uint32_t M = (1u << KB) - 1u;
+    const float2 neg = make_float2(-8388608.f, -8388608.f), c = make_float2(-off, -off);
+#pragma unroll
+    for (int i = 0; i < 64; i += 2) {
+      const int m = i / CPW, t = i % CPW;  // codes i and i + 1: positions t and t + 1 of word m
+      const uint32_t lo = w[m], hi = w[m] >> Magic<KB>::HI;
+      const float va = magic_f(magic_hi<KB>(t) ? hi : lo, M << magic_shift<KB>(t));
+      const float vb = magic_f(magic_hi<KB>(t + 1) ? hi : lo, M << magic_shift<KB>(t + 1));
+      const float2 q = fadd2(make_float2(va, vb), neg);  // (q_i 2^shift_i, q_i+1 2^shift_i+1)
+      const float2 a = ffma2(q, make_float2(pow2f(1 - magic_shift<KB>(t)), pow2f(1 - magic_shift<KB>(t + 1))), c);
+      out[(i >> 1) & 3] = bf16x2_bits(a.x, a.y);
+      if (((i >> 1) & 3) == 3) sts128(arow + 16 * (i >> 3), out);
+    }
+  }
 }
 
 // Batch B <= 4, one width bucket: the warp's units (local unit u for u = first, first + TW, ...) of 32 / B items
@@ -838,21 +901,19 @@ __global__ void __launch_bounds__(Cfg<B>::kThreads, 1) vbq_kernel(const __grid_c
             const int k = 1 << bk;
             const int jj = j0 + lane;
             const bool valid = jj < nb;
-            __nv_bfloat162* arow = reinterpret_cast<__nv_bfloat162*>(As + lane * kAStride);
+            const uint32_t ar = smem_u32(As + lane * kAStride);
             if (valid) {
-              const uint32_t* w = reinterpret_cast<const uint32_t*>(st + cbase + 8 * k * jj);
+              const uint32_t cw = sa + uint32_t(cbase + 8 * k * jj);
               const float off = float((1 << k) - 1 - ((grid_sym && k >= 2) ? 1 : 0));  // 2c: A = 2(q - c)
-              const uint32_t mask = (1u << k) - 1u;
-#pragma unroll 8
-              for (int i2 = 0; i2 < 64; i2 += 2) {
-                const int b0 = k * i2, b1 = k * (i2 + 1);
-                const uint32_t q0 = (w[b0 >> 5] >> (b0 & 31)) & mask;
-                const uint32_t q1 = (w[b1 >> 5] >> (b1 & 31)) & mask;
-                arow[i2 >> 1] = __floats2bfloat162_rn(2.f * float(q0) - off, 2.f * float(q1) - off);
-              }
+              // bk is the same for the whole warp (a unit holds one bucket)
+              if (bk == 0) dequant_a_row<1>(cw, ar, off);
+              else if (bk == 1) dequant_a_row<2>(cw, ar, off);
+              else if (bk == 2) dequant_a_row<4>(cw, ar, off);
+              else dequant_a_row<8>(cw, ar, off);
             } else {
+              const uint32_t z[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-              for (int i2 = 0; i2 < 32; ++i2) arow[i2] = __floats2bfloat162_rn(0.f, 0.f);
+              for (int q = 0; q < 8; ++q) sts128(ar + 16 * q, z);
             }
             __syncwarp();
             float scale_mine = 0.f;
