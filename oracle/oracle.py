@@ -7,6 +7,15 @@ The oracle is a plain fp64 CPU implementation of the VBQ dequantize-and-multiply
 ("Variable Bit-width Quantization", section 3.1: 64-weight groups with a per-group scale and a width from
 {1,2,4,8}; section 6, "Fused kernels over packed weights": dequantize per group, then accumulate W x) and
 FORMAT.md for the byte layout.
+
+Pins (tests/test_oracle_pins.py), besides those of the C part:
+- silu: textbook values of the logistic function at 0 and +-1, large-argument limits, and the identity
+  silu(g) - silu(-g) = g;
+- swiglu_bound: admits the bf16 rounding of an exact h;
+- quantize: weights that lie exactly on either grid come back as that scale and those codes; 1-bit groups give
+  sign times the mean magnitude; every dequantized weight lies within half a step of its input (plus the
+  scale's fp16 rounding); all-zero groups decode to zero; non-finite weights and scales beyond fp16 are
+  refused.
 """
 from __future__ import annotations
 
