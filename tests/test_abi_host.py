@@ -258,3 +258,29 @@ def test_suggest_tile_rows_rule():
     for rows, K in ((1, 64), (4096, 4096), (32000, 4096)):
         R = vbq.suggest_tile_rows(rows, K, 148)
         assert 16 <= R <= 1024 and R % 16 == 0
+
+
+def test_pack_and_quantize_are_thread_safe():
+    """The host entry points are pure (the bench packs layers on a thread pool): many threads packing and
+    quantizing different matrices at once give the same bytes as one thread doing it alone."""
+    import concurrent.futures as cf
+    rng = np.random.default_rng(21)
+    cases = []
+    for i in range(12):
+        N, K, R = int(rng.integers(1, 700)), 64 * int(rng.integers(1, 12)), 16 * int(rng.integers(1, 40))
+        m = S.Matrix("t", N, K, S.widths_iid(N, K // 64, S.P_BASE, rng), S.scales_uniform(N, K // 64, rng),
+                     np.zeros((N, K), np.uint8))
+        m.codes[:] = S.codes_uniform(m.widths, rng)
+        w = rng.normal(0, 0.05, size=(N, K)).astype(np.float32)
+        cases.append((m, R, w))
+
+    def work(c):
+        m, R, w = c
+        blob, _ = vbq.vbq_pack(m.N, m.K, R, m.widths, m.scales, m.codes)
+        sc, co = vbq.vbq_quantize(w, m.widths)
+        return blob.tobytes(), sc.tobytes(), co.tobytes()
+
+    alone = [work(c) for c in cases]
+    with cf.ThreadPoolExecutor(max_workers=8) as pool:
+        for _ in range(3):
+            assert list(pool.map(work, cases)) == alone

@@ -75,3 +75,23 @@ def test_replica_timing_is_the_slowest_rank_over_gloo():
         ms_max, gbps = res[rank]
         assert ms_max == 200.0
         assert abs(gbps - 1e9 * 10 * 2 / 0.2 / 1e9) < 1e-9
+
+
+def test_kernel_source_hash_ignores_comments_only():
+    """The bench keys its ncu traffic capture to the kernel source's code: comment and blank-line edits keep the
+    key, any code edit changes it."""
+    import hashlib
+    import re
+    sys.path.insert(0, ROOT)
+    import bench
+
+    def key(src):
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        src = re.sub(r"//[^\n]*", "", src)
+        return hashlib.sha256("\n".join(ln.rstrip() for ln in src.splitlines() if ln.strip()).encode()).hexdigest()
+
+    with open(os.path.join(ROOT, "decode_vbq_gemv_b200", "csrc", "gemv.cu")) as f:
+        src = f.read()
+    assert bench.kernel_source_sha256() == key(src)
+    assert key("// note\nint a;\n\n/* block\n comment */ int b;  // tail\n") == key("int a;\n int b;\n")
+    assert key("int a = 1;\n") != key("int a = 2;\n")
