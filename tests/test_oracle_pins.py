@@ -3,8 +3,8 @@
 - float decoders: numpy's binary16 and torch's bfloat16 conversions, over all 65536 bit patterns;
 - CRC-32: the published check value and zlib;
 - packing: the hand-derived golden blob of FORMAT.md's worked example, and a single-code bit-position sweep;
-- matvec: exact rational arithmetic on tiny shapes, closed forms on uniform widths, one-hot columns, and exact
-  power-of-two scale invariance.
+- matvec: exact rational arithmetic on tiny shapes, closed forms on uniform widths, one-hot columns, exact
+  power-of-two scale invariance, and numpy's BLAS on weights rebuilt from the definition.
 
 The method follows the VBQ paper ("Variable Bit-width Quantization", section 3.1, groups of 64 with a per-group
 scale and width from {1,2,4,8}; section 6, "Fused kernels over packed weights").
@@ -292,6 +292,25 @@ def test_power_of_two_scale_invariance():
     assert np.array_equal(f16(s2), 2 * f16(s))
     y2, a2 = O.matvec(w, s2, c, x)
     assert np.array_equal(y2, 2 * y1) and np.array_equal(a2, 2 * a1)
+
+
+def test_matvec_against_an_independent_library_matmul():
+    """T12, on the host: the weights rebuilt with numpy straight from the definition (fp16 scale times
+    q - (2^k - 1)/2, no oracle code) and multiplied by numpy's BLAS. In fp64 the two sums differ only by
+    rounding order (1e-12 of sum |w||x|); in fp32, BLAS stays inside the parity bar, as a fp32 kernel must."""
+    g = np.random.default_rng(12)
+    N, K, B = 384, 4096, 3
+    w, s, c = random_logical(g, N, K)
+    x = S.x_normal(B, K, g)
+    y_ref, a = O.matvec(w, s, c, x, os.cpu_count() or 1)
+    kk = np.repeat(w.astype(np.int64), 64, axis=1)
+    W = np.repeat(f16(s), 64, axis=1) * (c.astype(np.float64) - ((1 << kk) - 1) / 2)
+    X = bf16(x)
+    y64 = X @ W.T
+    assert np.all(np.abs(y64 - y_ref) <= 1e-12 * a + 1e-300)
+    y32 = (X.astype(np.float32) @ W.astype(np.float32).T).astype(np.float64)
+    assert np.array_equal(W.astype(np.float32).astype(np.float64), W)       # every weight exact in fp32
+    assert np.all(O.within_tolerance(y32, y_ref, a))
 
 
 def test_silu_pins_and_identities():
