@@ -17,6 +17,8 @@ namespace {
 
 constexpr uint32_t kMagic = 0x31514256u;  // "VBQ1"
 constexpr uint32_t kVersion = 1;
+// Directory entries count 16-byte units in 32 bits, so a blob's records span at most 2^32 - 1 units (64 GiB).
+constexpr uint64_t kMaxRecordUnits = 0xFFFFFFFFull;
 constexpr uint64_t kHeaderBytes = 64;
 
 inline uint64_t align16(uint64_t v) { return (v + 15) / 16 * 16; }
@@ -208,10 +210,11 @@ int vbq_packed_size(int64_t N, int64_t K, int64_t R, const uint8_t* widths, uint
   Geometry geo(N, K, R);
   std::vector<uint32_t> counts;
   if (int st = record_counts(geo, widths, counts)) return st;
-  uint64_t total = geo.rec_off;
+  uint64_t recs = 0;
   for (int64_t t = 0; t < geo.T; ++t)
-    for (int64_t g = 0; g < geo.G; ++g) total += RecordLayout(geo.tile_rows(t), &counts[size_t(t * geo.G + g) * 4]).bytes;
-  *out_bytes = total;
+    for (int64_t g = 0; g < geo.G; ++g) recs += RecordLayout(geo.tile_rows(t), &counts[size_t(t * geo.G + g) * 4]).bytes;
+  if (recs / 16 > kMaxRecordUnits) return VBQ_ERR_SHAPE;
+  *out_bytes = geo.rec_off + recs;
   return VBQ_OK;
 }
 
@@ -239,6 +242,7 @@ int vbq_pack_ex(int64_t N, int64_t K, int64_t R, const uint8_t* widths, const ui
       pos += RecordLayout(geo.tile_rows(t), &counts[size_t(t * geo.G + g) * 4]).bytes;
     }
   rec_start.back() = pos;
+  if (pos / 16 > kMaxRecordUnits) return VBQ_ERR_SHAPE;  // directory entries would not fit in 32 bits
   uint64_t max_rec = 0;
   for (size_t i = 0; i + 1 < rec_start.size(); ++i) max_rec = std::max(max_rec, rec_start[i + 1] - rec_start[i]);
   const uint64_t total = geo.rec_off + pos;

@@ -32,7 +32,8 @@ extern "C" {
 typedef enum vbq_status {
   VBQ_OK = 0,
   VBQ_ERR_NULL = -1,              /* a required pointer is NULL */
-  VBQ_ERR_SHAPE = -2,             /* N < 1, K < 64, K % 64 != 0, or N or K above 2^31 - 1 */
+  VBQ_ERR_SHAPE = -2,             /* N < 1, K < 64, K % 64 != 0, N or K above 2^31 - 1, or (pack) records above
+                                     64 GiB, which the 32-bit directory entries cannot address */
   VBQ_ERR_WIDTH = -3,             /* a width is not 1, 2, 4 or 8 */
   VBQ_ERR_CODE_RANGE = -4,        /* a code is >= 2^width */
   VBQ_ERR_BUFFER_TOO_SMALL = -5,  /* output capacity or blob size too small */

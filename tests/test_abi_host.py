@@ -284,3 +284,22 @@ def test_pack_and_quantize_are_thread_safe():
     with cf.ThreadPoolExecutor(max_workers=8) as pool:
         for _ in range(3):
             assert list(pool.map(work, cases)) == alone
+
+
+def test_packed_size_refuses_blobs_the_directory_cannot_address():
+    """Directory entries count 16-byte units in 32 bits: an all-8-bit matrix of 65536 x 1048576 (66 bytes per
+    group, 70 GB of records) is refused with VBQ_ERR_SHAPE; one of half the rows (35 GB) is sized normally."""
+    psutil = pytest.importorskip("psutil")
+    if psutil.virtual_memory().available < 4 << 30:
+        pytest.skip("needs about 1.1 GB for the width array")
+    G = 16384
+    widths = np.full((65536, G), 8, np.uint8)
+    L = vbq.lib()
+    out = ctypes.c_uint64(0)
+    st = L.vbq_packed_size(ctypes.c_int64(65536), ctypes.c_int64(64 * G), ctypes.c_int64(1024),
+                           widths.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8)), ctypes.byref(out))
+    assert st == vbq.VBQ_ERR_SHAPE
+    half = widths[:32768]
+    st = L.vbq_packed_size(ctypes.c_int64(32768), ctypes.c_int64(64 * G), ctypes.c_int64(1024),
+                           half.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8)), ctypes.byref(out))
+    assert st == 0 and out.value > 32 << 30
