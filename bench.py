@@ -241,6 +241,53 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def vbq_line(args, *, world, value, ms_max, step_bytes, weight_bytes, tile_rows, launches_per_step, t_setup,
+             launch_bytes, launch_ms, traffic, per_shape, e2e_val, h2d, d2h, fp16, n_launches, clocks, cpu, peak,
+             peak_kind) -> dict:
+    """The GPU arm's JSON line from its measurements (no device work here)."""
+    B = args.batch
+    achieved = launch_bytes / (launch_ms / 1e3) / 1e9
+    l2_bytes = 126e6
+    workload = WORKLOAD if (args.layers == 32 and not args.no_head) else (
+        f"{args.layers} of the 32 layers of the 9B-shaped decode step" + ("" if args.no_head else " plus the LM head"))
+    return {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "fp32", "data": "synthetic",
+        "config": {"workload": workload, "batch": B, "layers": args.layers, "lm_head": not args.no_head,
+                   "us_per_token": 1e3 * ms_max / args.steps,
+                   "weight_bytes_per_step": weight_bytes,
+                   "tile_rows": tile_rows,
+                   "launch": ("plain" if args.no_overlap else "programmatic dependent launch (VBQ_LAUNCH_OVERLAP)")
+                             + ("; one launch per linear" if args.no_fuse
+                                else "; q/k/v fused (vbq_gemm_skinny_multi); gate/up fused with the SwiGLU "
+                                     "epilogue (vbq_gemm_swiglu) writing the down projection's input; "
+                                     f"{launches_per_step} launches per step"),
+                   "weights": "seeded synthetic VBQ groups: P(1,2,4,8 bit) = (0.69,0.16,0.09,0.06), layer 0's "
+                              "MLP (0.40,0.35,0.15,0.10), LM head tiered to ~1.09 bits; fp16 scales "
+                              "U(0.01,0.1), uniform codes; x ~ N(0,1) bf16, one seeded x per linear",
+                   "l2": (f"inputs larger than L2: {step_bytes / 1e6:.0f} MB of distinct weights streamed once per "
+                          "step" if step_bytes > 2 * l2_bytes else
+                          f"inputs NOT larger than L2 ({step_bytes / 1e6:.0f} MB): L2-warm, not an HBM figure"),
+                   "setup_s": round(t_setup, 1),
+                   "parallelism": f"replicas x{world}"},
+        "pct_of_peak": 100.0 * value / world / peak,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": traffic, "peak_kind": peak_kind,
+                     "traffic_source": (f"ncu capture of {NCU_TRAFFIC['launches']} launches (layer 0 and the LM "
+                                        "head), scaled to this step's bytes per launch; "
+                                        + NCU_TRAFFIC["summary"]) if traffic is not None else None,
+                     "kernel": f"vbq_kernel<{B}>",
+                     "algorithmic_bytes_per_launch": launch_bytes, "avg_launch_us": launch_ms * 1e3},
+        "per_launch_group": per_shape,
+        "e2e": {"value": e2e_val, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "fp16_cublas_reference": fp16,
+        "gpu_launches": n_launches,
+        "clocks": clocks,
+        "cpu_baseline": cpu,
+    }
+
+
 def run_vbq(args):
     import concurrent.futures as cf
     import torch
@@ -436,47 +483,13 @@ def run_vbq(args):
 
     if rank == 0:
         peak, peak_kind = peaks()
-        achieved = launch_bytes / (launch_ms / 1e3) / 1e9
         cpu = cpu_baseline(B, args.cpu_budget) if (world == 1 and args.cpu_budget > 0) else None
-        l2_bytes = 126e6
-        workload = WORKLOAD if (args.layers == 32 and not args.no_head) else (
-            f"{args.layers} of the 32 layers of the 9B-shaped decode step" + ("" if args.no_head else " plus the LM head"))
-        line = {
-            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "fp32", "data": "synthetic",
-            "config": {"workload": workload, "batch": B, "layers": args.layers, "lm_head": not args.no_head,
-                       "us_per_token": 1e3 * ms_max / args.steps,
-                       "weight_bytes_per_step": sum(sum(mt.nbytes for mt in g.mats) for g in step),
-                       "tile_rows": {g.name.split(".")[-1]: g.R for g in step},
-                       "launch": ("plain" if args.no_overlap else "programmatic dependent launch (VBQ_LAUNCH_OVERLAP)")
-                                 + ("; one launch per linear" if args.no_fuse
-                                    else "; q/k/v fused (vbq_gemm_skinny_multi); gate/up fused with the SwiGLU "
-                                         "epilogue (vbq_gemm_swiglu) writing the down projection's input; "
-                                         f"{launches_per_step} launches per step"),
-                       "weights": "seeded synthetic VBQ groups: P(1,2,4,8 bit) = (0.69,0.16,0.09,0.06), layer 0's "
-                                  "MLP (0.40,0.35,0.15,0.10), LM head tiered to ~1.09 bits; fp16 scales "
-                                  "U(0.01,0.1), uniform codes; x ~ N(0,1) bf16, one seeded x per linear",
-                       "l2": (f"inputs larger than L2: {step_bytes / 1e6:.0f} MB of distinct weights streamed once per "
-                              "step" if step_bytes > 2 * l2_bytes else
-                              f"inputs NOT larger than L2 ({step_bytes / 1e6:.0f} MB): L2-warm, not an HBM figure"),
-                       "setup_s": round(t_setup, 1),
-                       "parallelism": f"replicas x{world}"},
-            "pct_of_peak": 100.0 * value / world / peak,
-            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak, "traffic": traffic, "peak_kind": peak_kind,
-                         "traffic_source": (f"ncu capture of {NCU_TRAFFIC['launches']} launches (layer 0 and the LM "
-                                            "head), scaled to this step's bytes per launch; "
-                                            + NCU_TRAFFIC["summary"]) if traffic is not None else None,
-                         "kernel": f"vbq_kernel<{B}>",
-                         "algorithmic_bytes_per_launch": launch_bytes, "avg_launch_us": launch_ms * 1e3},
-            "per_launch_group": per_shape,
-            "e2e": {"value": e2e_val, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-            "fp16_cublas_reference": fp16,
-            "gpu_launches": n_launches,
-            "clocks": clocks,
-            "cpu_baseline": cpu,
-        }
+        line = vbq_line(args, world=world, value=value, ms_max=ms_max, step_bytes=step_bytes,
+                        weight_bytes=sum(sum(mt.nbytes for mt in g.mats) for g in step),
+                        tile_rows={g.name.split(".")[-1]: g.R for g in step}, launches_per_step=launches_per_step,
+                        t_setup=t_setup, launch_bytes=launch_bytes, launch_ms=launch_ms, traffic=traffic,
+                        per_shape=per_shape, e2e_val=e2e_val, h2d=h2d, d2h=d2h, fp16=fp16, n_launches=n_launches,
+                        clocks=clocks, cpu=cpu, peak=peak, peak_kind=peak_kind)
         print(json.dumps(line), flush=True)
     del graph, graph_e2e
     if world > 1:
@@ -485,7 +498,7 @@ def run_vbq(args):
         dist.destroy_process_group()
 
 
-def main():
+def make_parser() -> argparse.ArgumentParser:
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=100)
@@ -504,6 +517,11 @@ def main():
                     help="plain launches instead of programmatic dependent launch between the linears")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds for the CPU-oracle baseline (0: skip)")
     ap.add_argument("--ref-rows", type=int, default=256, help="rows per linear per step for --impl reference")
+    return ap
+
+
+def main():
+    ap = make_parser()
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

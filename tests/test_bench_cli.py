@@ -95,3 +95,31 @@ def test_kernel_source_hash_ignores_comments_only():
     assert bench.kernel_source_sha256() == key(src)
     assert key("// note\nint a;\n\n/* block\n comment */ int b;  // tail\n") == key("int a;\n int b;\n")
     assert key("int a = 1;\n") != key("int a = 2;\n")
+
+
+def test_gpu_arm_line_has_the_contract_keys():
+    """The GPU arm's JSON line, built from stand-in measurements (no device): every contract key, a roofline
+    whose achieved bytes per launch over the average launch time matches frac x peak, and valid JSON."""
+    sys.path.insert(0, ROOT)
+    import bench
+    args = bench.make_parser().parse_args([])
+    line = bench.vbq_line(
+        args, world=1, value=690.0, ms_max=310.0, step_bytes=2.1286e9, weight_bytes=2.1219e9,
+        tile_rows={"q_k_v": 224, "o": 512, "gate_up": 224, "down": 224, "head": 224}, launches_per_step=129,
+        t_setup=9.0, launch_bytes=16.5e6, launch_ms=0.024, traffic=16.53e6, per_shape={}, e2e_val=340.0,
+        h2d=794624, d2h=6419456, fp16={"value": 4100.0}, n_launches=12900,
+        clocks={"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": []},
+        cpu={"value": 0.18, "unit": "GB/s", "cores": 16, "kind": "oracle", "sample": "s"},
+        peak=6551.0, peak_kind="measured")
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "roofline", "e2e", "gpu_launches", "clocks",
+                "cpu_baseline"):
+        assert key in line, key
+    assert line["steps"] == 100 and line["warmup"] == 5 and line["n_gpus"] == 1 and line["scaling"] == "weak"
+    assert "32 layers" in line["config"]["workload"] and line["config"]["us_per_token"] == 3100.0
+    r = line["roofline"]
+    assert {"bound", "achieved", "peak", "unit", "frac", "traffic"} <= set(r)
+    assert abs(r["achieved"] - 16.5e6 / 0.024e-3 / 1e9) < 1e-6 and abs(r["frac"] * r["peak"] - r["achieved"]) < 1e-6
+    assert set(line["e2e"]) == {"value", "unit", "h2d_bytes_per_step", "d2h_bytes_per_step"}
+    assert "inputs larger than L2" in line["config"]["l2"]
+    json.loads(json.dumps(line))
