@@ -7,8 +7,10 @@
  * a group, expand them with the group scale in registers, and accumulate the matrix-vector product. The
  * dense FP16 matrix is never built (section 6, paragraph "Fused kernels over packed weights").
  *
- * The dequantized weight is w = s * (q - (2^k - 1)/2), with q in [0, 2^k). The byte layout is "format v1" of
- * FORMAT.md: row tiles, one record per (tile, group column), and per-width buckets inside each record.
+ * The dequantized weight is w = s * (q - (2^k - 1)/2), with q in [0, 2^k). Format flag VBQ_FLAG_GRID_SYMMETRIC
+ * puts widths k >= 2 on the paper's Eq. 1 integer grid instead: w = s * (q - (2^(k-1) - 1)), q in [0, 2^k - 2].
+ * The byte layout is "format v1" of FORMAT.md: row tiles, one record per (tile, group column), and per-width
+ * buckets inside each record.
  *
  * Conventions for every function:
  *  - The return value is a status: VBQ_OK (0) or a negative VBQ_ERR_* code. No function aborts, exits or
@@ -35,7 +37,7 @@ typedef enum vbq_status {
   VBQ_ERR_SHAPE = -2,             /* N < 1, K < 64, K % 64 != 0, N or K above 2^31 - 1, or (pack) records above
                                      64 GiB, which the 32-bit directory entries cannot address */
   VBQ_ERR_WIDTH = -3,             /* a width is not 1, 2, 4 or 8 */
-  VBQ_ERR_CODE_RANGE = -4,        /* a code is >= 2^width */
+  VBQ_ERR_CODE_RANGE = -4,        /* a code is >= 2^width (above 2^width - 2 for widths >= 2 on the symmetric grid) */
   VBQ_ERR_BUFFER_TOO_SMALL = -5,  /* output capacity or blob size too small */
   VBQ_ERR_BAD_MAGIC = -6,         /* blob does not start with "VBQ1" */
   VBQ_ERR_VERSION = -7,           /* unsupported format version */
@@ -55,7 +57,7 @@ typedef enum vbq_status {
  * the device entry points, so the library never reads device memory from the host. */
 typedef struct vbq_desc {
   uint32_t version;      /* format version (1) */
-  uint32_t flags;        /* 0 */
+  uint32_t flags;        /* format flags of the blob header: 0 or VBQ_FLAG_GRID_SYMMETRIC */
   int64_t N;             /* output rows */
   int64_t K;             /* input columns, multiple of 64 */
   int64_t G;             /* K / 64 */
@@ -152,7 +154,7 @@ int vbq_gemv(const vbq_desc* d, const void* blob_dev, const void* x_bf16, float*
 /* Y[B][N] = X[B][K] W^T for B in {1, 2, 4, 8, 16} activation rows (skinny GEMM; decode with a small batch).
  * x_bf16: B*K bf16 values, row-major (row b is activation b), 16-byte aligned. y: B*N fp32, row-major.
  * B <= 4 runs on CUDA cores; B = 8 and 16 run the dequantized groups through tensor cores (bf16 operands
- * that hold the exact odd integers 2q - (2^k - 1), fp32 accumulation, the group scale applied in fp32).
+ * that hold the exact integers 2(q - c), fp32 accumulation, the group scale applied in fp32).
  * Other arguments and guarantees as in vbq_gemv. Errors: NULL, BATCH, ALIGN, WORKSPACE, FORMAT, CUDA. */
 int vbq_gemm_skinny(const vbq_desc* d, const void* blob_dev, const void* x_bf16, int B, float* y,
                     void* workspace, uint64_t workspace_bytes, void* stream);
