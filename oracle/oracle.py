@@ -6,12 +6,15 @@ use this module. The product package never imports it, and it never imports the 
 The oracle is a plain fp64 CPU implementation of the VBQ dequantize-and-multiply path. It follows the VBQ paper
 ("Variable Bit-width Quantization", section 3.1: 64-weight groups with a per-group scale and a width from
 {1,2,4,8}; section 6, "Fused kernels over packed weights": dequantize per group, then accumulate W x) and
-FORMAT.md for the byte layout.
+packed format v1 for the byte layout (row tiles, one record per tile and group column, width buckets
+inside each record).
 
 Pins (tests/test_oracle_pins.py), besides those of the C part:
 - silu: textbook values of the logistic function at 0 and +-1, large-argument limits, and the identity
   silu(g) - silu(-g) = g;
-- swiglu_bound: admits the bf16 rounding of an exact h;
+- swiglu_bound: admits the bf16 rounding of an exact h; its propagation term covers every admissible
+  perturbation of (g, u) on a grid that reaches |g| = 30 and the peak of silu' (where 1.1 > sup|silu'| is checked
+  against the textbook derivative and finite differences);
 - quantize: weights that lie exactly on either grid come back as that scale and those codes; 1-bit groups give
   sign times the mean magnitude; every dequantized weight lies within half a step of its input (plus the
   scale's fp16 rounding); all-zero groups decode to zero; non-finite weights and scales beyond fp16 are
@@ -222,13 +225,21 @@ def swiglu(y_gate, y_up) -> np.ndarray:
 
 
 def swiglu_bound(y_gate, y_up, bound_gate, bound_up) -> np.ndarray:
-    """Per-element bar for h computed from fp32 outputs that meet `within_tolerance` and rounded to bf16:
-    2^-8 |h| (bf16 rounding, with margin) + 1.1 |u| tol_g + |silu(g)| tol_u + tol_g tol_u + 1e-6, where
-    tol = 1e-3 * sum|w||x| + 1e-6 and 1.1 bounds |silu'|."""
+    """Per-element bar for h computed from fp32 outputs g', u' that meet `within_tolerance` (|g' - g| <= tol_g,
+    |u' - u| <= tol_u with tol = 1e-3 * sum|w||x| + 1e-6) and rounded once to bf16:
+
+        P   = 1.1 tol_g (|u| + tol_u) + |silu(g)| tol_u
+        bar = P + 2^-8 (|h| + P) + 1e-6,  h = silu(g) u.
+
+    P is the propagation term: silu(g') u' - silu(g) u = (silu(g') - silu(g)) u' + silu(g) (u' - u), and by the
+    mean value theorem |silu(g') - silu(g)| <= sup|silu'| tol_g with sup|silu'| = 1.0998... < 1.1 (at g = 2.40),
+    while |u'| <= |u| + tol_u. The computed h' lies within P of h; rounding it to bf16 moves it by at most
+    2^-9 |h'| <= 2^-9 (|h| + P), and 2^-8 leaves the other half for the fp32 evaluation of silu(g') u'."""
     g, u = np.asarray(y_gate, np.float64), np.asarray(y_up, np.float64)
     tg, tu = 1e-3 * np.asarray(bound_gate) + 1e-6, 1e-3 * np.asarray(bound_up) + 1e-6
     h = swiglu(g, u)
-    return 2.0 ** -8 * np.abs(h) + 1.1 * np.abs(u) * tg + np.abs(silu(g)) * tu + tg * tu + 1e-6
+    prop = 1.1 * tg * (np.abs(u) + tu) + np.abs(silu(g)) * tu
+    return prop + 2.0 ** -8 * (np.abs(h) + prop) + 1e-6
 
 
 def fp16_bits(v) -> np.ndarray:

@@ -2,7 +2,8 @@
 
 - float decoders: numpy's binary16 and torch's bfloat16 conversions, over all 65536 bit patterns;
 - CRC-32: the published check value and zlib;
-- packing: the hand-derived golden blob of FORMAT.md's worked example, and a single-code bit-position sweep;
+- packing: hand-derived golden blobs of the packed format's worked example (default grid, and Eq. 1's
+  symmetric grid flag with a top code), and a single-code bit-position sweep;
 - matvec: exact rational arithmetic on tiny shapes, closed forms on uniform widths, one-hot columns, exact
   power-of-two scale invariance, and numpy's BLAS on weights rebuilt from the definition.
 
@@ -105,6 +106,35 @@ def test_golden_blob_bytes():
     assert int.from_bytes(blob[crc["CRC32_HEADER"]:][:4], "little") == zlib.crc32(blob[0:60])
 
 
+GOLDEN_SYM = os.path.join(os.path.dirname(__file__), "golden", "format_n2_k64_r16_sym.txt")
+
+
+def test_golden_blob_symmetric_grid_flag():
+    """The worked example with header flag bit 0 (Eq. 1's grid) and a top-code (2 = 2^2 - 2) 2-bit row: every byte
+    as derived by hand, the round trip, and the dequantized rows on one-hot activations."""
+    N, K, R = 2, 64, 16
+    w = np.array([[1], [2]], np.uint8)
+    s = np.array([[0x3C00], [0x3800]], np.uint16)
+    c = np.zeros((2, 64), np.uint8)
+    c[0] = np.arange(64) % 2
+    c[1] = np.arange(64) % 3
+    blob = O.pack(N, K, R, w, s, c, flags=O.FLAG_GRID_SYMMETRIC)
+    expect, crc = parse_golden(GOLDEN_SYM)
+    b = blob.tobytes()
+    assert len(b) == 144 and set(expect) | {o + i for o in crc.values() for i in range(4)} == set(range(144))
+    for off, v in expect.items():
+        assert b[off] == v, f"byte {off}: got {b[off]:#04x} want {v:#04x}"
+    assert int.from_bytes(b[crc["CRC32_BODY"]:][:4], "little") == zlib.crc32(b[64:144])
+    assert int.from_bytes(b[crc["CRC32_HEADER"]:][:4], "little") == zlib.crc32(b[0:60])
+    assert O.header_flags(blob) == O.FLAG_GRID_SYMMETRIC
+    w2, s2, c2, R2 = O.unpack(blob)
+    assert R2 == R and np.array_equal(w2, w) and np.array_equal(s2, s) and np.array_equal(c2, c)
+    for i in (0, 1, 2, 63):
+        x = np.zeros((1, K), np.uint16); x[0, i] = 0x3F80
+        y, _ = O.matvec(w, s, c, x, flags=O.FLAG_GRID_SYMMETRIC)
+        assert y[0, 0] == (0.5 if i % 2 else -0.5) and y[0, 1] == 0.5 * (i % 3 - 1)
+
+
 @pytest.mark.parametrize("k", [1, 2, 4, 8])
 def test_single_code_bit_positions(k):
     # One 1-bit... 8-bit group (N=1, K=64, R=16): header 64 + directory 16 = 80; record: counts+width word
@@ -192,9 +222,19 @@ def test_pack_error_codes():
 
 
 # ------------------------------------------------------------------------------------------------ matvec
-def exact_y(w, s, c, xbits):
+def grid_offset(k, symmetric):
+    """The value-grid offset c of w = s (q - c), from its definition: (2^k - 1)/2 on the default half-integer grid;
+    on Eq. 1's symmetric integer grid of the VBQ paper (section 3.1, header flag bit 0) 2^(k-1) - 1 for k >= 2,
+    the 1-bit case (sign times the mean magnitude) staying +-s/2."""
+    if symmetric and k >= 2:
+        return Fraction((1 << (k - 1)) - 1)
+    return Fraction((1 << k) - 1, 2)
+
+
+def exact_y(w, s, c, xbits, flags=0):
     """Exact rational y and bound, decoding with numpy/torch (not the oracle)."""
     N, K = c.shape
+    sym = bool(flags & O.FLAG_GRID_SYMMETRIC)
     sv = [[Fraction(float(v)) for v in row] for row in f16(s)]
     xv = [Fraction(float(v)) for v in bf16(xbits)]
     ys, bs = [], []
@@ -202,42 +242,78 @@ def exact_y(w, s, c, xbits):
         acc, a = Fraction(0), Fraction(0)
         for i in range(K):
             k = int(w[r, i // 64])
-            wt = sv[r][i // 64] * (int(c[r, i]) - Fraction((1 << k) - 1, 2))
+            wt = sv[r][i // 64] * (int(c[r, i]) - grid_offset(k, sym))
             acc += wt * xv[i]
             a += abs(wt) * abs(xv[i])
         ys.append(acc); bs.append(a)
     return ys, bs
 
 
-def test_matvec_matches_exact_rationals_all_width_pairs():
-    # K=128 (2 groups): all 16 (width, width) pairs, one row each.
+def codes_on_grid(w, c, flags):
+    """Codes valid on the flagged grid: at most 2^k - 2 for k >= 2 on the symmetric grid; a code at the top of
+    each k >= 2 group so that the grid's extreme point is exercised."""
+    if not flags & O.FLAG_GRID_SYMMETRIC:
+        return c
+    kk = np.repeat(w.astype(np.int64), 64, axis=1)
+    top = np.where(kk >= 2, (1 << kk) - 2, 1)
+    c = np.minimum(c, top).astype(np.uint8)
+    c[:, ::64] = np.where(kk[:, ::64] >= 2, top[:, ::64], c[:, ::64])
+    return c
+
+
+@pytest.mark.parametrize("flags", [0, O.FLAG_GRID_SYMMETRIC])
+def test_matvec_matches_exact_rationals_all_width_pairs(flags):
+    # K=128 (2 groups): all 16 (width, width) pairs, one row each, on either value grid.
     g = np.random.default_rng(11)
     pairs = [(a, b) for a in (1, 2, 4, 8) for b in (1, 2, 4, 8)]
     w = np.array(pairs, np.uint8)
     s = S.scales_uniform(16, 2, g)
     s[3, 1] = 0xB555   # a negative scale
     s[5, 0] = 0x0003   # a subnormal scale
-    c = S.codes_uniform(w, g)
+    c = codes_on_grid(w, S.codes_uniform(w, g), flags)
     x = S.x_normal(1, 128, g)
     x[0, 7] = 0x0001   # a subnormal activation
     x[0, 9] = 0x7F00   # a large one
-    y, a = O.matvec(w, s, c, x)
-    ys, bs = exact_y(w, s, c, x[0])
+    y, a = O.matvec(w, s, c, x, flags=flags)
+    ys, bs = exact_y(w, s, c, x[0], flags)
     for r in range(16):
         assert abs(Fraction(y[0, r]) - ys[r]) <= Fraction(1, 2**50) * bs[r] + Fraction(1, 2**1000)
         assert abs(Fraction(a[0, r]) - bs[r]) <= Fraction(1, 2**50) * bs[r]
 
 
+@pytest.mark.parametrize("flags", [0, O.FLAG_GRID_SYMMETRIC])
 @pytest.mark.parametrize("N,K", [(1, 64), (3, 192), (5, 64)])
-def test_matvec_brute_force_small(N, K):
+def test_matvec_brute_force_small(N, K, flags):
     g = np.random.default_rng(N + K)
     w, s, c = random_logical(g, N, K, p=(0.25, 0.25, 0.25, 0.25))
+    c = codes_on_grid(w, c, flags)
     x = S.x_normal(2, K, g)
-    y, a = O.matvec(w, s, c, x)
+    y, a = O.matvec(w, s, c, x, flags=flags)
     for b in range(2):
-        ys, bs = exact_y(w, s, c, x[b])
+        ys, bs = exact_y(w, s, c, x[b], flags)
         for r in range(N):
             assert abs(Fraction(y[b, r]) - ys[r]) <= Fraction(1, 2**50) * bs[r]
+
+
+def test_symmetric_grid_closed_forms():
+    """Eq. 1's grid at its extreme and middle codes, on a one-hot activation: code 2^k - 2 is +(2^(k-1) - 1) s,
+    code 0 is -(2^(k-1) - 1) s, code 2^(k-1) - 1 is exactly 0; 1-bit codes stay +-s/2."""
+    K = 64
+    xe = np.zeros((1, K), np.uint16); xe[0, 5] = 0x3F80   # bf16 1.0 at column 5
+    s = np.full((1, 1), 0x3400, np.uint16)                 # 0.25
+    for k in (2, 4, 8):
+        L = (1 << (k - 1)) - 1
+        for code, want in ((2 * L, L * 0.25), (0, -L * 0.25), (L, 0.0)):
+            c = np.full((1, K), code, np.uint8)
+            y, a = O.matvec(np.full((1, 1), k, np.uint8), s, c, xe, flags=O.FLAG_GRID_SYMMETRIC)
+            assert y[0, 0] == want and a[0, 0] == abs(want), (k, code)
+    for code, want in ((1, 0.125), (0, -0.125)):
+        y, _ = O.matvec(np.ones((1, 1), np.uint8), s, np.full((1, K), code, np.uint8), xe,
+                        flags=O.FLAG_GRID_SYMMETRIC)
+        assert y[0, 0] == want
+    # codes above 2^k - 2 do not exist on the symmetric grid: the packer refuses them
+    assert O.pack_status(1, K, 16, np.full((1, 1), 2, np.uint8), s, np.full((1, K), 3, np.uint8),
+                         flags=O.FLAG_GRID_SYMMETRIC)[0] == O.ERR_CODE_RANGE
 
 
 @pytest.mark.parametrize("k", [1, 2, 4, 8])
@@ -337,6 +413,45 @@ def test_swiglu_bound_covers_bf16_rounding():
     hq = h_bf16.astype(np.uint32).view(np.float32).astype(np.float64)
     bound = O.swiglu_bound(g, u, np.zeros_like(g), np.zeros_like(u))
     assert np.all(np.abs(hq - h) <= bound)
+
+
+def silu_prime(g):
+    """Textbook derivative of g * sigma(g): sigma(g) (1 + g (1 - sigma(g))), sigma the logistic function."""
+    sg = 1.0 / (1.0 + np.exp(-np.asarray(g, np.float64)))
+    return sg * (1.0 + g * (1.0 - sg))
+
+
+def test_silu_derivative_is_below_the_bar_constant():
+    """The 1.1 of the h bar bounds |silu'|: the textbook derivative on a fine grid peaks at 1.0998 (g = 2.3994), and
+    central differences of the oracle's silu agree with it."""
+    g = np.concatenate([np.linspace(-40, 40, 160001), np.linspace(2.3, 2.5, 20001)])
+    d = silu_prime(g)
+    assert 1.0995 < d.max() < 1.1 and abs(g[np.argmax(d)] - 2.3994) < 1e-3
+    assert d.min() > -0.1
+    h = 1e-5
+    fd = (O.silu(g + h) - O.silu(g - h)) / (2 * h)
+    assert np.max(np.abs(fd - d)) < 1e-8
+
+
+def test_swiglu_bound_covers_every_admissible_perturbation():
+    """The propagation term P of the h bar (the bar without its rounding terms 2^-8 (|h| + P) + 1e-6) bounds
+    |silu(g') u' - silu(g) u| for every g' within tol_g of g and u' within tol_u of u: on a grid of (g, u) with |g|
+    up to 30, dense around the peak of silu', each with the corners and 21 interior points of the tolerance box."""
+    gs = np.concatenate([np.linspace(-30, 30, 241), np.linspace(2.2, 2.6, 41), [-1.2785]])
+    us = np.array([-30.0, -3.0, -0.5, 0.0, 0.5, 3.0, 30.0])
+    worst = 0.0
+    for tg, tu in ((1e-3, 1e-3), (0.05, 0.02), (0.5, 0.5), (2.0, 1.0)):
+        G, U = np.meshgrid(gs, us, indexing="ij")
+        A_g, A_u = (tg - 1e-6) / 1e-3, (tu - 1e-6) / 1e-3   # sum|w||x| that gives these tolerances
+        bar = O.swiglu_bound(G, U, np.full_like(G, A_g), np.full_like(U, A_u))
+        h = O.swiglu(G, U)
+        prop = (bar - 1e-6 - 2.0 ** -8 * np.abs(h)) / (1.0 + 2.0 ** -8)
+        for dg in np.concatenate([np.linspace(-1, 1, 21), [-1.0, 1.0]]):
+            for du in (-1.0, -0.5, 0.0, 0.5, 1.0):
+                d = np.abs(O.swiglu(G + dg * tg, U + du * tu) - h)
+                assert np.all(d <= prop * (1 + 1e-12) + 1e-12), (tg, tu, dg, du, float((d - prop).max()))
+                worst = max(worst, float((d / np.maximum(prop, 1e-300)).max()))
+    assert worst > 0.9   # the bar is tight somewhere: it is not loose by a large factor
 
 
 def test_recipe_workload_shape():
