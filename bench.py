@@ -275,8 +275,8 @@ def vbq_line(args, *, world, value, ms_max, step_bytes, weight_bytes, tile_rows,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic, "peak_kind": peak_kind,
                      "traffic_source": (f"ncu capture of {NCU_TRAFFIC['launches']} launches (layer 0 and the LM "
-                                        "head), scaled to this step's bytes per launch; "
-                                        + NCU_TRAFFIC["summary"]) if traffic is not None else None,
+                                        "head), scaled to this step's bytes per launch")
+                                       if traffic is not None else None,
                      "kernel": f"vbq_kernel<{B}>",
                      "algorithmic_bytes_per_launch": launch_bytes, "avg_launch_us": launch_ms * 1e3},
         "per_launch_group": per_shape,

@@ -27,6 +27,8 @@
 #include <cuda_fp16.h>
 #include <stdint.h>
 
+#include <algorithm>
+#include <atomic>
 #include <mutex>
 
 #include "vbq.h"
@@ -78,6 +80,13 @@ struct Params {
   int team_bytes;          // per team: S stages | tile accumulators [R][B] f32 | item results (B <= 4, 1-2 x R x B f32)
   int acc_off, res_off;
   int warps_off, warp_bytes;
+  // CUDA-core kernel (batch <= 4) only
+  int NB;                  // records per batch
+  int meta_off, dir_off;   // shared-memory offsets: per-record metadata blocks, directory cache
+  int res_rec, meta_rec;   // bytes per record: item results, metadata block
+  int cost[5];             // job costs for the split of a batch among warps: units of 1, 2, 4, 8 bits; meta job
+  int withhold;            // test hook: the record (global index) whose bulk copy is never issued, or -1
+  unsigned long long wait_ns;  // limit of every mbarrier wait
 };
 
 // Element m of a kernel-parameter array through a select chain (a dynamic index would copy the array to local
@@ -151,9 +160,10 @@ __device__ __forceinline__ unsigned long long now_ns() {
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
   return t;
 }
-// Wait for the phase with the given parity to complete. Gives up after kWaitNs: sets the status word and the
+// Wait for the phase with the given parity to complete. Gives up after limit_ns: sets the status word and the
 // CTA's abort flag, after which every wait of the CTA returns at once and nothing more is written.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, unsigned parity, unsigned* status, volatile int* abort) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, unsigned parity, unsigned* status, volatile int* abort,
+                                          unsigned long long limit_ns) {
   if (*abort) return false;
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = now_ns();
@@ -161,7 +171,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, unsigned parity, unsign
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 255u) == 0) {
       if (*abort) return false;
-      if (now_ns() - t0 > kWaitNs) {
+      if (now_ns() - t0 > limit_ns) {
         *abort = 1;
         atomicOr(status, kStatusTimeout);
         return false;
@@ -171,10 +181,10 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, unsigned parity, unsign
 }
 // Drain wait used after an abort: waits (bounded, ignoring the abort flag) for a bulk copy this CTA issued, so
 // that no copy into its shared memory is still in flight when the CTA exits.
-__device__ __forceinline__ void mbar_drain(uint64_t* bar, unsigned parity) {
+__device__ __forceinline__ void mbar_drain(uint64_t* bar, unsigned parity, unsigned long long limit_ns) {
   const unsigned long long t0 = now_ns();
   while (!mbar_try_wait(bar, parity))
-    if (now_ns() - t0 > kWaitNs) return;
+    if (now_ns() - t0 > limit_ns) return;
 }
 // Atomic add with acquire-release semantics at GPU scope; returns the old value.
 __device__ __forceinline__ unsigned atom_add_acq_rel(unsigned* addr, unsigned v) {
@@ -271,30 +281,17 @@ __device__ __forceinline__ float magic_f(uint32_t src, uint32_t mask_shifted) {
 }
 
 // Each returns sum_i (q_i - (2^k-1)/2) x_i for one 64-weight group; sg = sum_i x_i.
-// a += x when (w & bit) != 0, as a predicated add (no branch).
-__device__ __forceinline__ void add_if(float& a, uint32_t w, uint32_t bit, float x) {
-  asm("{\n\t.reg .pred p;\n\t.reg .b32 t;\n\tand.b32 t, %1, %2;\n\tsetp.ne.b32 p, t, 0;\n\t"
-      "@p add.f32 %0, %0, %3;\n\t}"
-      : "+f"(a) : "r"(w), "r"(bit), "f"(x));
-}
-// 1-bit: sum of the activations whose bit is set, minus half the group sum.
+// 1-bit: sum of the activations whose bit is set (predicated adds, eight independent sums), minus half the group
+// sum.
 __device__ __forceinline__ float dot_b1(uint2 w, const float (&xr)[64], float sg) {
-  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+  float a[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-  for (int i = 0; i < 32; i += 4) {
-    add_if(a0, w.x, 1u << i, xr[i]);
-    add_if(a1, w.x, 1u << (i + 1), xr[i + 1]);
-    add_if(a2, w.x, 1u << (i + 2), xr[i + 2]);
-    add_if(a3, w.x, 1u << (i + 3), xr[i + 3]);
-  }
+  for (int i = 0; i < 32; ++i)
+    if (w.x & (1u << i)) a[i & 7] += xr[i];
 #pragma unroll
-  for (int i = 0; i < 32; i += 4) {
-    add_if(a0, w.y, 1u << i, xr[32 + i]);
-    add_if(a1, w.y, 1u << (i + 1), xr[33 + i]);
-    add_if(a2, w.y, 1u << (i + 2), xr[34 + i]);
-    add_if(a3, w.y, 1u << (i + 3), xr[35 + i]);
-  }
-  return ((a0 + a1) + (a2 + a3)) - 0.5f * sg;
+  for (int i = 0; i < 32; ++i)
+    if (w.y & (1u << i)) a[i & 7] += xr[32 + i];
+  return (((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]))) - 0.5f * sg;
 }
 
 // 2- and 4-bit: xr holds x_i * 2^-shift(i). v - 2^23 = q * 2^shift exactly, so (v - 2^23) * xr_i = q * x_i.
@@ -470,7 +467,7 @@ __device__ __forceinline__ int item_row(const uint32_t* masks, const int* pref, 
 }
 
 // ----------------------------------------------------------------------------------------- record view
-// Offsets of the parts of a record with Rt rows and bucket counts n0..n3 (FORMAT.md).
+// Offsets of the parts of a packed-format-v1 record with Rt rows and bucket counts n0..n3.
 struct Rec {
   int n0, n1, n2, n3;
   int sc, c0, c1, c2, c3;     // byte offsets: scales and the four code buckets
@@ -589,6 +586,118 @@ struct TeamMap {
   }
 };
 
+
+// ---------------------------------------------------------------------------------------- end of a CTA
+// Runs after every whole-tile output and every partial slot of this CTA is written (all threads, after a barrier).
+//  - Tiles shared with other CTAs (only a CTA's first and last tile can be): one thread makes the CTA's slot writes
+//    visible GPU-wide and counts the CTA in on the tile's arrival counter; the last owner to arrive adds all owners'
+//    slots in CTA order and resets the counter. No CTA waits for another.
+//  - SwiGLU epilogue (p.swiglu): matrices 0 (gate) and 1 (up) have the same rows and tiles. Whoever writes a tile's
+//    final y counts it in on the pair counter of its tile index; the second of the pair computes h = silu(gate) * up
+//    for those rows from both final outputs, rounded once to bf16, and resets the counter.
+template <int B, int kThreads>
+__device__ void finish_cta(const Params& p, int L, int H, int* cta_flags, int* epi_tiles, int* epi_count) {
+  const int tid = threadIdx.x, G = p.G, R = p.R;
+  if (H <= L) return;
+  // Owners of tile t. With at least as many records as CTAs every CTA owns a contiguous, non-empty record range,
+  // so the owners are first..last. With fewer records than CTAs each CTA owns at most one record, so the owners
+  // are the owners of the tile's G records, one each.
+  const bool dense = p.nrec >= int(gridDim.x);
+  auto tile_owners = [&](int t, int& first) -> int {
+    first = owner(p, t * G);
+    return dense ? owner(p, t * G + G - 1) - first + 1 : G;
+  };
+  auto kth_owner = [&](int t, int first, int k) -> int { return dense ? first + k : owner(p, t * G + k); };
+  // Sums of all owners' partial slots of tiles ta (and tb2 when ntiles == 2), each in CTA order, into y. The
+  // elements of both tiles form one index space; each thread has the loads of up to 16 owners in flight.
+  auto reduce_tiles = [&](int ta, int tb2, int ntiles) {
+    int fa, fb = 0;
+    const int oa = tile_owners(ta, fa), ob = ntiles > 1 ? tile_owners(tb2, fb) : 0;
+    const TileOut ya = tile_out(p, ta), yb = tile_out(p, ntiles > 1 ? tb2 : ta);
+    const int n0 = ya.Rt * B, ntot = n0 + (ntiles > 1 ? yb.Rt * B : 0);
+    for (int e2 = tid; e2 < ntot; e2 += kThreads) {
+      const bool second = e2 >= n0;
+      const int e = second ? e2 - n0 : e2, t = second ? tb2 : ta, first = second ? fb : fa;
+      const int owners = second ? ob : oa;
+      float v = 0.f;
+      for (int o0 = 0; o0 < owners; o0 += 16) {
+        float part[16];
+#pragma unroll
+        for (int q = 0; q < 16; ++q)
+          part[q] = o0 + q < owners ? __ldcg(p.partial + size_t(kth_owner(t, first, o0 + q) + t) * R * B + e) : 0.f;
+#pragma unroll
+        for (int q = 0; q < 16; ++q)
+          if (o0 + q < owners) v += part[q];
+      }
+      const int r = e / B, b = e - r * B;
+      const TileOut& to = second ? yb : ya;
+      to.y[size_t(b) * to.ld + r] = v;
+    }
+  };
+
+  const int tfirst = L / G, tlast = (H - 1) / G;
+  const bool part0 = !(L <= tfirst * G && H >= (tfirst + 1) * G);
+  const bool part1 = tlast != tfirst && !(L <= tlast * G && H >= (tlast + 1) * G);
+  if (part0 || part1) {
+    __syncthreads();
+    if (tid == 0) {
+      // acq_rel at GPU scope: the release publishes the CTA's slot writes (ordered before it by the barrier),
+      // the acquire makes the other owners' slots visible to the reduction that follows.
+      int first;
+      const int own0 = part0 ? tile_owners(tfirst, first) : 0, own1 = part1 ? tile_owners(tlast, first) : 0;
+      const unsigned a0 = part0 ? atom_add_acq_rel(&p.arrive[tfirst], 1u) : 0u;
+      const unsigned a1 = part1 ? atom_add_acq_rel(&p.arrive[tlast], 1u) : 0u;
+      cta_flags[0] = part0 && a0 == unsigned(own0 - 1);
+      cta_flags[1] = part1 && a1 == unsigned(own1 - 1);
+    }
+    __syncthreads();
+    const int ntiles = cta_flags[0] + cta_flags[1];
+    if (ntiles > 0) {
+      const int ta = cta_flags[0] ? tfirst : tlast;
+      reduce_tiles(ta, tlast, ntiles);
+      if (tid == 0) {
+        p.arrive[ta] = 0u;
+        if (ntiles > 1) p.arrive[tlast] = 0u;
+      }
+    }
+  } else if (tid == 0) {
+    cta_flags[0] = cta_flags[1] = 0;
+  }
+  if (!p.swiglu) return;
+
+  // SwiGLU epilogue. This CTA wrote the final y of its whole tiles and of the shared tiles it reduced.
+  const int tiles_here = tlast - tfirst + 1;
+  for (int c0 = 0; c0 < tiles_here; c0 += kEpiChunk) {
+    __syncthreads();  // this CTA's y writes (and the previous chunk's epilogue) are done
+    if (tid == 0) {
+      int n = 0;
+      for (int k = c0; k < min(tiles_here, c0 + kEpiChunk); ++k) {
+        const int t = tfirst + k;
+        const bool whole = L <= t * G && H >= (t + 1) * G;
+        const bool reduced = (t == tfirst && part0 && cta_flags[0]) || (t == tlast && part1 && cta_flags[1]);
+        if (!whole && !reduced) continue;
+        const int m = mat_of_tile(p, t), tl = m == 0 ? t : t - p.tile_start[1];
+        if (atom_add_acq_rel(&p.pair[tl], 1u) == 1u) epi_tiles[n++] = tl;
+      }
+      *epi_count = n;
+    }
+    __syncthreads();
+    for (int k = 0; k < *epi_count; ++k) {
+      const int tl = epi_tiles[k];
+      const int N = p.N[0], Rt = min(R, N - tl * R);
+      const size_t row0 = size_t(tl) * R;
+      for (int e = tid; e < Rt * B; e += kThreads) {
+        const int b = e / Rt, r = e - b * Rt;
+        const size_t at = size_t(b) * N + row0 + r;
+        const float g = __ldcg(p.y[0] + at), u = __ldcg(p.y[1] + at);
+        const float silu = g / (1.f + expf(-g));
+        p.h[at] = __bfloat16_as_ushort(__float2bfloat16_rn(silu * u));
+      }
+      if (tid == 0) p.pair[tl] = 0u;
+    }
+  }
+}
+
 // ------------------------------------------------------------------------------------------------ kernel
 template <int B>
 __global__ void __launch_bounds__(Cfg<B>::kThreads, 1) vbq_kernel(const __grid_constant__ Params params) {
@@ -618,43 +727,6 @@ __global__ void __launch_bounds__(Cfg<B>::kThreads, 1) vbq_kernel(const __grid_c
   // A kernel launched after this one with programmatic dependent launch may start its own prologue (which reads
   // only its weights) as soon as SMs free up; it waits for this grid before touching activations or outputs.
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-
-  // Owners of tile t. With at least as many records as CTAs every CTA owns a contiguous, non-empty record range,
-  // so the owners are first..last. With fewer records than CTAs each CTA owns at most one record, so the owners
-  // are the owners of the tile's G records, one each.
-  const bool dense = p.nrec >= int(gridDim.x);
-  auto tile_owners = [&](int t, int& first) -> int {
-    first = owner(p, t * G);
-    return dense ? owner(p, t * G + G - 1) - first + 1 : G;
-  };
-  auto kth_owner = [&](int t, int first, int k) -> int { return dense ? first + k : owner(p, t * G + k); };
-
-  // Sums of all owners' partial slots of the tiles in ts[0..nt), each in CTA order, into y (all threads; the
-  // elements of both tiles form one index space). Each thread has the loads of up to 16 owners in flight.
-  auto reduce_tiles = [&](int ta, int tb2, int ntiles) {  // tiles ta (and tb2 when ntiles == 2)
-    int fa, fb = 0;
-    const int oa = tile_owners(ta, fa), ob = ntiles > 1 ? tile_owners(tb2, fb) : 0;
-    const TileOut ya = tile_out(p, ta), yb = tile_out(p, ntiles > 1 ? tb2 : ta);
-    const int n0 = ya.Rt * B, ntot = n0 + (ntiles > 1 ? yb.Rt * B : 0);
-    for (int e2 = tid; e2 < ntot; e2 += C::kThreads) {
-      const bool second = e2 >= n0;
-      const int e = second ? e2 - n0 : e2, t = second ? tb2 : ta, first = second ? fb : fa;
-      const int owners = second ? ob : oa;
-      float v = 0.f;
-      for (int o0 = 0; o0 < owners; o0 += 16) {
-        float part[16];
-#pragma unroll
-        for (int q = 0; q < 16; ++q)
-          part[q] = o0 + q < owners ? __ldcg(p.partial + size_t(kth_owner(t, first, o0 + q) + t) * R * B + e) : 0.f;
-#pragma unroll
-        for (int q = 0; q < 16; ++q)
-          if (o0 + q < owners) v += part[q];
-      }
-      const int r = e / B, b = e - r * B;
-      const TileOut& to = second ? yb : ya;
-      to.y[size_t(b) * to.ld + r] = v;
-    }
-  };
 
   const int team = warp / TW, tw = warp - team * TW;
   int tb = L, te = L, tseg = -1;
@@ -715,12 +787,12 @@ __global__ void __launch_bounds__(Cfg<B>::kThreads, 1) vbq_kernel(const __grid_c
       } else {
         stage_bad[team * S + s] = 0;
         mbar_arrive_tx(&bars[s], bytes + 128u * B);
-        tma_bulk_load(dst, pick(p.recs, m) + 16ull * a, bytes, &bars[s]);
+        if (tb + i != p.withhold) tma_bulk_load(dst, pick(p.recs, m) + 16ull * a, bytes, &bars[s]);
       }
     };
     auto issue_x = [&](int i) {  // lane 0
       const int s = i % S, j = tb + i, g = j % G;
-      if (stage_bad[team * S + s]) return;
+      if (stage_bad[team * S + s] || j == p.withhold) return;
       unsigned char* dst = tbase + s * p.stage_size + p.stage_bytes;
 #pragma unroll
       for (int bb = 0; bb < B; ++bb)
@@ -765,7 +837,7 @@ __global__ void __launch_bounds__(Cfg<B>::kThreads, 1) vbq_kernel(const __grid_c
       const int s = i % S;
       const unsigned char* st = tbase + s * p.stage_size;
       const uint32_t sa = smem_u32(st);
-      bool ok = mbar_wait(&bars[s], (i / S) & 1, p.status, abort_flag);
+      bool ok = mbar_wait(&bars[s], (i / S) & 1, p.status, abort_flag, p.wait_ns);
       if (ok && stage_bad[team * S + s]) ok = false;
       ok = __all_sync(0xFFFFFFFFu, ok);  // lanes can see an abort at different times; the warp decides as one
       const int j = tb + i, t = j / G;
@@ -991,7 +1063,7 @@ __global__ void __launch_bounds__(Cfg<B>::kThreads, 1) vbq_kernel(const __grid_c
     if (cur_t >= 0) flush(cur_t);
     // After an abort, wait (bounded) for this team's copies still in flight before the CTA can exit.
     if (*abort_flag && tw == 0 && lane == 0)
-      for (int r = max(0, issued - S); r < issued; ++r) mbar_drain(&bars[r % S], (r / S) & 1);
+      for (int r = max(0, issued - S); r < issued; ++r) mbar_drain(&bars[r % S], (r / S) & 1, p.wait_ns);
   }
 
   // =================================================================== combine of tiles shared by teams
@@ -1022,80 +1094,564 @@ __global__ void __launch_bounds__(Cfg<B>::kThreads, 1) vbq_kernel(const __grid_c
       }
     }
   }
-  // ================================================= tiles shared with other CTAs: only this CTA's first and last
-  // Every partial slot of this CTA is written. One thread makes them visible GPU-wide and counts the CTA in;
-  // the last owner of a tile to arrive adds all owners' slots in CTA order.
-  if (H <= L) return;
-  const int tfirst = L / G, tlast = (H - 1) / G;
-  const bool part0 = !(L <= tfirst * G && H >= (tfirst + 1) * G);
-  const bool part1 = tlast != tfirst && !(L <= tlast * G && H >= (tlast + 1) * G);
-  if (part0 || part1) {
-    __syncthreads();
-    if (tid == 0) {
-      // acq_rel at GPU scope: the release publishes the CTA's slot writes (ordered before it by the barrier),
-      // the acquire makes the other owners' slots visible to the reduction that follows. Both counters at once.
-      int first;
-      const int own0 = part0 ? tile_owners(tfirst, first) : 0, own1 = part1 ? tile_owners(tlast, first) : 0;
-      const unsigned a0 = part0 ? atom_add_acq_rel(&p.arrive[tfirst], 1u) : 0u;
-      const unsigned a1 = part1 ? atom_add_acq_rel(&p.arrive[tlast], 1u) : 0u;
-      cta_flags[0] = part0 && a0 == unsigned(own0 - 1);
-      cta_flags[1] = part1 && a1 == unsigned(own1 - 1);
-    }
-    __syncthreads();
-    const int ntiles = cta_flags[0] + cta_flags[1];
-    if (ntiles > 0) {
-      const int ta = cta_flags[0] ? tfirst : tlast;
-      reduce_tiles(ta, tlast, ntiles);
-      if (tid == 0) {
-        p.arrive[ta] = 0u;
-        if (ntiles > 1) p.arrive[tlast] = 0u;
-      }
-    }
-  }
-  if (!p.swiglu) return;
+  finish_cta<B, C::kThreads>(p, L, H, cta_flags, epi_tiles, &epi_count);
+}
 
-  // ================================================= SwiGLU epilogue: h = silu(gate) * up, bf16
-  // Matrix 0 is gate and matrix 1 is up, with the same rows and tiles, so gate tile tl and up tile tl cover the
-  // same rows. Whoever writes a tile's final y counts it in on the pair counter of tl; the second of the pair
-  // computes h for those rows from both (final) outputs. This CTA wrote the final y of its whole tiles and of
-  // the shared tiles it reduced.
-  const int tiles_here = tlast - tfirst + 1;
-  for (int c0 = 0; c0 < tiles_here; c0 += kEpiChunk) {
-    __syncthreads();  // this CTA's y writes (and the previous chunk's epilogue) are done
-    if (tid == 0) {
-      int n = 0;
-      for (int k = c0; k < min(tiles_here, c0 + kEpiChunk); ++k) {
-        const int t = tfirst + k;
-        const bool whole = L <= t * G && H >= (t + 1) * G;
-        const bool reduced = (t == tfirst && part0 && cta_flags[0]) || (t == tlast && part1 && cta_flags[1]);
-        if (!whole && !reduced) continue;
-        const int m = mat_of_tile(p, t), tl = m == 0 ? t : t - p.tile_start[1];
-        if (atom_add_acq_rel(&p.pair[tl], 1u) == 1u) epi_tiles[n++] = tl;
-      }
-      epi_count = n;
+
+// ====================================================================================== CUDA-core kernel
+// Batch B in {1, 2, 4}. One CTA per SM, 16 warps that work on the CTA's records together:
+//  - The CTA's record range is cut into batches of up to NB records of one row tile. Records stream HBM ->
+//    shared memory by cp.async.bulk (one copy per record plus one 128-byte copy per batch row of the column's
+//    activations), S batches ahead, each record in its own slot with its own mbarrier.
+//  - Each record gets a meta job one batch before its units run: validate it, build the width masks and item
+//    starts per 32-row word, the activation tables and the 1-bit nibble tables, and note where its buckets lie.
+//  - Per batch, the jobs are the width-bucket units of its records and the meta jobs of the next batch. Every warp
+//    computes the same job list from the meta blocks and takes the jobs whose cost midpoint falls in its 1/16 of
+//    the total, so the split is even to about one unit. A unit writes s * dot for each of its items (and batch
+//    rows) into the record's result buffer.
+//  - One CTA barrier per batch. Then each warp adds the results of its own 32-row words to its accumulators,
+//    record by record in record order (row r takes the result of its item: the start of its bucket in its word
+//    plus the rows of the same width before it), so every row is summed in a fixed order and results are bitwise
+//    identical from run to run. The batch's slots are refilled right after the barrier.
+//  - A finished tile goes to y when the CTA holds all its records, else to the CTA's partial slot; finish_cta then
+//    reduces the tiles shared with neighbouring CTAs and runs the SwiGLU epilogue.
+template <int B> struct CCfg {
+  static constexpr int kWarps = 16;
+  static constexpr int kThreads = kWarps * 32;
+  static constexpr int kIPU = 32 / B;                               // items per 2-, 4-, 8-bit unit
+  static constexpr int kWordsPerWarp = (32 + kWarps - 1) / kWarps;  // row-pass words per warp (R <= 1024)
+};
+constexpr int kMaxNB = 7;        // records per batch: the 1 + 4 NB job segments of a batch fit in one warp
+constexpr int kMaxSets = 4;      // batches in flight
+constexpr int kDirCache = 512;   // directory entries cached in shared memory
+
+// Per-record metadata block (256-byte aligned), written by the record's meta job:
+//  lut [B][16][16] f32: 1-bit nibble tables; entry n of position p is the sum of x[4p + i] over the set bits i of n
+//  xt  [3][B][64] f32:  x, x * 2^-shift for 2-bit codes, x * 2^-shift for 4-bit codes
+//  sg  [B] f32:         group sums of x
+//  mk  [4][32] u32:     width masks per 32-row word;  pf [4][32] u16: item index of the word's first row per width
+//  wc  [64] u32:        the record's width-code words
+//  fl  [12] i32:        bad, scales offset, bucket counts n[4], bucket code offsets c[4]
+struct MetaOff {
+  int lut, xt, sg, mk, pf, wc, fl, size;
+  __host__ __device__ explicit MetaOff(int B) {
+    lut = 0;
+    xt = 1024 * B;
+    sg = xt + 768 * B;
+    mk = sg + 16;
+    pf = mk + 512;
+    wc = pf + 256;
+    fl = wc + 256;
+    size = (fl + 48 + 255) & ~255;
+  }
+};
+
+// The CTA's batches: records [L, H) cut at row-tile boundaries, then into runs of at most NB records.
+struct Batches {
+  int L, H, G, NB, e0, nb0, bpt, tile0, nbatch;
+  __device__ Batches(int L_, int H_, int G_, int NB_)
+      : L(L_), H(H_), G(G_), NB(NB_), e0(0), nb0(0), bpt(1), tile0(0), nbatch(0) {
+    if (H <= L) return;
+    tile0 = L / G;
+    e0 = min(H, (tile0 + 1) * G);
+    nb0 = (e0 - L + NB - 1) / NB;
+    bpt = (G + NB - 1) / NB;
+    const int rest = H - e0, full = rest / G, last = rest - full * G;
+    nbatch = nb0 + full * bpt + (last + NB - 1) / NB;
+  }
+  __device__ void get(int n, int& rb, int& re) const {
+    if (n < nb0) {
+      rb = L + n * NB;
+      re = min(e0, rb + NB);
+      return;
     }
-    __syncthreads();
-    for (int k = 0; k < epi_count; ++k) {
-      const int tl = epi_tiles[k];
-      const int N = p.N[0], Rt = min(R, N - tl * R);
-      const size_t row0 = size_t(tl) * R;
-      for (int e = tid; e < Rt * B; e += C::kThreads) {
-        const int b = e / Rt, r = e - b * Rt;
-        const size_t at = size_t(b) * N + row0 + r;
-        const float g = __ldcg(p.y[0] + at), u = __ldcg(p.y[1] + at);
-        const float silu = g / (1.f + expf(-g));
-        p.h[at] = __bfloat16_as_ushort(__float2bfloat16_rn(silu * u));
-      }
-      if (tid == 0) p.pair[tl] = 0u;
+    const int m = n - nb0, q = m / bpt, t = tile0 + 1 + q;
+    rb = t * G + (m - q * bpt) * NB;
+    re = min(min(H, (t + 1) * G), rb + NB);
+  }
+};
+
+// 1-bit group against the nibble tables of B batch rows at shared address tab (256-byte aligned, table b at
+// tab + 1024 b): 16 lookups per row, one per four weights. Each nibble times 4 is moved by one byte permute into
+// the low byte of the table address. Returns sum_i (q_i - 1/2) x_i per row.
+template <int B>
+__device__ __forceinline__ void dot_b1_lut(uint2 w, uint32_t tab, const float (&sg)[B], float (&d)[B]) {
+  const uint32_t e0 = (w.x << 2) & 0x3C3C3C3Cu, o0 = (w.x >> 2) & 0x3C3C3C3Cu;  // nibbles 2k / 2k+1, times 4
+  const uint32_t e1 = (w.y << 2) & 0x3C3C3C3Cu, o1 = (w.y >> 2) & 0x3C3C3C3Cu;
+  constexpr int NA = B == 1 ? 8 : 4;
+  float a[B][NA];
+#pragma unroll
+  for (int b = 0; b < B; ++b)
+#pragma unroll
+    for (int i = 0; i < NA; ++i) a[b][i] = 0.f;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const uint32_t ae0 = __byte_perm(e0, tab, 0x7650u + k), ao0 = __byte_perm(o0, tab, 0x7650u + k);
+    const uint32_t ae1 = __byte_perm(e1, tab, 0x7650u + k), ao1 = __byte_perm(o1, tab, 0x7650u + k);
+#pragma unroll
+    for (int b = 0; b < B; ++b) {
+      a[b][(2 * k) % NA] += lds32f(ae0 + 1024 * b + 64 * (2 * k));
+      a[b][(2 * k + 1) % NA] += lds32f(ao0 + 1024 * b + 64 * (2 * k + 1));
+      a[b][(2 * k) % NA] += lds32f(ae1 + 1024 * b + 64 * (8 + 2 * k));
+      a[b][(2 * k + 1) % NA] += lds32f(ao1 + 1024 * b + 64 * (9 + 2 * k));
     }
   }
+#pragma unroll
+  for (int b = 0; b < B; ++b) {
+    float t = 0.f;
+    if constexpr (NA == 8) t = ((a[b][0] + a[b][1]) + (a[b][2] + a[b][3])) + ((a[b][4] + a[b][5]) + (a[b][6] + a[b][7]));
+    else t = (a[b][0] + a[b][1]) + (a[b][2] + a[b][3]);
+    d[b] = t - 0.5f * sg[b];
+  }
+}
+
+// 1-bit units [lo, hi) of 32 items each (lane = item, all B batch rows): s * dot into res[item][b].
+template <int B>
+__device__ __forceinline__ void unit_range_b1(int n, int lo, int hi, int lane, uint32_t codes, uint32_t scales,
+                                              uint32_t res, uint32_t tab, const float (&sg)[B]) {
+  for (int u = lo; u < hi; ++u) {
+    const int jj = 32 * u + lane;
+    if (jj >= n) break;
+    float d[B];
+    dot_b1_lut<B>(lds64(codes + 8 * jj), tab, sg, d);
+    const float s = __half2float(__ushort_as_half((unsigned short)lds16(scales + 2 * jj)));
+#pragma unroll
+    for (int b = 0; b < B; ++b) sts32f(res + 4 * (jj * B + b), s * d[b]);
+  }
+}
+
+// 2-, 4-, 8-bit units [lo, hi) of 32 / B items each (lane = item * B + b): s * dot of the item's group with batch
+// row b into res[item][b]. codes, scales and res are byte addresses of item 0 of the bucket.
+template <int KB, int B>
+__device__ __forceinline__ void unit_range(int n, int lo, int hi, int lane, uint32_t codes, uint32_t scales,
+                                           uint32_t res, const float (&xr)[64], float sg, float corr) {
+  constexpr int IPU = 32 / B;
+  const int sub = lane / B, b = lane - sub * B;
+  for (int u = lo; u < hi; ++u) {
+    const int jj = IPU * u + sub;
+    if (jj >= n) break;
+    float d;
+    if constexpr (KB == 2) {
+      const uint4 a = lds128(codes + 16 * jj);
+      const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+      d = dot_magic<2>(w, xr, sg, corr);
+    } else if constexpr (KB == 4) {
+      const uint4 a = lds128(codes + 32 * jj), c = lds128(codes + 32 * jj + 16);
+      const uint32_t w[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
+      d = dot_magic<4>(w, xr, sg, corr);
+    } else {
+      uint32_t w[16];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint4 a = lds128(codes + 64 * jj + 16 * q);
+        w[4 * q] = a.x; w[4 * q + 1] = a.y; w[4 * q + 2] = a.z; w[4 * q + 3] = a.w;
+      }
+      d = dot_b8(w, xr, sg, corr);
+    }
+    sts32f(res + 4 * (jj * B + b), __half2float(__ushort_as_half((unsigned short)lds16(scales + 2 * jj))) * d);
+  }
+}
+
+// First job (of count jobs costing c each, the segment starting at cost s0) whose cost midpoint reaches cost
+// cut2 / (2 W): the smallest j with W (2 s0 + c (2j + 1)) >= cut2, clamped to [0, count].
+__device__ __forceinline__ int first_job(int cut2, int s0, int c, int count, int W) {
+  if (count <= 0) return 0;
+  const int num = cut2 - (2 * s0 + c) * W;
+  if (num <= 0) return 0;
+  const int den = 2 * W * c;
+  return min(count, (num + den - 1) / den);
+}
+
+template <int B>
+__global__ void __launch_bounds__(CCfg<B>::kThreads, 1) vbq_cc_kernel(const __grid_constant__ Params params) {
+  using C = CCfg<B>;
+  constexpr int W = C::kWarps, IPU = C::kIPU, NWW = C::kWordsPerWarp;
+  extern __shared__ __align__(128) unsigned char smem[];
+  __shared__ uint64_t bar_full[kMaxNB * kMaxSets];
+  __shared__ int slot_bad[kMaxNB * kMaxSets];
+  __shared__ volatile int cta_abort;
+  __shared__ int cta_flags[2];
+  __shared__ int epi_tiles[kEpiChunk];
+  __shared__ int epi_count;
+  __shared__ __align__(16) Params p;
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  static_assert(sizeof(Params) % 4 == 0 && sizeof(Params) / 4 <= C::kThreads, "parameter copy");
+  if (tid < int(sizeof(Params) / 4))
+    reinterpret_cast<uint32_t*>(&p)[tid] = reinterpret_cast<const uint32_t*>(&params)[tid];
+  if (tid == 0) cta_abort = 0;
+  __syncthreads();
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  const int G = p.G, NB = p.NB, S = p.S, cta = blockIdx.x;
+  const int L = rec_lo(p, cta), H = rec_lo(p, cta + 1);
+  const Batches bt(L, H, G, NB);
+  if (bt.nbatch == 0) return;  // nothing to read or write
+  const MetaOff mo(B);
+
+  // -- directory cache: entries (start, end) of records [dbase, dbase + kDirCache), in 16-byte units
+  uint32_t* dlo = reinterpret_cast<uint32_t*>(smem + p.dir_off);
+  uint32_t* dhi = dlo + kDirCache;
+  int dbase = L;
+  auto fill_dir = [&](int from) {
+    for (int j = from + tid; j < min(H, from + kDirCache); j += C::kThreads) {
+      const int m = mat_of_rec(p, j);
+      const int jl = j - (m == 0 ? 0 : m == 1 ? p.rec_start[1] : m == 2 ? p.rec_start[2] : p.rec_start[3]);
+      const uint32_t* dir = pick(p.dir, m);
+      dlo[j - from] = __ldg(dir + jl);
+      dhi[j - from] = __ldg(dir + jl + 1);
+    }
+  };
+  fill_dir(L);
+  if (tid == 0) {
+    for (int i = 0; i < NB * S; ++i) mbar_init(&bar_full[i], 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+
+  // Record j (CTA-local index j - L) streams into slot (j - L) % NS; its use of that slot is number (j - L) / NS,
+  // which sets the mbarrier phase parity. A batch is issued only when the batch S before it is done, and the S
+  // batches from there hold at most NS records, so a slot's previous record is always finished.
+  const int NS = NB * S;
+  auto slot_ptr = [&](int slot) { return smem + slot * p.stage_size; };
+  // metadata blocks from the first 256-byte boundary of their region (the nibble-table lookups put an index in
+  // the low byte of a table address); the plan leaves 256 bytes of room for this
+  const int meta0 = int(((smem_u32(smem + p.meta_off) + 255u) & ~255u) - smem_u32(smem));
+  auto meta_ptr = [&](int mp, int pos) { return smem + meta0 + (mp * NB + pos) * p.meta_rec; };
+  auto res_addr = [&](int n, int pos) { return smem_u32(smem + p.res_off + ((n & 1) * NB + pos) * p.res_rec); };
+
+  // Bulk copies of records [rb, re) (warp 0, one record per lane, at most 32): the records (with_rec) and the
+  // activation rows (with_x) into their slots. The mbarrier of a slot expects both.
+  auto issue = [&](int rb, int re, bool with_rec, bool with_x) {
+    const int j = rb + lane;
+    if (j >= re) return;
+    const int slot = (j - L) % NS;
+    uint64_t* bar = &bar_full[slot];
+    unsigned char* dst = slot_ptr(slot);
+    if (with_rec) {
+      const uint32_t a = dlo[j - dbase], b = dhi[j - dbase];
+      const int m = mat_of_rec(p, j);
+      const unsigned bytes = 16u * (b - a);
+      if (b < a || b > pick(p.units_total, m) || bytes > unsigned(p.stage_bytes)) {  // not what was promised
+        slot_bad[slot] = 1;
+        atomicOr(p.status, kStatusOversize);
+        mbar_arrive(bar);
+        return;
+      }
+      slot_bad[slot] = 0;
+      mbar_arrive_tx(bar, bytes + 128u * B);
+      if (j != p.withhold) tma_bulk_load(dst, pick(p.recs, m) + 16ull * a, bytes, bar);
+    }
+    if (with_x && !slot_bad[slot] && j != p.withhold) {
+      const int g = j % G;
+#pragma unroll
+      for (int bb = 0; bb < B; ++bb)
+        tma_bulk_load(dst + p.stage_bytes + 128 * bb, p.x + size_t(bb) * p.K + size_t(g) * 64, 128u, bar);
+    }
+  };
+
+  // Meta job of record j (whole warp) into meta set mp: wait for the record, validate it, write its metadata.
+  auto meta_job = [&](int j, int mp, int pos) {
+    const int slot = (j - L) % NS;
+    const unsigned char* st = slot_ptr(slot);
+    const uint32_t sa = smem_u32(st);
+    unsigned char* mb = meta_ptr(mp, pos);
+    bool ok = mbar_wait(&bar_full[slot], ((j - L) / NS) & 1, p.status, &cta_abort, p.wait_ns);
+    ok = __all_sync(0xFFFFFFFFu, ok) && !slot_bad[slot];
+    const int Rt = tile_out(p, j / G).Rt;
+    int n0 = 0, n1 = 0, n2 = 0, n3 = 0;
+    if (ok) {
+      const uint2 cnt = lds64(sa);
+      n0 = cnt.x & 0xFFFF; n1 = cnt.x >> 16; n2 = cnt.y & 0xFFFF; n3 = cnt.y >> 16;
+      const Rec rc(Rt, n0, n1, n2, n3);
+      if (n0 + n1 + n2 + n3 != Rt || rc.c3 + 64 * n3 > p.stage_bytes) {
+        if (lane == 0) atomicOr(p.status, kStatusRecord);
+        ok = false;
+      }
+    }
+    uint32_t m0 = 0, m1 = 0, m2 = 0, m3 = 0;
+    unsigned long long v = 0, pre = 0;
+    if (ok) {
+      // width masks and item starts per 32-row word (lane = word)
+      const int nvalid = max(0, min(32, Rt - 32 * lane));
+      if (nvalid > 0) {
+        const uint2 v2 = lds64(sa + 8 + 8 * lane);
+        v = (unsigned long long)v2.x | ((unsigned long long)v2.y << 32);
+      }
+      const uint32_t lo = even_bits(v), hi = even_bits(v >> 1);
+      const uint32_t valid = nvalid >= 32 ? 0xFFFFFFFFu : ((1u << nvalid) - 1u);
+      m0 = ~hi & ~lo & valid;
+      m1 = ~hi & lo & valid;
+      m2 = hi & ~lo & valid;
+      m3 = hi & lo & valid;
+      const unsigned long long mine = (unsigned long long)__popc(m0) | ((unsigned long long)__popc(m1) << 16) |
+                                      ((unsigned long long)__popc(m2) << 32) | ((unsigned long long)__popc(m3) << 48);
+      unsigned long long incl = mine;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const unsigned long long u = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+        if (lane >= off) incl += u;
+      }
+      pre = incl - mine;
+      const unsigned long long tot = __shfl_sync(0xFFFFFFFFu, incl, 31);
+      if (tot != ((unsigned long long)n0 | ((unsigned long long)n1 << 16) | ((unsigned long long)n2 << 32) |
+                  ((unsigned long long)n3 << 48))) {
+        if (lane == 0) atomicOr(p.status, kStatusRecord);
+        ok = false;
+      }
+    }
+    int* fl = reinterpret_cast<int*>(mb + mo.fl);
+    if (ok) {
+      uint32_t* mk = reinterpret_cast<uint32_t*>(mb + mo.mk);
+      uint16_t* pf = reinterpret_cast<uint16_t*>(mb + mo.pf);
+      uint32_t* wc = reinterpret_cast<uint32_t*>(mb + mo.wc);
+      mk[lane] = m0; mk[32 + lane] = m1; mk[64 + lane] = m2; mk[96 + lane] = m3;
+      pf[lane] = uint16_t(pre & 0xFFFFull);
+      pf[32 + lane] = uint16_t(n0 + int((pre >> 16) & 0xFFFFull));
+      pf[64 + lane] = uint16_t(n0 + n1 + int((pre >> 32) & 0xFFFFull));
+      pf[96 + lane] = uint16_t(n0 + n1 + n2 + int(pre >> 48));
+      wc[2 * lane] = uint32_t(v);
+      wc[2 * lane + 1] = uint32_t(v >> 32);
+      // activation tables [3][B][64]: x, x * 2^-shift (2-bit codes), x * 2^-shift (4-bit codes); group sums
+      const uint16_t* xg = reinterpret_cast<const uint16_t*>(st + p.stage_bytes);
+      float* xv = reinterpret_cast<float*>(mb + mo.xt);
+      float* sgv = reinterpret_cast<float*>(mb + mo.sg);
+      const float s2a = __uint_as_float(uint32_t(127 - code_shift<2>(lane)) << 23);
+      const float s2b = __uint_as_float(uint32_t(127 - code_shift<2>(32 + lane)) << 23);
+      const float s4a = __uint_as_float(uint32_t(127 - code_shift<4>(lane)) << 23);
+      const float s4b = __uint_as_float(uint32_t(127 - code_shift<4>(32 + lane)) << 23);
+#pragma unroll
+      for (int b = 0; b < B; ++b) {
+        const float x0 = __uint_as_float(uint32_t(xg[b * 64 + lane]) << 16);
+        const float x1 = __uint_as_float(uint32_t(xg[b * 64 + 32 + lane]) << 16);
+        xv[b * 64 + lane] = x0;
+        xv[b * 64 + 32 + lane] = x1;
+        xv[(B + b) * 64 + lane] = x0 * s2a;
+        xv[(B + b) * 64 + 32 + lane] = x1 * s2b;
+        xv[(2 * B + b) * 64 + lane] = x0 * s4a;
+        xv[(2 * B + b) * 64 + 32 + lane] = x1 * s4b;
+        float sg = x0 + x1;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) sg += __shfl_xor_sync(0xFFFFFFFFu, sg, off);
+        if (lane == 0) sgv[b] = sg;
+      }
+      __syncwarp();
+      // 1-bit nibble tables: lane = (position p, half h) builds entries 8h .. 8h + 7 of position p of each row
+      const int pp = lane >> 1, hh = lane & 1;
+      const uint32_t xa = smem_u32(mb + mo.xt), ta = smem_u32(mb + mo.lut) + 64 * pp + 32 * hh;
+#pragma unroll
+      for (int b = 0; b < B; ++b) {
+        const float4 q = lds128f(xa + 256 * b + 16 * pp);
+        const float base = hh ? q.w : 0.f;
+        const float e1 = base + q.x, e2 = base + q.y, e3 = e1 + q.y;
+        const uint32_t lo4[4] = {__float_as_uint(base), __float_as_uint(e1), __float_as_uint(e2), __float_as_uint(e3)};
+        const uint32_t hi4[4] = {__float_as_uint(base + q.z), __float_as_uint(e1 + q.z), __float_as_uint(e2 + q.z),
+                                 __float_as_uint(e3 + q.z)};
+        sts128(ta + 1024 * b, lo4);
+        sts128(ta + 1024 * b + 16, hi4);
+      }
+      if (lane == 0) {
+        const Rec rc(Rt, n0, n1, n2, n3);
+        fl[1] = rc.sc;
+        fl[2] = n0; fl[3] = n1; fl[4] = n2; fl[5] = n3;
+        fl[6] = rc.c0; fl[7] = rc.c1; fl[8] = rc.c2; fl[9] = rc.c3;
+      }
+    } else if (lane == 0) {
+      fl[2] = fl[3] = fl[4] = fl[5] = 0;
+    }
+    if (lane == 0) fl[0] = ok ? 0 : 1;
+  };
+
+  // Jobs of batch [rb, re) (meta set mp) for this warp: the meta jobs of the next batch [nrb, nre) (segment 0,
+  // into meta set mpn) and the units of this batch's records, buckets in the order 1, 8, 2, 4 bits (8-bit units
+  // read the raw activation table, which the 1-bit units leave in place).
+  auto jobs = [&](int n, int rb, int re, int mp, int nrb, int nre, int mpn) {
+    const int nrec = re - rb;
+    int count = 0, cost = 0;
+    if (lane == 0) {
+      count = nre - nrb;
+      cost = p.cost[4];
+    } else if (lane - 1 < 4 * nrec) {
+      const int pos = (lane - 1) >> 2, q = (lane - 1) & 3;
+      const int k = q == 0 ? 0 : q == 1 ? 3 : q == 2 ? 1 : 2;
+      const int* fl = reinterpret_cast<const int*>(meta_ptr(mp, pos) + mo.fl);
+      const int nk = fl[2 + k];
+      count = k == 0 ? (nk + 31) >> 5 : (nk + IPU - 1) / IPU;
+      cost = p.cost[k];
+    }
+    const int tot = count * cost;
+    int incl = tot;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int u = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+      if (lane >= off) incl += u;
+    }
+    const int s0 = incl - tot, total = __shfl_sync(0xFFFFFFFFu, incl, 31);
+    const int jlo = first_job(2 * total * warp, s0, max(cost, 1), count, W);
+    const int jhi = first_job(2 * total * (warp + 1), s0, max(cost, 1), count, W);
+    // units first, the meta jobs last (their records were issued most recently)
+    unsigned todo = __ballot_sync(0xFFFFFFFFu, jhi > jlo);
+    todo = (todo >> 1) | ((todo & 1u) << 31);
+    float xr[64];
+    int loaded = -1;
+    const int t = rb / G;
+    const float corr = pick(p.sym, mat_of_tile(p, t)) != 0 ? 1.f : 0.5f;
+    int slot0 = (rb - L) % NS;
+    while (todo) {
+      const int sgi = __ffs(todo) & 31;  // bit i holds segment i + 1; bit 31 holds segment 0
+      todo &= todo - 1;
+      const int lo = __shfl_sync(0xFFFFFFFFu, jlo, sgi), hi = __shfl_sync(0xFFFFFFFFu, jhi, sgi);
+      if (sgi == 0) {
+        for (int jb = lo; jb < hi; ++jb) meta_job(nrb + jb, mpn, jb);
+        continue;
+      }
+      const int pos = (sgi - 1) >> 2, q = (sgi - 1) & 3;
+      const int k = q == 0 ? 0 : q == 1 ? 3 : q == 2 ? 1 : 2;
+      const unsigned char* mb = meta_ptr(mp, pos);
+      const int* fl = reinterpret_cast<const int*>(mb + mo.fl);
+      const int nk = fl[2 + k], cb = fl[6 + k], sc = fl[1];
+      const int ib = k == 0 ? 0 : k == 1 ? fl[2] : k == 2 ? fl[2] + fl[3] : fl[2] + fl[3] + fl[4];
+      int slot = slot0 + pos;
+      if (slot >= NS) slot -= NS;
+      const uint32_t sa = smem_u32(slot_ptr(slot));
+      const uint32_t res = res_addr(n, pos) + 4 * B * ib;
+      const uint32_t sca = sa + sc + 2 * ib;
+      if (k == 0) {
+        float sgb[B];
+#pragma unroll
+        for (int b = 0; b < B; ++b) sgb[b] = reinterpret_cast<const float*>(mb + mo.sg)[b];
+        unit_range_b1<B>(nk, lo, hi, lane, sa + cb, sca, res, smem_u32(mb + mo.lut), sgb);
+        continue;
+      }
+      const int tbl = k == 1 ? 1 : k == 2 ? 2 : 0;
+      const int b = lane % B;
+      if (loaded != pos * 4 + tbl) {
+        const uint32_t xa = smem_u32(mb + mo.xt) + 256 * (tbl * B + b);
+#pragma unroll
+        for (int qq = 0; qq < 16; ++qq) {
+          const float4 f = lds128f(xa + 16 * qq);
+          xr[4 * qq] = f.x; xr[4 * qq + 1] = f.y; xr[4 * qq + 2] = f.z; xr[4 * qq + 3] = f.w;
+        }
+        loaded = pos * 4 + tbl;
+      }
+      const float sg = reinterpret_cast<const float*>(mb + mo.sg)[b];
+      if (k == 1) unit_range<2, B>(nk, lo, hi, lane, sa + cb, sca, res, xr, sg, corr);
+      else if (k == 2) unit_range<4, B>(nk, lo, hi, lane, sa + cb, sca, res, xr, sg, corr);
+      else unit_range<8, B>(nk, lo, hi, lane, sa + cb, sca, res, xr, sg, corr);
+    }
+  };
+
+  // -- prologue: the first S batches' records, then (once the kernel before this one has finished, under
+  // programmatic dependent launch) their activations; the meta jobs of batch 0
+  const int pre_batches = min(S, bt.nbatch);
+  int rb, re, pre_end;
+  bt.get(0, rb, re);
+  {
+    int a0, a1;
+    bt.get(pre_batches - 1, a0, a1);
+    pre_end = a1;  // the first S batches are records [L, pre_end), at most NS <= 32 of them
+  }
+  if (warp == 0) issue(L, pre_end, true, false);
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  if (warp == 0) {
+    __syncwarp();
+    issue(L, pre_end, false, true);
+  }
+  for (int pos = warp; pos < re - rb; pos += W) meta_job(rb + pos, 0, pos);
+  // every thread leaves each barrier with the same verdict on the CTA's abort flag
+  bool aborted = __syncthreads_or(cta_abort != 0) != 0;
+
+  float acc[NWW][B];
+#pragma unroll
+  for (int ww = 0; ww < NWW; ++ww)
+#pragma unroll
+    for (int b = 0; b < B; ++b) acc[ww][b] = 0.f;
+  int last_issued_end = pre_end;
+  int mp = 0;  // meta set of batch n (n % 3)
+  for (int n = 0; n < bt.nbatch && !aborted; ++n) {
+    int nrb = 0, nre = 0;
+    if (n + 1 < bt.nbatch) bt.get(n + 1, nrb, nre);
+    const int mpn = mp == 2 ? 0 : mp + 1;
+    jobs(n, rb, re, mp, nrb, nre, mpn);
+    aborted = __syncthreads_or(cta_abort != 0) != 0;
+    if (aborted) break;
+    // refill the slots of batch n with batch n + S (their records and activation rows)
+    if (n + S < bt.nbatch) {
+      int rb2, re2;
+      bt.get(n + S, rb2, re2);
+      if (re2 > dbase + kDirCache) {  // uniform: every thread takes this branch together
+        dbase = rb2;
+        fill_dir(rb2);
+        __syncthreads();
+      }
+      if (warp == 0) {
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        issue(rb2, re2, true, true);
+      }
+      last_issued_end = re2;
+    }
+    // row pass of batch n: this warp's words, records in order
+    const int t = rb / G;
+    const TileOut to = tile_out(p, t);
+    const int Rt = to.Rt;
+    for (int pos = 0; pos < re - rb; ++pos) {
+      const unsigned char* mb = meta_ptr(mp, pos);
+      if (reinterpret_cast<const int*>(mb + mo.fl)[0]) continue;  // bad record (status already set)
+      const uint32_t* mk = reinterpret_cast<const uint32_t*>(mb + mo.mk);
+      const uint16_t* pf = reinterpret_cast<const uint16_t*>(mb + mo.pf);
+      const uint32_t* wc = reinterpret_cast<const uint32_t*>(mb + mo.wc);
+      const uint32_t res = res_addr(n, pos);
+#pragma unroll
+      for (int ww = 0; ww < NWW; ++ww) {
+        const int word = warp + ww * W, r = 32 * word + lane;
+        if (r < Rt) {
+          const int c = int(wc[r >> 4] >> (2 * (r & 15))) & 3;
+          const int item = pf[c * 32 + word] + __popc(mk[c * 32 + word] & ((1u << lane) - 1u));
+#pragma unroll
+          for (int b = 0; b < B; ++b) acc[ww][b] += lds32f(res + 4 * (item * B + b));
+        }
+      }
+    }
+    // tile end: this CTA's share of tile t is complete
+    if (n + 1 == bt.nbatch || nrb / G != t) {
+      const bool whole = L <= t * G && H >= (t + 1) * G;
+      float* slot = p.partial + size_t(cta + t) * p.R * B;
+#pragma unroll
+      for (int ww = 0; ww < NWW; ++ww) {
+        const int r = 32 * (warp + ww * W) + lane;
+        if (r < Rt) {
+#pragma unroll
+          for (int b = 0; b < B; ++b) {
+            if (whole) to.y[size_t(b) * to.ld + r] = acc[ww][b];
+            else slot[r * B + b] = acc[ww][b];
+          }
+        }
+#pragma unroll
+        for (int b = 0; b < B; ++b) acc[ww][b] = 0.f;
+      }
+    }
+    rb = nrb;
+    re = nre;
+    mp = mpn;
+  }
+  if (aborted) {
+    // wait (bounded) for the copies still in flight before the CTA exits; publish nothing. Only the last use of
+    // each slot can still be in flight: the last NS records issued.
+    if (warp == 0) {
+      const int j = last_issued_end - NS + lane;
+      if (lane < NS && j >= L) mbar_drain(&bar_full[(j - L) % NS], ((j - L) / NS) & 1, p.wait_ns);
+    }
+    return;
+  }
+  finish_cta<B, C::kThreads>(p, L, H, cta_flags, epi_tiles, &epi_count);
 }
 
 // ------------------------------------------------------------------------------------------ launch plan
 struct Plan {
   int grid, threads, NT, TW, S, stage_bytes, stage_size, team_bytes, acc_off, res_off, warps_off, warp_bytes, smem;
+  int NB, meta_off, dir_off, res_rec, meta_rec;  // CUDA-core kernel
   uint64_t ws_bytes, status_off, counters_off;
 };
+
 
 inline int num_sms() {
   int dev = 0, sms = 148;
@@ -1146,6 +1702,15 @@ inline int make_problem(int nmat, const vbq_desc* const* d, Problem& pr) {
   return VBQ_OK;
 }
 
+// Workspace: partial slots [nCTA + T][R][B] f32 of the row tiles that CTAs share, then an arrival counter and a
+// SwiGLU pair counter per tile, then the status word.
+inline void plan_workspace(const Problem& pr, int B, Plan& pl) {
+  const uint64_t slots = uint64_t(pl.grid) + uint64_t(pr.T);
+  pl.counters_off = slots * uint64_t(pr.R) * B * 4;
+  pl.ws_bytes = (pl.counters_off + uint64_t(pr.T) * 8 + 4 + 15) / 16 * 16;
+  pl.status_off = pl.ws_bytes - 4;
+}
+
 // Teams per CTA, warps per team and stages per team. A team's record copies overlap its arithmetic when it has
 // two stages; with one, every record's load latency is exposed. The plan that fits in shared memory with the
 // fewest exposed load latencies (records per team / stages, rounded up) wins; ties go to more warps, then to
@@ -1188,29 +1753,70 @@ inline bool make_plan_t(const Problem& pr, int sms, Plan& pl) {
     }
   }
   if (best_key < 0) return false;
-  const uint64_t slots = uint64_t(pl.grid) + uint64_t(pr.T);
-  pl.counters_off = slots * uint64_t(R) * B * 4;
-  // counters: arrivals per tile, then SwiGLU pair counters per tile; then the status word
-  pl.ws_bytes = (pl.counters_off + uint64_t(pr.T) * 8 + 4 + 15) / 16 * 16;
-  pl.status_off = pl.ws_bytes - 4;
+  plan_workspace(pr, B, pl);
+  return true;
+}
+
+// CUDA-core kernel (B <= 4): records per batch NB and batches in flight S. NB aims at about three jobs per warp
+// per batch (from an estimate of the units per record at the paper's allocation); S = 3 when it fits (the meta
+// jobs of a batch read records issued two batches earlier), else 2. Fewer records per batch before fewer sets.
+template <int B>
+inline bool make_plan_cc(const Problem& pr, int sms, Plan& pl) {
+  using C = CCfg<B>;
+  pl.grid = sms;
+  pl.threads = C::kThreads;
+  const int R = pr.R;
+  pl.stage_bytes = align128i(int(pr.max_record_bytes));
+  pl.stage_size = pl.stage_bytes + align128i(128 * B);
+  pl.res_rec = align128i(R * B * 4);
+  pl.meta_rec = MetaOff(B).size;
+  const int dir_bytes = 8 * kDirCache;
+  // units per record at the paper's allocation: 1-bit units of 32 items, the others of 32 / B; bucket tails
+  const int upr = (7 * R / 10 + 31) / 32 + (3 * R / 10 + C::kIPU - 1) / C::kIPU + 2;
+  const int nb_want = std::min(kMaxNB, std::max(1, (4 * C::kWarps + upr - 1) / upr));
+  pl.NB = 0;
+  for (int NB = nb_want; NB >= 1 && pl.NB == 0; --NB)
+    for (int S = 3; S >= 2; --S) {
+      const long long smem = (long long)S * NB * pl.stage_size + 2ll * NB * pl.res_rec + 256 +
+                             3ll * NB * pl.meta_rec + dir_bytes;
+      if (smem <= kSmemBudget) {
+        pl.NB = NB;
+        pl.S = S;
+        break;
+      }
+    }
+  if (pl.NB == 0) return false;
+  pl.res_off = pl.S * pl.NB * pl.stage_size;
+  pl.meta_off = pl.res_off + 2 * pl.NB * pl.res_rec;
+  pl.dir_off = pl.meta_off + 256 + 3 * pl.NB * pl.meta_rec;
+  pl.smem = pl.dir_off + dir_bytes;
+  pl.NT = pl.TW = 1;
+  pl.team_bytes = pl.acc_off = pl.warps_off = pl.warp_bytes = 0;
+  plan_workspace(pr, B, pl);
   return true;
 }
 
 inline bool make_plan(const Problem& pr, int B, int sms, Plan& pl) {
   switch (B) {
-    case 1: return make_plan_t<1>(pr, sms, pl);
-    case 2: return make_plan_t<2>(pr, sms, pl);
-    case 4: return make_plan_t<4>(pr, sms, pl);
+    case 1: return make_plan_cc<1>(pr, sms, pl);
+    case 2: return make_plan_cc<2>(pr, sms, pl);
+    case 4: return make_plan_cc<4>(pr, sms, pl);
     case 8: return make_plan_t<8>(pr, sms, pl);
     default: return make_plan_t<16>(pr, sms, pl);
   }
 }
 
+// Test hook (vbq_test_set_fault): a shorter limit for the kernels' bounded waits and one record whose bulk copy
+// is never issued, so that a wait runs out. Off by default.
+std::atomic<unsigned long long> g_test_wait_ns{0};
+std::atomic<long long> g_test_withhold{-1};
+
 template <int B>
 int launch(const Problem& pr, const void* const* blobs, const void* x, float* const* ys, void* ws, uint64_t ws_bytes,
-           unsigned flags, cudaStream_t stream, uint16_t* h = nullptr) {
+           unsigned flags, cudaStream_t stream, uint16_t* h = nullptr, unsigned* status = nullptr) {
+  constexpr bool cc = B <= 4;  // CUDA-core kernel; batch 8 and 16 run the tensor-core kernel
   Plan pl;
-  if (!make_plan_t<B>(pr, num_sms(), pl)) return VBQ_ERR_FORMAT;
+  if (!(cc ? make_plan_cc<B>(pr, num_sms(), pl) : make_plan_t<B>(pr, num_sms(), pl))) return VBQ_ERR_FORMAT;
   if (!ws || (reinterpret_cast<uintptr_t>(ws) & 15) || ws_bytes < pl.ws_bytes) return VBQ_ERR_WORKSPACE;
   Params p = {};
   p.nmat = pr.nmat;
@@ -1239,7 +1845,7 @@ int launch(const Problem& pr, const void* const* blobs, const void* x, float* co
   p.pair = p.arrive + tiles;
   p.swiglu = h != nullptr;
   p.h = h;
-  p.status = reinterpret_cast<unsigned*>(w + pl.status_off);
+  p.status = status ? status : reinterpret_cast<unsigned*>(w + pl.status_off);
   p.K = pr.K; p.G = pr.G; p.R = pr.R; p.T = tiles;
   p.nrec = recs;
   p.NT = pl.NT; p.TW = pl.TW; p.S = pl.S;
@@ -1250,13 +1856,29 @@ int launch(const Problem& pr, const void* const* blobs, const void* x, float* co
   p.res_off = pl.res_off;
   p.warps_off = pl.warps_off;
   p.warp_bytes = pl.warp_bytes;
+  p.NB = pl.NB;
+  p.meta_off = pl.meta_off;
+  p.dir_off = pl.dir_off;
+  p.res_rec = pl.res_rec;
+  p.meta_rec = pl.meta_rec;
+  // job costs (about the instructions a warp spends): units of 1-, 2-, 4-, 8-bit groups; a meta job
+  p.cost[0] = 30 + 40 * B;
+  p.cost[1] = 145;
+  p.cost[2] = 150;
+  p.cost[3] = 145;
+  p.cost[4] = 150 + 30 * B;
+  const unsigned long long wl = g_test_wait_ns.load();
+  p.wait_ns = wl ? wl : kWaitNs;
+  const long long wh = g_test_withhold.load();
+  p.withhold = (wh >= 0 && wh < recs) ? int(wh) : -1;
+  auto kern = cc ? vbq_cc_kernel<(B <= 4 ? B : 1)> : vbq_kernel<B>;
   // Opt in to the dynamic shared memory once per device and size.
   static int opted[64] = {0};
   int dev = 0;
   cudaGetDevice(&dev);
   int& done = opted[dev & 63];
   if (pl.smem > done) {
-    if (cudaFuncSetAttribute(vbq_kernel<B>, cudaFuncAttributeMaxDynamicSharedMemorySize, pl.smem) != cudaSuccess)
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, pl.smem) != cudaSuccess)
       return VBQ_ERR_CUDA;
     done = pl.smem;
   }
@@ -1270,11 +1892,12 @@ int launch(const Problem& pr, const void* const* blobs, const void* x, float* co
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = (flags & VBQ_LAUNCH_OVERLAP) ? 1 : 0;
-  if (cudaLaunchKernelEx(&cfg, vbq_kernel<B>, p) != cudaSuccess) return VBQ_ERR_CUDA;
+  if (cudaLaunchKernelEx(&cfg, kern, p) != cudaSuccess) return VBQ_ERR_CUDA;
   return cudaPeekAtLastError() == cudaSuccess ? VBQ_OK : VBQ_ERR_CUDA;
 }
 
 inline bool batch_ok(int B) { return B == 1 || B == 2 || B == 4 || B == 8 || B == 16; }
+
 
 }  // namespace vbq
 
@@ -1376,17 +1999,27 @@ int vbq_gemv(const vbq_desc* d, const void* blob_dev, const void* x_bf16, float*
   return vbq_gemm_skinny(d, blob_dev, x_bf16, 1, y, workspace, workspace_bytes, stream);
 }
 
+int vbq_test_set_fault(uint64_t wait_limit_ns, int64_t withheld_record) {
+  vbq::g_test_wait_ns.store(wait_limit_ns);
+  vbq::g_test_withhold.store(withheld_record < 0 ? -1 : withheld_record);
+  return VBQ_OK;
+}
+
 }  // extern "C"
 
 // ------------------------------------------------------------------------------ allocation-free variant
 // Scratch for vbq_gemm_skinny_noalloc: one fixed buffer per device, created when the library is loaded on that
-// device and kept until the process exits. It replaces the caller-provided workspace of vbq_gemm_skinny.
+// device and kept until the process exits. It replaces the caller-provided workspace of vbq_gemm_skinny: the
+// split-K partial sums and the counters take its first 16 MiB - 256 bytes, and its last 256 bytes hold the status
+// word, at a fixed place so that vbq_noalloc_status can read it.
 namespace vbq {
 constexpr uint64_t kStaticScratchBytes = 16ull << 20;  // 16 MiB
+constexpr uint64_t kStaticStatusOff = kStaticScratchBytes - 256;
 static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
 
 // Device address of g_static_scratch on the current device. In host code the array's name is only a host-side
-// stand-in, so the address is looked up once per device with cudaGetSymbolAddress (that device current).
+// stand-in, so the address is looked up once per device with cudaGetSymbolAddress (that device current) and
+// kept; a device reset (cudaDeviceReset) would void it.
 int static_scratch(void** out) {
   static std::mutex mu;
   static void* addr[64] = {nullptr};
@@ -1410,18 +2043,40 @@ extern "C" int vbq_gemm_skinny_noalloc(const vbq_desc* d, const void* blob_dev, 
   if (!vbq::desc_ok(d)) return VBQ_ERR_FORMAT;
   uint64_t need = 0;
   if (int st = vbq_workspace_size(d, B, &need)) return st;
-  if (need > vbq::kStaticScratchBytes) return VBQ_ERR_SCRATCH_LIMIT;
+  if (need > vbq::kStaticStatusOff) return VBQ_ERR_SCRATCH_LIMIT;
+  if ((reinterpret_cast<uintptr_t>(x_bf16) & 15) || (reinterpret_cast<uintptr_t>(blob_dev) & 15) ||
+      (reinterpret_cast<uintptr_t>(y) & 3))
+    return VBQ_ERR_ALIGN;
   void* scratch = nullptr;
   if (int st = vbq::static_scratch(&scratch)) return st;
-  // The buffer keeps the previous call's contents: clear the arrival counters and the status word, which the
-  // kernel needs at zero. The partial-sum area is always written before it is read.
+  unsigned char* base = static_cast<unsigned char*>(scratch);
   vbq::Problem pr;
   if (int st = vbq::make_problem(1, &d, pr)) return st;
   vbq::Plan pl;
   if (!vbq::make_plan(pr, B, vbq::num_sms(), pl)) return VBQ_ERR_FORMAT;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(static_cast<unsigned char*>(scratch) + pl.counters_off, 0,
-                      size_t(need - pl.counters_off), st) != cudaSuccess)
+  // The buffer keeps the previous call's contents: clear the arrival counters and the status word, which the
+  // kernel needs at zero. The partial-sum area is always written before it is read.
+  if (cudaMemsetAsync(base + pl.counters_off, 0, size_t(need - pl.counters_off), st) != cudaSuccess ||
+      cudaMemsetAsync(base + vbq::kStaticStatusOff, 0, 4, st) != cudaSuccess)
     return VBQ_ERR_CUDA;
-  return vbq_gemm_skinny(d, blob_dev, x_bf16, B, y, scratch, need, stream);
+  unsigned* status = reinterpret_cast<unsigned*>(base + vbq::kStaticStatusOff);
+  const void* blobs[1] = {blob_dev};
+  float* ys[1] = {y};
+  switch (B) {
+    case 1: return vbq::launch<1>(pr, blobs, x_bf16, ys, base, need, 0u, st, nullptr, status);
+    case 2: return vbq::launch<2>(pr, blobs, x_bf16, ys, base, need, 0u, st, nullptr, status);
+    case 4: return vbq::launch<4>(pr, blobs, x_bf16, ys, base, need, 0u, st, nullptr, status);
+    case 8: return vbq::launch<8>(pr, blobs, x_bf16, ys, base, need, 0u, st, nullptr, status);
+    default: return vbq::launch<16>(pr, blobs, x_bf16, ys, base, need, 0u, st, nullptr, status);
+  }
+}
+
+extern "C" int vbq_noalloc_status(uint32_t* status_host, void* stream) {
+  if (!status_host) return VBQ_ERR_NULL;
+  void* scratch = nullptr;
+  if (int st = vbq::static_scratch(&scratch)) return st;
+  return cudaMemcpyAsync(status_host, static_cast<unsigned char*>(scratch) + vbq::kStaticStatusOff, 4,
+                         cudaMemcpyDeviceToHost, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? VBQ_OK : VBQ_ERR_CUDA;
 }

@@ -1,4 +1,4 @@
-// Host side of libvbq: the format-v1 packer, unpacker and blob validator (FORMAT.md).
+// Host side of libvbq: the packer, unpacker and blob validator of packed format v1.
 //
 // VBQ groups ("Variable Bit-width Quantization", section 3.1) are 64 contiguous weights along K of one output
 // row, each with its own fp16 scale and a width from {1,2,4,8}. The packer is the export-time contract check

@@ -87,6 +87,8 @@ def lib() -> ctypes.CDLL:
             "vbq_workspace_size_swiglu": (i32, [dp, dp, i32, ctypes.POINTER(u64)]),
             "vbq_gemm_swiglu": (i32, [dp, dp, vp, vp, vp, i32, vp, vp, vp, vp, u64, ctypes.c_uint, vp]),
             "vbq_gemm_skinny_noalloc": (i32, [dp, vp, vp, i32, vp, vp]),
+            "vbq_noalloc_status": (i32, [vp, vp]),
+            "vbq_test_set_fault": (i32, [u64, i64]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -308,6 +310,22 @@ def vbq_gemm_skinny_noalloc_status(desc, blob_dev, x_bf16, B, y, stream=None) ->
 
 def vbq_gemm_skinny_noalloc(desc, blob_dev, x_bf16, B, y, stream=None) -> None:
     _check(vbq_gemm_skinny_noalloc_status(desc, blob_dev, x_bf16, B, y, stream), "vbq_gemm_skinny_noalloc")
+
+
+def vbq_noalloc_status(stream=None) -> int:
+    """Device status word of the last vbq_gemm_skinny_noalloc call on the current device (0: no device-side
+    error). Enqueues the read on `stream` and synchronizes that stream."""
+    import torch
+    out = np.zeros(1, np.uint32)
+    st = _stream_ptr(stream)
+    _check(lib().vbq_noalloc_status(_np_ptr(out), st), "vbq_noalloc_status")
+    (stream or torch.cuda.current_stream()).synchronize()
+    return int(out[0])
+
+
+def vbq_test_set_fault(wait_limit_ns: int = 0, withheld_record: int = -1) -> None:
+    """Test hook of the failure-detection path: the kernels' wait limit and a record whose copy is withheld."""
+    _check(lib().vbq_test_set_fault(wait_limit_ns, withheld_record), "vbq_test_set_fault")
 
 
 def vbq_gemv(desc, blob_dev, x_bf16, y, workspace=None, stream=None) -> None:

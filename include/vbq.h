@@ -9,7 +9,7 @@
  *
  * The dequantized weight is w = s * (q - (2^k - 1)/2), with q in [0, 2^k). Format flag VBQ_FLAG_GRID_SYMMETRIC
  * puts widths k >= 2 on the paper's Eq. 1 integer grid instead: w = s * (q - (2^(k-1) - 1)), q in [0, 2^k - 2].
- * The byte layout is "format v1" of FORMAT.md: row tiles, one record per (tile, group column), and per-width
+ * The byte layout is packed format v1: row tiles, one record per (tile, group column), and per-width
  * buckets inside each record.
  *
  * Conventions for every function:
@@ -77,7 +77,7 @@ uint32_t vbq_version(void);
 
 /* ---------------------------------------------------------------------------------------------- host */
 
-/* Bytes of the canonical blob for this logical matrix (FORMAT.md, "Physical layout").
+/* Bytes of the canonical packed-format-v1 blob for this logical matrix.
  * widths: [N*G] in {1,2,4,8}. R: tile rows. Errors: NULL, SHAPE, TILE, WIDTH. Thread-safe, pure. */
 int vbq_packed_size(int64_t N, int64_t K, int64_t R, const uint8_t* widths, uint64_t* out_bytes);
 
@@ -200,8 +200,9 @@ int vbq_gemm_skinny_multi(int nmat, const vbq_desc* const* d, const void* const*
  * of the down projection. gate and up must have the same N (SHAPE), K (SHAPE) and tile rows (TILE).
  * h_bf16: B*N bf16 values, row-major, 2-byte aligned; y_gate, y_up as in vbq_gemm_skinny (also written).
  * workspace: vbq_workspace_size_swiglu(gate, up, B) bytes, zeroed once by vbq_workspace_init.
- * h meets |h - h_exact| <= 2^-8 |h_exact| + 1.1 |u| tol_g + |silu(g)| tol_u + tol_g tol_u + 1e-6, where
- * tol_g, tol_u are the vbq_gemv tolerances of y_gate, y_up; every output is bitwise identical from run to run.
+ * h meets |h - h_exact| <= P + 2^-8 (|h_exact| + P) + 1e-6 with P = 1.1 tol_g (|u| + tol_u) + |silu(g)| tol_u,
+ * where tol_g, tol_u are the vbq_gemv tolerances of y_gate, y_up (1.1 bounds |silu'|); every output is bitwise
+ * identical from run to run.
  * Errors: as vbq_gemm_skinny_multi. */
 int vbq_workspace_size_swiglu(const vbq_desc* gate, const vbq_desc* up, int B, uint64_t* out_bytes);
 int vbq_gemm_swiglu(const vbq_desc* gate, const vbq_desc* up, const void* blob_gate, const void* blob_up,
@@ -217,17 +218,36 @@ int vbq_gemm_swiglu(const vbq_desc* gate, const vbq_desc* up, const void* blob_g
  * (split-K partial sums, arrival counters, status word) lives in one fixed 16 MiB device buffer inside the
  * library. Every GPU that loads the library holds that buffer until the process exits.
  *
- * - Limit: problems whose vbq_workspace_size(d, B) exceeds 16 MiB are rejected with VBQ_ERR_SCRATCH_LIMIT, and
- *   nothing is launched. With 1024-row tiles that covers any N at B <= 4, and N up to about 110K at B = 16.
+ * - Limit: problems whose vbq_workspace_size(d, B) exceeds 16 MiB - 256 bytes are rejected with
+ *   VBQ_ERR_SCRATCH_LIMIT, and nothing is launched. With 1024-row tiles that covers any N at B <= 4, and N up to
+ *   about 110K at B = 16. The buffer's last 256 bytes hold the status word.
  * - First call per device: it looks up the buffer's device address (cudaGetSymbolAddress, with that device
- *   current). Make this first call before any stream capture.
- * - Each call clears the counters and the status word with one cudaMemsetAsync on `stream`, then launches the
+ *   current) and keeps it; a device reset voids it. Make this first call before any stream capture.
+ * - Each call clears the counters and the status word with cudaMemsetAsync on `stream`, then launches the
  *   same kernel as vbq_gemm_skinny. It allocates nothing and frees nothing.
  * - All calls on a device share the one buffer, which keeps the last call's contents. Calls that can overlap
  *   on the GPU (different streams, different host threads) race on it: serialize them.
+ * - Errors found on the device (a bounded wait that ran out, a record the kernel refused; the bits of the
+ *   vbq_workspace_size status word) are not returned by this call, which only enqueues the work: read them with
+ *   vbq_noalloc_status, enqueued on the same stream after the call and before the next noalloc call.
  * Errors: as vbq_gemm_skinny, plus SCRATCH_LIMIT; CUDA if the buffer's address cannot be obtained. */
 int vbq_gemm_skinny_noalloc(const vbq_desc* d, const void* blob_dev, const void* x_bf16, int B, float* y,
                             void* stream);
+
+/* Status word of the last vbq_gemm_skinny_noalloc call on the current device, as described for the workspace
+ * status word under vbq_workspace_size (0: no device-side error). It enqueues one cudaMemcpyAsync of 4 bytes on
+ * `stream` into *status_host; *status_host is valid once the stream has reached it (synchronize the stream or
+ * an event recorded after this call). The next noalloc call clears the word. Errors: NULL, CUDA. */
+int vbq_noalloc_status(uint32_t* status_host, void* stream);
+
+/* Test hook of the failure-detection path (the VBQ paper has no counterpart). Sets, for every later launch in
+ * this process: wait_limit_ns, the limit of the kernels' bounded mbarrier waits (0 restores the default of
+ * 2 s); withheld_record, a record of each launch (its index in the launch's record sequence: records of matrix 0
+ * first, tile-major) whose bulk copy is never issued, or -1 for none. A launch that withholds a record waits for
+ * it until the limit, then sets bit 0 of its status word, publishes nothing and returns; its workspace must be
+ * zeroed again before the next use. Not thread-safe against concurrent launches; meant for tests only.
+ * Returns VBQ_OK. */
+int vbq_test_set_fault(uint64_t wait_limit_ns, int64_t withheld_record);
 
 #ifdef __cplusplus
 }

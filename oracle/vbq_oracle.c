@@ -5,7 +5,8 @@
  * TEST INFRASTRUCTURE ONLY. Only the tests, the smoke check and the CPU-baseline
  * leg of the benchmark may load this file. The product path never does.
  * It shares no code with the CUDA library: it has its own packer, CRC, and
- * float decoders, written from FORMAT.md and from the IEEE definitions.
+ * float decoders, written from the packed-format-v1 specification and from the IEEE
+ * definitions.
  *
  * Method source: "Variable Bit-width Quantization: Learning Per-Group Precision
  * for 'Bigger-but-Smaller' Language Models", section 3.1 (contiguous groups of
@@ -126,7 +127,8 @@ static int check_logical(int64_t N, int64_t K, const uint8_t* widths, const uint
   return O_OK;
 }
 
-/* Size in bytes of record (t, g): FORMAT.md "Record (t, g)". */
+/* Size in bytes of record (t, g) of packed format v1: counts, width codes, scales, then the
+ * four code buckets, each part padded to 16 bytes. */
 static uint64_t record_bytes(int64_t Rt, const int64_t cnt[4]) {
   uint64_t sz = a16(8 + 4 * (uint64_t)((Rt + 15) / 16));
   sz += a16(2 * (uint64_t)Rt);
