@@ -39,6 +39,8 @@ GROUPS = (("q", "k", "v"), ("o",), ("gate", "up"), ("down",))   # projections th
 WORKLOAD = ("9B-shaped decode step: 32 layers of q,k,v,o 4096x4096, gate,up 4096->14336, down 14336->4096, "
             "plus the LM head 4096->32000")
 SYNTH_CFG = 5   # seed family of the full decode-step stack in vbq_synth
+RECIPE_CFG = 6  # seed family of the fixed-recipe stack (one width per projection, tiered LM head)
+L2_BYTES = 126e6
 
 # DRAM traffic of the kernel from one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum, cold L2) of the
 # first five launches of `python bench.py --layers 1 --steps 3 --warmup 3 --cpu-budget 0`: layer 0's four launch
@@ -125,9 +127,14 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------------------------------------ setup
-def step_matrices(layer: int):
-    """The seven linears of decoder layer `layer` (layer 0's MLP at the first-block mix)."""
-    return S.cfg5_layer(layer)
+def step_matrices(layer: int, recipe: bool = False):
+    """The seven linears of decoder layer `layer`: the paper's allocation (layer 0's MLP at the first-block mix),
+    or the fixed deployment recipe (one width per projection)."""
+    return S.cfg6_recipe_layer(layer) if recipe else S.cfg5_layer(layer)
+
+
+def head_matrix(recipe: bool = False):
+    return S.cfg6_recipe_head() if recipe else S.cfg5_head()
 
 
 def sample_matrices(with_head: bool = True):
@@ -250,6 +257,9 @@ def vbq_line(args, *, world, value, ms_max, step_bytes, weight_bytes, tile_rows,
     l2_bytes = 126e6
     workload = WORKLOAD if (args.layers == 32 and not args.no_head) else (
         f"{args.layers} of the 32 layers of the 9B-shaped decode step" + ("" if args.no_head else " plus the LM head"))
+    if args.workload == "recipe":
+        workload += ("; fixed deployment recipe: one width per projection (2-bit, first-block MLP 4-bit), LM head "
+                     "tiered by token frequency to 1.18 mean bits")
     return {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
@@ -263,9 +273,13 @@ def vbq_line(args, *, world, value, ms_max, step_bytes, weight_bytes, tile_rows,
                                 else "; q/k/v fused (vbq_gemm_skinny_multi); gate/up fused with the SwiGLU "
                                      "epilogue (vbq_gemm_swiglu) writing the down projection's input; "
                                      f"{launches_per_step} launches per step"),
-                   "weights": "seeded synthetic VBQ groups: P(1,2,4,8 bit) = (0.69,0.16,0.09,0.06), layer 0's "
-                              "MLP (0.40,0.35,0.15,0.10), LM head tiered to ~1.09 bits; fp16 scales "
-                              "U(0.01,0.1), uniform codes; x ~ N(0,1) bf16, one seeded x per linear",
+                   "weights": ("seeded synthetic VBQ groups: P(1,2,4,8 bit) = (0.69,0.16,0.09,0.06), layer 0's "
+                               "MLP (0.40,0.35,0.15,0.10), LM head tiered to ~1.09 bits; fp16 scales "
+                               "U(0.01,0.1), uniform codes; x ~ N(0,1) bf16, one seeded x per linear")
+                              if args.workload == "step" else
+                              ("seeded synthetic VBQ groups under the fixed recipe: uniform 2-bit projections, 4-bit "
+                               "layer-0 MLP, LM head rows 0.5/1.5/10/88% at 8/4/2/1 bits; fp16 scales U(0.01,0.1), "
+                               "uniform codes; x ~ N(0,1) bf16, one seeded x per linear"),
                    "l2": (f"inputs larger than L2: {step_bytes / 1e6:.0f} MB of distinct weights streamed once per "
                           "step" if step_bytes > 2 * l2_bytes else
                           f"inputs NOT larger than L2 ({step_bytes / 1e6:.0f} MB): L2-warm, not an HBM figure"),
@@ -306,16 +320,19 @@ def run_vbq(args):
     def tile_rows(ms):
         return R if R > 0 else vbq.suggest_tile_rows(sum(m.N for m in ms), ms[0].K, sms)
 
+    recipe = args.workload == "recipe"
+    xcfg = RECIPE_CFG if recipe else SYNTH_CFG
+
     def prepare(layer):
         """Host side of one layer (or the head, layer -1): seeded matrices, packed; logical arrays dropped."""
-        mats = [S.cfg5_head()] if layer < 0 else step_matrices(layer)
+        mats = [head_matrix(recipe)] if layer < 0 else step_matrices(layer, recipe)
         by_name = {m.name: m for m in mats}
         out = []
         for names in ([("head",)] if layer < 0 else groups):
             ms = [by_name[n] for n in names]
             rt = tile_rows(ms)
             blobs = [vbq.vbq_pack(m.N, m.K, rt, m.widths, m.scales, m.codes)[0] for m in ms]
-            x = S.make_x(SYNTH_CFG, names[0], B, ms[0].K, layer=max(layer, 0))
+            x = S.make_x(xcfg, names[0], B, ms[0].K, layer=max(layer, 0))
             out.append((names, rt, [(m.N, m.K) for m in ms], blobs, x))
         return layer, out
 
@@ -331,11 +348,9 @@ def run_vbq(args):
             g.shapes = shapes
             g.mats = [vbq.DeviceMatrix(bl, dev, max_batch=B) for bl in blobs]
             g.fused = vbq.FusedMatrices(g.mats, max_batch=B) if len(g.mats) > 1 else None
-            g.xh = torch.from_numpy(xb.astype(np.int16)).view(torch.bfloat16).pin_memory()
-            g.xd = g.xh.to(dev)
-            g.yd = [torch.empty((B, N), dtype=torch.float32, device=dev) for N, _ in shapes]
-            g.yh = [torch.empty((B, N), dtype=torch.float32).pin_memory() for N, _ in shapes]
-            g.nbytes = sum(mt.nbytes for mt in g.mats) + B * shapes[0][1] * 2 + sum(B * N * 4 for N, _ in shapes)
+            g.xb = xb
+            g.K = shapes[0][1]
+            g.nbytes = sum(mt.nbytes for mt in g.mats) + B * g.K * 2 + sum(B * N * 4 for N, _ in shapes)
             g.h = None
             g.x_from_device = False
             lin.append(g)
@@ -344,9 +359,9 @@ def run_vbq(args):
         names = [g.name.split(".")[-1] for g in lin]
         if "gate_up" in names and "down" in names:
             gu, dn = lin[names.index("gate_up")], lin[names.index("down")]
-            gu.h = dn.xd
-            gu.nbytes += dn.xd.numel() * 2
             dn.x_from_device = True
+            gu.h_of = dn
+            gu.nbytes += B * dn.K * 2
         return lin
 
     # Host preparation runs on a few threads (the packer and most of the generator release the GIL); device
@@ -357,6 +372,36 @@ def run_vbq(args):
     with cf.ThreadPoolExecutor(max_workers=min(4, os.cpu_count() or 1)) as pool:
         for layer, prepared in pool.map(prepare, order):
             step.extend(upload(layer, prepared))
+    # Activations and outputs live in one device buffer each, so that the end-to-end step moves them with one
+    # copy per direction from and to one pinned host buffer each. A down projection's input is the SwiGLU output
+    # of its gate/up launch, produced on the device: it has a buffer of its own and is not copied.
+    x_off, n_x = {}, 0
+    for i, g in enumerate(step):
+        if not g.x_from_device:
+            x_off[i] = n_x
+            n_x += B * g.K
+    n_y = sum(B * N for g in step for N, _ in g.shapes)
+    X_h = torch.empty(n_x, dtype=torch.bfloat16).pin_memory()
+    X_d = torch.empty(n_x, dtype=torch.bfloat16, device=dev)
+    Y_h = torch.empty(n_y, dtype=torch.float32).pin_memory()
+    Y_d = torch.empty(n_y, dtype=torch.float32, device=dev)
+    yo = 0
+    for i, g in enumerate(step):
+        if g.x_from_device:
+            g.xd = torch.empty((B, g.K), dtype=torch.bfloat16, device=dev)
+        else:
+            o = x_off[i]
+            X_h[o:o + B * g.K].copy_(torch.from_numpy(g.xb.astype(np.int16).reshape(-1)).view(torch.bfloat16))
+            g.xd = X_d[o:o + B * g.K].view(B, g.K)
+        g.yd = []
+        for N, _ in g.shapes:
+            g.yd.append(Y_d[yo:yo + B * N].view(B, N))
+            yo += B * N
+        del g.xb
+    for g in step:
+        if hasattr(g, "h_of"):
+            g.h = g.h_of.xd
+    X_d.copy_(X_h)
     t_setup = time.perf_counter() - t_setup
     step_bytes = sum(g.nbytes for g in step)
     flags = 0 if args.no_overlap else vbq.VBQ_LAUNCH_OVERLAP
@@ -383,12 +428,10 @@ def run_vbq(args):
                 launch(g, stream)
         graph_e2e = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph_e2e, stream=stream):
+            X_d.copy_(X_h, non_blocking=True)
             for g in step:
-                if not g.x_from_device:
-                    g.xd.copy_(g.xh, non_blocking=True)
                 launch(g, stream)
-                for yd, yh in zip(g.yd, g.yh):
-                    yh.copy_(yd, non_blocking=True)
+            Y_h.copy_(Y_d, non_blocking=True)
     torch.cuda.synchronize()
     launches_per_step = len(step)
 
@@ -444,8 +487,8 @@ def run_vbq(args):
         per_shape[g.name] = {"us": us, "GBps": g.nbytes / (us / 1e6) / 1e9, "note": "same launch repeated (L2-warm)"}
 
     # End to end through host buffers.
-    h2d = sum(g.xh.numel() * 2 for g in step if not g.x_from_device)
-    d2h = sum(sum(y.numel() * 4 for y in g.yh) for g in step)
+    h2d = X_h.numel() * 2
+    d2h = Y_h.numel() * 4
     e2e_ms = allreduce_max(timed(graph_e2e), world)
     e2e_val = whole_job_gbps(step_bytes, args.steps, world, e2e_ms)
     n_launches = args.steps * launches_per_step
@@ -498,6 +541,103 @@ def run_vbq(args):
         dist.destroy_process_group()
 
 
+# ------------------------------------------------------------------------------------------- config 4
+CFG4 = (("q", 4096, 4096), ("gate", 14336, 4096), ("down", 4096, 14336))
+
+
+def run_cfg4(args):
+    """The 9B-shaped single linears (q/k/v/o 4096x4096, gate/up 4096->14336, down 14336->4096) at batch 1, 2, 4,
+    8 and 16, each timed alone: M distinct device copies of the packed matrix, together at least 4x the L2, are
+    launched round-robin in one CUDA graph (chained by programmatic dependent launch), so every launch streams its
+    weights from HBM; time per launch = replay time / M, the best of three replays after warm-up. The headline
+    value is the batch-1 GB/s of the two 15.7 MB MLP matrices (their mean); every (matrix, batch) is in `cfg4`."""
+    import torch
+    from decode_vbq_gemv_b200 import vbq
+    world, rank, local = dist_setup()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    peak, peak_kind = peaks()
+    stream = torch.cuda.Stream(dev)
+    batches = (1, 2, 4, 8, 16) if args.batch == 1 else (args.batch,)
+    results, n_launches, t_setup = {}, 0, time.perf_counter()
+    sampler = ClockSampler(local)
+    sampler.start()
+    for name, N, K in CFG4:
+        m = S.cfg4((name,))[0]
+        R = args.tile_rows if args.tile_rows > 0 else vbq.suggest_tile_rows(N, K, sms)
+        blob, desc = vbq.vbq_pack(m.N, m.K, R, m.widths, m.scales, m.codes)
+        stride = (blob.size + 255) // 256 * 256
+        M = max(2, int(np.ceil(4 * L2_BYTES / stride)))
+        copies = torch.empty(M * stride, dtype=torch.uint8, device=dev)
+        first = torch.from_numpy(blob).to(dev)
+        for c in range(M):
+            copies[c * stride:c * stride + blob.size].copy_(first)
+        del first
+        for B in batches:
+            ws_bytes = vbq.vbq_workspace_size(desc, B)
+            ws = torch.zeros(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+            x = torch.from_numpy(S.make_x(4, name, B, K).astype(np.int16)).view(torch.bfloat16).to(dev)
+            y = torch.empty((B, N), dtype=torch.float32, device=dev)
+            flags = 0 if args.no_overlap else vbq.VBQ_LAUNCH_OVERLAP
+            with torch.cuda.stream(stream):
+                def run_all():
+                    for c in range(M):
+                        vbq.vbq_gemm_skinny_ex(desc, copies[c * stride:c * stride + blob.size], x, B, y, ws, flags,
+                                               stream)
+                run_all()
+                torch.cuda.synchronize()
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=stream):
+                    run_all()
+                for _ in range(args.warmup):
+                    g.replay()
+                torch.cuda.synchronize()
+                best = None
+                for _ in range(3):
+                    e0 = torch.cuda.Event(enable_timing=True)
+                    e1 = torch.cuda.Event(enable_timing=True)
+                    e0.record(stream)
+                    g.replay()
+                    e1.record(stream)
+                    torch.cuda.synchronize()
+                    t = e0.elapsed_time(e1) / M
+                    best = t if best is None else min(best, t)
+                n_launches += M * (args.warmup + 3)
+            status = int(ws[ws_bytes - 4:ws_bytes].cpu().numpy().view(np.uint32)[0]) if ws_bytes >= 4 else 0
+            nbytes = blob.size + B * K * 2 + B * N * 4
+            gbps = nbytes / (best / 1e3) / 1e9
+            results[f"{name} {N}x{K} B={B}"] = {"us": best * 1e3, "GBps": gbps, "frac": gbps / peak, "tile_rows": R,
+                                                "copies": M, "status": status}
+            del g, ws
+        del copies
+        torch.cuda.empty_cache()
+    clocks = sampler.stop()
+    t_setup = time.perf_counter() - t_setup
+    head = [results[f"{n} {N}x{K} B=1"]["GBps"] for n, N, K in CFG4 if n in ("gate", "down")] if 1 in batches else \
+        [results[k]["GBps"] for k in results]
+    value = float(np.mean(head))
+    if rank == 0:
+        line = {"metric": METRIC, "value": value * world, "unit": UNIT, "n_gpus": world, "steps": 3,
+                "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "fp32", "data": "synthetic",
+                "config": {"workload": "9B-shaped single linears (q 4096x4096, gate 4096->14336, down 14336->4096), "
+                                       "each alone with >= 4x L2 of distinct copies in rotation",
+                           "batch": list(batches), "l2": "inputs larger than L2: copies in rotation",
+                           "parallelism": f"replicas x{world}"},
+                "pct_of_peak": 100.0 * value / peak,
+                "roofline": {"bound": "hbm", "achieved": value, "peak": peak, "unit": "GB/s", "frac": value / peak,
+                             "traffic": None, "peak_kind": peak_kind,
+                             "kernel": "vbq_cc_kernel<1> (batch 1, 2, 4), vbq_kernel<8|16> (batch 8, 16)"},
+                "cfg4": results, "gpu_launches": n_launches, "clocks": clocks, "setup_s": round(t_setup, 1),
+                "e2e": None, "cpu_baseline": None}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        barrier(world)
+        dist.destroy_process_group()
+
+
 def make_parser() -> argparse.ArgumentParser:
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -505,6 +645,10 @@ def make_parser() -> argparse.ArgumentParser:
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--batch", type=int, default=1, choices=(1, 2, 4, 8, 16))
     ap.add_argument("--impl", default="vbq", choices=("vbq", "reference"))
+    ap.add_argument("--workload", default="step", choices=("step", "recipe", "cfg4"),
+                    help="step: the 9B-shaped decode step at the paper's allocation (default); recipe: the same step "
+                         "under the fixed deployment recipe; cfg4: each 9B-shaped linear alone at batch 1..16, "
+                         "rotating copies larger than L2")
     ap.add_argument("--layers", type=int, default=32, help="decoder layers in the step (1..32)")
     ap.add_argument("--no-head", action="store_true", help="leave the LM head out of the step")
     ap.add_argument("--no-fp16-ref", action="store_true",
@@ -529,6 +673,8 @@ def main():
         ap.error("--layers must be in 1..32")
     if args.impl == "reference":
         run_reference(args)
+    elif args.workload == "cfg4":
+        run_cfg4(args)
     else:
         run_vbq(args)
 

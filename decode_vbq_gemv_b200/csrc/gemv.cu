@@ -29,6 +29,7 @@
 
 #include <algorithm>
 #include <atomic>
+#include <type_traits>
 #include <mutex>
 
 #include "vbq.h"
@@ -82,7 +83,7 @@ struct Params {
   int warps_off, warp_bytes;
   // CUDA-core kernel (batch <= 4) only
   int NB;                  // records per batch
-  int meta_off, dir_off;   // shared-memory offsets: per-record metadata blocks, directory cache
+  int meta_off, row_off, dir_off;  // shared-memory offsets: table blocks, row blocks, directory cache
   int res_rec, meta_rec;   // bytes per record: item results, metadata block
   int cost[5];             // job costs for the split of a batch among warps: units of 1, 2, 4, 8 bits; meta job
   int withhold;            // test hook: the record (global index) whose bulk copy is never issued, or -1
@@ -223,6 +224,21 @@ __device__ __forceinline__ uint32_t lds32(uint32_t a) {
 __device__ __forceinline__ float lds32f(uint32_t a) {
   float v;
   asm("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(a) : "memory");
+  return v;
+}
+// f(integral_constant<int, I>) for I = I0 .. N-1, unrolled at compile time (for immediates that must be constants)
+template <int I, int N, typename F>
+__device__ __forceinline__ void static_for(F&& f) {
+  if constexpr (I < N) {
+    f(std::integral_constant<int, I>{});
+    static_for<I + 1, N>(f);
+  }
+}
+// ld.shared.f32 at a + OFF, the offset an immediate of the instruction
+template <int OFF>
+__device__ __forceinline__ float lds32f_off(uint32_t a) {
+  float v;
+  asm("ld.shared.f32 %0, [%1+%2];" : "=f"(v) : "r"(a), "n"(OFF) : "memory");
   return v;
 }
 __device__ __forceinline__ uint32_t lds16(uint32_t a) {
@@ -640,15 +656,19 @@ __device__ void finish_cta(const Params& p, int L, int H, int* cta_flags, int* e
   const bool part1 = tlast != tfirst && !(L <= tlast * G && H >= (tlast + 1) * G);
   if (part0 || part1) {
     __syncthreads();
-    if (tid == 0) {
-      // acq_rel at GPU scope: the release publishes the CTA's slot writes (ordered before it by the barrier),
-      // the acquire makes the other owners' slots visible to the reduction that follows.
-      int first;
-      const int own0 = part0 ? tile_owners(tfirst, first) : 0, own1 = part1 ? tile_owners(tlast, first) : 0;
-      const unsigned a0 = part0 ? atom_add_acq_rel(&p.arrive[tfirst], 1u) : 0u;
-      const unsigned a1 = part1 ? atom_add_acq_rel(&p.arrive[tlast], 1u) : 0u;
-      cta_flags[0] = part0 && a0 == unsigned(own0 - 1);
-      cta_flags[1] = part1 && a1 == unsigned(own1 - 1);
+    // Thread 0 counts the CTA in on its first tile, thread 32 on its last, at the same time. Each atomic is
+    // acq_rel at GPU scope: the release publishes the CTA's slot writes (ordered before it by the barrier), the
+    // acquire makes the other owners' slots visible to the reduction that follows.
+    if (tid == 0 || tid == 32) {
+      const bool last = tid == 32;
+      if (last ? part1 : part0) {
+        const int t = last ? tlast : tfirst;
+        int first;
+        const int own = tile_owners(t, first);
+        cta_flags[last] = atom_add_acq_rel(&p.arrive[t], 1u) == unsigned(own - 1);
+      } else {
+        cta_flags[last] = 0;
+      }
     }
     __syncthreads();
     const int ntiles = cta_flags[0] + cta_flags[1];
@@ -1115,8 +1135,10 @@ __global__ void __launch_bounds__(Cfg<B>::kThreads, 1) vbq_kernel(const __grid_c
 //    identical from run to run. The batch's slots are refilled right after the barrier.
 //  - A finished tile goes to y when the CTA holds all its records, else to the CTA's partial slot; finish_cta then
 //    reduces the tiles shared with neighbouring CTAs and runs the SwiGLU epilogue.
+constexpr int kCCWarps = 16;      // warps per CTA of the CUDA-core kernel
+constexpr int kCCCtasPerSM = 1;   // CTAs per SM in its grid
 template <int B> struct CCfg {
-  static constexpr int kWarps = 16;
+  static constexpr int kWarps = kCCWarps;
   static constexpr int kThreads = kWarps * 32;
   static constexpr int kIPU = 32 / B;                               // items per 2-, 4-, 8-bit unit
   static constexpr int kWordsPerWarp = (32 + kWarps - 1) / kWarps;  // row-pass words per warp (R <= 1024)
@@ -1125,102 +1147,126 @@ constexpr int kMaxNB = 7;        // records per batch: the 1 + 4 NB job segments
 constexpr int kMaxSets = 4;      // batches in flight
 constexpr int kDirCache = 512;   // directory entries cached in shared memory
 
-// Per-record metadata block (256-byte aligned), written by the record's meta job:
-//  lut [B][16][16] f32: 1-bit nibble tables; entry n of position p is the sum of x[4p + i] over the set bits i of n
-//  xt  [3][B][64] f32:  x, x * 2^-shift for 2-bit codes, x * 2^-shift for 4-bit codes
-//  sg  [B] f32:         group sums of x
-//  mk  [4][32] u32:     width masks per 32-row word;  pf [4][32] u16: item index of the word's first row per width
-//  wc  [64] u32:        the record's width-code words
-//  fl  [12] i32:        bad, scales offset, bucket counts n[4], bucket code offsets c[4]
+// Per-record metadata, written by the record's meta job one batch before its units run, in two blocks.
+// Table block (256-byte aligned; read only by the units, so two sets serve alternate batches):
+//  t1 [B][16][16] f32: 1-bit nibble tables; entry n of position p is the sum of x[4p + i] over the set bits i of n
+//  t2 [B][32][16] f32: 2-bit nibble tables; entry n of position p is (n & 3) x[2p] + (n >> 2) x[2p + 1]
+//  xt [2][B][64] f32:  x, and x * 2^-shift for the magic-number expansion of 4-bit codes
+//  sg [B] f32:         group sums of x
+//  fl [16] i32:        bad, scales offset, bucket counts n[4], bucket code offsets c[4], bucket item starts i[4]
+// Row block (read by the row pass, which can still run while the next batch's units write: three sets):
+//  mk [4][32] u32:     width masks per 32-row word;  pf [4][32] u16: item index of the word's first row per width
+//  wc [64] u32:        the record's width-code words;  bad (i32)
 struct MetaOff {
-  int lut, xt, sg, mk, pf, wc, fl, size;
+  int t1, t2, xt, sg, fl, size;      // table block
+  int mk, pf, wc, bad, row_size;     // row block
   __host__ __device__ explicit MetaOff(int B) {
-    lut = 0;
-    xt = 1024 * B;
-    sg = xt + 768 * B;
-    mk = sg + 16;
-    pf = mk + 512;
-    wc = pf + 256;
-    fl = wc + 256;
-    size = (fl + 48 + 255) & ~255;
+    t1 = 0;
+    t2 = 1024 * B;
+    xt = t2 + 2048 * B;
+    sg = xt + 512 * B;
+    fl = sg + 16;
+    size = (fl + 64 + 255) & ~255;
+    mk = 0;
+    pf = 512;
+    wc = 768;
+    bad = 1024;
+    row_size = 1040;
   }
 };
 
-// The CTA's batches: records [L, H) cut at row-tile boundaries, then into runs of at most NB records.
-struct Batches {
-  int L, H, G, NB, e0, nb0, bpt, tile0, nbatch;
-  __device__ Batches(int L_, int H_, int G_, int NB_)
-      : L(L_), H(H_), G(G_), NB(NB_), e0(0), nb0(0), bpt(1), tile0(0), nbatch(0) {
-    if (H <= L) return;
-    tile0 = L / G;
-    e0 = min(H, (tile0 + 1) * G);
-    nb0 = (e0 - L + NB - 1) / NB;
-    bpt = (G + NB - 1) / NB;
-    const int rest = H - e0, full = rest / G, last = rest - full * G;
-    nbatch = nb0 + full * bpt + (last + NB - 1) / NB;
+// The CTA's batches, in order: records [L, H) cut at row-tile boundaries, then into runs of at most NB records.
+// Also tracks where batch's first record streams: slot s0 of the NS slots, its use u0 of that slot (mbarrier phase).
+struct BatchIt {
+  int rb, re, t, te, s0, u0;
+  int H, G, NB, NS;
+  __device__ void init(int L, int H_, int G_, int NB_, int NS_) {
+    H = H_; G = G_; NB = NB_; NS = NS_;
+    rb = L;
+    t = L / G;
+    te = min(H, (t + 1) * G);
+    re = min(te, rb + NB);
+    s0 = 0;
+    u0 = 0;
   }
-  __device__ void get(int n, int& rb, int& re) const {
-    if (n < nb0) {
-      rb = L + n * NB;
-      re = min(e0, rb + NB);
-      return;
+  __device__ bool valid() const { return rb < H; }
+  __device__ void next() {
+    s0 += re - rb;
+    if (s0 >= NS) { s0 -= NS; ++u0; }
+    rb = re;
+    if (rb >= te) {
+      ++t;
+      te = min(H, te + G);
     }
-    const int m = n - nb0, q = m / bpt, t = tile0 + 1 + q;
-    rb = t * G + (m - q * bpt) * NB;
-    re = min(min(H, (t + 1) * G), rb + NB);
+    re = min(te, rb + NB);
+  }
+  // slot and mbarrier phase parity of record rb + pos
+  __device__ void slot_of(int pos, int& slot, unsigned& parity) const {
+    slot = s0 + pos;
+    int u = u0;
+    if (slot >= NS) { slot -= NS; ++u; }
+    parity = unsigned(u) & 1u;
   }
 };
 
-// 1-bit group against the nibble tables of B batch rows at shared address tab (256-byte aligned, table b at
-// tab + 1024 b): 16 lookups per row, one per four weights. Each nibble times 4 is moved by one byte permute into
-// the low byte of the table address. Returns sum_i (q_i - 1/2) x_i per row.
-template <int B>
-__device__ __forceinline__ void dot_b1_lut(uint2 w, uint32_t tab, const float (&sg)[B], float (&d)[B]) {
-  const uint32_t e0 = (w.x << 2) & 0x3C3C3C3Cu, o0 = (w.x >> 2) & 0x3C3C3C3Cu;  // nibbles 2k / 2k+1, times 4
-  const uint32_t e1 = (w.y << 2) & 0x3C3C3C3Cu, o1 = (w.y >> 2) & 0x3C3C3C3Cu;
+// 1- and 2-bit groups against nibble tables of B batch rows at shared address tab (256-byte aligned, table b at
+// tab + TB * b; entry n of position p at + 64 p + 4 n): one lookup per nibble. Each nibble times 4 is moved by one
+// byte permute into the low byte of the table address. KB = 1: 16 positions of four 1-bit codes; KB = 2: 32
+// positions of two 2-bit codes. Returns sum_i q_i x_i per row in d.
+template <int KB, int B>
+__device__ __forceinline__ void dot_lut(const uint32_t (&w)[2 * KB], uint32_t tab, float (&d)[B]) {
+  constexpr int TB = KB == 1 ? 1024 : 2048;
   constexpr int NA = B == 1 ? 8 : 4;
   float a[B][NA];
 #pragma unroll
   for (int b = 0; b < B; ++b)
 #pragma unroll
     for (int i = 0; i < NA; ++i) a[b][i] = 0.f;
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const uint32_t ae0 = __byte_perm(e0, tab, 0x7650u + k), ao0 = __byte_perm(o0, tab, 0x7650u + k);
-    const uint32_t ae1 = __byte_perm(e1, tab, 0x7650u + k), ao1 = __byte_perm(o1, tab, 0x7650u + k);
-#pragma unroll
-    for (int b = 0; b < B; ++b) {
-      a[b][(2 * k) % NA] += lds32f(ae0 + 1024 * b + 64 * (2 * k));
-      a[b][(2 * k + 1) % NA] += lds32f(ao0 + 1024 * b + 64 * (2 * k + 1));
-      a[b][(2 * k) % NA] += lds32f(ae1 + 1024 * b + 64 * (8 + 2 * k));
-      a[b][(2 * k + 1) % NA] += lds32f(ao1 + 1024 * b + 64 * (9 + 2 * k));
-    }
-  }
+  static_for<0, 2 * KB>([&](auto mc) {
+    constexpr int m = decltype(mc)::value;                                        // word m: positions 8m .. 8m + 7
+    const uint32_t e = (w[m] << 2) & 0x3C3C3C3Cu, o = (w[m] >> 2) & 0x3C3C3C3Cu;  // nibbles 2k / 2k+1, times 4
+    static_for<0, 4>([&](auto kc) {
+      constexpr int k = decltype(kc)::value;
+      const uint32_t ae = __byte_perm(e, tab, 0x7650u + k), ao = __byte_perm(o, tab, 0x7650u + k);
+      static_for<0, B>([&](auto bc) {
+        constexpr int b = decltype(bc)::value;
+        a[b][(2 * k) % NA] += lds32f_off<TB * b + 64 * (8 * m + 2 * k)>(ae);
+        a[b][(2 * k + 1) % NA] += lds32f_off<TB * b + 64 * (8 * m + 2 * k + 1)>(ao);
+      });
+    });
+  });
 #pragma unroll
   for (int b = 0; b < B; ++b) {
-    float t = 0.f;
-    if constexpr (NA == 8) t = ((a[b][0] + a[b][1]) + (a[b][2] + a[b][3])) + ((a[b][4] + a[b][5]) + (a[b][6] + a[b][7]));
-    else t = (a[b][0] + a[b][1]) + (a[b][2] + a[b][3]);
-    d[b] = t - 0.5f * sg[b];
+    if constexpr (NA == 8) d[b] = ((a[b][0] + a[b][1]) + (a[b][2] + a[b][3])) + ((a[b][4] + a[b][5]) + (a[b][6] + a[b][7]));
+    else d[b] = (a[b][0] + a[b][1]) + (a[b][2] + a[b][3]);
   }
 }
 
-// 1-bit units [lo, hi) of 32 items each (lane = item, all B batch rows): s * dot into res[item][b].
-template <int B>
-__device__ __forceinline__ void unit_range_b1(int n, int lo, int hi, int lane, uint32_t codes, uint32_t scales,
-                                              uint32_t res, uint32_t tab, const float (&sg)[B]) {
+// 1- or 2-bit units [lo, hi) of 32 items each (lane = item, all B batch rows): s * (sum q x - off * S_g) into
+// res[item][b], off = 1/2 (1-bit) or 2 - corr (2-bit).
+template <int KB, int B>
+__device__ __forceinline__ void unit_range_lut(int n, int lo, int hi, int lane, uint32_t codes, uint32_t scales,
+                                               uint32_t res, uint32_t tab, const float (&sg)[B], float off) {
   for (int u = lo; u < hi; ++u) {
     const int jj = 32 * u + lane;
     if (jj >= n) break;
+    uint32_t w[2 * KB];
+    if constexpr (KB == 1) {
+      const uint2 v = lds64(codes + 8 * jj);
+      w[0] = v.x; w[1] = v.y;
+    } else {
+      const uint4 v = lds128(codes + 16 * jj);
+      w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
+    }
     float d[B];
-    dot_b1_lut<B>(lds64(codes + 8 * jj), tab, sg, d);
+    dot_lut<KB, B>(w, tab, d);
     const float s = __half2float(__ushort_as_half((unsigned short)lds16(scales + 2 * jj)));
 #pragma unroll
-    for (int b = 0; b < B; ++b) sts32f(res + 4 * (jj * B + b), s * d[b]);
+    for (int b = 0; b < B; ++b) sts32f(res + 4 * (jj * B + b), s * (d[b] - off * sg[b]));
   }
 }
 
-// 2-, 4-, 8-bit units [lo, hi) of 32 / B items each (lane = item * B + b): s * dot of the item's group with batch
+// 4- and 8-bit units [lo, hi) of 32 / B items each (lane = item * B + b): s * dot of the item's group with batch
 // row b into res[item][b]. codes, scales and res are byte addresses of item 0 of the bucket.
 template <int KB, int B>
 __device__ __forceinline__ void unit_range(int n, int lo, int hi, int lane, uint32_t codes, uint32_t scales,
@@ -1231,11 +1277,7 @@ __device__ __forceinline__ void unit_range(int n, int lo, int hi, int lane, uint
     const int jj = IPU * u + sub;
     if (jj >= n) break;
     float d;
-    if constexpr (KB == 2) {
-      const uint4 a = lds128(codes + 16 * jj);
-      const uint32_t w[4] = {a.x, a.y, a.z, a.w};
-      d = dot_magic<2>(w, xr, sg, corr);
-    } else if constexpr (KB == 4) {
+    if constexpr (KB == 4) {
       const uint4 a = lds128(codes + 32 * jj), c = lds128(codes + 32 * jj + 16);
       const uint32_t w[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
       d = dot_magic<4>(w, xr, sg, corr);
@@ -1252,18 +1294,22 @@ __device__ __forceinline__ void unit_range(int n, int lo, int hi, int lane, uint
   }
 }
 
-// First job (of count jobs costing c each, the segment starting at cost s0) whose cost midpoint reaches cost
-// cut2 / (2 W): the smallest j with W (2 s0 + c (2j + 1)) >= cut2, clamped to [0, count].
+// First job (of count jobs costing c each, in the segment starting at cost s0) whose cost midpoint reaches
+// cut2 / (2 W): the smallest j >= 0 with W (2 s0 + c (2j + 1)) >= cut2, at most count. The quotient comes from a
+// float division (all values are below 2^24), corrected to the exact integer.
 __device__ __forceinline__ int first_job(int cut2, int s0, int c, int count, int W) {
   if (count <= 0) return 0;
   const int num = cut2 - (2 * s0 + c) * W;
   if (num <= 0) return 0;
   const int den = 2 * W * c;
-  return min(count, (num + den - 1) / den);
+  int j = __float2int_ru(__fdividef(float(num), float(den)));
+  if (j * den < num) ++j;
+  else if (j > 0 && (j - 1) * den >= num) --j;
+  return min(count, j);
 }
 
 template <int B>
-__global__ void __launch_bounds__(CCfg<B>::kThreads, 1) vbq_cc_kernel(const __grid_constant__ Params params) {
+__global__ void __launch_bounds__(CCfg<B>::kThreads, 16 / kCCWarps) vbq_cc_kernel(const __grid_constant__ Params params) {
   using C = CCfg<B>;
   constexpr int W = C::kWarps, IPU = C::kIPU, NWW = C::kWordsPerWarp;
   extern __shared__ __align__(128) unsigned char smem[];
@@ -1284,9 +1330,9 @@ __global__ void __launch_bounds__(CCfg<B>::kThreads, 1) vbq_cc_kernel(const __gr
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int G = p.G, NB = p.NB, S = p.S, cta = blockIdx.x;
   const int L = rec_lo(p, cta), H = rec_lo(p, cta + 1);
-  const Batches bt(L, H, G, NB);
-  if (bt.nbatch == 0) return;  // nothing to read or write
+  if (H <= L) return;  // nothing to read or write
   const MetaOff mo(B);
+  const int NS = NB * S;
 
   // -- directory cache: entries (start, end) of records [dbase, dbase + kDirCache), in 16-byte units
   uint32_t* dlo = reinterpret_cast<uint32_t*>(smem + p.dir_off);
@@ -1303,28 +1349,30 @@ __global__ void __launch_bounds__(CCfg<B>::kThreads, 1) vbq_cc_kernel(const __gr
   };
   fill_dir(L);
   if (tid == 0) {
-    for (int i = 0; i < NB * S; ++i) mbar_init(&bar_full[i], 1);
+    for (int i = 0; i < NS; ++i) mbar_init(&bar_full[i], 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
 
-  // Record j (CTA-local index j - L) streams into slot (j - L) % NS; its use of that slot is number (j - L) / NS,
-  // which sets the mbarrier phase parity. A batch is issued only when the batch S before it is done, and the S
+  // Record j streams into slot (j - L) % NS; its use of that slot is number (j - L) / NS, which sets the mbarrier
+  // phase parity (BatchIt tracks both). A batch is issued only when the batch S before it is done, and the S
   // batches from there hold at most NS records, so a slot's previous record is always finished.
-  const int NS = NB * S;
   auto slot_ptr = [&](int slot) { return smem + slot * p.stage_size; };
   // metadata blocks from the first 256-byte boundary of their region (the nibble-table lookups put an index in
   // the low byte of a table address); the plan leaves 256 bytes of room for this
   const int meta0 = int(((smem_u32(smem + p.meta_off) + 255u) & ~255u) - smem_u32(smem));
-  auto meta_ptr = [&](int mp, int pos) { return smem + meta0 + (mp * NB + pos) * p.meta_rec; };
-  auto res_addr = [&](int n, int pos) { return smem_u32(smem + p.res_off + ((n & 1) * NB + pos) * p.res_rec); };
+  auto meta_ptr = [&](int tp, int pos) { return smem + meta0 + (tp * NB + pos) * p.meta_rec; };   // table block
+  auto row_ptr = [&](int mp, int pos) { return smem + p.row_off + (mp * NB + pos) * MetaOff(B).row_size; };
+  auto res_addr = [&](int rp, int pos) { return smem_u32(smem + p.res_off + (rp * NB + pos) * p.res_rec); };
 
-  // Bulk copies of records [rb, re) (warp 0, one record per lane, at most 32): the records (with_rec) and the
+  // Bulk copies of batch `it` (warp 0, one record per lane, at most NB <= 32): the records (with_rec) and the
   // activation rows (with_x) into their slots. The mbarrier of a slot expects both.
-  auto issue = [&](int rb, int re, bool with_rec, bool with_x) {
-    const int j = rb + lane;
-    if (j >= re) return;
-    const int slot = (j - L) % NS;
+  auto issue = [&](const BatchIt& it, bool with_rec, bool with_x) {
+    const int j = it.rb + lane;
+    if (j >= it.re) return;
+    int slot;
+    unsigned parity;
+    it.slot_of(lane, slot, parity);
     uint64_t* bar = &bar_full[slot];
     unsigned char* dst = slot_ptr(slot);
     if (with_rec) {
@@ -1342,22 +1390,26 @@ __global__ void __launch_bounds__(CCfg<B>::kThreads, 1) vbq_cc_kernel(const __gr
       if (j != p.withhold) tma_bulk_load(dst, pick(p.recs, m) + 16ull * a, bytes, bar);
     }
     if (with_x && !slot_bad[slot] && j != p.withhold) {
-      const int g = j % G;
+      const int g = j - it.t * G;
 #pragma unroll
       for (int bb = 0; bb < B; ++bb)
         tma_bulk_load(dst + p.stage_bytes + 128 * bb, p.x + size_t(bb) * p.K + size_t(g) * 64, 128u, bar);
     }
   };
 
-  // Meta job of record j (whole warp) into meta set mp: wait for the record, validate it, write its metadata.
-  auto meta_job = [&](int j, int mp, int pos) {
-    const int slot = (j - L) % NS;
+  // Meta job of record pos of batch `it` (whole warp) into table set tp and row set mp: wait for the record,
+  // validate it, write its metadata.
+  auto meta_job = [&](const BatchIt& it, int pos, int tp, int mp) {
+    int slot;
+    unsigned parity;
+    it.slot_of(pos, slot, parity);
     const unsigned char* st = slot_ptr(slot);
     const uint32_t sa = smem_u32(st);
-    unsigned char* mb = meta_ptr(mp, pos);
-    bool ok = mbar_wait(&bar_full[slot], ((j - L) / NS) & 1, p.status, &cta_abort, p.wait_ns);
+    unsigned char* mb = meta_ptr(tp, pos);
+    unsigned char* rb_ = row_ptr(mp, pos);
+    bool ok = mbar_wait(&bar_full[slot], parity, p.status, &cta_abort, p.wait_ns);
     ok = __all_sync(0xFFFFFFFFu, ok) && !slot_bad[slot];
-    const int Rt = tile_out(p, j / G).Rt;
+    const int Rt = tile_out(p, it.t).Rt;
     int n0 = 0, n1 = 0, n2 = 0, n3 = 0;
     if (ok) {
       const uint2 cnt = lds64(sa);
@@ -1401,9 +1453,9 @@ __global__ void __launch_bounds__(CCfg<B>::kThreads, 1) vbq_cc_kernel(const __gr
     }
     int* fl = reinterpret_cast<int*>(mb + mo.fl);
     if (ok) {
-      uint32_t* mk = reinterpret_cast<uint32_t*>(mb + mo.mk);
-      uint16_t* pf = reinterpret_cast<uint16_t*>(mb + mo.pf);
-      uint32_t* wc = reinterpret_cast<uint32_t*>(mb + mo.wc);
+      uint32_t* mk = reinterpret_cast<uint32_t*>(rb_ + mo.mk);
+      uint16_t* pf = reinterpret_cast<uint16_t*>(rb_ + mo.pf);
+      uint32_t* wc = reinterpret_cast<uint32_t*>(rb_ + mo.wc);
       mk[lane] = m0; mk[32 + lane] = m1; mk[64 + lane] = m2; mk[96 + lane] = m3;
       pf[lane] = uint16_t(pre & 0xFFFFull);
       pf[32 + lane] = uint16_t(n0 + int((pre >> 16) & 0xFFFFull));
@@ -1411,12 +1463,10 @@ __global__ void __launch_bounds__(CCfg<B>::kThreads, 1) vbq_cc_kernel(const __gr
       pf[96 + lane] = uint16_t(n0 + n1 + n2 + int(pre >> 48));
       wc[2 * lane] = uint32_t(v);
       wc[2 * lane + 1] = uint32_t(v >> 32);
-      // activation tables [3][B][64]: x, x * 2^-shift (2-bit codes), x * 2^-shift (4-bit codes); group sums
+      // activation tables [2][B][64]: x, x * 2^-shift (4-bit codes); group sums
       const uint16_t* xg = reinterpret_cast<const uint16_t*>(st + p.stage_bytes);
       float* xv = reinterpret_cast<float*>(mb + mo.xt);
       float* sgv = reinterpret_cast<float*>(mb + mo.sg);
-      const float s2a = __uint_as_float(uint32_t(127 - code_shift<2>(lane)) << 23);
-      const float s2b = __uint_as_float(uint32_t(127 - code_shift<2>(32 + lane)) << 23);
       const float s4a = __uint_as_float(uint32_t(127 - code_shift<4>(lane)) << 23);
       const float s4b = __uint_as_float(uint32_t(127 - code_shift<4>(32 + lane)) << 23);
 #pragma unroll
@@ -1425,19 +1475,19 @@ __global__ void __launch_bounds__(CCfg<B>::kThreads, 1) vbq_cc_kernel(const __gr
         const float x1 = __uint_as_float(uint32_t(xg[b * 64 + 32 + lane]) << 16);
         xv[b * 64 + lane] = x0;
         xv[b * 64 + 32 + lane] = x1;
-        xv[(B + b) * 64 + lane] = x0 * s2a;
-        xv[(B + b) * 64 + 32 + lane] = x1 * s2b;
-        xv[(2 * B + b) * 64 + lane] = x0 * s4a;
-        xv[(2 * B + b) * 64 + 32 + lane] = x1 * s4b;
+        xv[(B + b) * 64 + lane] = x0 * s4a;
+        xv[(B + b) * 64 + 32 + lane] = x1 * s4b;
         float sg = x0 + x1;
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) sg += __shfl_xor_sync(0xFFFFFFFFu, sg, off);
         if (lane == 0) sgv[b] = sg;
       }
       __syncwarp();
-      // 1-bit nibble tables: lane = (position p, half h) builds entries 8h .. 8h + 7 of position p of each row
+      // nibble tables. 1-bit: lane = (position p, half h) builds entries 8h .. 8h + 7 of position p.
+      // 2-bit: lane = position p (codes 2p, 2p + 1) builds its 16 entries.
+      const uint32_t xa = smem_u32(mb + mo.xt);
       const int pp = lane >> 1, hh = lane & 1;
-      const uint32_t xa = smem_u32(mb + mo.xt), ta = smem_u32(mb + mo.lut) + 64 * pp + 32 * hh;
+      const uint32_t t1a = smem_u32(mb + mo.t1) + 64 * pp + 32 * hh, t2a = smem_u32(mb + mo.t2) + 64 * lane;
 #pragma unroll
       for (int b = 0; b < B; ++b) {
         const float4 q = lds128f(xa + 256 * b + 16 * pp);
@@ -1446,36 +1496,50 @@ __global__ void __launch_bounds__(CCfg<B>::kThreads, 1) vbq_cc_kernel(const __gr
         const uint32_t lo4[4] = {__float_as_uint(base), __float_as_uint(e1), __float_as_uint(e2), __float_as_uint(e3)};
         const uint32_t hi4[4] = {__float_as_uint(base + q.z), __float_as_uint(e1 + q.z), __float_as_uint(e2 + q.z),
                                  __float_as_uint(e3 + q.z)};
-        sts128(ta + 1024 * b, lo4);
-        sts128(ta + 1024 * b + 16, hi4);
+        sts128(t1a + 1024 * b, lo4);
+        sts128(t1a + 1024 * b + 16, hi4);
+        const uint2 xp = lds64(xa + 256 * b + 8 * lane);
+        const float xa0 = __uint_as_float(xp.x), xb0 = __uint_as_float(xp.y);
+#pragma unroll
+        for (int qb = 0; qb < 4; ++qb) {
+          const float hb = float(qb) * xb0;
+          const uint32_t row[4] = {__float_as_uint(hb), __float_as_uint(fmaf(1.f, xa0, hb)),
+                                   __float_as_uint(fmaf(2.f, xa0, hb)), __float_as_uint(fmaf(3.f, xa0, hb))};
+          sts128(t2a + 2048 * b + 16 * qb, row);
+        }
       }
       if (lane == 0) {
         const Rec rc(Rt, n0, n1, n2, n3);
         fl[1] = rc.sc;
         fl[2] = n0; fl[3] = n1; fl[4] = n2; fl[5] = n3;
         fl[6] = rc.c0; fl[7] = rc.c1; fl[8] = rc.c2; fl[9] = rc.c3;
+        fl[10] = 0; fl[11] = n0; fl[12] = n0 + n1; fl[13] = n0 + n1 + n2;
       }
     } else if (lane == 0) {
       fl[2] = fl[3] = fl[4] = fl[5] = 0;
     }
-    if (lane == 0) fl[0] = ok ? 0 : 1;
+    if (lane == 0) {
+      fl[0] = ok ? 0 : 1;
+      *reinterpret_cast<int*>(rb_ + mo.bad) = ok ? 0 : 1;
+    }
   };
 
-  // Jobs of batch [rb, re) (meta set mp) for this warp: the meta jobs of the next batch [nrb, nre) (segment 0,
-  // into meta set mpn) and the units of this batch's records, buckets in the order 1, 8, 2, 4 bits (8-bit units
-  // read the raw activation table, which the 1-bit units leave in place).
-  auto jobs = [&](int n, int rb, int re, int mp, int nrb, int nre, int mpn) {
-    const int nrec = re - rb;
+  // Jobs of batch `cur` (meta set mp, result set rp) for this warp: the units of its records, buckets in the order
+  // 1, 2, 8, 4 bits, then the meta jobs of the next batch `nxt` (into meta set mpn). 1- and 2-bit units take 32
+  // items (all batch rows per lane); 4- and 8-bit units 32 / B items.
+  auto jobs = [&](const BatchIt& cur, const BatchIt& nxt, int rp, int mpn) {
+    const int nrec = cur.re - cur.rb;
+    // segment of this lane: 4 pos + q = record pos, bucket order q; lane 31 = the meta jobs
     int count = 0, cost = 0;
-    if (lane == 0) {
-      count = nre - nrb;
+    if (lane == 31) {
+      count = nxt.valid() ? nxt.re - nxt.rb : 0;
       cost = p.cost[4];
-    } else if (lane - 1 < 4 * nrec) {
-      const int pos = (lane - 1) >> 2, q = (lane - 1) & 3;
-      const int k = q == 0 ? 0 : q == 1 ? 3 : q == 2 ? 1 : 2;
-      const int* fl = reinterpret_cast<const int*>(meta_ptr(mp, pos) + mo.fl);
+    } else if (lane < 4 * nrec) {
+      const int pos = lane >> 2, q = lane & 3;
+      const int k = q == 0 ? 0 : q == 1 ? 1 : q == 2 ? 3 : 2;
+      const int* fl = reinterpret_cast<const int*>(meta_ptr(rp, pos) + mo.fl);
       const int nk = fl[2 + k];
-      count = k == 0 ? (nk + 31) >> 5 : (nk + IPU - 1) / IPU;
+      count = k < 2 ? (nk + 31) >> 5 : (nk + IPU - 1) / IPU;
       cost = p.cost[k];
     }
     const int tot = count * cost;
@@ -1488,75 +1552,70 @@ __global__ void __launch_bounds__(CCfg<B>::kThreads, 1) vbq_cc_kernel(const __gr
     const int s0 = incl - tot, total = __shfl_sync(0xFFFFFFFFu, incl, 31);
     const int jlo = first_job(2 * total * warp, s0, max(cost, 1), count, W);
     const int jhi = first_job(2 * total * (warp + 1), s0, max(cost, 1), count, W);
-    // units first, the meta jobs last (their records were issued most recently)
     unsigned todo = __ballot_sync(0xFFFFFFFFu, jhi > jlo);
-    todo = (todo >> 1) | ((todo & 1u) << 31);
     float xr[64];
     int loaded = -1;
-    const int t = rb / G;
-    const float corr = pick(p.sym, mat_of_tile(p, t)) != 0 ? 1.f : 0.5f;
-    int slot0 = (rb - L) % NS;
+    const float corr = pick(p.sym, mat_of_tile(p, cur.t)) != 0 ? 1.f : 0.5f;
     while (todo) {
-      const int sgi = __ffs(todo) & 31;  // bit i holds segment i + 1; bit 31 holds segment 0
+      const int sgi = __ffs(todo) - 1;
       todo &= todo - 1;
       const int lo = __shfl_sync(0xFFFFFFFFu, jlo, sgi), hi = __shfl_sync(0xFFFFFFFFu, jhi, sgi);
-      if (sgi == 0) {
-        for (int jb = lo; jb < hi; ++jb) meta_job(nrb + jb, mpn, jb);
+      if (sgi == 31) {
+        for (int jb = lo; jb < hi; ++jb) meta_job(nxt, jb, rp ^ 1, mpn);
         continue;
       }
-      const int pos = (sgi - 1) >> 2, q = (sgi - 1) & 3;
-      const int k = q == 0 ? 0 : q == 1 ? 3 : q == 2 ? 1 : 2;
-      const unsigned char* mb = meta_ptr(mp, pos);
+      const int pos = sgi >> 2, q = sgi & 3;
+      const int k = q == 0 ? 0 : q == 1 ? 1 : q == 2 ? 3 : 2;
+      const unsigned char* mb = meta_ptr(rp, pos);
       const int* fl = reinterpret_cast<const int*>(mb + mo.fl);
-      const int nk = fl[2 + k], cb = fl[6 + k], sc = fl[1];
-      const int ib = k == 0 ? 0 : k == 1 ? fl[2] : k == 2 ? fl[2] + fl[3] : fl[2] + fl[3] + fl[4];
-      int slot = slot0 + pos;
-      if (slot >= NS) slot -= NS;
+      const int nk = fl[2 + k], cb = fl[6 + k], ib = fl[10 + k], sc = fl[1];
+      int slot;
+      unsigned parity;
+      cur.slot_of(pos, slot, parity);
       const uint32_t sa = smem_u32(slot_ptr(slot));
-      const uint32_t res = res_addr(n, pos) + 4 * B * ib;
+      const uint32_t res = res_addr(rp, pos) + 4 * B * ib;
       const uint32_t sca = sa + sc + 2 * ib;
-      if (k == 0) {
+      if (k < 2) {
         float sgb[B];
 #pragma unroll
         for (int b = 0; b < B; ++b) sgb[b] = reinterpret_cast<const float*>(mb + mo.sg)[b];
-        unit_range_b1<B>(nk, lo, hi, lane, sa + cb, sca, res, smem_u32(mb + mo.lut), sgb);
+        if (k == 0) unit_range_lut<1, B>(nk, lo, hi, lane, sa + cb, sca, res, smem_u32(mb + mo.t1), sgb, 0.5f);
+        else unit_range_lut<2, B>(nk, lo, hi, lane, sa + cb, sca, res, smem_u32(mb + mo.t2), sgb, 2.f - corr);
         continue;
       }
-      const int tbl = k == 1 ? 1 : k == 2 ? 2 : 0;
+      const int tbl = k == 2 ? 1 : 0;
       const int b = lane % B;
-      if (loaded != pos * 4 + tbl) {
+      if (loaded != pos * 2 + tbl) {
         const uint32_t xa = smem_u32(mb + mo.xt) + 256 * (tbl * B + b);
 #pragma unroll
         for (int qq = 0; qq < 16; ++qq) {
           const float4 f = lds128f(xa + 16 * qq);
           xr[4 * qq] = f.x; xr[4 * qq + 1] = f.y; xr[4 * qq + 2] = f.z; xr[4 * qq + 3] = f.w;
         }
-        loaded = pos * 4 + tbl;
+        loaded = pos * 2 + tbl;
       }
       const float sg = reinterpret_cast<const float*>(mb + mo.sg)[b];
-      if (k == 1) unit_range<2, B>(nk, lo, hi, lane, sa + cb, sca, res, xr, sg, corr);
-      else if (k == 2) unit_range<4, B>(nk, lo, hi, lane, sa + cb, sca, res, xr, sg, corr);
+      if (k == 2) unit_range<4, B>(nk, lo, hi, lane, sa + cb, sca, res, xr, sg, corr);
       else unit_range<8, B>(nk, lo, hi, lane, sa + cb, sca, res, xr, sg, corr);
     }
   };
 
   // -- prologue: the first S batches' records, then (once the kernel before this one has finished, under
   // programmatic dependent launch) their activations; the meta jobs of batch 0
-  const int pre_batches = min(S, bt.nbatch);
-  int rb, re, pre_end;
-  bt.get(0, rb, re);
-  {
-    int a0, a1;
-    bt.get(pre_batches - 1, a0, a1);
-    pre_end = a1;  // the first S batches are records [L, pre_end), at most NS <= 32 of them
-  }
-  if (warp == 0) issue(L, pre_end, true, false);
+  BatchIt cur, nxt, iss;
+  cur.init(L, H, G, NB, NS);
+  iss = cur;
+  if (warp == 0)
+    for (int n = 0; n < S && iss.valid(); ++n, iss.next()) issue(iss, true, false);
+  else
+    for (int n = 0; n < S && iss.valid(); ++n) iss.next();
   asm volatile("griddepcontrol.wait;" ::: "memory");
   if (warp == 0) {
     __syncwarp();
-    issue(L, pre_end, false, true);
+    BatchIt it = cur;
+    for (; it.rb < iss.rb; it.next()) issue(it, false, true);
   }
-  for (int pos = warp; pos < re - rb; pos += W) meta_job(rb + pos, 0, pos);
+  for (int pos = warp; pos < cur.re - cur.rb; pos += W) meta_job(cur, pos, 0, 0);
   // every thread leaves each barrier with the same verdict on the CTA's abort flag
   bool aborted = __syncthreads_or(cta_abort != 0) != 0;
 
@@ -1565,54 +1624,61 @@ __global__ void __launch_bounds__(CCfg<B>::kThreads, 1) vbq_cc_kernel(const __gr
   for (int ww = 0; ww < NWW; ++ww)
 #pragma unroll
     for (int b = 0; b < B; ++b) acc[ww][b] = 0.f;
-  int last_issued_end = pre_end;
-  int mp = 0;  // meta set of batch n (n % 3)
-  for (int n = 0; n < bt.nbatch && !aborted; ++n) {
-    int nrb = 0, nre = 0;
-    if (n + 1 < bt.nbatch) bt.get(n + 1, nrb, nre);
+  int mp = 0, rp = 0;  // meta set (batch index % 3) and result set (batch index % 2) of the current batch
+  while (cur.valid() && !aborted) {
+    nxt = cur;
+    nxt.next();
     const int mpn = mp == 2 ? 0 : mp + 1;
-    jobs(n, rb, re, mp, nrb, nre, mpn);
+    jobs(cur, nxt, rp, mpn);
     aborted = __syncthreads_or(cta_abort != 0) != 0;
     if (aborted) break;
     // refill the slots of batch n with batch n + S (their records and activation rows)
-    if (n + S < bt.nbatch) {
-      int rb2, re2;
-      bt.get(n + S, rb2, re2);
-      if (re2 > dbase + kDirCache) {  // uniform: every thread takes this branch together
-        dbase = rb2;
-        fill_dir(rb2);
+    if (iss.valid()) {
+      if (iss.re > dbase + kDirCache) {  // uniform: every thread takes this branch together
+        dbase = iss.rb;
+        fill_dir(iss.rb);
         __syncthreads();
       }
       if (warp == 0) {
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        issue(rb2, re2, true, true);
+        issue(iss, true, true);
       }
-      last_issued_end = re2;
+      iss.next();
     }
-    // row pass of batch n: this warp's words, records in order
-    const int t = rb / G;
-    const TileOut to = tile_out(p, t);
+    // row pass of batch n: this warp's words, records in order. First every record's item index for the row
+    // (independent loads, issued together), then the results added in record order.
+    const TileOut to = tile_out(p, cur.t);
     const int Rt = to.Rt;
-    for (int pos = 0; pos < re - rb; ++pos) {
-      const unsigned char* mb = meta_ptr(mp, pos);
-      if (reinterpret_cast<const int*>(mb + mo.fl)[0]) continue;  // bad record (status already set)
-      const uint32_t* mk = reinterpret_cast<const uint32_t*>(mb + mo.mk);
-      const uint16_t* pf = reinterpret_cast<const uint16_t*>(mb + mo.pf);
-      const uint32_t* wc = reinterpret_cast<const uint32_t*>(mb + mo.wc);
-      const uint32_t res = res_addr(n, pos);
+    const int nrec = cur.re - cur.rb;
 #pragma unroll
-      for (int ww = 0; ww < NWW; ++ww) {
-        const int word = warp + ww * W, r = 32 * word + lane;
-        if (r < Rt) {
-          const int c = int(wc[r >> 4] >> (2 * (r & 15))) & 3;
-          const int item = pf[c * 32 + word] + __popc(mk[c * 32 + word] & ((1u << lane) - 1u));
+    for (int ww = 0; ww < NWW; ++ww) {
+      const int word = warp + ww * W, r = 32 * word + lane;
+      if (32 * word >= Rt) continue;
+      int item[kMaxNB];
 #pragma unroll
-          for (int b = 0; b < B; ++b) acc[ww][b] += lds32f(res + 4 * (item * B + b));
+      for (int pos = 0; pos < kMaxNB; ++pos) {
+        item[pos] = -1;
+        if (pos < nrec && r < Rt) {
+          const unsigned char* rm = row_ptr(mp, pos);
+          const uint32_t* mk = reinterpret_cast<const uint32_t*>(rm + mo.mk);
+          const uint16_t* pf = reinterpret_cast<const uint16_t*>(rm + mo.pf);
+          const uint32_t wcw = reinterpret_cast<const uint32_t*>(rm + mo.wc)[r >> 4];
+          const int c = int(wcw >> (2 * (r & 15))) & 3;
+          const int it = pf[c * 32 + word] + __popc(mk[c * 32 + word] & ((1u << lane) - 1u));
+          item[pos] = *reinterpret_cast<const int*>(rm + mo.bad) ? -1 : it;   // a bad record adds nothing
         }
       }
+#pragma unroll
+      for (int pos = 0; pos < kMaxNB; ++pos)
+        if (item[pos] >= 0) {
+          const uint32_t res = res_addr(rp, pos) + 4 * (item[pos] * B);
+#pragma unroll
+          for (int b = 0; b < B; ++b) acc[ww][b] += lds32f(res + 4 * b);
+        }
     }
-    // tile end: this CTA's share of tile t is complete
-    if (n + 1 == bt.nbatch || nrb / G != t) {
+    // tile end: this CTA's share of tile cur.t is complete
+    if (!nxt.valid() || nxt.t != cur.t) {
+      const int t = cur.t;
       const bool whole = L <= t * G && H >= (t + 1) * G;
       float* slot = p.partial + size_t(cta + t) * p.R * B;
 #pragma unroll
@@ -1629,15 +1695,15 @@ __global__ void __launch_bounds__(CCfg<B>::kThreads, 1) vbq_cc_kernel(const __gr
         for (int b = 0; b < B; ++b) acc[ww][b] = 0.f;
       }
     }
-    rb = nrb;
-    re = nre;
+    cur = nxt;
     mp = mpn;
+    rp ^= 1;
   }
   if (aborted) {
     // wait (bounded) for the copies still in flight before the CTA exits; publish nothing. Only the last use of
-    // each slot can still be in flight: the last NS records issued.
+    // each slot can still be in flight: the last NS records issued, which end at iss.rb.
     if (warp == 0) {
-      const int j = last_issued_end - NS + lane;
+      const int j = iss.rb - NS + lane;
       if (lane < NS && j >= L) mbar_drain(&bar_full[(j - L) % NS], ((j - L) / NS) & 1, p.wait_ns);
     }
     return;
@@ -1648,7 +1714,7 @@ __global__ void __launch_bounds__(CCfg<B>::kThreads, 1) vbq_cc_kernel(const __gr
 // ------------------------------------------------------------------------------------------ launch plan
 struct Plan {
   int grid, threads, NT, TW, S, stage_bytes, stage_size, team_bytes, acc_off, res_off, warps_off, warp_bytes, smem;
-  int NB, meta_off, dir_off, res_rec, meta_rec;  // CUDA-core kernel
+  int NB, meta_off, row_off, dir_off, res_rec, meta_rec;  // CUDA-core kernel
   uint64_t ws_bytes, status_off, counters_off;
 };
 
@@ -1763,7 +1829,7 @@ inline bool make_plan_t(const Problem& pr, int sms, Plan& pl) {
 template <int B>
 inline bool make_plan_cc(const Problem& pr, int sms, Plan& pl) {
   using C = CCfg<B>;
-  pl.grid = sms;
+  pl.grid = sms * kCCCtasPerSM;
   pl.threads = C::kThreads;
   const int R = pr.R;
   pl.stage_bytes = align128i(int(pr.max_record_bytes));
@@ -1772,23 +1838,26 @@ inline bool make_plan_cc(const Problem& pr, int sms, Plan& pl) {
   pl.meta_rec = MetaOff(B).size;
   const int dir_bytes = 8 * kDirCache;
   // units per record at the paper's allocation: 1-bit units of 32 items, the others of 32 / B; bucket tails
-  const int upr = (7 * R / 10 + 31) / 32 + (3 * R / 10 + C::kIPU - 1) / C::kIPU + 2;
-  const int nb_want = std::min(kMaxNB, std::max(1, (4 * C::kWarps + upr - 1) / upr));
+  const int upr = (7 * R / 10 + 31) / 32 + (16 * R / 100 + 31) / 32 + (15 * R / 100 + C::kIPU - 1) / C::kIPU + 2;
+  const int nb_want = std::min(kMaxNB, std::max(1, (5 * C::kWarps + upr - 1) / upr));
+  const MetaOff mo(B);
+  auto need = [&](int NB, int S) {
+    return (long long)S * NB * pl.stage_size + 2ll * NB * pl.res_rec + 256 + 2ll * NB * pl.meta_rec +
+           3ll * NB * mo.row_size + dir_bytes;
+  };
   pl.NB = 0;
   for (int NB = nb_want; NB >= 1 && pl.NB == 0; --NB)
-    for (int S = 3; S >= 2; --S) {
-      const long long smem = (long long)S * NB * pl.stage_size + 2ll * NB * pl.res_rec + 256 +
-                             3ll * NB * pl.meta_rec + dir_bytes;
-      if (smem <= kSmemBudget) {
+    for (int S = 3; S >= 2; --S)
+      if (need(NB, S) <= kSmemBudget / (16 / kCCWarps)) {  // a CTA of fewer warps leaves room for a second one
         pl.NB = NB;
         pl.S = S;
         break;
       }
-    }
   if (pl.NB == 0) return false;
   pl.res_off = pl.S * pl.NB * pl.stage_size;
   pl.meta_off = pl.res_off + 2 * pl.NB * pl.res_rec;
-  pl.dir_off = pl.meta_off + 256 + 3 * pl.NB * pl.meta_rec;
+  pl.row_off = pl.meta_off + 256 + 2 * pl.NB * pl.meta_rec;
+  pl.dir_off = pl.row_off + 3 * pl.NB * mo.row_size;
   pl.smem = pl.dir_off + dir_bytes;
   pl.NT = pl.TW = 1;
   pl.team_bytes = pl.acc_off = pl.warps_off = pl.warp_bytes = 0;
@@ -1858,15 +1927,18 @@ int launch(const Problem& pr, const void* const* blobs, const void* x, float* co
   p.warp_bytes = pl.warp_bytes;
   p.NB = pl.NB;
   p.meta_off = pl.meta_off;
+  p.row_off = pl.row_off;
   p.dir_off = pl.dir_off;
   p.res_rec = pl.res_rec;
   p.meta_rec = pl.meta_rec;
   // job costs (about the instructions a warp spends): units of 1-, 2-, 4-, 8-bit groups; a meta job
-  p.cost[0] = 30 + 40 * B;
-  p.cost[1] = 145;
-  p.cost[2] = 150;
-  p.cost[3] = 145;
-  p.cost[4] = 150 + 30 * B;
+  // job costs, in scheduler cycles of one lane (integer and packed fp32 instructions take two, fp32 one):
+  // 1- and 2-bit units (nibble tables, all batch rows), 4- and 8-bit units (magic-number expansion), a meta job
+  p.cost[0] = 60 + 20 * B;
+  p.cost[1] = 100 + 35 * B;
+  p.cost[2] = 285;
+  p.cost[3] = 275;
+  p.cost[4] = 400 + 100 * B;
   const unsigned long long wl = g_test_wait_ns.load();
   p.wait_ns = wl ? wl : kWaitNs;
   const long long wh = g_test_withhold.load();

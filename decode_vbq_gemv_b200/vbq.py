@@ -27,15 +27,18 @@ DEFAULT_TILE_ROWS = 256
 
 def suggest_tile_rows(rows: int, K: int, sms: int = 148) -> int:
     """Tile rows for packing a matrix (or the matrices of one fused launch, `rows` in total) on a GPU with `sms`
-    SMs, for batch 1: 224 unless 256-row tiles would leave fewer than 10 records per SM, then 512.
+    SMs: the largest of 1024, 512 and 256 that still gives every SM at least 7 records (tile, group column).
 
-    From a sweep of 128..512-row tiles over the 9B-shaped launch groups on B200 (graph-timed, batch 1):
-    224-row tiles ran fused q/k/v in 21.1 us (256: 21.2), fused gate/up with the SwiGLU epilogue in 37.2 us
-    (38.5), down in 21.4 us (21.8) and the 32000-row LM head in 42.6 us (43.8); 512-row tiles ran the lone
-    4096x4096 projection in 15.3 us (256: 17.5). At 224 rows, sixteen single-warp teams with two record stages
-    each fit in shared memory for these width mixes; at 256 only fifteen do."""
-    records = -(-rows // 256) * (K // 64)
-    return 512 if records < 10 * sms else 224
+    Larger tiles fill the width-bucket units better and cut per-record work; too few records per SM leave the
+    CTAs' batches short. From graph-timed launch groups of the 9B-shaped decode step on B200 at batch 1, this
+    picks the fastest of the three sizes for each: fused q/k/v 512 rows (21.8 us; 1024: 22.2), the lone 4096x4096
+    projection 256 (12.8 us; 512: 15.3), fused gate/up 1024 (34.1 us; 512: 40.3), down 512 (25.4 us; 1024:
+    27.7) and the LM head 1024 (33.3 us; 512: 40.3)."""
+    G = max(K // 64, 1)
+    for R in (1024, 512, 256):
+        if -(-rows // R) * G >= 7 * sms:
+            return R
+    return 256
 
 
 class VbqError(RuntimeError):

@@ -77,7 +77,9 @@ uint32_t vbq_version(void);
 
 /* ---------------------------------------------------------------------------------------------- host */
 
-/* Bytes of the canonical packed-format-v1 blob for this logical matrix.
+/* Bytes of the canonical packed-format-v1 blob for this logical matrix. No passage of the VBQ paper defines it:
+ * the paper fixes the group size and the width set, not a byte layout. R (tile rows) is a parameter of the
+ * layout, so the size depends on it.
  * widths: [N*G] in {1,2,4,8}. R: tile rows. Errors: NULL, SHAPE, TILE, WIDTH. Thread-safe, pure. */
 int vbq_packed_size(int64_t N, int64_t K, int64_t R, const uint8_t* widths, uint64_t* out_bytes);
 
@@ -113,12 +115,14 @@ int vbq_pack_ex(int64_t N, int64_t K, int64_t R, const uint8_t* widths, const ui
 int vbq_quantize(int64_t N, int64_t K, const float* w, const uint8_t* widths, unsigned format_flags,
                  uint16_t* scales, uint8_t* codes);
 
-/* Validate a host copy of a blob and fill *out_desc. Checks, in order: size >= 64 (BUFFER_TOO_SMALL), magic
+/* Validate a host copy of a blob and fill *out_desc (no passage of the VBQ paper: the blob's header and CRCs are
+ * this library's). Checks, in order: size >= 64 (BUFFER_TOO_SMALL), magic
  * (BAD_MAGIC), version (VERSION), header CRC (CRC), header fields (FORMAT), total_bytes <= blob_bytes
  * (BUFFER_TOO_SMALL), body CRC (CRC). It does not walk the records; vbq_unpack does. */
 int vbq_describe(const void* blob_host, uint64_t blob_bytes, vbq_desc* out_desc);
 
-/* Unpack a canonical blob (host memory) back into logical arrays sized from its header (N*G, N*G, N*K).
+/* Unpack a canonical blob (host memory) back into logical arrays sized from its header (N*G, N*G, N*K); the
+ * inverse of vbq_pack (no passage of the VBQ paper; the paper's kernels consume the packed form directly).
  * Performs every vbq_describe check, then checks each record: counts agree with the width codes, and every
  * padding byte and unused bit is zero (FORMAT). Any output pointer may be NULL to validate only. */
 int vbq_unpack(const void* blob_host, uint64_t blob_bytes, uint8_t* widths, uint16_t* scales,
@@ -127,7 +131,8 @@ int vbq_unpack(const void* blob_host, uint64_t blob_bytes, uint8_t* widths, uint
 /* -------------------------------------------------------------------------------------------- device */
 
 /* Workspace bytes that vbq_gemv / vbq_gemm_skinny need for this matrix and batch on the CURRENT device (the
- * launch shape depends on its SM count). The workspace holds the partial sums of row tiles that several CTAs
+ * launch shape depends on its SM count). No passage of the VBQ paper: the workspace exists because the kernels
+ * split the K dimension of a row tile among CTAs and reduce the partial sums without floating-point atomics. The workspace holds the partial sums of row tiles that several CTAs
  * share, one arrival counter per row tile, and, in its 4 bytes at offset (size - 4), a device status word: 0 after every
  * successful call; nonzero if a kernel gave up a bounded wait (bit 0), met a record larger than the staging
  * size its descriptor promised or a directory entry past the end of the records (bit 1), or met a record whose
@@ -140,7 +145,10 @@ int vbq_workspace_size(const vbq_desc* d, int B, uint64_t* out_bytes);
  * counters at zero again, so one zeroing per workspace is enough. Errors: NULL, CUDA. */
 int vbq_workspace_init(void* workspace, uint64_t workspace_bytes, void* stream);
 
-/* y[N] = W x for one activation vector (batch 1): vbq_gemm_skinny with B = 1.
+/* y[N] = W x for one activation vector (batch 1): vbq_gemm_skinny with B = 1. This is the VBQ paper's fused
+ * kernel (section 6, paragraph "Fused kernels over packed weights": the packed low-bit bytes of each group are
+ * expanded with the group scale in registers and the matrix-vector product accumulated; the FP16 matrix is never
+ * built), over the per-group widths and scales of section 3.1.
  * blob_dev: byte-identical device copy of the packed blob, 16-byte aligned (ALIGN).
  * x_bf16:   K bf16 values (device), 16-byte aligned (ALIGN).
  * y:        N fp32 values (device), 4-byte aligned; fully overwritten.
@@ -151,7 +159,10 @@ int vbq_workspace_init(void* workspace, uint64_t workspace_bytes, void* stream);
 int vbq_gemv(const vbq_desc* d, const void* blob_dev, const void* x_bf16, float* y, void* workspace,
              uint64_t workspace_bytes, void* stream);
 
-/* Y[B][N] = X[B][K] W^T for B in {1, 2, 4, 8, 16} activation rows (skinny GEMM; decode with a small batch).
+/* Y[B][N] = X[B][K] W^T for B in {1, 2, 4, 8, 16} activation rows (skinny GEMM; decode with a small batch). The
+ * same fused dequantize-and-multiply as vbq_gemv (VBQ paper, section 6, "Fused kernels over packed weights"),
+ * applied to several activation rows at once; the paper decodes at batch 1, the small batches are this library's
+ * extension.
  * x_bf16: B*K bf16 values, row-major (row b is activation b), 16-byte aligned. y: B*N fp32, row-major.
  * B <= 4 runs on CUDA cores; B = 8 and 16 run the dequantized groups through tensor cores (bf16 operands
  * that hold the exact integers 2(q - c), fp32 accumulation, the group scale applied in fp32).
