@@ -248,13 +248,13 @@ def test_symmetric_grid_pack_unpack_and_errors():
 
 
 def test_suggest_tile_rows_rule():
-    # 512-row tiles when 256-row tiles would leave fewer than 10 records per SM, else 224
-    assert vbq.suggest_tile_rows(4096, 4096, 148) == 512
-    assert vbq.suggest_tile_rows(3 * 4096, 4096, 148) == 224
-    assert vbq.suggest_tile_rows(2 * 14336, 4096, 148) == 224
-    assert vbq.suggest_tile_rows(4096, 14336, 148) == 224
-    assert vbq.suggest_tile_rows(32000, 4096, 148) == 224
-    assert vbq.suggest_tile_rows(768, 768, 148) == 512
+    # the largest of 1024, 512, 256 rows that leaves every SM at least 7 records (tile, group column)
+    assert vbq.suggest_tile_rows(4096, 4096, 148) == 256            # 1024 records at 256 rows: 6.9 per SM
+    assert vbq.suggest_tile_rows(3 * 4096, 4096, 148) == 512        # fused q/k/v
+    assert vbq.suggest_tile_rows(2 * 14336, 4096, 148) == 1024      # fused gate/up
+    assert vbq.suggest_tile_rows(4096, 14336, 148) == 512           # down: 224 group columns
+    assert vbq.suggest_tile_rows(32000, 4096, 148) == 1024          # LM head
+    assert vbq.suggest_tile_rows(768, 768, 148) == 256              # too small for any: the smallest
     for rows, K in ((1, 64), (4096, 4096), (32000, 4096)):
         R = vbq.suggest_tile_rows(rows, K, 148)
         assert 16 <= R <= 1024 and R % 16 == 0
