@@ -628,7 +628,7 @@ def run_cfg4(args):
                 "pct_of_peak": 100.0 * value / peak,
                 "roofline": {"bound": "hbm", "achieved": value, "peak": peak, "unit": "GB/s", "frac": value / peak,
                              "traffic": None, "peak_kind": peak_kind,
-                             "kernel": "vbq_cc_kernel<1> (batch 1, 2, 4), vbq_kernel<8|16> (batch 8, 16)"},
+                             "kernel": "vbq_kernel<B> (CUDA-core units at batch 1, 2, 4; mma.sync units at 8, 16)"},
                 "cfg4": results, "gpu_launches": n_launches, "clocks": clocks, "setup_s": round(t_setup, 1),
                 "e2e": None, "cpu_baseline": None}
         print(json.dumps(line), flush=True)

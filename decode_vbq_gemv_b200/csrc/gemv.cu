@@ -37,22 +37,11 @@
 namespace vbq {
 
 constexpr int kMaxTileRows = 1024;
-constexpr int kAStride = 72;            // bf16 per staged A row for ldmatrix (64 + 8 pad: conflict-free rows)
-constexpr int kMaxTeams = 16;
-constexpr int kMaxStages = 2;
 constexpr int kEpiChunk = 32;          // SwiGLU epilogue: tiles counted in per round
 constexpr int kSmemBudget = 227 * 1024 - 2048;  // dynamic shared memory; the rest is the static part
 constexpr unsigned long long kWaitNs = 2000000000ull;  // bounded mbarrier waits: 2 s
 constexpr unsigned kSuspendNs = 20000;                  // a waiting thread sleeps (no issue slots) up to 20 us per poll
 constexpr unsigned kStatusTimeout = 1u, kStatusOversize = 2u, kStatusRecord = 4u;
-
-template <int B> struct Cfg {
-  static constexpr int kWarps = (B == 1) ? 16 : (B < 8 ? 12 : 8);
-  static constexpr int kThreads = kWarps * 32;
-  // per-warp activation buffer: B <= 4: three fp32 tables [3][B][64]: x, x*2^-shift for 2-bit codes,
-  // x*2^-shift for 4-bit codes; B=8,16: the bf16 A tile of the tensor-core path, [32][kAStride]
-  static constexpr int kXBytes = (B <= 4) ? 3 * B * 64 * 4 : 32 * kAStride * 2;
-};
 
 // Up to kMaxMats matrices with the same K and tile rows run as one sequence of records (and row tiles): matrix m
 // holds global records [rec_start[m], rec_start[m+1]) and tiles [tile_start[m], tile_start[m+1]).
@@ -71,20 +60,17 @@ struct Params {
   uint16_t* h;             // bf16 bits, [B][N_0] (SwiGLU only)
   unsigned* pair;          // [T_0] row tiles of the gate/up pair already final; zero between calls (SwiGLU only)
   const uint16_t* x;       // bf16 bits, [B][K], shared by all matrices
-  float* partial;          // [nCTA + T][R][B] partial sums of shared row tiles
+  float* partial;          // [nCTA + T][B][R] partial sums of shared row tiles
   unsigned* arrive;        // [T] owners that have published their partial sums; zero between calls
   unsigned* status;        // device status word
   int K, G, R, T, nrec;    // T, nrec: all matrices
-  int NT, TW, S;           // teams per CTA, warps per team, stages per team
-  int stage_bytes;         // record capacity of one stage (multiple of 128)
-  int stage_size;          // stage: record, then the column's bf16 activations [B][64]
-  int team_bytes;          // per team: S stages | tile accumulators [R][B] f32 | item results (B <= 4, 1-2 x R x B f32)
-  int acc_off, res_off;
-  int warps_off, warp_bytes;
-  // CUDA-core kernel (batch <= 4) only
+  int S;                   // batches in flight (record slots: NB x S)
+  int stage_bytes;         // record capacity of one slot (multiple of 128)
+  int stage_size;          // slot: record, then the column's bf16 activations [B][64]
   int NB;                  // records per batch
-  int meta_off, row_off, dir_off;  // shared-memory offsets: table blocks, row blocks, directory cache
-  int res_rec, meta_rec;   // bytes per record: item results, metadata block
+  int res_off, meta_off, row_off, dir_off;  // shared-memory offsets: item results, table blocks, row blocks, directory
+  int res_rec, meta_rec;   // bytes per record: item results [R][B] f32, table block
+  int res_sets;            // item-result sets: 2 (alternate batches) or 1
   int cost[5];             // job costs for the split of a batch among warps: units of 1, 2, 4, 8 bits; meta job
   int withhold;            // test hook: the record (global index) whose bulk copy is never issued, or -1
   unsigned long long wait_ns;  // limit of every mbarrier wait
@@ -119,21 +105,6 @@ __device__ __forceinline__ TileOut tile_out(const Params& p, int t) {
 
 __host__ __device__ constexpr int align16i(int v) { return (v + 15) & ~15; }
 __host__ __device__ constexpr int align128i(int v) { return (v + 127) & ~127; }
-
-// Per-warp scratch: activations | group sums (B f32) | width masks [4][32] u32 | item starts [4][32] i32 |
-// width-code words of the record (up to 64 u32)
-struct WarpOff {
-  int x, sg, mk, pf, wd, sz;
-  __host__ __device__ WarpOff(int xbytes, int /*B*/) {
-    x = 0;
-    sg = align16i(xbytes);
-    mk = sg + 64;
-    pf = mk + 512;
-    wd = pf + 512;
-    sz = align128i(wd + 256);
-  }
-  __host__ __device__ int size() const { return sz; }
-};
 
 // ------------------------------------------------------------------------------------------ PTX helpers
 __device__ __forceinline__ uint32_t smem_u32(const void* p) { return uint32_t(__cvta_generic_to_shared(p)); }
@@ -254,6 +225,9 @@ __device__ __forceinline__ uint32_t lds8(uint32_t a) {
 __device__ __forceinline__ void sts32f(uint32_t a, float v) {
   asm volatile("st.shared.f32 [%0], %1;" ::"r"(a), "f"(v) : "memory");
 }
+__device__ __forceinline__ void sts64f(uint32_t a, float v0, float v1) {
+  asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(a), "f"(v0), "f"(v1) : "memory");
+}
 __device__ __forceinline__ void sts128(uint32_t a, const uint32_t (&v)[4]) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3])
                : "memory");
@@ -296,20 +270,7 @@ __device__ __forceinline__ float magic_f(uint32_t src, uint32_t mask_shifted) {
   return __uint_as_float((src & mask_shifted) | 0x4B000000u);
 }
 
-// Each returns sum_i (q_i - (2^k-1)/2) x_i for one 64-weight group; sg = sum_i x_i.
-// 1-bit: sum of the activations whose bit is set (predicated adds, eight independent sums), minus half the group
-// sum.
-__device__ __forceinline__ float dot_b1(uint2 w, const float (&xr)[64], float sg) {
-  float a[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-  for (int i = 0; i < 32; ++i)
-    if (w.x & (1u << i)) a[i & 7] += xr[i];
-#pragma unroll
-  for (int i = 0; i < 32; ++i)
-    if (w.y & (1u << i)) a[i & 7] += xr[32 + i];
-  return (((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]))) - 0.5f * sg;
-}
-
+// Each returns sum_i (q_i - c) x_i for one 64-weight group; sg = sum_i x_i.
 // 2- and 4-bit: xr holds x_i * 2^-shift(i). v - 2^23 = q * 2^shift exactly, so (v - 2^23) * xr_i = q * x_i.
 // The grid offset is c = 2^(k-1) - corr: corr = 1/2 on the default grid, 1 on Eq. 1's symmetric grid.
 template <int KB>
@@ -364,124 +325,6 @@ __device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
 // code words at byte address codes; off = 2c. Every value is an integer of magnitude at most 255, so every step
 // is exact: the magic-number expansion gives q * 2^shift (as in the batch-1 loops), one packed FMA scales it by
 // 2^(1 - shift) and subtracts 2c, and bf16 holds the result. 8-bit codes use the byte-permute form.
-template <int KB>
-__device__ __forceinline__ void dequant_a_row(uint32_t codes, uint32_t arow, float off) {
-  uint32_t w[2 * KB];
-  if constexpr (KB == 1) {
-    const uint2 a = lds64(codes);
-    w[0] = a.x; w[1] = a.y;
-  } else {
-#pragma unroll
-    for (int q = 0; q < KB / 2; ++q) {
-      const uint4 a = lds128(codes + 16 * q);
-      w[4 * q] = a.x; w[4 * q + 1] = a.y; w[4 * q + 2] = a.z; w[4 * q + 3] = a.w;
-    }
-  }
-  uint32_t out[4];
-  if constexpr (KB == 8) {
-    const float2 neg = make_float2(-8388736.f, -8388736.f);  // -(2^23 + 128)
-    const float2 two = make_float2(2.f, 2.f), c = make_float2(256.f - off, 256.f - off);
-#pragma unroll
-    for (int m = 0; m < 16; ++m) {
-      const float2 q0 = fadd2(make_float2(__uint_as_float(__byte_perm(w[m], 0x4B000000u, 0x7440u)),
-                                          __uint_as_float(__byte_perm(w[m], 0x4B000000u, 0x7441u))), neg);
-      const float2 q1 = fadd2(make_float2(__uint_as_float(__byte_perm(w[m], 0x4B000000u, 0x7442u)),
-                                          __uint_as_float(__byte_perm(w[m], 0x4B000000u, 0x7443u))), neg);
-      const float2 a0 = ffma2(q0, two, c), a1 = ffma2(q1, two, c);  // 2(q - 128) + 256 - 2c
-      out[(2 * m) & 3] = bf16x2_bits(a0.x, a0.y);
-      out[(2 * m + 1) & 3] = bf16x2_bits(a1.x, a1.y);
-      if (m & 1) sts128(arow + 16 * (m >> 1), out);
-    }
-  } else {
-    constexpr int CPW = 32 / KB;
-    constexpr uint32_t M = (1u << KB) - 1u;
-    const float2 neg = make_float2(-8388608.f, -8388608.f), c = make_float2(-off, -off);
-#pragma unroll
-    for (int i = 0; i < 64; i += 2) {
-      const int m = i / CPW, t = i % CPW;  // codes i and i + 1: positions t and t + 1 of word m
-      const uint32_t lo = w[m], hi = w[m] >> Magic<KB>::HI;
-      const float va = magic_f(magic_hi<KB>(t) ? hi : lo, M << magic_shift<KB>(t));
-      const float vb = magic_f(magic_hi<KB>(t + 1) ? hi : lo, M << magic_shift<KB>(t + 1));
-      const float2 q = fadd2(make_float2(va, vb), neg);  // (q_i 2^shift_i, q_i+1 2^shift_i+1)
-      const float2 a = ffma2(q, make_float2(pow2f(1 - magic_shift<KB>(t)), pow2f(1 - magic_shift<KB>(t + 1))), c);
-      out[(i >> 1) & 3] = bf16x2_bits(a.x, a.y);
-      if (((i >> 1) & 3) == 3) sts128(arow + 16 * (i >> 3), out);
-    }
-  }
-}
-
-// Batch B <= 4, one width bucket: the warp's units (local unit u for u = first, first + TW, ...) of 32 / B items
-// each. Lane = item * B + b: the lane computes the dot of its item's group with batch row b of the activations,
-// whose 64 values it holds in registers. The result s * dot goes to res[item][b] (byte addresses: codes, scales
-// and res for item 0 of the bucket; xtab is the activation table this width reads, [B][64] fp32). The
-// activations are loaded into registers unless `load` is false (they are already there). sg = sum of x of row b.
-template <int KB, int B>
-__device__ __forceinline__ void bucket_units(int n, int U, int first, int TW, int lane, uint32_t codes,
-                                             uint32_t scales, uint32_t res, float (&xr)[64], uint32_t xtab,
-                                             float sg, bool load, float corr) {
-  constexpr int IPU = 32 / B;  // items per unit
-  if (first >= U) return;
-  const int sub = lane / B, b = lane - sub * B;
-  if (load) {
-    const uint32_t xcopy = xtab + 256 * b;
-#pragma unroll
-    for (int q = 0; q < 16; ++q) {
-      const float4 f = lds128f(xcopy + 16 * q);
-      xr[4 * q] = f.x; xr[4 * q + 1] = f.y; xr[4 * q + 2] = f.z; xr[4 * q + 3] = f.w;
-    }
-  }
-  for (int u = first; u < U; u += TW) {
-    const int jj = IPU * u + sub;
-    if (jj >= n) continue;
-    float d;
-    if constexpr (KB == 1) {
-      d = dot_b1(lds64(codes + 8 * jj), xr, sg);
-    } else if constexpr (KB == 2) {
-      const uint4 a = lds128(codes + 16 * jj);
-      const uint32_t w[4] = {a.x, a.y, a.z, a.w};
-      d = dot_magic<2>(w, xr, sg, corr);
-    } else if constexpr (KB == 4) {
-      const uint4 a = lds128(codes + 32 * jj), c = lds128(codes + 32 * jj + 16);
-      const uint32_t w[8] = {a.x, a.y, a.z, a.w, c.x, c.y, c.z, c.w};
-      d = dot_magic<4>(w, xr, sg, corr);
-    } else {
-      uint32_t w[16];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const uint4 a = lds128(codes + 64 * jj + 16 * q);
-        w[4 * q] = a.x; w[4 * q + 1] = a.y; w[4 * q + 2] = a.z; w[4 * q + 3] = a.w;
-      }
-      d = dot_b8(w, xr, sg, corr);
-    }
-    sts32f(res + 4 * (jj * B + b), __half2float(__ushort_as_half((unsigned short)lds16(scales + 2 * jj))) * d);
-  }
-}
-// First local unit of a bucket for warp tw of TW, when the bucket's units follow `before` units of the record.
-__device__ __forceinline__ int first_unit(int tw, int before, int TW) {
-  if (TW == 1) return 0;
-  const int r = (tw - before) % TW;
-  return r < 0 ? r + TW : r;
-}
-
-// Row (within the tile) of item `item` of bucket c. masks[c][w] marks the rows of 32-row word w whose width code
-// is c; pref[c][w] is the item index of the first such row (bucket start + rows of code c in earlier words).
-// Binary search for the word, then select the k-th set bit of its mask.
-__device__ __forceinline__ int item_row(const uint32_t* masks, const int* pref, int c, int item) {
-  const int* P = pref + c * 32;
-  int w = 0;
-#pragma unroll
-  for (int step = 16; step > 0; step >>= 1)
-    if (P[w + step] <= item) w += step;
-  uint32_t m = masks[c * 32 + w];
-  int k = item - P[w], pos = 0, cnt;
-  cnt = __popc(m & 0xFFFFu); if (k >= cnt) { k -= cnt; m >>= 16; pos += 16; }
-  cnt = __popc(m & 0xFFu);   if (k >= cnt) { k -= cnt; m >>= 8;  pos += 8; }
-  cnt = __popc(m & 0xFu);    if (k >= cnt) { k -= cnt; m >>= 4;  pos += 4; }
-  cnt = __popc(m & 0x3u);    if (k >= cnt) { k -= cnt; m >>= 2;  pos += 2; }
-  if (k >= int(m & 1u)) pos += 1;
-  return 32 * w + pos;
-}
-
 // ----------------------------------------------------------------------------------------- record view
 // Offsets of the parts of a packed-format-v1 record with Rt rows and bucket counts n0..n3.
 struct Rec {
@@ -538,81 +381,17 @@ __device__ __forceinline__ int owner(const Params& p, int j) {
   return int(min(c, (long long)gridDim.x - 1));
 }
 
-// Barrier of one team: the warp itself, or a named hardware barrier (ids 1..15, one per team) over its warps.
-__device__ __forceinline__ void team_sync(int team, int TW) {
-  if (TW == 1) {
-    __syncwarp();
-  } else {
-    asm volatile("bar.sync %0, %1;" ::"r"(team + 1), "r"(TW * 32) : "memory");
-  }
-}
-
-// floor(a / b) for 0 <= a and 0 < b: through a float quotient when both are below 2^20 (then it is within one of
-// the exact quotient, and one correction step fixes it), else by integer division.
-__device__ __forceinline__ int div_floor(int a, int b) {
-  if ((a | b) < (1 << 20)) {
-    int q = __float2int_rz(__fdividef(float(a), float(b)));
-    if (q * b > a) --q;
-    else if ((q + 1) * b <= a) ++q;
-    return q;
-  }
-  return a / b;
-}
-
-// Closed-form split of the CTA's records [L, H) among its NT teams. The records fall into segments, one per row
-// tile. Every team computes its own share; nothing is exchanged.
-//  - At most NT segments: each segment gets one team plus a share of the NT - nseg spare teams proportional to its
-//    records (cumulative rounding), and is cut evenly among its teams. A team then never leaves its tile, and a
-//    segment with several teams is summed in shared memory at the end.
-//  - More segments than teams: each team takes whole segments, spread evenly by count.
-struct TeamMap {
-  int L, H, G, NT, n, tL, nseg;
-  __device__ TeamMap(int L_, int H_, int G_, int NT_) : L(L_), H(H_), G(G_), NT(NT_), n(H_ - L_), tL(0), nseg(0) {
-    if (n > 0) {
-      tL = div_floor(L, G);
-      nseg = div_floor(H - 1, G) - tL + 1;
-    }
-  }
-  __device__ bool split() const { return nseg <= NT; }
-  __device__ int seg_lo(int i) const { return max(L, (tL + i) * G); }
-  __device__ int seg_hi(int i) const { return min(H, (tL + i + 1) * G); }
-  // first team of segment i (split mode); seg_team0(nseg) == NT
-  __device__ int seg_team0(int i) const {
-    if (i >= nseg) return NT;
-    const unsigned num = unsigned(NT - nseg) * unsigned(seg_lo(i) - L);  // < 16 * n
-    return i + (n < (1 << 27) ? div_floor(int(num), n) : int((long long)(NT - nseg) * (seg_lo(i) - L) / n));
-  }
-  // records [lo, hi) of team k; seg = its segment when that segment has several teams, else -1
-  __device__ void team(int k, int& lo, int& hi, int& seg) const {
-    seg = -1;
-    if (n <= 0) { lo = hi = L; return; }
-    if (split()) {
-      int i = 0;
-      while (i + 1 < nseg && seg_team0(i + 1) <= k) ++i;
-      const int f = seg_team0(i), cnt = seg_team0(i + 1) - f;
-      const int s0 = seg_lo(i), len = seg_hi(i) - s0, q = k - f;
-      lo = s0 + div_floor(q * len, cnt);
-      hi = s0 + div_floor((q + 1) * len, cnt);
-      if (cnt >= 2) seg = i;
-    } else {
-      const int a = int((long long)k * nseg / NT), b = int((long long)(k + 1) * nseg / NT);
-      lo = max(L, (tL + a) * G);
-      hi = min(H, (tL + b) * G);
-    }
-  }
-};
-
-
 // ---------------------------------------------------------------------------------------- end of a CTA
 // Runs after every whole-tile output and every partial slot of this CTA is written (all threads, after a barrier).
 //  - Tiles shared with other CTAs (only a CTA's first and last tile can be): one thread makes the CTA's slot writes
 //    visible GPU-wide and counts the CTA in on the tile's arrival counter; the last owner to arrive adds all owners'
-//    slots in CTA order and resets the counter. No CTA waits for another.
+//    slots in an order fixed by the tile's shape and owner count, and resets the counter. No CTA waits for another.
 //  - SwiGLU epilogue (p.swiglu): matrices 0 (gate) and 1 (up) have the same rows and tiles. Whoever writes a tile's
 //    final y counts it in on the pair counter of its tile index; the second of the pair computes h = silu(gate) * up
 //    for those rows from both final outputs, rounded once to bf16, and resets the counter.
 template <int B, int kThreads>
-__device__ void finish_cta(const Params& p, int L, int H, int* cta_flags, int* epi_tiles, int* epi_count) {
+__device__ void finish_cta(const Params& p, int L, int H, int* cta_flags, int* epi_tiles, int* epi_count,
+                           unsigned char* scratch) {
   const int tid = threadIdx.x, G = p.G, R = p.R;
   if (H <= L) return;
   // Owners of tile t. With at least as many records as CTAs every CTA owns a contiguous, non-empty record range,
@@ -624,30 +403,82 @@ __device__ void finish_cta(const Params& p, int L, int H, int* cta_flags, int* e
     return dense ? owner(p, t * G + G - 1) - first + 1 : G;
   };
   auto kth_owner = [&](int t, int first, int k) -> int { return dense ? first + k : owner(p, t * G + k); };
-  // Sums of all owners' partial slots of tiles ta (and tb2 when ntiles == 2), each in CTA order, into y. The
-  // elements of both tiles form one index space; each thread has the loads of up to 16 owners in flight.
-  auto reduce_tiles = [&](int ta, int tb2, int ntiles) {
-    int fa, fb = 0;
-    const int oa = tile_owners(ta, fa), ob = ntiles > 1 ? tile_owners(tb2, fb) : 0;
-    const TileOut ya = tile_out(p, ta), yb = tile_out(p, ntiles > 1 ? tb2 : ta);
-    const int n0 = ya.Rt * B, ntot = n0 + (ntiles > 1 ? yb.Rt * B : 0);
-    for (int e2 = tid; e2 < ntot; e2 += kThreads) {
-      const bool second = e2 >= n0;
-      const int e = second ? e2 - n0 : e2, t = second ? tb2 : ta, first = second ? fb : fa;
-      const int owners = second ? ob : oa;
-      float v = 0.f;
-      for (int o0 = 0; o0 < owners; o0 += 16) {
-        float part[16];
+  // Sum of all owners' partial slots of tile t into y, in a fixed order. A slot holds [B][R] f32, so four rows of
+  // one batch row are one 16-byte load (item f: batch row f / nq, rows 4 (f % nq) ..). Large tiles: each thread
+  // sums U items over all owners in CTA order, OC owners' loads in flight. Small tiles: the owners are cut into C
+  // consecutive chunks summed by separate threads (OC loads in flight each), and the C chunk sums are added in
+  // chunk order through shared memory.
+  auto reduce_tile = [&](int t) {
+    constexpr int U = kThreads >= 512 ? 1 : 2, OC = 8;
+    int first;
+    const int owners = tile_owners(t, first);
+    const TileOut yo = tile_out(p, t);
+    const int nq = (yo.Rt + 3) >> 2, nf = nq * B;
+    auto load = [&](int o, int f) {
+      const int b = f / nq, r = 4 * (f - b * nq);
+      return __ldcg(reinterpret_cast<const float4*>(p.partial + size_t(kth_owner(t, first, o) + t) * R * B +
+                                                    size_t(b) * R + r));
+    };
+    auto store = [&](int f, float4 v) {
+      const int b = f / nq, r = 4 * (f - b * nq);
+      float* yr = yo.y + size_t(b) * yo.ld + r;
+      const float vv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-        for (int q = 0; q < 16; ++q)
-          part[q] = o0 + q < owners ? __ldcg(p.partial + size_t(kth_owner(t, first, o0 + q) + t) * R * B + e) : 0.f;
+      for (int i = 0; i < 4; ++i)
+        if (r + i < yo.Rt) yr[i] = vv[i];
+    };
+    auto add4 = [](float4& v, const float4& a) { v.x += a.x; v.y += a.y; v.z += a.z; v.w += a.w; };
+    // owners [o_begin, o_end) summed in order into v, for the item f of this thread
+    auto sum_owners = [&](int f, int o_begin, int o_end, float4& v) {
+      for (int o0 = o_begin; o0 < o_end; o0 += OC) {
+        float4 part[OC];
 #pragma unroll
-        for (int q = 0; q < 16; ++q)
-          if (o0 + q < owners) v += part[q];
+        for (int q = 0; q < OC; ++q) part[q] = o0 + q < o_end ? load(o0 + q, f) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int q = 0; q < OC; ++q)
+          if (o0 + q < o_end) add4(v, part[q]);
       }
-      const int r = e / B, b = e - r * B;
-      const TileOut& to = second ? yb : ya;
-      to.y[size_t(b) * to.ld + r] = v;
+    };
+    if (2 * nf > kThreads) {
+      for (int f0 = tid; f0 < nf; f0 += U * kThreads) {
+        float4 v[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int o0 = 0; o0 < owners; o0 += OC) {
+          float4 part[OC][U];
+#pragma unroll
+          for (int q = 0; q < OC; ++q)
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+              const int f = f0 + u * kThreads;
+              part[q][u] = (o0 + q < owners && f < nf) ? load(o0 + q, f) : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+          for (int q = 0; q < OC; ++q)
+            if (o0 + q < owners)
+#pragma unroll
+              for (int u = 0; u < U; ++u) add4(v[u], part[q][u]);
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+          if (f0 + u * kThreads < nf) store(f0 + u * kThreads, v[u]);
+      }
+    } else {
+      const int C = max(1, min(kThreads / nf, (owners + OC - 1) / OC)), per = (owners + C - 1) / C;
+      const int c = tid / nf, f = tid - c * nf;
+      float4* chunk = reinterpret_cast<float4*>(scratch);
+      if (c < C) {
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        sum_owners(f, c * per, min(owners, (c + 1) * per), v);
+        chunk[c * nf + f] = v;
+      }
+      __syncthreads();
+      if (tid < nf) {
+        float4 v = chunk[f];
+        for (int k = 1; k < C; ++k) add4(v, chunk[k * nf + f]);
+        store(f, v);
+      }
+      __syncthreads();
     }
   };
 
@@ -671,14 +502,11 @@ __device__ void finish_cta(const Params& p, int L, int H, int* cta_flags, int* e
       }
     }
     __syncthreads();
-    const int ntiles = cta_flags[0] + cta_flags[1];
-    if (ntiles > 0) {
-      const int ta = cta_flags[0] ? tfirst : tlast;
-      reduce_tiles(ta, tlast, ntiles);
-      if (tid == 0) {
-        p.arrive[ta] = 0u;
-        if (ntiles > 1) p.arrive[tlast] = 0u;
-      }
+    if (cta_flags[0]) reduce_tile(tfirst);
+    if (cta_flags[1]) reduce_tile(tlast);
+    if (tid == 0) {
+      if (cta_flags[0]) p.arrive[tfirst] = 0u;
+      if (cta_flags[1]) p.arrive[tlast] = 0u;
     }
   } else if (tid == 0) {
     cta_flags[0] = cta_flags[1] = 0;
@@ -718,429 +546,32 @@ __device__ void finish_cta(const Params& p, int L, int H, int* cta_flags, int* e
   }
 }
 
-// ------------------------------------------------------------------------------------------------ kernel
-template <int B>
-__global__ void __launch_bounds__(Cfg<B>::kThreads, 1) vbq_kernel(const __grid_constant__ Params params) {
-  using C = Cfg<B>;
-  extern __shared__ __align__(128) unsigned char smem[];
-  __shared__ uint64_t bar_full[kMaxTeams * kMaxStages];
-  __shared__ int stage_bad[kMaxTeams * kMaxStages];
-  __shared__ volatile int team_abort[kMaxTeams];
-  __shared__ int team_live[kMaxTeams];  // team has records (its accumulators hold a partial sum)
-  __shared__ int cta_flags[2];
-  __shared__ int epi_tiles[kEpiChunk];
-  __shared__ int epi_count;
-  __shared__ __align__(16) Params p;    // the launch parameters, read from here
-
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  // Copy the parameters to shared memory once, every word by its own thread: the first read of a parameter
-  // line misses the constant cache, and here those misses overlap instead of queuing up one after another
-  // wherever the parameters are first used.
-  static_assert(sizeof(Params) % 4 == 0 && sizeof(Params) / 4 <= Cfg<8>::kThreads, "parameter copy");
-  if (tid < int(sizeof(Params) / 4))
-    reinterpret_cast<uint32_t*>(&p)[tid] = reinterpret_cast<const uint32_t*>(&params)[tid];
-  __syncthreads();
-  const int NT = p.NT, TW = p.TW, S = p.S, G = p.G, R = p.R;
-  const int cta = blockIdx.x;
-  const int L = rec_lo(p, cta), H = rec_lo(p, cta + 1);
-  const TeamMap tm(L, H, G, NT);
-  // A kernel launched after this one with programmatic dependent launch may start its own prologue (which reads
-  // only its weights) as soon as SMs free up; it waits for this grid before touching activations or outputs.
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-
-  const int team = warp / TW, tw = warp - team * TW;
-  int tb = L, te = L, tseg = -1;
-  if (team < NT) tm.team(team, tb, te, tseg);
-  if (team < NT && tw == 0 && lane == 0) {
-    team_abort[team] = 0;
-    team_live[team] = tb < te;
-  }
-  if (team < NT && tb < te) {
-    // ================================================================== one team: records [tb, te)
-    const int nt = te - tb;
-    volatile int* abort_flag = &team_abort[team];
-    unsigned char* tbase = smem + team * p.team_bytes;
-    float* acc = reinterpret_cast<float*>(tbase + p.acc_off);       // tile accumulators [R][B]
-    unsigned char* wbase = smem + p.warps_off + warp * p.warp_bytes;
-    const WarpOff wo(C::kXBytes, B);
-    uint32_t* mk = reinterpret_cast<uint32_t*>(wbase + wo.mk);      // [4][32] width masks per 32-row word
-    int* pf = reinterpret_cast<int*>(wbase + wo.pf);                // [4][32] item index of the word's first row
-    uint32_t* wd = reinterpret_cast<uint32_t*>(wbase + wo.wd);      // width-code words of the record
-    const int sl0 = div_floor(tw * R, TW), sl1 = div_floor((tw + 1) * R, TW);  // this warp's rows (flush, row pass)
-    uint64_t* bars = bar_full + team * S;
-
-    // -- the team's first warp streams the records: directory entries 32 at a time in its lanes, loaded first
-    // (their latency is what the first copy waits for); lane 0 sets up the team's barriers and issues the copies
-    int issued = 0;
-    int win = 0;
-    uint32_t d_lo = 0, d_hi = 0;  // directory entries (start, end) of record tb + win + lane
-    int d_m = 0;                  // its matrix
-    auto load_dir = [&]() {
-      const int j = tb + win + lane;
-      if (win + lane < nt) {
-        d_m = mat_of_rec(p, j);
-        const int jl = j - (d_m == 0 ? 0 : d_m == 1 ? p.rec_start[1] : d_m == 2 ? p.rec_start[2] : p.rec_start[3]);
-        const uint32_t* dir = pick(p.dir, d_m);
-        d_lo = __ldg(dir + jl);
-        d_hi = __ldg(dir + jl + 1);
-      }
-    };
-    if (tw == 0) load_dir();
-    // Record i's bulk copy into stage i % S (whole warp, i non-decreasing between calls; lane 0 issues). The
-    // activations follow with issue_x.
-    auto issue_record = [&](int i) {
-      if (i >= win + 32) {
-        win = i;
-        load_dir();
-      }
-      const uint32_t a = __shfl_sync(0xFFFFFFFFu, d_lo, i - win);
-      const uint32_t b = __shfl_sync(0xFFFFFFFFu, d_hi, i - win);
-      const int m = __shfl_sync(0xFFFFFFFFu, d_m, i - win);
-      if (lane != 0) return;
-      const int s = i % S;
-      unsigned char* dst = tbase + s * p.stage_size;
-      const unsigned bytes = 16u * (b - a);
-      if (b < a || b > pick(p.units_total, m) || bytes > unsigned(p.stage_bytes)) {  // not what was promised
-        stage_bad[team * S + s] = 1;
-        atomicOr(p.status, kStatusOversize);
-        mbar_arrive(&bars[s]);
-      } else {
-        stage_bad[team * S + s] = 0;
-        mbar_arrive_tx(&bars[s], bytes + 128u * B);
-        if (tb + i != p.withhold) tma_bulk_load(dst, pick(p.recs, m) + 16ull * a, bytes, &bars[s]);
-      }
-    };
-    auto issue_x = [&](int i) {  // lane 0
-      const int s = i % S, j = tb + i, g = j % G;
-      if (stage_bad[team * S + s] || j == p.withhold) return;
-      unsigned char* dst = tbase + s * p.stage_size + p.stage_bytes;
-#pragma unroll
-      for (int bb = 0; bb < B; ++bb)
-        tma_bulk_load(dst + 128 * bb, p.x + size_t(bb) * p.K + size_t(g) * 64, 128u, &bars[s]);
-    };
-    if (tw == 0) {
-      if (lane == 0) {
-        for (int i = 0; i < S; ++i) mbar_init(&bars[i], 1);
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-      }
-      __syncwarp();
-      issued = min(S, nt);
-      for (int i = 0; i < issued; ++i) issue_record(i);
-    }
-    team_sync(team, TW);  // the team's barriers are initialized
-    // The weights never depend on an earlier kernel; the activations, outputs and workspace may. Under
-    // programmatic dependent launch this waits for the previous kernel; otherwise it returns at once.
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-    if (tw == 0 && lane == 0)
-      for (int i = 0; i < issued; ++i) issue_x(i);
-
-    // -- flush of a finished tile: straight into y when this team covers the whole tile. A partial tile that no
-    // other team of the CTA shares goes to the CTA's partial slot, counted in at the end of the kernel; a
-    // partial tile shared inside the CTA stays here for the combine at the end.
-    auto flush = [&](int t) {
-      if (tseg >= 0) return;  // shared inside the CTA: the combine at the end writes it
-      const TileOut to = tile_out(p, t);
-      const int Rt = to.Rt;
-      if (tb <= t * G && tb + nt >= (t + 1) * G) {
-        for (int r = sl0 + lane; r < min(sl1, Rt); r += 32)
-#pragma unroll
-          for (int b = 0; b < B; ++b) to.y[size_t(b) * to.ld + r] = acc[r * B + b];
-      } else {
-        float* slot = p.partial + size_t(cta + t) * R * B;
-        for (int e = sl0 * B + lane; e < min(sl1, Rt) * B; e += 32) slot[e] = acc[e];
-      }
-    };
-
-    int cur_t = -1;
-    float xr[B <= 4 ? 64 : 1];
-    for (int i = 0; i < nt; ++i) {
-      const int s = i % S;
-      const unsigned char* st = tbase + s * p.stage_size;
-      const uint32_t sa = smem_u32(st);
-      bool ok = mbar_wait(&bars[s], (i / S) & 1, p.status, abort_flag, p.wait_ns);
-      if (ok && stage_bad[team * S + s]) ok = false;
-      ok = __all_sync(0xFFFFFFFFu, ok);  // lanes can see an abort at different times; the warp decides as one
-      const int j = tb + i, t = j / G;
-      const int Rt = tile_out(p, t).Rt;
-      const bool grid_sym = pick(p.sym, mat_of_tile(p, t)) != 0;
-      const float corr = grid_sym ? 1.f : 0.5f;  // (q - c) = (q - 2^(k-1)) + corr for k >= 2
-      if (t != cur_t) {
-        if (cur_t >= 0) flush(cur_t);
-        for (int e = sl0 * B + lane; e < sl1 * B; e += 32) acc[e] = 0.f;
-        if (B >= 8) team_sync(team, TW);  // the tensor-core path accumulates any row of the tile
-        cur_t = t;
-      }
-      int n0 = 0, n1 = 0, n2 = 0, n3 = 0;
-      if (ok) {
-        const uint2 cnt = lds64(sa);
-        n0 = cnt.x & 0xFFFF; n1 = cnt.x >> 16; n2 = cnt.y & 0xFFFF; n3 = cnt.y >> 16;
-        // a record whose counts disagree with its tile, or whose buckets overrun the stage, is not read
-        const Rec rc(Rt, n0, n1, n2, n3);
-        if (n0 + n1 + n2 + n3 != Rt || rc.c3 + 64 * n3 > p.stage_bytes) {
-          if (lane == 0) atomicOr(p.status, kStatusRecord);
-          ok = false;
-        }
-      }
-      const Rec rc(Rt, n0, n1, n2, n3);
-      uint32_t m0 = 0, m1 = 0, m2 = 0, m3 = 0;
-      unsigned long long v = 0, pre = 0;
-      if (ok) {
-        // -- width masks and item starts per 32-row word (lane = word), and a copy of the width codes
-        const int nvalid = max(0, min(32, Rt - 32 * lane));
-        if (nvalid > 0) {
-          const uint2 v2 = lds64(sa + 8 + 8 * lane);
-          v = (unsigned long long)v2.x | ((unsigned long long)v2.y << 32);
-        }
-        // bit r of lo / hi: the low / high bit of row r's width code
-        const uint32_t lo = even_bits(v), hi = even_bits(v >> 1);
-        const uint32_t valid = nvalid >= 32 ? 0xFFFFFFFFu : ((1u << nvalid) - 1u);
-        m0 = ~hi & ~lo & valid;
-        m1 = ~hi & lo & valid;
-        m2 = hi & ~lo & valid;
-        m3 = hi & lo & valid;
-        const unsigned long long mine = (unsigned long long)__popc(m0) | ((unsigned long long)__popc(m1) << 16) |
-                                        ((unsigned long long)__popc(m2) << 32) |
-                                        ((unsigned long long)__popc(m3) << 48);
-        unsigned long long incl = mine;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-          const unsigned long long u = __shfl_up_sync(0xFFFFFFFFu, incl, off);
-          if (lane >= off) incl += u;
-        }
-        pre = incl - mine;
-        // the width codes must agree with the bucket counts, or no item index derived from them is in range
-        const unsigned long long tot = __shfl_sync(0xFFFFFFFFu, incl, 31);
-        if (tot != ((unsigned long long)n0 | ((unsigned long long)n1 << 16) | ((unsigned long long)n2 << 32) |
-                    ((unsigned long long)n3 << 48))) {
-          if (lane == 0) atomicOr(p.status, kStatusRecord);
-          ok = false;
-        }
-      }
-      if (ok) {
-        mk[lane] = m0; mk[32 + lane] = m1; mk[64 + lane] = m2; mk[96 + lane] = m3;
-        pf[lane] = int(pre & 0xFFFFull);
-        pf[32 + lane] = n0 + int((pre >> 16) & 0xFFFFull);
-        pf[64 + lane] = n0 + n1 + int((pre >> 32) & 0xFFFFull);
-        pf[96 + lane] = n0 + n1 + n2 + int(pre >> 48);
-        wd[2 * lane] = uint32_t(v);
-        wd[2 * lane + 1] = uint32_t(v >> 32);
-        // -- the column's activations, from the bf16 copy that landed with the record
-        const uint16_t* xg = reinterpret_cast<const uint16_t*>(st + p.stage_bytes);  // [B][64]
-        float* xv = reinterpret_cast<float*>(wbase + wo.x);
-        float* sgv = reinterpret_cast<float*>(wbase + wo.sg);
-        if constexpr (B <= 4) {
-          // tables [3][B][64]: x, x * 2^-shift for 2-bit codes, x * 2^-shift for 4-bit codes; row b's group sum
-          const float s2a = __uint_as_float(uint32_t(127 - code_shift<2>(lane)) << 23);
-          const float s2b = __uint_as_float(uint32_t(127 - code_shift<2>(32 + lane)) << 23);
-          const float s4a = __uint_as_float(uint32_t(127 - code_shift<4>(lane)) << 23);
-          const float s4b = __uint_as_float(uint32_t(127 - code_shift<4>(32 + lane)) << 23);
-#pragma unroll
-          for (int b = 0; b < B; ++b) {
-            const float x0 = __uint_as_float(uint32_t(xg[b * 64 + lane]) << 16);
-            const float x1 = __uint_as_float(uint32_t(xg[b * 64 + 32 + lane]) << 16);
-            xv[b * 64 + lane] = x0;
-            xv[b * 64 + 32 + lane] = x1;
-            xv[(B + b) * 64 + lane] = x0 * s2a;
-            xv[(B + b) * 64 + 32 + lane] = x1 * s2b;
-            xv[(2 * B + b) * 64 + lane] = x0 * s4a;
-            xv[(2 * B + b) * 64 + 32 + lane] = x1 * s4b;
-            float sg = x0 + x1;
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) sg += __shfl_xor_sync(0xFFFFFFFFu, sg, off);
-            if (lane == 0) sgv[b] = sg;
-          }
-        }
-        __syncwarp();
-
-        if constexpr (B <= 4) {
-          // -- CUDA cores, B <= 4: item results s * dot into the team's result buffer ([item][B], item order),
-          // one bucket at a time; lane = item * B + b. Units of 32 / B items are numbered across the buckets and
-          // dealt round-robin to the team's warps.
-          constexpr int IPU = 32 / B;
-          const float sg = sgv[lane % B];
-          const uint32_t xa = smem_u32(xv);
-          const uint32_t ra = smem_u32(tbase + p.res_off) + (TW > 1 ? 4 * R * B * (i & 1) : 0);
-          const uint32_t sca = sa + rc.sc;
-          const int c0 = (n0 + IPU - 1) / IPU, c1 = c0 + (n1 + IPU - 1) / IPU, c2 = c1 + (n2 + IPU - 1) / IPU,
-                    cU = c2 + (n3 + IPU - 1) / IPU;
-          // 1-bit and 8-bit units read the same (raw) activations, so they run back to back on one load.
-          bucket_units<1, B>(n0, c0, first_unit(tw, 0, TW), TW, lane, sa + rc.c0, sca, ra, xr, xa, sg, true, 0.5f);
-          bucket_units<8, B>(n3, cU - c2, first_unit(tw, c2, TW), TW, lane, sa + rc.c3, sca + 2 * (n0 + n1 + n2),
-                             ra + 4 * B * (n0 + n1 + n2), xr, xa, sg, first_unit(tw, 0, TW) >= c0, corr);
-          bucket_units<2, B>(n1, c1 - c0, first_unit(tw, c0, TW), TW, lane, sa + rc.c1, sca + 2 * n0,
-                             ra + 4 * B * n0, xr, xa + 256 * B, sg, true, corr);
-          bucket_units<4, B>(n2, c2 - c1, first_unit(tw, c1, TW), TW, lane, sa + rc.c2, sca + 2 * (n0 + n1),
-                             ra + 4 * B * (n0 + n1), xr, xa + 512 * B, sg, true, corr);
-        } else {
-          // -- tensor cores, B in {8, 16}: lane = group, dequantized to bf16 2(q - c) (2q-(2^k-1) on the default grid,
-          // 2q-(2^k-2) on the symmetric one; both exact) in this warp's A tile;
-          // two m16 tiles per unit through mma.sync m16n8k16 (bf16 in, fp32 accumulate), then s/2 per row.
-          constexpr int NTL = B >= 8 ? B / 8 : 1;
-          __nv_bfloat16* As = reinterpret_cast<__nv_bfloat16*>(wbase + wo.x);
-          const uint32_t* xb = reinterpret_cast<const uint32_t*>(st + p.stage_bytes);
-          uint32_t bfr[4][NTL][2];
-#pragma unroll
-          for (int ks = 0; ks < 4; ++ks)
-#pragma unroll
-            for (int nt2 = 0; nt2 < NTL; ++nt2) {
-              const int nb2 = nt2 * 8 + (lane >> 2);
-              bfr[ks][nt2][0] = xb[nb2 * 32 + 8 * ks + (lane & 3)];
-              bfr[ks][nt2][1] = xb[nb2 * 32 + 8 * ks + 4 + (lane & 3)];
-            }
-          for (int u = tw; u < rc.U; u += TW) {
-            int bk, j0, ibase, cbase, nb;
-            rc.unit(u, bk, j0, ibase, cbase, nb);
-            const int k = 1 << bk;
-            const int jj = j0 + lane;
-            const bool valid = jj < nb;
-            const uint32_t ar = smem_u32(As + lane * kAStride);
-            if (valid) {
-              const uint32_t cw = sa + uint32_t(cbase + 8 * k * jj);
-              const float off = float((1 << k) - 1 - ((grid_sym && k >= 2) ? 1 : 0));  // 2c: A = 2(q - c)
-              // bk is the same for the whole warp (a unit holds one bucket)
-              if (bk == 0) dequant_a_row<1>(cw, ar, off);
-              else if (bk == 1) dequant_a_row<2>(cw, ar, off);
-              else if (bk == 2) dequant_a_row<4>(cw, ar, off);
-              else dequant_a_row<8>(cw, ar, off);
-            } else {
-              const uint32_t z[4] = {0u, 0u, 0u, 0u};
-#pragma unroll
-              for (int q = 0; q < 8; ++q) sts128(ar + 16 * q, z);
-            }
-            __syncwarp();
-            float scale_mine = 0.f;
-            int row_mine = 0;
-            if (valid) {
-              scale_mine = 0.5f * __half2float(reinterpret_cast<const __half*>(st + rc.sc)[ibase + jj]);
-              row_mine = item_row(mk, pf, bk, ibase + jj);
-            }
-#pragma unroll
-            for (int mt = 0; mt < 2; ++mt) {
-              float c4[NTL][4];
-#pragma unroll
-              for (int nt2 = 0; nt2 < NTL; ++nt2) c4[nt2][0] = c4[nt2][1] = c4[nt2][2] = c4[nt2][3] = 0.f;
-#pragma unroll
-              for (int ks = 0; ks < 4; ++ks) {
-                const int r = mt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-                const int kk = ks * 16 + (lane >> 4) * 8;
-                uint32_t a0, a1, a2, a3;
-                asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-                             : "=r"(a0), "=r"(a1), "=r"(a2), "=r"(a3) : "r"(smem_u32(As + r * kAStride + kk)));
-#pragma unroll
-                for (int nt2 = 0; nt2 < NTL; ++nt2)
-                  asm volatile(
-                      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-                      "{%0,%1,%2,%3};"
-                      : "+f"(c4[nt2][0]), "+f"(c4[nt2][1]), "+f"(c4[nt2][2]), "+f"(c4[nt2][3])
-                      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(bfr[ks][nt2][0]), "r"(bfr[ks][nt2][1]));
-              }
-              // c4[nt][0..1]: tile row lane/4, batch nt*8 + 2(lane%4) + {0,1}; c4[nt][2..3]: tile row lane/4 + 8.
-#pragma unroll
-              for (int h = 0; h < 2; ++h) {
-                const int src = mt * 16 + (lane >> 2) + 8 * h;
-                const float sc = __shfl_sync(0xFFFFFFFFu, scale_mine, src);
-                const int row = __shfl_sync(0xFFFFFFFFu, row_mine, src);
-                if (j0 + src < nb) {
-#pragma unroll
-                  for (int nt2 = 0; nt2 < NTL; ++nt2) {
-                    const int b = nt2 * 8 + 2 * (lane & 3);
-                    acc[row * B + b] = fmaf(sc, c4[nt2][2 * h], acc[row * B + b]);
-                    acc[row * B + b + 1] = fmaf(sc, c4[nt2][2 * h + 1], acc[row * B + b + 1]);
-                  }
-                }
-              }
-            }
-            __syncwarp();
-          }
-        }
-      }
-      // every warp of the team is done with stage s (and, for B <= 4, has written its item results)
-      team_sync(team, TW);
-      if (tw == 0 && i + S < nt) {
-        const int go = __shfl_sync(0xFFFFFFFFu, *abort_flag ? 0 : 1, 0);
-        if (go) {
-          if (lane == 0) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-          issue_record(i + S);
-          if (lane == 0) issue_x(i + S);
-          ++issued;
-        }
-      }
-      if constexpr (B <= 4) {
-        if (ok) {
-          // -- row pass: row r of this warp's slice takes the results of its item (bucket start for its 32-row
-          // word, plus the rows of the same width before it in that word)
-          const uint32_t ra = smem_u32(tbase + p.res_off) + (TW > 1 ? 4 * R * B * (i & 1) : 0);
-          for (int r = sl0 + lane; r < min(sl1, Rt); r += 32) {
-            const int cc = int(wd[r >> 4] >> (2 * (r & 15))) & 3;
-            const int w = r >> 5;
-            const int item = pf[cc * 32 + w] + __popc(mk[cc * 32 + w] & ((1u << (r & 31)) - 1u));
-#pragma unroll
-            for (int b = 0; b < B; ++b) acc[r * B + b] += lds32f(ra + 4 * (item * B + b));
-          }
-        }
-      }
-    }
-    if (cur_t >= 0) flush(cur_t);
-    // After an abort, wait (bounded) for this team's copies still in flight before the CTA can exit.
-    if (*abort_flag && tw == 0 && lane == 0)
-      for (int r = max(0, issued - S); r < issued; ++r) mbar_drain(&bars[r % S], (r / S) & 1, p.wait_ns);
-  }
-
-  // =================================================================== combine of tiles shared by teams
-  asm volatile("griddepcontrol.wait;" ::: "memory");  // warps without records reach this point directly
-  __syncthreads();
-  for (int k = 0; k < NT; ++k)
-    if (team_abort[k]) return;  // a team gave up a wait: its outputs are not valid, publish nothing
-  if (tm.split()) {
-    for (int i = 0; i < tm.nseg; ++i) {
-      const int k0 = tm.seg_team0(i), m = tm.seg_team0(i + 1) - k0;
-      if (m < 2) continue;
-      const int s0 = tm.seg_lo(i), s1 = tm.seg_hi(i);
-      const int t = s0 / G;
-      const TileOut to = tile_out(p, t);
-      const int Rt = to.Rt;
-      const bool whole = s0 <= t * G && s1 >= (t + 1) * G;
-      float* slot = p.partial + size_t(cta + t) * R * B;
-      for (int e = tid; e < Rt * B; e += C::kThreads) {
-        float v = 0.f;
-        for (int q = 0; q < m; ++q)
-          if (team_live[k0 + q]) v += reinterpret_cast<const float*>(smem + (k0 + q) * p.team_bytes + p.acc_off)[e];
-        if (whole) {
-          const int r = e / B, b = e - r * B;
-          to.y[size_t(b) * to.ld + r] = v;
-        } else {
-          slot[e] = v;
-        }
-      }
-    }
-  }
-  finish_cta<B, C::kThreads>(p, L, H, cta_flags, epi_tiles, &epi_count);
-}
-
-
-// ====================================================================================== CUDA-core kernel
-// Batch B in {1, 2, 4}. One CTA per SM, 16 warps that work on the CTA's records together:
+// ===================================================================================== record-batch kernel
+// Every batch B in {1, 2, 4, 8, 16}. One CTA per SM whose warps (16 at B = 1, 2; 12 at B = 4, 8; 8 at B = 16:
+// as many as the registers of each batch size allow) work on the CTA's records together:
 //  - The CTA's record range is cut into batches of up to NB records of one row tile. Records stream HBM ->
 //    shared memory by cp.async.bulk (one copy per record plus one 128-byte copy per batch row of the column's
 //    activations), S batches ahead, each record in its own slot with its own mbarrier.
 //  - Each record gets a meta job one batch before its units run: validate it, build the width masks and item
-//    starts per 32-row word, the activation tables and the 1-bit nibble tables, and note where its buckets lie.
+//    starts per 32-row word, the group sums of x (and for B <= 4 the activation and nibble tables), and note where
+//    its buckets lie.
 //  - Per batch, the jobs are the width-bucket units of its records and the meta jobs of the next batch. Every warp
-//    computes the same job list from the meta blocks and takes the jobs whose cost midpoint falls in its 1/16 of
+//    computes the same job list from the meta blocks and takes the jobs whose cost midpoint falls in its share of
 //    the total, so the split is even to about one unit. A unit writes s * dot for each of its items (and batch
-//    rows) into the record's result buffer.
+//    rows) into the record's result buffer: on CUDA cores for B <= 4, through mma.sync for B = 8, 16.
 //  - One CTA barrier per batch. Then each warp adds the results of its own 32-row words to its accumulators,
 //    record by record in record order (row r takes the result of its item: the start of its bucket in its word
 //    plus the rows of the same width before it), so every row is summed in a fixed order and results are bitwise
 //    identical from run to run. The batch's slots are refilled right after the barrier.
 //  - A finished tile goes to y when the CTA holds all its records, else to the CTA's partial slot; finish_cta then
 //    reduces the tiles shared with neighbouring CTAs and runs the SwiGLU epilogue.
-constexpr int kCCWarps = 16;      // warps per CTA of the CUDA-core kernel
-constexpr int kCCCtasPerSM = 1;   // CTAs per SM in its grid
-template <int B> struct CCfg {
-  static constexpr int kWarps = kCCWarps;
+constexpr int kCudaCoreWarps = 16;      // warps per CTA at B = 1, 2
+constexpr int kCtasPerSM = 1;   // CTAs per SM in its grid
+template <int B> struct KCfg {
+  static constexpr bool kTC = B >= 8;                               // tensor-core units (batch 8, 16)
+  static constexpr int kWarps = B <= 2 ? kCudaCoreWarps : B <= 8 ? 12 : 8;
   static constexpr int kThreads = kWarps * 32;
-  static constexpr int kIPU = 32 / B;                               // items per 2-, 4-, 8-bit unit
+  static constexpr int kIPU = kTC ? 32 : 32 / B;                    // items per 4-, 8-bit unit
   static constexpr int kWordsPerWarp = (32 + kWarps - 1) / kWarps;  // row-pass words per warp (R <= 1024)
 };
 constexpr int kMaxNB = 7;        // records per batch: the 1 + 4 NB job segments of a batch fit in one warp
@@ -1161,11 +592,12 @@ struct MetaOff {
   int t1, t2, xt, sg, fl, size;      // table block
   int mk, pf, wc, bad, row_size;     // row block
   __host__ __device__ explicit MetaOff(int B) {
+    const int tb = B >= 8 ? 0 : B;   // the tensor-core path (batch 8, 16) needs no activation tables
     t1 = 0;
-    t2 = 1024 * B;
-    xt = t2 + 2048 * B;
-    sg = xt + 512 * B;
-    fl = sg + 16;
+    t2 = 1024 * tb;
+    xt = t2 + 2048 * tb;
+    sg = xt + 512 * tb;
+    fl = sg + 4 * (B < 4 ? 4 : B);     // group sums of x, one per batch row
     size = (fl + 64 + 255) & ~255;
     mk = 0;
     pf = 512;
@@ -1294,6 +726,130 @@ __device__ __forceinline__ void unit_range(int n, int lo, int hi, int lane, uint
   }
 }
 
+// Tensor-core A fragments (batch 8, 16). Lane (g, t) = (lane / 4, lane % 4) of an mma.sync m16n8k16 holds, for
+// each k-step ks, two bf16 pairs of A row g: logical columns 16 ks + 2t + {0, 1} and + {8, 9}. Logical columns
+// map to codes so that lane t reads one contiguous run of its item's codes: 16t .. 16t + 15, as 8 bf16 pairs
+// a[0..7], a[2 ks] and a[2 ks + 1] feeding k-step ks. The activations take the same map (tc_x_frags), so any
+// pairing of codes into registers is allowed; each width takes its cheapest exact one:
+//   1, 2 bits: pairs of adjacent codes (c_2r, c_2r+1), exact values q - c from a 16-entry nibble table;
+//   4 bits:    (c_r, c_r+4) and (c_8+r, c_12+r), r < 4: the bf16 bits 0x4300 | q = 128 + q, minus 136: q - 8;
+//   8 bits:    adjacent codes, q - 128 through fp32 (2^23 + q as bits, minus 2^23 + 128), then packed to bf16.
+// Every value is a small integer or half-integer, exact in bf16; the grid offset left over in the 4- and 8-bit
+// forms, (2^(k-1) - c) x group sum of x, seeds the accumulator.
+template <int KB>
+__device__ __forceinline__ void tc_a_frag(uint32_t addr, bool ok, uint32_t tab, uint32_t (&a)[8]) {
+  if constexpr (KB == 1) {
+    const uint32_t h = ok ? lds16(addr) : 0u;
+    const uint32_t e = (h << 3) & 0x7878u, o = (h >> 1) & 0x7878u;   // nibbles times 8: codes 0-3, 8-11 / 4-7, 12-15
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const uint2 lo = lds64(__byte_perm(e, tab, 0x7650u + k)), hi = lds64(__byte_perm(o, tab, 0x7650u + k));
+      a[4 * k] = lo.x; a[4 * k + 1] = lo.y; a[4 * k + 2] = hi.x; a[4 * k + 3] = hi.y;
+    }
+  } else if constexpr (KB == 2) {
+    const uint32_t w = ok ? lds32(addr) : 0u;
+    const uint32_t e = (w << 2) & 0x3C3C3C3Cu, o = (w >> 2) & 0x3C3C3C3Cu;   // nibbles times 4
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      a[2 * k] = lds32(__byte_perm(e, tab, 0x7650u + k));       // codes 4k, 4k + 1
+      a[2 * k + 1] = lds32(__byte_perm(o, tab, 0x7650u + k));   // codes 4k + 2, 4k + 3
+    }
+  } else if constexpr (KB == 4) {
+    uint2 w = make_uint2(0u, 0u);
+    if (ok) w = lds64(addr);
+    const __nv_bfloat162 m136 = __floats2bfloat162_rn(136.f, 136.f);
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const uint32_t v = (((r < 4 ? w.x : w.y) >> (4 * (r & 3))) & 0x000F000Fu) | 0x43004300u;
+      const __nv_bfloat162 d = __hsub2(*reinterpret_cast<const __nv_bfloat162*>(&v), m136);
+      a[r] = *reinterpret_cast<const uint32_t*>(&d);
+    }
+  } else {
+    uint4 w = make_uint4(0u, 0u, 0u, 0u);
+    if (ok) w = lds128(addr);
+    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+    const float2 neg = make_float2(-8388736.f, -8388736.f);   // -(2^23 + 128)
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const uint32_t x = ww[r >> 1], j = 2 * (r & 1);
+      const float2 q = fadd2(make_float2(__uint_as_float(__byte_perm(x, 0x4B000000u, 0x7440u + j)),
+                                         __uint_as_float(__byte_perm(x, 0x4B000000u, 0x7441u + j))), neg);
+      a[r] = bf16x2_bits(q.x, q.y);
+    }
+  }
+}
+
+// The activations of one group as mma B fragments in the code map of tc_a_frag: lane (g, t), batch row
+// b = 8 nt + g, k-step ks: bfr[ks][nt][0] pairs with a[2 ks], bfr[ks][nt][1] with a[2 ks + 1]. xb: the staged
+// bf16 activations [B][64] of the record's group. perm4: the 4-bit map, else adjacent pairs.
+template <int B>
+__device__ __forceinline__ void tc_x_frags(uint32_t xb, int lane, bool perm4, uint32_t (&bfr)[4][B / 8][2]) {
+  const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+  for (int nt = 0; nt < B / 8; ++nt) {
+    const uint32_t row = xb + 128 * (nt * 8 + g) + 32 * t;
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks) {
+      if (perm4) {   // codes base, base + 4 | base + 1, base + 5 with base = 2 ks + 4 (ks / 2)
+        const uint32_t base = 2 * ks + 4 * (ks >> 1);
+        const uint32_t u = lds32(row + 2 * base), v = lds32(row + 2 * base + 8);
+        bfr[ks][nt][0] = __byte_perm(u, v, 0x5410u);
+        bfr[ks][nt][1] = __byte_perm(u, v, 0x7632u);
+      } else {       // codes 4 ks, 4 ks + 1 | 4 ks + 2, 4 ks + 3
+        const uint2 u = lds64(row + 8 * ks);
+        bfr[ks][nt][0] = u.x;
+        bfr[ks][nt][1] = u.y;
+      }
+    }
+  }
+}
+
+// Tensor-core units [lo, hi) of one width bucket, 32 items each (B = 8, 16): per 16-item m-tile, lane (g, t) builds
+// the fragments of items 16 mt + g and + 8 from their codes, mma.sync m16n8k16 (bf16 in, fp32 accumulate, seeded
+// with the grid-offset term init[nt]) against the activations bfr, and writes s times each result to res[item][b].
+template <int B, int KB>
+__device__ __forceinline__ void unit_range_tc(int n, int lo, int hi, int lane, uint32_t codes, uint32_t scales,
+                                              uint32_t res, uint32_t tab, const float2 (&init)[B / 8],
+                                              const uint32_t (&bfr)[4][B / 8][2]) {
+  constexpr int NTL = B / 8;
+  const int g = lane >> 2, t = lane & 3;
+  for (int u = lo; u < hi; ++u) {
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt) {
+      const int i0 = 32 * u + 16 * mt + g, i1 = i0 + 8;
+      const bool ok0 = i0 < n, ok1 = i1 < n;
+      uint32_t a0[8], a1[8];
+      tc_a_frag<KB>(codes + 8 * KB * i0 + 2 * KB * t, ok0, tab, a0);
+      tc_a_frag<KB>(codes + 8 * KB * i1 + 2 * KB * t, ok1, tab, a1);
+      float c4[NTL][4];
+#pragma unroll
+      for (int nt = 0; nt < NTL; ++nt) {
+        c4[nt][0] = c4[nt][2] = init[nt].x;
+        c4[nt][1] = c4[nt][3] = init[nt].y;
+      }
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks)
+#pragma unroll
+        for (int nt = 0; nt < NTL; ++nt)
+          asm volatile(
+              "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+              "{%0,%1,%2,%3};"
+              : "+f"(c4[nt][0]), "+f"(c4[nt][1]), "+f"(c4[nt][2]), "+f"(c4[nt][3])
+              : "r"(a0[2 * ks]), "r"(a1[2 * ks]), "r"(a0[2 * ks + 1]), "r"(a1[2 * ks + 1]), "r"(bfr[ks][nt][0]),
+                "r"(bfr[ks][nt][1]));
+      // c4[nt][0..1]: item i0, batch rows 8 nt + 2t + {0, 1}; c4[nt][2..3]: item i1
+      const float s0 = ok0 ? __half2float(__ushort_as_half((unsigned short)lds16(scales + 2 * i0))) : 0.f;
+      const float s1 = ok1 ? __half2float(__ushort_as_half((unsigned short)lds16(scales + 2 * i1))) : 0.f;
+#pragma unroll
+      for (int nt = 0; nt < NTL; ++nt) {
+        const int b = nt * 8 + 2 * t;
+        if (ok0) sts64f(res + 4 * (i0 * B + b), s0 * c4[nt][0], s0 * c4[nt][1]);
+        if (ok1) sts64f(res + 4 * (i1 * B + b), s1 * c4[nt][2], s1 * c4[nt][3]);
+      }
+    }
+  }
+}
+
 // First job (of count jobs costing c each, in the segment starting at cost s0) whose cost midpoint reaches
 // cut2 / (2 W): the smallest j >= 0 with W (2 s0 + c (2j + 1)) >= cut2, at most count. The quotient comes from a
 // float division (all values are below 2^24), corrected to the exact integer.
@@ -1309,8 +865,8 @@ __device__ __forceinline__ int first_job(int cut2, int s0, int c, int count, int
 }
 
 template <int B>
-__global__ void __launch_bounds__(CCfg<B>::kThreads, 16 / kCCWarps) vbq_cc_kernel(const __grid_constant__ Params params) {
-  using C = CCfg<B>;
+__global__ void __launch_bounds__(KCfg<B>::kThreads, 1) vbq_kernel(const __grid_constant__ Params params) {
+  using C = KCfg<B>;
   constexpr int W = C::kWarps, IPU = C::kIPU, NWW = C::kWordsPerWarp;
   extern __shared__ __align__(128) unsigned char smem[];
   __shared__ uint64_t bar_full[kMaxNB * kMaxSets];
@@ -1320,12 +876,27 @@ __global__ void __launch_bounds__(CCfg<B>::kThreads, 16 / kCCWarps) vbq_cc_kerne
   __shared__ int epi_tiles[kEpiChunk];
   __shared__ int epi_count;
   __shared__ __align__(16) Params p;
+  // tensor-core path: nibble tables of exact A values. [0, 32): 1-bit, 16 entries of four bf16 (bit_i(n) - 1/2);
+  // [64, 80): 2-bit on the default grid, 16 entries of two bf16 (q - 3/2, q = n & 3 and n >> 2); [128, 144): 2-bit
+  // on the symmetric grid (q - 1)
+  __shared__ __align__(256) uint32_t tc_tab[192];
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   static_assert(sizeof(Params) % 4 == 0 && sizeof(Params) / 4 <= C::kThreads, "parameter copy");
   if (tid < int(sizeof(Params) / 4))
     reinterpret_cast<uint32_t*>(&p)[tid] = reinterpret_cast<const uint32_t*>(&params)[tid];
   if (tid == 0) cta_abort = 0;
+  if constexpr (C::kTC) {
+    if (tid < 32) {   // 1-bit: entry tid / 2, bf16 pair (tid & 1)
+      const int nib = tid >> 1, i0 = 2 * (tid & 1);
+      tc_tab[tid] = bf16x2_bits(float((nib >> i0) & 1) - 0.5f, float((nib >> (i0 + 1)) & 1) - 0.5f);
+    } else if (tid < 64) {   // 2-bit: default grid at [64, 80), symmetric grid at [128, 144)
+      const int e = tid & 15;
+      const bool sym = tid >= 48;
+      const float c = sym ? 1.f : 1.5f;
+      tc_tab[(sym ? 128 : 64) + e] = bf16x2_bits(float(e & 3) - c, float(e >> 2) - c);
+    }
+  }
   __syncthreads();
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int G = p.G, NB = p.NB, S = p.S, cta = blockIdx.x;
@@ -1363,7 +934,10 @@ __global__ void __launch_bounds__(CCfg<B>::kThreads, 16 / kCCWarps) vbq_cc_kerne
   const int meta0 = int(((smem_u32(smem + p.meta_off) + 255u) & ~255u) - smem_u32(smem));
   auto meta_ptr = [&](int tp, int pos) { return smem + meta0 + (tp * NB + pos) * p.meta_rec; };   // table block
   auto row_ptr = [&](int mp, int pos) { return smem + p.row_off + (mp * NB + pos) * MetaOff(B).row_size; };
-  auto res_addr = [&](int rp, int pos) { return smem_u32(smem + p.res_off + (rp * NB + pos) * p.res_rec); };
+  // result set of a batch: alternate sets when there are two, else the one set (and a barrier after each row pass)
+  auto res_addr = [&](int rp, int pos) {
+    return smem_u32(smem + p.res_off + ((p.res_sets > 1 ? rp : 0) * NB + pos) * p.res_rec);
+  };
 
   // Bulk copies of batch `it` (warp 0, one record per lane, at most NB <= 32): the records (with_rec) and the
   // activation rows (with_x) into their slots. The mbarrier of a slot expects both.
@@ -1463,6 +1037,24 @@ __global__ void __launch_bounds__(CCfg<B>::kThreads, 16 / kCCWarps) vbq_cc_kerne
       pf[96 + lane] = uint16_t(n0 + n1 + n2 + int(pre >> 48));
       wc[2 * lane] = uint32_t(v);
       wc[2 * lane + 1] = uint32_t(v >> 32);
+      if constexpr (C::kTC) {
+        // group sums of x per batch row: 32 / B lanes per row, each over 2B consecutive values
+        constexpr int LPR = 32 / B, VPL = 64 / LPR;
+        const uint32_t xa = smem_u32(st + p.stage_bytes) + 128 * (lane / LPR) + 2 * VPL * (lane % LPR);
+        float2 acc2 = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int q = 0; q < VPL / 8; ++q) {
+          const uint4 u = lds128(xa + 16 * q);
+          const uint32_t uu[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            acc2 = fadd2(acc2, make_float2(__uint_as_float(uu[i] << 16), __uint_as_float(uu[i] & 0xFFFF0000u)));
+        }
+        float sgl = acc2.x + acc2.y;
+#pragma unroll
+        for (int off = 1; off < LPR; off <<= 1) sgl += __shfl_xor_sync(0xFFFFFFFFu, sgl, off);
+        if (lane % LPR == 0) reinterpret_cast<float*>(mb + mo.sg)[lane / LPR] = sgl;
+      } else {
       // activation tables [2][B][64]: x, x * 2^-shift (4-bit codes); group sums
       const uint16_t* xg = reinterpret_cast<const uint16_t*>(st + p.stage_bytes);
       float* xv = reinterpret_cast<float*>(mb + mo.xt);
@@ -1508,6 +1100,7 @@ __global__ void __launch_bounds__(CCfg<B>::kThreads, 16 / kCCWarps) vbq_cc_kerne
           sts128(t2a + 2048 * b + 16 * qb, row);
         }
       }
+      }
       if (lane == 0) {
         const Rec rc(Rt, n0, n1, n2, n3);
         fl[1] = rc.sc;
@@ -1539,7 +1132,7 @@ __global__ void __launch_bounds__(CCfg<B>::kThreads, 16 / kCCWarps) vbq_cc_kerne
       const int k = q == 0 ? 0 : q == 1 ? 1 : q == 2 ? 3 : 2;
       const int* fl = reinterpret_cast<const int*>(meta_ptr(rp, pos) + mo.fl);
       const int nk = fl[2 + k];
-      count = k < 2 ? (nk + 31) >> 5 : (nk + IPU - 1) / IPU;
+      count = (k < 2 || C::kTC) ? (nk + 31) >> 5 : (nk + IPU - 1) / IPU;
       cost = p.cost[k];
     }
     const int tot = count * cost;
@@ -1553,9 +1146,11 @@ __global__ void __launch_bounds__(CCfg<B>::kThreads, 16 / kCCWarps) vbq_cc_kerne
     const int jlo = first_job(2 * total * warp, s0, max(cost, 1), count, W);
     const int jhi = first_job(2 * total * (warp + 1), s0, max(cost, 1), count, W);
     unsigned todo = __ballot_sync(0xFFFFFFFFu, jhi > jlo);
-    float xr[64];
+    float xr[C::kTC ? 1 : 64];
     int loaded = -1;
-    const float corr = pick(p.sym, mat_of_tile(p, cur.t)) != 0 ? 1.f : 0.5f;
+    const bool grid_sym = pick(p.sym, mat_of_tile(p, cur.t)) != 0;
+    const float corr = grid_sym ? 1.f : 0.5f;
+    uint32_t bfr[4][C::kTC ? B / 8 : 1][2];   // tensor-core path: the record's activations as mma B fragments
     while (todo) {
       const int sgi = __ffs(todo) - 1;
       todo &= todo - 1;
@@ -1575,6 +1170,27 @@ __global__ void __launch_bounds__(CCfg<B>::kThreads, 16 / kCCWarps) vbq_cc_kerne
       const uint32_t sa = smem_u32(slot_ptr(slot));
       const uint32_t res = res_addr(rp, pos) + 4 * B * ib;
       const uint32_t sca = sa + sc + 2 * ib;
+      if constexpr (C::kTC) {
+        const int kind = pos * 2 + (k == 2 ? 1 : 0);   // the 4-bit code map differs from the others'
+        if (loaded != kind) {
+          tc_x_frags<B>(smem_u32(slot_ptr(slot) + p.stage_bytes), lane, k == 2, bfr);
+          loaded = kind;
+        }
+        // accumulator seed: (2^(k-1) - c) sum x for 4 and 8 bits (1/2 on the default grid, 1 on the symmetric)
+        float2 init[B / 8];
+        const float* sgv = reinterpret_cast<const float*>(mb + mo.sg);
+        const float f = k < 2 ? 0.f : corr;
+#pragma unroll
+        for (int nt = 0; nt < B / 8; ++nt) {
+          const float2 sg2 = *reinterpret_cast<const float2*>(sgv + nt * 8 + 2 * (lane & 3));
+          init[nt] = make_float2(f * sg2.x, f * sg2.y);
+        }
+        const uint32_t tb = smem_u32(tc_tab);
+        if (k == 0) unit_range_tc<B, 1>(nk, lo, hi, lane, sa + cb, sca, res, tb, init, bfr);
+        else if (k == 1) unit_range_tc<B, 2>(nk, lo, hi, lane, sa + cb, sca, res, tb + (grid_sym ? 512 : 256), init, bfr);
+        else if (k == 2) unit_range_tc<B, 4>(nk, lo, hi, lane, sa + cb, sca, res, tb, init, bfr);
+        else unit_range_tc<B, 8>(nk, lo, hi, lane, sa + cb, sca, res, tb, init, bfr);
+      } else {
       if (k < 2) {
         float sgb[B];
 #pragma unroll
@@ -1597,6 +1213,7 @@ __global__ void __launch_bounds__(CCfg<B>::kThreads, 16 / kCCWarps) vbq_cc_kerne
       const float sg = reinterpret_cast<const float*>(mb + mo.sg)[b];
       if (k == 2) unit_range<4, B>(nk, lo, hi, lane, sa + cb, sca, res, xr, sg, corr);
       else unit_range<8, B>(nk, lo, hi, lane, sa + cb, sca, res, xr, sg, corr);
+      }
     }
   };
 
@@ -1672,8 +1289,16 @@ __global__ void __launch_bounds__(CCfg<B>::kThreads, 16 / kCCWarps) vbq_cc_kerne
       for (int pos = 0; pos < kMaxNB; ++pos)
         if (item[pos] >= 0) {
           const uint32_t res = res_addr(rp, pos) + 4 * (item[pos] * B);
+          if constexpr (B >= 4) {
 #pragma unroll
-          for (int b = 0; b < B; ++b) acc[ww][b] += lds32f(res + 4 * b);
+            for (int b = 0; b < B; b += 4) {
+              const float4 v = lds128f(res + 4 * b);
+              acc[ww][b] += v.x; acc[ww][b + 1] += v.y; acc[ww][b + 2] += v.z; acc[ww][b + 3] += v.w;
+            }
+          } else {
+#pragma unroll
+            for (int b = 0; b < B; ++b) acc[ww][b] += lds32f(res + 4 * b);
+          }
         }
     }
     // tile end: this CTA's share of tile cur.t is complete
@@ -1688,7 +1313,7 @@ __global__ void __launch_bounds__(CCfg<B>::kThreads, 16 / kCCWarps) vbq_cc_kerne
 #pragma unroll
           for (int b = 0; b < B; ++b) {
             if (whole) to.y[size_t(b) * to.ld + r] = acc[ww][b];
-            else slot[r * B + b] = acc[ww][b];
+            else slot[b * p.R + r] = acc[ww][b];
           }
         }
 #pragma unroll
@@ -1698,6 +1323,7 @@ __global__ void __launch_bounds__(CCfg<B>::kThreads, 16 / kCCWarps) vbq_cc_kerne
     cur = nxt;
     mp = mpn;
     rp ^= 1;
+    if (p.res_sets == 1) __syncthreads();   // the next batch's units overwrite the one result set
   }
   if (aborted) {
     // wait (bounded) for the copies still in flight before the CTA exits; publish nothing. Only the last use of
@@ -1708,13 +1334,13 @@ __global__ void __launch_bounds__(CCfg<B>::kThreads, 16 / kCCWarps) vbq_cc_kerne
     }
     return;
   }
-  finish_cta<B, C::kThreads>(p, L, H, cta_flags, epi_tiles, &epi_count);
+  finish_cta<B, C::kThreads>(p, L, H, cta_flags, epi_tiles, &epi_count, smem);
 }
 
 // ------------------------------------------------------------------------------------------ launch plan
 struct Plan {
-  int grid, threads, NT, TW, S, stage_bytes, stage_size, team_bytes, acc_off, res_off, warps_off, warp_bytes, smem;
-  int NB, meta_off, row_off, dir_off, res_rec, meta_rec;  // CUDA-core kernel
+  int grid, threads, S, stage_bytes, stage_size, res_off, smem;
+  int NB, RS, meta_off, row_off, dir_off, res_rec, meta_rec;  // record-batch kernel
   uint64_t ws_bytes, status_off, counters_off;
 };
 
@@ -1768,7 +1394,7 @@ inline int make_problem(int nmat, const vbq_desc* const* d, Problem& pr) {
   return VBQ_OK;
 }
 
-// Workspace: partial slots [nCTA + T][R][B] f32 of the row tiles that CTAs share, then an arrival counter and a
+// Workspace: partial slots [nCTA + T][B][R] f32 of the row tiles that CTAs share, then an arrival counter and a
 // SwiGLU pair counter per tile, then the status word.
 inline void plan_workspace(const Problem& pr, int B, Plan& pl) {
   const uint64_t slots = uint64_t(pl.grid) + uint64_t(pr.T);
@@ -1777,59 +1403,13 @@ inline void plan_workspace(const Problem& pr, int B, Plan& pl) {
   pl.status_off = pl.ws_bytes - 4;
 }
 
-// Teams per CTA, warps per team and stages per team. A team's record copies overlap its arithmetic when it has
-// two stages; with one, every record's load latency is exposed. The plan that fits in shared memory with the
-// fewest exposed load latencies (records per team / stages, rounded up) wins; ties go to more warps, then to
-// more teams.
-template <int B>
-inline bool make_plan_t(const Problem& pr, int sms, Plan& pl) {
-  using C = Cfg<B>;
-  pl.grid = sms;
-  pl.threads = C::kThreads;
-  const int R = pr.R;
-  const int rpc = int((pr.nrec + pl.grid - 1) / pl.grid);
-  pl.stage_bytes = align128i(int(pr.max_record_bytes));
-  pl.stage_size = pl.stage_bytes + align128i(128 * B);
-  const int acc_bytes = align128i(R * B * 4);
-  pl.warp_bytes = WarpOff(C::kXBytes, B).size();
-  const int W = C::kWarps;
-  long long best_key = -1;
-  for (int NT = min(min(W, kMaxTeams), max(rpc, 1)); NT >= 1; --NT) {
-    const int TW = W / NT;
-    if (TW > 1 && NT > 15) continue;  // named barrier ids 1..15
-    const int rpt = (rpc + NT - 1) / NT;
-    // batch <= 4: item results, double-buffered when several warps share a record
-    const int res_bytes = B <= 4 ? align128i((TW > 1 ? 2 : 1) * R * B * 4) : 0;
-    for (int S = min(max(rpt, 1), kMaxStages); S >= 1; --S) {
-      const int team_bytes = S * pl.stage_size + acc_bytes + res_bytes;
-      const long long smem = (long long)NT * team_bytes + (long long)NT * TW * pl.warp_bytes;
-      if (smem > kSmemBudget) continue;
-      const long long exposed = (rpt + S - 1) / S;
-      const long long key = (1000000 - exposed) * 10000 + (long long)NT * TW * 100 + NT;
-      if (key > best_key) {
-        best_key = key;
-        pl.NT = NT; pl.TW = TW; pl.S = S;
-        pl.team_bytes = team_bytes;
-        pl.acc_off = S * pl.stage_size;
-        pl.res_off = pl.acc_off + acc_bytes;
-        pl.warps_off = NT * team_bytes;
-        pl.smem = int(smem);
-      }
-      break;  // fewer stages only expose more latency
-    }
-  }
-  if (best_key < 0) return false;
-  plan_workspace(pr, B, pl);
-  return true;
-}
-
-// CUDA-core kernel (B <= 4): records per batch NB and batches in flight S. NB aims at about three jobs per warp
+// Records per batch NB and batches in flight S. NB aims at about three jobs per warp
 // per batch (from an estimate of the units per record at the paper's allocation); S = 3 when it fits (the meta
 // jobs of a batch read records issued two batches earlier), else 2. Fewer records per batch before fewer sets.
 template <int B>
-inline bool make_plan_cc(const Problem& pr, int sms, Plan& pl) {
-  using C = CCfg<B>;
-  pl.grid = sms * kCCCtasPerSM;
+inline bool make_plan_b(const Problem& pr, int sms, Plan& pl) {
+  using C = KCfg<B>;
+  pl.grid = sms * kCtasPerSM;
   pl.threads = C::kThreads;
   const int R = pr.R;
   pl.stage_bytes = align128i(int(pr.max_record_bytes));
@@ -1841,37 +1421,39 @@ inline bool make_plan_cc(const Problem& pr, int sms, Plan& pl) {
   const int upr = (7 * R / 10 + 31) / 32 + (16 * R / 100 + 31) / 32 + (15 * R / 100 + C::kIPU - 1) / C::kIPU + 2;
   const int nb_want = std::min(kMaxNB, std::max(1, (5 * C::kWarps + upr - 1) / upr));
   const MetaOff mo(B);
-  auto need = [&](int NB, int S) {
-    return (long long)S * NB * pl.stage_size + 2ll * NB * pl.res_rec + 256 + 2ll * NB * pl.meta_rec +
+  auto need = [&](int NB, int S, int RS) {
+    return (long long)S * NB * pl.stage_size + (long long)RS * NB * pl.res_rec + 256 + 2ll * NB * pl.meta_rec +
            3ll * NB * mo.row_size + dir_bytes;
   };
+  // two result sets let the next batch's units start before every warp has finished this batch's row pass; one
+  // set (with a barrier after each row pass) is the last resort for large records at batch 16
   pl.NB = 0;
-  for (int NB = nb_want; NB >= 1 && pl.NB == 0; --NB)
-    for (int S = 3; S >= 2; --S)
-      if (need(NB, S) <= kSmemBudget / (16 / kCCWarps)) {  // a CTA of fewer warps leaves room for a second one
-        pl.NB = NB;
-        pl.S = S;
-        break;
-      }
+  for (int RS = 2; RS >= 1 && pl.NB == 0; --RS)
+    for (int NB = nb_want; NB >= 1 && pl.NB == 0; --NB)
+      for (int S = 3; S >= 2; --S)
+        if (need(NB, S, RS) <= kSmemBudget) {
+          pl.NB = NB;
+          pl.S = S;
+          pl.RS = RS;
+          break;
+        }
   if (pl.NB == 0) return false;
   pl.res_off = pl.S * pl.NB * pl.stage_size;
-  pl.meta_off = pl.res_off + 2 * pl.NB * pl.res_rec;
+  pl.meta_off = pl.res_off + pl.RS * pl.NB * pl.res_rec;
   pl.row_off = pl.meta_off + 256 + 2 * pl.NB * pl.meta_rec;
   pl.dir_off = pl.row_off + 3 * pl.NB * mo.row_size;
   pl.smem = pl.dir_off + dir_bytes;
-  pl.NT = pl.TW = 1;
-  pl.team_bytes = pl.acc_off = pl.warps_off = pl.warp_bytes = 0;
   plan_workspace(pr, B, pl);
   return true;
 }
 
 inline bool make_plan(const Problem& pr, int B, int sms, Plan& pl) {
   switch (B) {
-    case 1: return make_plan_cc<1>(pr, sms, pl);
-    case 2: return make_plan_cc<2>(pr, sms, pl);
-    case 4: return make_plan_cc<4>(pr, sms, pl);
-    case 8: return make_plan_t<8>(pr, sms, pl);
-    default: return make_plan_t<16>(pr, sms, pl);
+    case 1: return make_plan_b<1>(pr, sms, pl);
+    case 2: return make_plan_b<2>(pr, sms, pl);
+    case 4: return make_plan_b<4>(pr, sms, pl);
+    case 8: return make_plan_b<8>(pr, sms, pl);
+    default: return make_plan_b<16>(pr, sms, pl);
   }
 }
 
@@ -1883,9 +1465,8 @@ std::atomic<long long> g_test_withhold{-1};
 template <int B>
 int launch(const Problem& pr, const void* const* blobs, const void* x, float* const* ys, void* ws, uint64_t ws_bytes,
            unsigned flags, cudaStream_t stream, uint16_t* h = nullptr, unsigned* status = nullptr) {
-  constexpr bool cc = B <= 4;  // CUDA-core kernel; batch 8 and 16 run the tensor-core kernel
   Plan pl;
-  if (!(cc ? make_plan_cc<B>(pr, num_sms(), pl) : make_plan_t<B>(pr, num_sms(), pl))) return VBQ_ERR_FORMAT;
+  if (!make_plan_b<B>(pr, num_sms(), pl)) return VBQ_ERR_FORMAT;
   if (!ws || (reinterpret_cast<uintptr_t>(ws) & 15) || ws_bytes < pl.ws_bytes) return VBQ_ERR_WORKSPACE;
   Params p = {};
   p.nmat = pr.nmat;
@@ -1917,33 +1498,39 @@ int launch(const Problem& pr, const void* const* blobs, const void* x, float* co
   p.status = status ? status : reinterpret_cast<unsigned*>(w + pl.status_off);
   p.K = pr.K; p.G = pr.G; p.R = pr.R; p.T = tiles;
   p.nrec = recs;
-  p.NT = pl.NT; p.TW = pl.TW; p.S = pl.S;
+  p.S = pl.S;
   p.stage_bytes = pl.stage_bytes;
   p.stage_size = pl.stage_size;
-  p.team_bytes = pl.team_bytes;
-  p.acc_off = pl.acc_off;
   p.res_off = pl.res_off;
-  p.warps_off = pl.warps_off;
-  p.warp_bytes = pl.warp_bytes;
   p.NB = pl.NB;
   p.meta_off = pl.meta_off;
   p.row_off = pl.row_off;
   p.dir_off = pl.dir_off;
   p.res_rec = pl.res_rec;
   p.meta_rec = pl.meta_rec;
+  p.res_sets = pl.RS;
   // job costs (about the instructions a warp spends): units of 1-, 2-, 4-, 8-bit groups; a meta job
   // job costs, in scheduler cycles of one lane (integer and packed fp32 instructions take two, fp32 one):
   // 1- and 2-bit units (nibble tables, all batch rows), 4- and 8-bit units (magic-number expansion), a meta job
-  p.cost[0] = 60 + 20 * B;
-  p.cost[1] = 100 + 35 * B;
-  p.cost[2] = 285;
-  p.cost[3] = 275;
-  p.cost[4] = 400 + 100 * B;
+  // batch 8, 16: tensor-core units of 32 items (fragment building dominates; mma.sync adds 8 B / 8 per unit)
+  if (B <= 4) {
+    p.cost[0] = 60 + 20 * B;
+    p.cost[1] = 100 + 35 * B;
+    p.cost[2] = 285;
+    p.cost[3] = 275;
+    p.cost[4] = 400 + 100 * B;
+  } else {
+    p.cost[0] = 110 + 4 * B;
+    p.cost[1] = 150 + 4 * B;
+    p.cost[2] = 190 + 4 * B;
+    p.cost[3] = 260 + 4 * B;
+    p.cost[4] = 500;
+  }
   const unsigned long long wl = g_test_wait_ns.load();
   p.wait_ns = wl ? wl : kWaitNs;
   const long long wh = g_test_withhold.load();
   p.withhold = (wh >= 0 && wh < recs) ? int(wh) : -1;
-  auto kern = cc ? vbq_cc_kernel<(B <= 4 ? B : 1)> : vbq_kernel<B>;
+  auto kern = vbq_kernel<B>;
   // Opt in to the dynamic shared memory once per device and size.
   static int opted[64] = {0};
   int dev = 0;
