@@ -390,8 +390,7 @@ __device__ __forceinline__ int owner(const Params& p, int j) {
 //    final y counts it in on the pair counter of its tile index; the second of the pair computes h = silu(gate) * up
 //    for those rows from both final outputs, rounded once to bf16, and resets the counter.
 template <int B, int kThreads>
-__device__ void finish_cta(const Params& p, int L, int H, int* cta_flags, int* epi_tiles, int* epi_count,
-                           unsigned char* scratch) {
+__device__ void finish_cta(const Params& p, int L, int H, int* cta_flags, int* epi_tiles, int* epi_count) {
   const int tid = threadIdx.x, G = p.G, R = p.R;
   if (H <= L) return;
   // Owners of tile t. With at least as many records as CTAs every CTA owns a contiguous, non-empty record range,
@@ -403,82 +402,81 @@ __device__ void finish_cta(const Params& p, int L, int H, int* cta_flags, int* e
     return dense ? owner(p, t * G + G - 1) - first + 1 : G;
   };
   auto kth_owner = [&](int t, int first, int k) -> int { return dense ? first + k : owner(p, t * G + k); };
-  // Sum of all owners' partial slots of tile t into y, in a fixed order. A slot holds [B][R] f32, so four rows of
-  // one batch row are one 16-byte load (item f: batch row f / nq, rows 4 (f % nq) ..). Large tiles: each thread
-  // sums U items over all owners in CTA order, OC owners' loads in flight. Small tiles: the owners are cut into C
-  // consecutive chunks summed by separate threads (OC loads in flight each), and the C chunk sums are added in
-  // chunk order through shared memory.
-  auto reduce_tile = [&](int t) {
+  // Sums of all owners' partial slots of the tiles this CTA reduces (one or two) into y, each element over the
+  // owners in CTA order (so the result does not depend on which CTA reduces). A slot holds [B][R] f32. The
+  // elements of both tiles form one index space, so their loads overlap. Few elements: one element per thread and
+  // step, 16 owners' loads in flight. Many: four rows of one batch row per 16-byte load (item f of a tile: batch
+  // row f / nq, rows 4 (f % nq) ..), U items per thread and step, 8 owners' loads in flight each.
+  auto reduce_tiles = [&](int ta, int tb, int ntiles) {
+    // tile i in {0, 1} (selected by value: an indexed local array would live in local memory)
+    int first0, first1 = 0;
+    const int own0 = tile_owners(ta, first0), own1 = ntiles > 1 ? tile_owners(tb, first1) : 0;
+    const TileOut y0 = tile_out(p, ta), y1 = tile_out(p, ntiles > 1 ? tb : ta);
+    const int omax = max(own0, own1);
+    auto slot_of = [&](bool sec, int o) {
+      const int t = sec ? tb : ta;
+      return p.partial + size_t(kth_owner(t, sec ? first1 : first0, o) + t) * R * B;
+    };
+    const int ne0 = y0.Rt * B, ne = ne0 + (ntiles > 1 ? y1.Rt * B : 0);
+    if (ne <= 2 * kThreads) {
+      constexpr int OC = 16;
+      for (int e2 = tid; e2 < ne; e2 += kThreads) {
+        const bool sec = e2 >= ne0;
+        const int e = e2 - (sec ? ne0 : 0), Rt = sec ? y1.Rt : y0.Rt, own = sec ? own1 : own0;
+        const int b = e / Rt, r = e - b * Rt;
+        float v = 0.f;
+        for (int o0 = 0; o0 < own; o0 += OC) {
+          float part[OC];
+#pragma unroll
+          for (int q = 0; q < OC; ++q) part[q] = o0 + q < own ? __ldcg(slot_of(sec, o0 + q) + size_t(b) * R + r) : 0.f;
+#pragma unroll
+          for (int q = 0; q < OC; ++q)
+            if (o0 + q < own) v += part[q];
+        }
+        (sec ? y1.y : y0.y)[size_t(b) * (sec ? y1.ld : y0.ld) + r] = v;
+      }
+      return;
+    }
     constexpr int U = kThreads >= 512 ? 1 : 2, OC = 8;
-    int first;
-    const int owners = tile_owners(t, first);
-    const TileOut yo = tile_out(p, t);
-    const int nq = (yo.Rt + 3) >> 2, nf = nq * B;
-    auto load = [&](int o, int f) {
-      const int b = f / nq, r = 4 * (f - b * nq);
-      return __ldcg(reinterpret_cast<const float4*>(p.partial + size_t(kth_owner(t, first, o) + t) * R * B +
-                                                    size_t(b) * R + r));
-    };
-    auto store = [&](int f, float4 v) {
-      const int b = f / nq, r = 4 * (f - b * nq);
-      float* yr = yo.y + size_t(b) * yo.ld + r;
-      const float vv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-        if (r + i < yo.Rt) yr[i] = vv[i];
-    };
+    const int nq0 = (y0.Rt + 3) >> 2, nq1 = (y1.Rt + 3) >> 2;
+    const int nf0 = nq0 * B, nf = nf0 + (ntiles > 1 ? nq1 * B : 0);
     auto add4 = [](float4& v, const float4& a) { v.x += a.x; v.y += a.y; v.z += a.z; v.w += a.w; };
-    // owners [o_begin, o_end) summed in order into v, for the item f of this thread
-    auto sum_owners = [&](int f, int o_begin, int o_end, float4& v) {
-      for (int o0 = o_begin; o0 < o_end; o0 += OC) {
-        float4 part[OC];
+    for (int f0 = tid; f0 < nf; f0 += U * kThreads) {
+      float4 v[U];
 #pragma unroll
-        for (int q = 0; q < OC; ++q) part[q] = o0 + q < o_end ? load(o0 + q, f) : make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int u = 0; u < U; ++u) v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int o0 = 0; o0 < omax; o0 += OC) {
+        float4 part[OC][U];
 #pragma unroll
         for (int q = 0; q < OC; ++q)
-          if (o0 + q < o_end) add4(v, part[q]);
+#pragma unroll
+          for (int u = 0; u < U; ++u) {
+            const int f = f0 + u * kThreads;
+            const bool sec = f >= nf0;
+            const int fl = f - (sec ? nf0 : 0), nq = sec ? nq1 : nq0, b = fl / nq, r = 4 * (fl - b * nq);
+            part[q][u] = (f < nf && o0 + q < (sec ? own1 : own0))
+                             ? __ldcg(reinterpret_cast<const float4*>(slot_of(sec, o0 + q) + size_t(b) * R + r))
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+#pragma unroll
+        for (int q = 0; q < OC; ++q)
+#pragma unroll
+          for (int u = 0; u < U; ++u)
+            if (o0 + q < (f0 + u * kThreads >= nf0 ? own1 : own0)) add4(v[u], part[q][u]);
       }
-    };
-    if (2 * nf > kThreads) {
-      for (int f0 = tid; f0 < nf; f0 += U * kThreads) {
-        float4 v[U];
 #pragma unroll
-        for (int u = 0; u < U; ++u) v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int o0 = 0; o0 < owners; o0 += OC) {
-          float4 part[OC][U];
+      for (int u = 0; u < U; ++u) {
+        const int f = f0 + u * kThreads;
+        if (f >= nf) continue;
+        const bool sec = f >= nf0;
+        const int fl = f - (sec ? nf0 : 0), nq = sec ? nq1 : nq0, b = fl / nq, r = 4 * (fl - b * nq);
+        const int Rt = sec ? y1.Rt : y0.Rt;
+        float* yr = (sec ? y1.y : y0.y) + size_t(b) * (sec ? y1.ld : y0.ld) + r;
+        const float vv[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
 #pragma unroll
-          for (int q = 0; q < OC; ++q)
-#pragma unroll
-            for (int u = 0; u < U; ++u) {
-              const int f = f0 + u * kThreads;
-              part[q][u] = (o0 + q < owners && f < nf) ? load(o0 + q, f) : make_float4(0.f, 0.f, 0.f, 0.f);
-            }
-#pragma unroll
-          for (int q = 0; q < OC; ++q)
-            if (o0 + q < owners)
-#pragma unroll
-              for (int u = 0; u < U; ++u) add4(v[u], part[q][u]);
-        }
-#pragma unroll
-        for (int u = 0; u < U; ++u)
-          if (f0 + u * kThreads < nf) store(f0 + u * kThreads, v[u]);
+        for (int i = 0; i < 4; ++i)
+          if (r + i < Rt) yr[i] = vv[i];
       }
-    } else {
-      const int C = max(1, min(kThreads / nf, (owners + OC - 1) / OC)), per = (owners + C - 1) / C;
-      const int c = tid / nf, f = tid - c * nf;
-      float4* chunk = reinterpret_cast<float4*>(scratch);
-      if (c < C) {
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        sum_owners(f, c * per, min(owners, (c + 1) * per), v);
-        chunk[c * nf + f] = v;
-      }
-      __syncthreads();
-      if (tid < nf) {
-        float4 v = chunk[f];
-        for (int k = 1; k < C; ++k) add4(v, chunk[k * nf + f]);
-        store(f, v);
-      }
-      __syncthreads();
     }
   };
 
@@ -502,8 +500,8 @@ __device__ void finish_cta(const Params& p, int L, int H, int* cta_flags, int* e
       }
     }
     __syncthreads();
-    if (cta_flags[0]) reduce_tile(tfirst);
-    if (cta_flags[1]) reduce_tile(tlast);
+    const int ntiles = cta_flags[0] + cta_flags[1];
+    if (ntiles > 0) reduce_tiles(cta_flags[0] ? tfirst : tlast, tlast, ntiles);
     if (tid == 0) {
       if (cta_flags[0]) p.arrive[tfirst] = 0u;
       if (cta_flags[1]) p.arrive[tlast] = 0u;
@@ -935,9 +933,10 @@ __global__ void __launch_bounds__(KCfg<B>::kThreads, 1) vbq_kernel(const __grid_
   auto meta_ptr = [&](int tp, int pos) { return smem + meta0 + (tp * NB + pos) * p.meta_rec; };   // table block
   auto row_ptr = [&](int mp, int pos) { return smem + p.row_off + (mp * NB + pos) * MetaOff(B).row_size; };
   // result set of a batch: alternate sets when there are two, else the one set (and a barrier after each row pass)
-  auto res_addr = [&](int rp, int pos) {
-    return smem_u32(smem + p.res_off + ((p.res_sets > 1 ? rp : 0) * NB + pos) * p.res_rec);
-  };
+  const bool two_sets = B < 8 || p.res_sets > 1;   // one set is planned only for batch 8, 16
+  const uint32_t res0 = smem_u32(smem + p.res_off);
+  const int res_rec = p.res_rec;
+  auto res_addr = [=](int rp, int pos) { return res0 + uint32_t(((two_sets ? rp : 0) * NB + pos) * res_rec); };
 
   // Bulk copies of batch `it` (warp 0, one record per lane, at most NB <= 32): the records (with_rec) and the
   // activation rows (with_x) into their slots. The mbarrier of a slot expects both.
@@ -1242,11 +1241,83 @@ __global__ void __launch_bounds__(KCfg<B>::kThreads, 1) vbq_kernel(const __grid_
 #pragma unroll
     for (int b = 0; b < B; ++b) acc[ww][b] = 0.f;
   int mp = 0, rp = 0;  // meta set (batch index % 3) and result set (batch index % 2) of the current batch
-  while (cur.valid() && !aborted) {
-    nxt = cur;
-    nxt.next();
-    const int mpn = mp == 2 ? 0 : mp + 1;
-    jobs(cur, nxt, rp, mpn);
+  // Row pass of batch bt (row set mp_, result set rp_): this warp's words, records in order. First every record's
+  // item index for the row (independent loads, issued together), then the results added in record order. At a
+  // tile end (tile_end: the next batch is in another tile, or there is none), this CTA's share of the tile goes to
+  // y or to its partial slot.
+  auto row_pass = [&](int t, int nrec, int mp_, int rp_, bool tile_end) {
+    const TileOut to = tile_out(p, t);
+    const int Rt = to.Rt;
+#pragma unroll
+    for (int ww = 0; ww < NWW; ++ww) {
+      const int word = warp + ww * W, r = 32 * word + lane;
+      if (32 * word >= Rt) continue;
+      int item[kMaxNB];
+#pragma unroll
+      for (int pos = 0; pos < kMaxNB; ++pos) {
+        item[pos] = -1;
+        if (pos < nrec && r < Rt) {
+          const unsigned char* rm = row_ptr(mp_, pos);
+          const uint32_t* mk = reinterpret_cast<const uint32_t*>(rm + mo.mk);
+          const uint16_t* pf = reinterpret_cast<const uint16_t*>(rm + mo.pf);
+          const uint32_t wcw = reinterpret_cast<const uint32_t*>(rm + mo.wc)[r >> 4];
+          const int c = int(wcw >> (2 * (r & 15))) & 3;
+          const int it = pf[c * 32 + word] + __popc(mk[c * 32 + word] & ((1u << lane) - 1u));
+          item[pos] = *reinterpret_cast<const int*>(rm + mo.bad) ? -1 : it;   // a bad record adds nothing
+        }
+      }
+#pragma unroll
+      for (int pos = 0; pos < kMaxNB; ++pos)
+        if (item[pos] >= 0) {
+          const uint32_t res = res_addr(rp_, pos) + 4 * (item[pos] * B);
+          if constexpr (B >= 4) {
+#pragma unroll
+            for (int b = 0; b < B; b += 4) {
+              const float4 v = lds128f(res + 4 * b);
+              acc[ww][b] += v.x; acc[ww][b + 1] += v.y; acc[ww][b + 2] += v.z; acc[ww][b + 3] += v.w;
+            }
+          } else {
+#pragma unroll
+            for (int b = 0; b < B; ++b) acc[ww][b] += lds32f(res + 4 * b);
+          }
+        }
+    }
+    if (!tile_end) return;
+    const bool whole = L <= t * G && H >= (t + 1) * G;
+    float* slot = p.partial + size_t(cta + t) * p.R * B;
+#pragma unroll
+    for (int ww = 0; ww < NWW; ++ww) {
+      const int r = 32 * (warp + ww * W) + lane;
+      if (r < Rt) {
+#pragma unroll
+        for (int b = 0; b < B; ++b) {
+          if (whole) to.y[size_t(b) * to.ld + r] = acc[ww][b];
+          else slot[b * p.R + r] = acc[ww][b];
+        }
+      }
+#pragma unroll
+      for (int b = 0; b < B; ++b) acc[ww][b] = 0.f;
+    }
+  };
+
+  // With two result sets, batch n's row pass runs after the warp's jobs of batch n + 1, before the barrier that
+  // ends them: a warp that finishes its units early sums rows instead of waiting. (Batch n + 1's units write the
+  // other result set; the row, result and table sets batch n's row pass reads are next written by batch n + 2's
+  // and n + 3's meta jobs and units, which start after that barrier.) With one set, the row pass follows the
+  // batch's own barrier and a second barrier guards the set.
+  int pt = 0, pn = 0, pmp = 0, prp = 0;   // the previous batch: tile, records, row and result sets
+  bool have_prev = false;
+  while (!aborted) {
+    const bool live = cur.valid();   // one more round after the last batch, for its row pass
+    int mpn = 0;
+    if (live) {
+      nxt = cur;
+      nxt.next();
+      mpn = mp == 2 ? 0 : mp + 1;
+      jobs(cur, nxt, rp, mpn);
+    }
+    if (two_sets && have_prev) row_pass(pt, pn, pmp, prp, !live || pt != cur.t);
+    if (!live) break;
     aborted = __syncthreads_or(cta_abort != 0) != 0;
     if (aborted) break;
     // refill the slots of batch n with batch n + S (their records and activation rows)
@@ -1262,68 +1333,19 @@ __global__ void __launch_bounds__(KCfg<B>::kThreads, 1) vbq_kernel(const __grid_
       }
       iss.next();
     }
-    // row pass of batch n: this warp's words, records in order. First every record's item index for the row
-    // (independent loads, issued together), then the results added in record order.
-    const TileOut to = tile_out(p, cur.t);
-    const int Rt = to.Rt;
-    const int nrec = cur.re - cur.rb;
-#pragma unroll
-    for (int ww = 0; ww < NWW; ++ww) {
-      const int word = warp + ww * W, r = 32 * word + lane;
-      if (32 * word >= Rt) continue;
-      int item[kMaxNB];
-#pragma unroll
-      for (int pos = 0; pos < kMaxNB; ++pos) {
-        item[pos] = -1;
-        if (pos < nrec && r < Rt) {
-          const unsigned char* rm = row_ptr(mp, pos);
-          const uint32_t* mk = reinterpret_cast<const uint32_t*>(rm + mo.mk);
-          const uint16_t* pf = reinterpret_cast<const uint16_t*>(rm + mo.pf);
-          const uint32_t wcw = reinterpret_cast<const uint32_t*>(rm + mo.wc)[r >> 4];
-          const int c = int(wcw >> (2 * (r & 15))) & 3;
-          const int it = pf[c * 32 + word] + __popc(mk[c * 32 + word] & ((1u << lane) - 1u));
-          item[pos] = *reinterpret_cast<const int*>(rm + mo.bad) ? -1 : it;   // a bad record adds nothing
-        }
-      }
-#pragma unroll
-      for (int pos = 0; pos < kMaxNB; ++pos)
-        if (item[pos] >= 0) {
-          const uint32_t res = res_addr(rp, pos) + 4 * (item[pos] * B);
-          if constexpr (B >= 4) {
-#pragma unroll
-            for (int b = 0; b < B; b += 4) {
-              const float4 v = lds128f(res + 4 * b);
-              acc[ww][b] += v.x; acc[ww][b + 1] += v.y; acc[ww][b + 2] += v.z; acc[ww][b + 3] += v.w;
-            }
-          } else {
-#pragma unroll
-            for (int b = 0; b < B; ++b) acc[ww][b] += lds32f(res + 4 * b);
-          }
-        }
-    }
-    // tile end: this CTA's share of tile cur.t is complete
-    if (!nxt.valid() || nxt.t != cur.t) {
-      const int t = cur.t;
-      const bool whole = L <= t * G && H >= (t + 1) * G;
-      float* slot = p.partial + size_t(cta + t) * p.R * B;
-#pragma unroll
-      for (int ww = 0; ww < NWW; ++ww) {
-        const int r = 32 * (warp + ww * W) + lane;
-        if (r < Rt) {
-#pragma unroll
-          for (int b = 0; b < B; ++b) {
-            if (whole) to.y[size_t(b) * to.ld + r] = acc[ww][b];
-            else slot[b * p.R + r] = acc[ww][b];
-          }
-        }
-#pragma unroll
-        for (int b = 0; b < B; ++b) acc[ww][b] = 0.f;
-      }
+    if (two_sets) {
+      pt = cur.t;
+      pn = cur.re - cur.rb;
+      pmp = mp;
+      prp = rp;
+      have_prev = true;
+    } else {
+      row_pass(cur.t, cur.re - cur.rb, mp, rp, !nxt.valid() || nxt.t != cur.t);
+      __syncthreads();   // the next batch's units overwrite the one result set
     }
     cur = nxt;
     mp = mpn;
     rp ^= 1;
-    if (p.res_sets == 1) __syncthreads();   // the next batch's units overwrite the one result set
   }
   if (aborted) {
     // wait (bounded) for the copies still in flight before the CTA exits; publish nothing. Only the last use of
@@ -1334,7 +1356,7 @@ __global__ void __launch_bounds__(KCfg<B>::kThreads, 1) vbq_kernel(const __grid_
     }
     return;
   }
-  finish_cta<B, C::kThreads>(p, L, H, cta_flags, epi_tiles, &epi_count, smem);
+  finish_cta<B, C::kThreads>(p, L, H, cta_flags, epi_tiles, &epi_count);
 }
 
 // ------------------------------------------------------------------------------------------ launch plan
@@ -1428,7 +1450,7 @@ inline bool make_plan_b(const Problem& pr, int sms, Plan& pl) {
   // two result sets let the next batch's units start before every warp has finished this batch's row pass; one
   // set (with a barrier after each row pass) is the last resort for large records at batch 16
   pl.NB = 0;
-  for (int RS = 2; RS >= 1 && pl.NB == 0; --RS)
+  for (int RS = 2; RS >= (B < 8 ? 2 : 1) && pl.NB == 0; --RS)
     for (int NB = nb_want; NB >= 1 && pl.NB == 0; --NB)
       for (int S = 3; S >= 2; --S)
         if (need(NB, S, RS) <= kSmemBudget) {
