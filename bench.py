@@ -9,6 +9,11 @@ the 126 MB L2, so every step streams them from HBM. One step is one token: 129 l
 fused, o, gate/up fused with the SwiGLU epilogue feeding down's input, down; then the head).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--batch B] [--layers L] [--impl vbq|reference]
+                    [--workload step|recipe|cfg4|pad512]
+
+Other workloads: ``recipe`` is the same step under the paper's fixed deployment recipe (one width per
+projection); ``cfg4`` times each 9B-shaped linear alone at batch 1..16; ``pad512`` compares an 8960-wide MLP
+packed as is with its zero-padded 9216-wide form.
 
 Under torchrun (N > 1) every rank runs an independent replica on its own GPU. The path has no cross-GPU
 exchange. Time is the max over ranks, and the value is the bytes of all ranks divided by that time.
@@ -638,6 +643,116 @@ def run_cfg4(args):
         dist.destroy_process_group()
 
 
+def run_pad512(args):
+    """The 8960-wide MLP (gate/up 8960x1536 with the fused SwiGLU epilogue, then down 1536x8960 on h), packed as
+    is and zero-padded to an intermediate width of 9216 (a multiple of 512), at batch 1 and 16 (or --batch). Each
+    form is timed like cfg4: M distinct device copies of its three blobs, together at least 4x the L2, run
+    round-robin in one CUDA graph; time per MLP = replay time / M, the best of three replays. GB/s counts the
+    blobs, x, both y, h and the down output of the logical (unpadded) problem for both forms, so the padded form
+    pays for its extra bytes."""
+    import torch
+    from decode_vbq_gemv_b200 import vbq
+    world, rank, local = dist_setup()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    peak, peak_kind = peaks()
+    stream = torch.cuda.Stream(dev)
+    batches = (1, 16) if args.batch == 1 else (args.batch,)
+    gm, um, dm = S.cfg7_mlp()
+    I, H, I_pad = gm.N, gm.K, 9216
+    R = args.tile_rows if args.tile_rows > 0 else vbq.suggest_tile_rows(I, H, sms)
+    Rd = args.tile_rows if args.tile_rows > 0 else vbq.suggest_tile_rows(H, I, sms)
+    results, n_launches, t_setup = {}, 0, time.perf_counter()
+    sampler = ClockSampler(local)
+    sampler.start()
+    for pad in (False, True):
+        if pad:
+            packed = [vbq.vbq_pack_padded(m.N, m.K, R, m.widths, m.scales, m.codes, I_pad, H) for m in (gm, um)]
+            packed.append(vbq.vbq_pack_padded(dm.N, dm.K, Rd, dm.widths, dm.scales, dm.codes, H, I_pad))
+        else:
+            packed = [vbq.vbq_pack(m.N, m.K, R, m.widths, m.scales, m.codes) for m in (gm, um)]
+            packed.append(vbq.vbq_pack(dm.N, dm.K, Rd, dm.widths, dm.scales, dm.codes))
+        blobs, descs = [b for b, _ in packed], [d for _, d in packed]
+        strides = [(b.size + 255) // 256 * 256 for b in blobs]
+        unit = sum(strides)
+        M = max(2, int(np.ceil(4 * L2_BYTES / unit)))
+        copies = torch.empty(M * unit, dtype=torch.uint8, device=dev)
+        offs = [0, strides[0], strides[0] + strides[1]]
+        for i, b in enumerate(blobs):
+            src = torch.from_numpy(b).to(dev)
+            for c in range(M):
+                copies[c * unit + offs[i]:c * unit + offs[i] + b.size].copy_(src)
+        Np = descs[0].N
+        for B in batches:
+            ws_gu = torch.zeros(vbq.vbq_workspace_size_swiglu(descs[0], descs[1], B), dtype=torch.uint8, device=dev)
+            ws_d = torch.zeros(max(vbq.vbq_workspace_size(descs[2], B), 16), dtype=torch.uint8, device=dev)
+            x = torch.from_numpy(S.make_x(7, "gate", B, H).astype(np.int16)).view(torch.bfloat16).to(dev)
+            yg = torch.empty((B, Np), dtype=torch.float32, device=dev)
+            yu = torch.empty((B, Np), dtype=torch.float32, device=dev)
+            h = torch.empty((B, Np), dtype=torch.bfloat16, device=dev)
+            yd = torch.empty((B, H), dtype=torch.float32, device=dev)
+            flags = 0 if args.no_overlap else vbq.VBQ_LAUNCH_OVERLAP
+
+            def blob(c, i):
+                return copies[c * unit + offs[i]:c * unit + offs[i] + blobs[i].size]
+
+            with torch.cuda.stream(stream):
+                def run_all():
+                    for c in range(M):
+                        vbq.vbq_gemm_swiglu(descs[0], descs[1], blob(c, 0), blob(c, 1), x, B, yg, yu, h, ws_gu,
+                                            flags, stream)
+                        vbq.vbq_gemm_skinny_ex(descs[2], blob(c, 2), h, B, yd, ws_d, flags, stream)
+                run_all()
+                torch.cuda.synchronize()
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=stream):
+                    run_all()
+                for _ in range(args.warmup):
+                    g.replay()
+                torch.cuda.synchronize()
+                best = None
+                for _ in range(3):
+                    e0 = torch.cuda.Event(enable_timing=True)
+                    e1 = torch.cuda.Event(enable_timing=True)
+                    e0.record(stream)
+                    g.replay()
+                    e1.record(stream)
+                    torch.cuda.synchronize()
+                    t = e0.elapsed_time(e1) / M
+                    best = t if best is None else min(best, t)
+                n_launches += 2 * M * (args.warmup + 3)
+            logical_bytes = sum(vbq.vbq_packed_size(m.N, m.K, r, m.widths) for m, r in ((gm, R), (um, R), (dm, Rd)))
+            nbytes = logical_bytes + B * H * 2 + 2 * B * I * 4 + B * I * 2 + B * I * 2 + B * H * 4
+            gbps = nbytes / (best / 1e3) / 1e9
+            results[f"{'padded to 9216' if pad else 'unpadded 8960'} B={B}"] = {
+                "us": best * 1e3, "GBps": gbps, "frac": gbps / peak, "blob_bytes": int(sum(b.size for b in blobs)),
+                "copies": M, "tile_rows": [R, Rd]}
+            del g, ws_gu, ws_d
+        del copies
+        torch.cuda.empty_cache()
+    clocks = sampler.stop()
+    t_setup = time.perf_counter() - t_setup
+    value = results["unpadded 8960 B=1"]["GBps"] if 1 in batches else next(iter(results.values()))["GBps"]
+    if rank == 0:
+        line = {"metric": METRIC, "value": value * world, "unit": UNIT, "n_gpus": world, "steps": 3,
+                "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "fp32", "data": "synthetic",
+                "config": {"workload": "8960-wide MLP (gate/up 8960x1536 + SwiGLU, down 1536x8960), unpadded and "
+                                       "zero-padded to 9216, >= 4x L2 of distinct copies in rotation",
+                           "batch": list(batches), "l2": "inputs larger than L2: copies in rotation",
+                           "parallelism": f"replicas x{world}"},
+                "roofline": {"bound": "hbm", "achieved": value, "peak": peak, "unit": "GB/s", "frac": value / peak,
+                             "traffic": None, "peak_kind": peak_kind, "kernel": "vbq_kernel<B>"},
+                "pad512": results, "gpu_launches": n_launches, "clocks": clocks, "setup_s": round(t_setup, 1),
+                "e2e": None, "cpu_baseline": None}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        barrier(world)
+        dist.destroy_process_group()
+
+
 def make_parser() -> argparse.ArgumentParser:
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -645,10 +760,11 @@ def make_parser() -> argparse.ArgumentParser:
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--batch", type=int, default=1, choices=(1, 2, 4, 8, 16))
     ap.add_argument("--impl", default="vbq", choices=("vbq", "reference"))
-    ap.add_argument("--workload", default="step", choices=("step", "recipe", "cfg4"),
+    ap.add_argument("--workload", default="step", choices=("step", "recipe", "cfg4", "pad512"),
                     help="step: the 9B-shaped decode step at the paper's allocation (default); recipe: the same step "
                          "under the fixed deployment recipe; cfg4: each 9B-shaped linear alone at batch 1..16, "
-                         "rotating copies larger than L2")
+                         "rotating copies larger than L2; pad512: an 8960-wide MLP unpadded and zero-padded to "
+                         "9216")
     ap.add_argument("--layers", type=int, default=32, help="decoder layers in the step (1..32)")
     ap.add_argument("--no-head", action="store_true", help="leave the LM head out of the step")
     ap.add_argument("--no-fp16-ref", action="store_true",
@@ -675,6 +791,8 @@ def main():
         run_reference(args)
     elif args.workload == "cfg4":
         run_cfg4(args)
+    elif args.workload == "pad512":
+        run_pad512(args)
     else:
         run_vbq(args)
 

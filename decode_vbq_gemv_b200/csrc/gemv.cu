@@ -577,18 +577,21 @@ constexpr int kMaxSets = 4;      // batches in flight
 constexpr int kDirCache = 512;   // directory entries cached in shared memory
 
 // Per-record metadata, written by the record's meta job one batch before its units run, in two blocks.
-// Table block (256-byte aligned; read only by the units, so two sets serve alternate batches):
+// Table block (256-byte aligned; read only by the units, so two sets serve alternate batches). The tables exist
+// for B <= 4 only, and each is built only when the record has rows of the widths that read it:
 //  t1 [B][16][16] f32: 1-bit nibble tables; entry n of position p is the sum of x[4p + i] over the set bits i of n
 //  t2 [B][32][16] f32: 2-bit nibble tables; entry n of position p is (n & 3) x[2p] + (n >> 2) x[2p + 1]
 //  xt [2][B][64] f32:  x, and x * 2^-shift for the magic-number expansion of 4-bit codes
 //  sg [B] f32:         group sums of x
 //  fl [16] i32:        bad, scales offset, bucket counts n[4], bucket code offsets c[4], bucket item starts i[4]
-// Row block (read by the row pass, which can still run while the next batch's units write: three sets):
+// Row block (read by the row pass, which can run while the next batch's units write: three sets):
 //  mk [4][32] u32:     width masks per 32-row word;  pf [4][32] u16: item index of the word's first row per width
-//  wc [64] u32:        the record's width-code words;  bad (i32)
+//  wc [64] u32:        the record's width-code words
+//  kind (i32):         0 mixed widths; 1 bad record (adds nothing); 2 + c every row has width code c, so the item
+//                      index of a row is the row itself and the row pass reads no masks
 struct MetaOff {
   int t1, t2, xt, sg, fl, size;      // table block
-  int mk, pf, wc, bad, row_size;     // row block
+  int mk, pf, wc, kind, row_size;    // row block
   __host__ __device__ explicit MetaOff(int B) {
     const int tb = B >= 8 ? 0 : B;   // the tensor-core path (batch 8, 16) needs no activation tables
     t1 = 0;
@@ -600,7 +603,7 @@ struct MetaOff {
     mk = 0;
     pf = 512;
     wc = 768;
-    bad = 1024;
+    kind = 1024;
     row_size = 1040;
   }
 };
@@ -1066,21 +1069,24 @@ __global__ void __launch_bounds__(KCfg<B>::kThreads, 1) vbq_kernel(const __grid_
         const float x1 = __uint_as_float(uint32_t(xg[b * 64 + 32 + lane]) << 16);
         xv[b * 64 + lane] = x0;
         xv[b * 64 + 32 + lane] = x1;
-        xv[(B + b) * 64 + lane] = x0 * s4a;
-        xv[(B + b) * 64 + 32 + lane] = x1 * s4b;
+        if (n2 > 0) {   // the 4-bit copy: only for a record with 4-bit rows
+          xv[(B + b) * 64 + lane] = x0 * s4a;
+          xv[(B + b) * 64 + 32 + lane] = x1 * s4b;
+        }
         float sg = x0 + x1;
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) sg += __shfl_xor_sync(0xFFFFFFFFu, sg, off);
         if (lane == 0) sgv[b] = sg;
       }
       __syncwarp();
-      // nibble tables. 1-bit: lane = (position p, half h) builds entries 8h .. 8h + 7 of position p.
-      // 2-bit: lane = position p (codes 2p, 2p + 1) builds its 16 entries.
+      // nibble tables, each only for a record with rows of its width. 1-bit: lane = (position p, half h) builds
+      // entries 8h .. 8h + 7 of position p. 2-bit: lane = position p (codes 2p, 2p + 1) builds its 16 entries.
       const uint32_t xa = smem_u32(mb + mo.xt);
       const int pp = lane >> 1, hh = lane & 1;
       const uint32_t t1a = smem_u32(mb + mo.t1) + 64 * pp + 32 * hh, t2a = smem_u32(mb + mo.t2) + 64 * lane;
 #pragma unroll
       for (int b = 0; b < B; ++b) {
+        if (n0 > 0) {
         const float4 q = lds128f(xa + 256 * b + 16 * pp);
         const float base = hh ? q.w : 0.f;
         const float e1 = base + q.x, e2 = base + q.y, e3 = e1 + q.y;
@@ -1089,6 +1095,8 @@ __global__ void __launch_bounds__(KCfg<B>::kThreads, 1) vbq_kernel(const __grid_
                                  __float_as_uint(e3 + q.z)};
         sts128(t1a + 1024 * b, lo4);
         sts128(t1a + 1024 * b + 16, hi4);
+        }
+        if (n1 == 0) continue;
         const uint2 xp = lds64(xa + 256 * b + 8 * lane);
         const float xa0 = __uint_as_float(xp.x), xb0 = __uint_as_float(xp.y);
 #pragma unroll
@@ -1112,7 +1120,9 @@ __global__ void __launch_bounds__(KCfg<B>::kThreads, 1) vbq_kernel(const __grid_
     }
     if (lane == 0) {
       fl[0] = ok ? 0 : 1;
-      *reinterpret_cast<int*>(rb_ + mo.bad) = ok ? 0 : 1;
+      // 1: bad record (adds nothing); 2 + c: every row has width code c (item index = row); 0: mixed widths
+      const int uni = n0 == Rt ? 0 : n1 == Rt ? 1 : n2 == Rt ? 2 : n3 == Rt ? 3 : -1;
+      *reinterpret_cast<int*>(rb_ + mo.kind) = !ok ? 1 : uni >= 0 ? 2 + uni : 0;
     }
   };
 
@@ -1258,12 +1268,17 @@ __global__ void __launch_bounds__(KCfg<B>::kThreads, 1) vbq_kernel(const __grid_
         item[pos] = -1;
         if (pos < nrec && r < Rt) {
           const unsigned char* rm = row_ptr(mp_, pos);
-          const uint32_t* mk = reinterpret_cast<const uint32_t*>(rm + mo.mk);
-          const uint16_t* pf = reinterpret_cast<const uint16_t*>(rm + mo.pf);
-          const uint32_t wcw = reinterpret_cast<const uint32_t*>(rm + mo.wc)[r >> 4];
-          const int c = int(wcw >> (2 * (r & 15))) & 3;
-          const int it = pf[c * 32 + word] + __popc(mk[c * 32 + word] & ((1u << lane) - 1u));
-          item[pos] = *reinterpret_cast<const int*>(rm + mo.bad) ? -1 : it;   // a bad record adds nothing
+          const int kd = *reinterpret_cast<const int*>(rm + mo.kind);
+          if (kd >= 2) {   // one width: the items are the rows
+            item[pos] = r;
+          } else {
+            const uint32_t* mk = reinterpret_cast<const uint32_t*>(rm + mo.mk);
+            const uint16_t* pf = reinterpret_cast<const uint16_t*>(rm + mo.pf);
+            const uint32_t wcw = reinterpret_cast<const uint32_t*>(rm + mo.wc)[r >> 4];
+            const int c = int(wcw >> (2 * (r & 15))) & 3;
+            const int it = pf[c * 32 + word] + __popc(mk[c * 32 + word] & ((1u << lane) - 1u));
+            item[pos] = kd ? -1 : it;   // a bad record adds nothing
+          }
         }
       }
 #pragma unroll

@@ -300,6 +300,54 @@ int vbq_pack(int64_t N, int64_t K, int64_t R, const uint8_t* widths, const uint1
   return vbq_pack_ex(N, K, R, widths, scales, codes, 0u, out, out_cap, out_desc);
 }
 
+namespace {
+// The logical arrays of an N x K matrix embedded in an N_pad x K_pad one: rows N.. and columns K.. are 1-bit
+// groups with scale +0 (every weight exactly 0) and code 0.
+struct Padded {
+  std::vector<uint8_t> widths, codes;
+  std::vector<uint16_t> scales;
+};
+int pad_status(int64_t N, int64_t K, int64_t N_pad, int64_t K_pad) {
+  if (N_pad < N || K_pad < K || K_pad % 64 != 0 || N_pad < 1) return VBQ_ERR_SHAPE;
+  if (N_pad > (int64_t(1) << 31) || K_pad > (int64_t(1) << 31)) return VBQ_ERR_SHAPE;
+  return VBQ_OK;
+}
+void pad_logical(int64_t N, int64_t K, const uint8_t* widths, const uint16_t* scales, const uint8_t* codes,
+                 int64_t N_pad, int64_t K_pad, Padded& out) {
+  const int64_t G = K / 64, Gp = K_pad / 64;
+  out.widths.assign(size_t(N_pad * Gp), uint8_t(1));
+  if (scales) out.scales.assign(size_t(N_pad * Gp), uint16_t(0));
+  if (codes) out.codes.assign(size_t(N_pad * K_pad), uint8_t(0));
+  for (int64_t r = 0; r < N; ++r) {
+    std::memcpy(&out.widths[size_t(r * Gp)], widths + r * G, size_t(G));
+    if (scales) std::memcpy(&out.scales[size_t(r * Gp)], scales + r * G, size_t(G) * 2);
+    if (codes) std::memcpy(&out.codes[size_t(r * K_pad)], codes + r * K, size_t(K));
+  }
+}
+}  // namespace
+
+int vbq_packed_size_padded(int64_t N, int64_t K, int64_t R, const uint8_t* widths, int64_t N_pad, int64_t K_pad,
+                           uint64_t* out_bytes) {
+  if (!widths || !out_bytes) return VBQ_ERR_NULL;
+  if (int st = shape_status(N, K, R)) return st;
+  if (int st = pad_status(N, K, N_pad, K_pad)) return st;
+  Padded pd;
+  pad_logical(N, K, widths, nullptr, nullptr, N_pad, K_pad, pd);
+  return vbq_packed_size(N_pad, K_pad, R, pd.widths.data(), out_bytes);
+}
+
+int vbq_pack_padded(int64_t N, int64_t K, int64_t R, const uint8_t* widths, const uint16_t* scales,
+                    const uint8_t* codes, int64_t N_pad, int64_t K_pad, unsigned format_flags, void* out,
+                    uint64_t out_cap, vbq_desc* out_desc) {
+  if (!widths || !scales || !codes || !out) return VBQ_ERR_NULL;
+  if (int st = shape_status(N, K, R)) return st;
+  if (int st = pad_status(N, K, N_pad, K_pad)) return st;
+  Padded pd;
+  pad_logical(N, K, widths, scales, codes, N_pad, K_pad, pd);
+  return vbq_pack_ex(N_pad, K_pad, R, pd.widths.data(), pd.scales.data(), pd.codes.data(), format_flags, out,
+                     out_cap, out_desc);
+}
+
 int vbq_describe(const void* blob_host, uint64_t blob_bytes, vbq_desc* out_desc) {
   if (!blob_host || !out_desc) return VBQ_ERR_NULL;
   const uint8_t* b = static_cast<const uint8_t*>(blob_host);

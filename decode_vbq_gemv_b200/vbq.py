@@ -78,6 +78,8 @@ def lib() -> ctypes.CDLL:
             "vbq_pack": (i32, [i64, i64, i64, vp, vp, vp, vp, u64, dp]),
             "vbq_pack_ex": (i32, [i64, i64, i64, vp, vp, vp, ctypes.c_uint, vp, u64, dp]),
             "vbq_quantize": (i32, [i64, i64, vp, vp, ctypes.c_uint, vp, vp]),
+            "vbq_packed_size_padded": (i32, [i64, i64, i64, vp, i64, i64, ctypes.POINTER(u64)]),
+            "vbq_pack_padded": (i32, [i64, i64, i64, vp, vp, vp, i64, i64, ctypes.c_uint, vp, u64, dp]),
             "vbq_describe": (i32, [vp, u64, dp]),
             "vbq_unpack": (i32, [vp, u64, vp, vp, vp]),
             "vbq_workspace_size": (i32, [dp, i32, ctypes.POINTER(u64)]),
@@ -163,6 +165,31 @@ def vbq_pack(N: int, K: int, R: int, widths, scales, codes, format_flags: int = 
     """Packs a logical matrix (vbq_pack_ex). Returns (blob as uint8 numpy array, vbq_desc)."""
     st, blob, d = vbq_pack_status(N, K, R, widths, scales, codes, format_flags=format_flags)
     _check(st, "vbq_pack")
+    return blob, d
+
+
+def vbq_pack_padded_status(N, K, R, widths, scales, codes, N_pad, K_pad, format_flags: int = 0):
+    """Returns (status, blob[uint8] or None, vbq_desc) of the N x K matrix packed as N_pad x K_pad with zero
+    weights in the added rows and columns (vbq_pack_padded)."""
+    w = np.ascontiguousarray(widths, np.uint8)
+    s = np.ascontiguousarray(scales, np.uint16)
+    c = np.ascontiguousarray(codes, np.uint8)
+    d = vbq_desc()
+    out = ctypes.c_uint64()
+    st = lib().vbq_packed_size_padded(N, K, R, _np_ptr(w), N_pad, K_pad, ctypes.byref(out))
+    if st != VBQ_OK:
+        return st, None, d
+    cap = int(out.value)
+    blob = np.zeros(max(cap, 1), np.uint8)
+    st = lib().vbq_pack_padded(N, K, R, _np_ptr(w), _np_ptr(s), _np_ptr(c), N_pad, K_pad, format_flags,
+                               _np_ptr(blob), cap, ctypes.byref(d))
+    return st, (blob[: d.total_bytes] if st == VBQ_OK else None), d
+
+
+def vbq_pack_padded(N: int, K: int, R: int, widths, scales, codes, N_pad: int, K_pad: int, format_flags: int = 0):
+    """Packs with zero padding to N_pad x K_pad (vbq_pack_padded). Returns (blob, vbq_desc)."""
+    st, blob, d = vbq_pack_padded_status(N, K, R, widths, scales, codes, N_pad, K_pad, format_flags)
+    _check(st, "vbq_pack_padded")
     return blob, d
 
 

@@ -100,6 +100,19 @@ int vbq_pack(int64_t N, int64_t K, int64_t R, const uint8_t* widths, const uint1
 int vbq_pack_ex(int64_t N, int64_t K, int64_t R, const uint8_t* widths, const uint16_t* scales,
                 const uint8_t* codes, unsigned format_flags, void* out, uint64_t out_cap, vbq_desc* out_desc);
 
+/* Zero-padded packing (VBQ paper, section 6, "Granularity is deployment-friendly": MLP intermediate widths are
+ * zero-padded to a multiple of 512, which changes nothing because silu(0) * 0 = 0). The N x K logical matrix is
+ * packed as an N_pad x K_pad one whose extra rows and columns are 1-bit groups with scale +0 and code 0, so every
+ * added weight is exactly 0: padded gate/up rows give h = silu(0) * 0 = 0, and padded down-projection columns
+ * multiply those zeros. Nothing in this library's kernels needs K % 512; the padded form is offered for blobs
+ * shared with kernels that do, and its cost is measured against the unpadded one.
+ * Requires N_pad >= N, K_pad >= K, K_pad % 64 == 0 (SHAPE otherwise). Other errors: as vbq_pack_ex. Pure. */
+int vbq_packed_size_padded(int64_t N, int64_t K, int64_t R, const uint8_t* widths, int64_t N_pad, int64_t K_pad,
+                           uint64_t* out_bytes);
+int vbq_pack_padded(int64_t N, int64_t K, int64_t R, const uint8_t* widths, const uint16_t* scales,
+                    const uint8_t* codes, int64_t N_pad, int64_t K_pad, unsigned format_flags, void* out,
+                    uint64_t out_cap, vbq_desc* out_desc);
+
 /* Quantize float32 weights w[N*K] (row-major) to the logical arrays for given widths[N*G] (VBQ paper,
  * section 3.1), group by group (64 weights):
  *  - width 1: scale s = 2 * mean|w| (the grid points +-s/2 are +-mean|w|: sign times the mean magnitude), the

@@ -303,3 +303,39 @@ def test_packed_size_refuses_blobs_the_directory_cannot_address():
     st = L.vbq_packed_size(ctypes.c_int64(32768), ctypes.c_int64(64 * G), ctypes.c_int64(1024),
                            half.ctypes.data_as(ctypes.POINTER(ctypes.c_uint8)), ctypes.byref(out))
     assert st == 0 and out.value > 32 << 30
+
+
+def pad_numpy(w, s, c, N_pad, K_pad):
+    """Zero padding written independently of the library: 1-bit groups, scale +0, code 0."""
+    N, G = w.shape
+    K = c.shape[1]
+    wp = np.ones((N_pad, K_pad // 64), np.uint8)
+    sp = np.zeros((N_pad, K_pad // 64), np.uint16)
+    cp = np.zeros((N_pad, K_pad), np.uint8)
+    wp[:N, :G], sp[:N, :G], cp[:N, :K] = w, s, c
+    return wp, sp, cp
+
+
+@pytest.mark.parametrize("N,K,N_pad,K_pad,R", [(100, 192, 512, 512, 64), (1030, 256, 1536, 256, 512),
+                                                (64, 448, 64, 512, 16), (7, 64, 7, 64, 16)])
+def test_padded_pack_matches_oracle_pack_of_padded_arrays(N, K, N_pad, K_pad, R):
+    """vbq_pack_padded equals the oracle's pack of the logical arrays padded with zero weights, and unpacks to
+    them; the added weights dequantize to exactly 0 (VBQ paper, section 6, zero padding to a multiple of 512)."""
+    w, s, c = logical(N + K + N_pad, N, K)
+    for flags in (0, O.FLAG_GRID_SYMMETRIC):
+        if flags:
+            c = np.minimum(c, (1 << w.repeat(64, axis=1)) - 2 + (w.repeat(64, axis=1) == 1)).astype(np.uint8)
+        blob, d = vbq.vbq_pack_padded(N, K, R, w, s, c, N_pad, K_pad, format_flags=flags)
+        wp, sp, cp = pad_numpy(w, s, c, N_pad, K_pad)
+        assert np.array_equal(blob, O.pack(N_pad, K_pad, R, wp, sp, cp, flags=flags))
+        assert (d.N, d.K, d.flags) == (N_pad, K_pad, flags)
+        assert vbq.lib().vbq_packed_size_padded is not None
+        wq = O.dequant(wp, sp, cp, flags)
+        assert not wq[N:, :].any() and not wq[:, K:].any()
+
+
+def test_padded_pack_refuses_shrinking_or_unaligned_padding():
+    w, s, c = logical(3, 10, 128)
+    for N_pad, K_pad in ((9, 128), (10, 64), (10, 200), (0, 128)):
+        st, blob, _ = vbq.vbq_pack_padded_status(10, 128, 16, w, s, c, N_pad, K_pad)
+        assert st == vbq.VBQ_ERR_SHAPE and blob is None

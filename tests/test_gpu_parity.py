@@ -553,3 +553,42 @@ def test_decode_step_in_the_bench_launch_configuration():
         got = yd.cpu().numpy().astype(np.float64)[0, rows]
         bad = np.abs(got - y_ref) > 1e-3 * (A + E) + 1e-6 + E
         assert not bad.any(), f"{what} (down): {int(bad.sum())} rows out of bar; first row {rows[bad][0]}"
+
+
+@pytest.mark.parametrize("B", [1, 4, 16])
+def test_zero_padded_mlp_matches_unpadded_and_oracle(B):
+    """The 8960-wide MLP (gate/up 8960x1536, down 1536x8960) packed as is and zero-padded to 9216 (a multiple of
+    512; VBQ paper, section 6, "Granularity is deployment-friendly"): in both forms gate/up with the fused SwiGLU
+    epilogue, then down on h. h against the oracle within its bar, the padded h exactly 0 past row 8960, and the
+    down output against the oracle's fp64 down projection of the oracle's h within the propagated bar."""
+    gm, um, dm = S.cfg7_mlp()
+    I, H, I_pad = gm.N, gm.K, 9216
+    R = vbq.suggest_tile_rows(I, H, 148)
+    x = S.make_x(7, "gate", B, H)
+    g_ref, bg = O.matvec(gm.widths, gm.scales, gm.codes, x, NTH)
+    u_ref, bu = O.matvec(um.widths, um.scales, um.codes, x, NTH)
+    h_ref, bar_h = O.swiglu(g_ref, u_ref), O.swiglu_bound(g_ref, u_ref, bg, bu)
+    W = O.dequant(dm.widths, dm.scales, dm.codes)
+    y_ref, A, E = h_ref @ W.T, np.abs(h_ref) @ np.abs(W).T, bar_h @ np.abs(W).T
+    for pad in (False, True):
+        if pad:
+            pk = [vbq.vbq_pack_padded(m.N, m.K, R, m.widths, m.scales, m.codes, I_pad, H)[0] for m in (gm, um)]
+            pd = vbq.vbq_pack_padded(dm.N, dm.K, 256, dm.widths, dm.scales, dm.codes, H, I_pad)[0]
+        else:
+            pk = [vbq.vbq_pack(m.N, m.K, R, m.widths, m.scales, m.codes)[0] for m in (gm, um)]
+            pd = vbq.vbq_pack(dm.N, dm.K, 256, dm.widths, dm.scales, dm.codes)[0]
+        fused = vbq.FusedMatrices([vbq.DeviceMatrix(b, dev(), max_batch=B) for b in pk], max_batch=B)
+        down = vbq.DeviceMatrix(pd, dev(), max_batch=B)
+        _, _, h = fused.swiglu(to_dev_x(x))
+        y = down.matmul(h)
+        torch_sync()
+        assert fused_status(fused, B) == 0
+        hh = bf16_to_f64(h)
+        what = f"{'padded' if pad else 'unpadded'} MLP B={B}"
+        assert hh.shape == (B, I_pad if pad else I)
+        if pad:
+            assert not hh[:, I:].any(), f"{what}: padded rows of h are not 0"
+        check_swiglu(hh[:, :I], g_ref, u_ref, bg, bu, what + " (h)")
+        got = y.cpu().numpy().astype(np.float64)
+        bad = np.abs(got - y_ref) > 1e-3 * (A + E) + 1e-6 + E
+        assert not bad.any(), f"{what} (down): {int(bad.sum())} outputs out of bar"

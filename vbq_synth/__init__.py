@@ -190,3 +190,14 @@ def cfg6_recipe_layer(layer: int):
 def cfg6_recipe_head(N: int = 32000, K: int = 4096):
     """LM head 4096 -> 32000 under the recipe's frequency tiers (mean 1.18 bits)."""
     return make_matrix(6, "head", N, K, widths=widths_head_tiered(N, K // 64))
+
+
+MLP8960 = {"hidden": 1536, "inter": 8960}   # an MLP whose intermediate width is not a multiple of 512
+
+
+def cfg7_mlp(hidden: int = MLP8960["hidden"], inter: int = MLP8960["inter"]):
+    """gate and up (inter x hidden) and down (hidden x inter) at the base width distribution: the shape on which
+    the zero-padded packing (intermediate width rounded up to a multiple of 512) is compared with the unpadded
+    one."""
+    return [make_matrix(7, "gate", inter, hidden), make_matrix(7, "up", inter, hidden),
+            make_matrix(7, "down", hidden, inter)]
