@@ -73,6 +73,10 @@ struct Params {
   int res_sets;            // item-result sets: 2 (alternate batches) or 1
   int cost[5];             // job costs for the split of a batch among warps: units of 1, 2, 4, 8 bits; meta job
   int withhold;            // test hook: the record (global index) whose bulk copy is never issued, or -1
+  int balanced;            // CTAs split the records by estimated cost (directory search) instead of by count
+  unsigned long long base16[kMaxMats];  // start of matrix m's records in the byte sequence of all records, 16-B units
+  unsigned long long rec_w16;           // cost of a record beyond its bytes, in 16-byte units
+  unsigned long long total_w;           // cost of all records: 16-byte units + nrec * rec_w16
   unsigned long long wait_ns;  // limit of every mbarrier wait
 };
 
@@ -381,6 +385,45 @@ __device__ __forceinline__ int owner(const Params& p, int j) {
   return int(min(c, (long long)gridDim.x - 1));
 }
 
+// Split by cost (p.balanced, for matrices whose records differ much in size, such as an LM head whose frequent
+// rows are wider, or a small last row tile). A record costs its bytes plus a fixed part (p.rec_w16, a few mean
+// records: its meta job and row pass, and the rows' units whatever their width). With off(j) the cost of the
+// records before j and T the total, CTA c owns the records j with c T <= n off(j) < (c + 1) T (n CTAs). So lo(c)
+// is the first j with n off(j) >= c T, and the owner of record j is floor(n off(j) / T); a CTA can own nothing.
+__device__ __forceinline__ unsigned long long rec_off16(const Params& p, int j) {   // j in [0, nrec]
+  const int m = mat_of_rec(p, j);
+  const int jl = j - (m == 0 ? 0 : m == 1 ? p.rec_start[1] : m == 2 ? p.rec_start[2] : p.rec_start[3]);
+  return pick(p.base16, m) + __ldg(pick(p.dir, m) + jl) + (unsigned long long)j * p.rec_w16;
+}
+__device__ __forceinline__ int byte_owner(const Params& p, int j) {
+  return int(rec_off16(p, j) * gridDim.x / p.total_w);
+}
+// lo(c) by a 128-way search of one warp (four probes per lane and round; the directory is read through L2).
+__device__ int byte_lo(const Params& p, int c, int lane) {
+  const unsigned long long tgt = (unsigned long long)c * p.total_w, n = gridDim.x;
+  int lo = 0, hi = p.nrec;   // the answer is in [lo, hi]; off(nrec) = T satisfies every target
+  while (lo < hi) {
+    const int step = (hi - lo + 127) / 128;
+    bool pr[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int j = lo + (4 * lane + q) * step;
+      pr[q] = j >= hi || rec_off16(p, j) * n >= tgt;
+    }
+    unsigned first = 128;   // first probe (in probe order) that holds
+#pragma unroll
+    for (int q = 3; q >= 0; --q)
+      if (pr[q]) first = 4 * lane + q;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) first = min(first, __shfl_xor_sync(0xFFFFFFFFu, first, off));
+    if (first == 0) return lo;
+    const int prev = lo + int(first - 1) * step;   // the last probe that fails
+    hi = first == 128 ? hi : min(hi, lo + int(first) * step);
+    lo = prev + 1;
+  }
+  return lo;
+}
+
 // ---------------------------------------------------------------------------------------- end of a CTA
 // Runs after every whole-tile output and every partial slot of this CTA is written (all threads, after a barrier).
 //  - Tiles shared with other CTAs (only a CTA's first and last tile can be): one thread makes the CTA's slot writes
@@ -393,15 +436,52 @@ template <int B, int kThreads>
 __device__ void finish_cta(const Params& p, int L, int H, int* cta_flags, int* epi_tiles, int* epi_count) {
   const int tid = threadIdx.x, G = p.G, R = p.R;
   if (H <= L) return;
-  // Owners of tile t. With at least as many records as CTAs every CTA owns a contiguous, non-empty record range,
-  // so the owners are first..last. With fewer records than CTAs each CTA owns at most one record, so the owners
-  // are the owners of the tile's G records, one each.
-  const bool dense = p.nrec >= int(gridDim.x);
+  extern __shared__ __align__(128) unsigned char smem_fin[];   // the kernel's dynamic shared memory, free by now
+  int* own_list = reinterpret_cast<int*>(smem_fin);
+  __shared__ int own_cnt[2];
+  const int tfirst = L / G, tlast = (H - 1) / G;
+  const bool part0 = !(L <= tfirst * G && H >= (tfirst + 1) * G);
+  const bool part1 = tlast != tfirst && !(L <= tlast * G && H >= (tlast + 1) * G);
+  // Owners of tile t, in CTA order. Split by count: with at least as many records as CTAs every CTA owns a
+  // contiguous, non-empty record range, so the owners are first..last; with fewer records than CTAs each CTA owns
+  // at most one record, so the owners are the owners of the tile's G records, one each. Split by bytes: the
+  // distinct owners of the tile's records, listed by warp 0 (first tile) and warp 1 (last tile) in own_list.
+  const bool dense = p.nrec >= int(gridDim.x), bal = p.balanced != 0;
+  const int stride = int(gridDim.x) + 1;
+  if (bal && (part0 || part1)) {
+    __syncthreads();   // own_list reuses shared memory that the last row pass may still read
+    const int w = tid >> 5, lane = tid & 31;
+    if (w < 2 && (w == 0 ? part0 : part1)) {
+      const int t = w == 0 ? tfirst : tlast, j0 = t * G, j1 = min(j0 + G, p.nrec);
+      int cnt = 0, prev_q = -1;
+      for (int jb = j0; jb < j1; jb += 32) {
+        const int j = jb + lane;
+        const int q = j < j1 ? byte_owner(p, j) : 0x7FFFFFFF;
+        int up = __shfl_up_sync(0xFFFFFFFFu, q, 1);
+        if (lane == 0) up = prev_q;
+        const bool start = j < j1 && q != up;
+        const unsigned m = __ballot_sync(0xFFFFFFFFu, start);
+        if (start) own_list[w * stride + cnt + __popc(m & ((1u << lane) - 1u))] = q;
+        cnt += __popc(m);
+        prev_q = __shfl_sync(0xFFFFFFFFu, q, 31);
+      }
+      if (lane == 0) own_cnt[w] = cnt;
+    }
+    __syncthreads();
+  }
+  // tile t is the first (index 0) or last (index 1) tile of this CTA
   auto tile_owners = [&](int t, int& first) -> int {
+    if (bal) {
+      first = t == tfirst ? 0 : 1;   // the list
+      return own_cnt[first];
+    }
     first = owner(p, t * G);
     return dense ? owner(p, t * G + G - 1) - first + 1 : G;
   };
-  auto kth_owner = [&](int t, int first, int k) -> int { return dense ? first + k : owner(p, t * G + k); };
+  auto kth_owner = [&](int t, int first, int k) -> int {
+    if (bal) return own_list[first * stride + k];
+    return dense ? first + k : owner(p, t * G + k);
+  };
   // Sums of all owners' partial slots of the tiles this CTA reduces (one or two) into y, each element over the
   // owners in CTA order (so the result does not depend on which CTA reduces). A slot holds [B][R] f32. The
   // elements of both tiles form one index space, so their loads overlap. Few elements: one element per thread and
@@ -480,9 +560,6 @@ __device__ void finish_cta(const Params& p, int L, int H, int* cta_flags, int* e
     }
   };
 
-  const int tfirst = L / G, tlast = (H - 1) / G;
-  const bool part0 = !(L <= tfirst * G && H >= (tfirst + 1) * G);
-  const bool part1 = tlast != tfirst && !(L <= tlast * G && H >= (tlast + 1) * G);
   if (part0 || part1) {
     __syncthreads();
     // Thread 0 counts the CTA in on its first tile, thread 32 on its last, at the same time. Each atomic is
@@ -588,7 +665,7 @@ constexpr int kDirCache = 512;   // directory entries cached in shared memory
 //  mk [4][32] u32:     width masks per 32-row word;  pf [4][32] u16: item index of the word's first row per width
 //  wc [64] u32:        the record's width-code words
 //  kind (i32):         0 mixed widths; 1 bad record (adds nothing); 2 + c every row has width code c, so the item
-//                      index of a row is the row itself and the row pass reads no masks
+//                      index of a row is the row itself
 struct MetaOff {
   int t1, t2, xt, sg, fl, size;      // table block
   int mk, pf, wc, kind, row_size;    // row block
@@ -901,7 +978,15 @@ __global__ void __launch_bounds__(KCfg<B>::kThreads, 1) vbq_kernel(const __grid_
   __syncthreads();
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int G = p.G, NB = p.NB, S = p.S, cta = blockIdx.x;
-  const int L = rec_lo(p, cta), H = rec_lo(p, cta + 1);
+  __shared__ int lo_hi[2];
+  if (p.balanced) {
+    if (warp < 2) {
+      const int v = byte_lo(p, cta + warp, lane);
+      if (lane == 0) lo_hi[warp] = v;
+    }
+    __syncthreads();
+  }
+  const int L = p.balanced ? lo_hi[0] : rec_lo(p, cta), H = p.balanced ? lo_hi[1] : rec_lo(p, cta + 1);
   if (H <= L) return;  // nothing to read or write
   const MetaOff mo(B);
   const int NS = NB * S;
@@ -1269,16 +1354,14 @@ __global__ void __launch_bounds__(KCfg<B>::kThreads, 1) vbq_kernel(const __grid_
         if (pos < nrec && r < Rt) {
           const unsigned char* rm = row_ptr(mp_, pos);
           const int kd = *reinterpret_cast<const int*>(rm + mo.kind);
-          if (kd >= 2) {   // one width: the items are the rows
-            item[pos] = r;
-          } else {
-            const uint32_t* mk = reinterpret_cast<const uint32_t*>(rm + mo.mk);
-            const uint16_t* pf = reinterpret_cast<const uint16_t*>(rm + mo.pf);
-            const uint32_t wcw = reinterpret_cast<const uint32_t*>(rm + mo.wc)[r >> 4];
-            const int c = int(wcw >> (2 * (r & 15))) & 3;
-            const int it = pf[c * 32 + word] + __popc(mk[c * 32 + word] & ((1u << lane) - 1u));
-            item[pos] = kd ? -1 : it;   // a bad record adds nothing
-          }
+          // the mixed-width item index, its loads issued alongside kind's (the meta job writes the masks of every
+          // record, so they are valid for one-width records too)
+          const uint32_t* mk = reinterpret_cast<const uint32_t*>(rm + mo.mk);
+          const uint16_t* pf = reinterpret_cast<const uint16_t*>(rm + mo.pf);
+          const uint32_t wcw = reinterpret_cast<const uint32_t*>(rm + mo.wc)[r >> 4];
+          const int c = int(wcw >> (2 * (r & 15))) & 3;
+          const int it = pf[c * 32 + word] + __popc(mk[c * 32 + word] & ((1u << lane) - 1u));
+          item[pos] = kd >= 2 ? r : kd ? -1 : it;   // one width: the items are the rows; a bad record adds nothing
         }
       }
 #pragma unroll
@@ -1508,6 +1591,7 @@ int launch(const Problem& pr, const void* const* blobs, const void* x, float* co
   Params p = {};
   p.nmat = pr.nmat;
   int tiles = 0, recs = 0;
+  unsigned long long total16 = 0;
   for (int m = 0; m < kMaxMats; ++m) {
     p.tile_start[m] = tiles;
     p.rec_start[m] = recs;
@@ -1520,11 +1604,20 @@ int launch(const Problem& pr, const void* const* blobs, const void* x, float* co
     p.N[m] = int(d->N);
     p.sym[m] = (d->flags & VBQ_FLAG_GRID_SYMMETRIC) ? 1 : 0;
     p.units_total[m] = uint32_t((d->total_bytes - d->rec_offset) / 16);
+    p.base16[m] = total16;
+    total16 += p.units_total[m];
     tiles += int(d->T);
     recs += int(d->T * d->G);
   }
   p.tile_start[kMaxMats] = tiles;
   p.rec_start[kMaxMats] = recs;
+  // Split by cost when record sizes differ much (the largest record over 1.3 times the mean, as in an LM head
+  // whose frequent rows are wider); otherwise by count, which needs no directory search.
+  p.balanced = (double(pr.max_record_bytes) > 1.3 * 16.0 * double(total16) / double(recs)) ? 1 : 0;
+  // the fixed part of a record's cost, measured on LM heads: four mean records at batch 1 (the per-record work
+  // dominates), two at larger batches (the units' share grows with B)
+  p.rec_w16 = std::max<unsigned long long>(1, (B == 1 ? 4ull : 2ull) * total16 / unsigned(recs));
+  p.total_w = total16 + p.rec_w16 * unsigned(recs);
   p.x = static_cast<const uint16_t*>(x);
   uint8_t* w = static_cast<uint8_t*>(ws);
   p.partial = reinterpret_cast<float*>(w);

@@ -592,3 +592,39 @@ def test_zero_padded_mlp_matches_unpadded_and_oracle(B):
         got = y.cpu().numpy().astype(np.float64)
         bad = np.abs(got - y_ref) > 1e-3 * (A + E) + 1e-6 + E
         assert not bad.any(), f"{what} (down): {int(bad.sum())} outputs out of bar"
+
+
+def uneven(seed, N, K, heavy_rows, heavy_width=8):
+    """Rows [0, heavy_rows) at heavy_width bits, the rest 1-bit: records of very different sizes, as in an LM head
+    whose frequent rows are wider (VBQ paper, section 6: frequency-grouped row buckets), so that CTAs split the
+    records by bytes."""
+    g = np.random.default_rng(seed)
+    w = np.ones((N, K // 64), np.uint8)
+    w[:heavy_rows] = heavy_width
+    return S.Matrix("uneven", N, K, w, S.scales_uniform(N, K // 64, g), S.codes_uniform(w, g))
+
+
+@pytest.mark.parametrize("B", [1, 4, 16])
+def test_byte_split_on_uneven_records(B):
+    """Matrices whose records differ up to eightfold in size, so the launch splits them among CTAs by bytes: a
+    ragged 3000-row matrix, one with fewer records than CTAs (CTAs that own nothing), and a fused launch of an
+    all-8-bit matrix with an all-1-bit one. Every output against the oracle."""
+    cases = [(uneven(1 + B, 3000, 512, 300), 64), (uneven(2 + B, 100, 2048, 10), 16),
+             (uneven(3 + B, 40, 256, 7), 16)]
+    for m, R in cases:
+        mat = vbq.DeviceMatrix(vbq.vbq_pack(m.N, m.K, R, m.widths, m.scales, m.codes)[0], dev(), max_batch=B)
+        x = S.x_normal(B, m.K, np.random.default_rng(m.N + B))
+        y, _ = gpu_y(m, x, mat=mat)
+        yref, bound = O.matvec(m.widths, m.scales, m.codes, x, NTH)
+        check(y, yref, bound, f"uneven {m.N}x{m.K} R={R} B={B}")
+    a, b = uneven(5 + B, 500, 512, 500), uneven(6 + B, 2000, 512, 0)
+    mats = [vbq.DeviceMatrix(vbq.vbq_pack(m.N, m.K, 64, m.widths, m.scales, m.codes)[0], dev(), max_batch=B)
+            for m in (a, b)]
+    fused = vbq.FusedMatrices(mats, max_batch=B)
+    x = S.x_normal(B, 512, np.random.default_rng(77 + B))
+    ys = fused.matmul(to_dev_x(x))
+    torch_sync()
+    assert fused_status(fused, B) == 0
+    for m, y in zip((a, b), ys):
+        yref, bound = O.matvec(m.widths, m.scales, m.codes, x, NTH)
+        check(y.cpu().numpy().astype(np.float64), yref, bound, f"fused uneven {m.N} B={B}")
