@@ -1398,11 +1398,12 @@ __global__ void __launch_bounds__(KCfg<B>::kThreads, 1) vbq_kernel(const __grid_
     }
   };
 
-  // With two result sets, batch n's row pass runs after the warp's jobs of batch n + 1, before the barrier that
-  // ends them: a warp that finishes its units early sums rows instead of waiting. (Batch n + 1's units write the
-  // other result set; the row, result and table sets batch n's row pass reads are next written by batch n + 2's
-  // and n + 3's meta jobs and units, which start after that barrier.) With one set, the row pass follows the
-  // batch's own barrier and a second barrier guards the set.
+  // At B >= 4 with two result sets, batch n's row pass runs after the warp's jobs of batch n + 1, before the
+  // barrier that ends them: a warp that finishes its units early sums rows instead of waiting. (Batch n + 1's
+  // units write the other result set; the row, result and table sets batch n's row pass reads are next written by
+  // batch n + 2's and n + 3's meta jobs and units, which start after that barrier.) At B <= 2 the row pass is short
+  // and follows the batch's own barrier (measured faster there). With one set, a second barrier guards the set.
+  constexpr bool kDefer = B >= 4;
   int pt = 0, pn = 0, pmp = 0, prp = 0;   // the previous batch: tile, records, row and result sets
   bool have_prev = false;
   while (!aborted) {
@@ -1414,7 +1415,7 @@ __global__ void __launch_bounds__(KCfg<B>::kThreads, 1) vbq_kernel(const __grid_
       mpn = mp == 2 ? 0 : mp + 1;
       jobs(cur, nxt, rp, mpn);
     }
-    if (two_sets && have_prev) row_pass(pt, pn, pmp, prp, !live || pt != cur.t);
+    if (kDefer && two_sets && have_prev) row_pass(pt, pn, pmp, prp, !live || pt != cur.t);
     if (!live) break;
     aborted = __syncthreads_or(cta_abort != 0) != 0;
     if (aborted) break;
@@ -1431,7 +1432,7 @@ __global__ void __launch_bounds__(KCfg<B>::kThreads, 1) vbq_kernel(const __grid_
       }
       iss.next();
     }
-    if (two_sets) {
+    if (kDefer && two_sets) {
       pt = cur.t;
       pn = cur.re - cur.rb;
       pmp = mp;
@@ -1439,7 +1440,7 @@ __global__ void __launch_bounds__(KCfg<B>::kThreads, 1) vbq_kernel(const __grid_
       have_prev = true;
     } else {
       row_pass(cur.t, cur.re - cur.rb, mp, rp, !nxt.valid() || nxt.t != cur.t);
-      __syncthreads();   // the next batch's units overwrite the one result set
+      if (!two_sets) __syncthreads();   // the next batch's units overwrite the one result set
     }
     cur = nxt;
     mp = mpn;
@@ -1523,7 +1524,7 @@ inline void plan_workspace(const Problem& pr, int B, Plan& pl) {
   pl.status_off = pl.ws_bytes - 4;
 }
 
-// Records per batch NB and batches in flight S. NB aims at about three jobs per warp
+// Records per batch NB and batches in flight S. Above batch 2, NB aims at about three jobs per warp
 // per batch (from an estimate of the units per record at the paper's allocation); S = 3 when it fits (the meta
 // jobs of a batch read records issued two batches earlier), else 2. Fewer records per batch before fewer sets.
 template <int B>
@@ -1539,7 +1540,8 @@ inline bool make_plan_b(const Problem& pr, int sms, Plan& pl) {
   const int dir_bytes = 8 * kDirCache;
   // units per record at the paper's allocation: 1-bit units of 32 items, the others of 32 / B; bucket tails
   const int upr = (7 * R / 10 + 31) / 32 + (16 * R / 100 + 31) / 32 + (15 * R / 100 + C::kIPU - 1) / C::kIPU + 2;
-  const int nb_want = std::min(kMaxNB, std::max(1, (5 * C::kWarps + upr - 1) / upr));
+  // batch 1 and 2: as many records per batch as fit (fewer batches, less per-batch bookkeeping: measured faster)
+  const int nb_want = B <= 2 ? kMaxNB : std::min(kMaxNB, std::max(1, (5 * C::kWarps + upr - 1) / upr));
   const MetaOff mo(B);
   auto need = [&](int NB, int S, int RS) {
     return (long long)S * NB * pl.stage_size + (long long)RS * NB * pl.res_rec + 256 + 2ll * NB * pl.meta_rec +
