@@ -53,10 +53,9 @@ L2_BYTES = 126e6
 # this step's algorithmic bytes per launch (traffic grows in proportion: the five launches span 4.5 to 41 MB, each
 # at 0.999 to 1.019 times its algorithmic bytes), and only while the kernel source and the tile rows are the
 # captured ones.
-NCU_TRAFFIC = {"kernel_source_sha256": "d6593dba6f9e3797de02ec23fbc0e6694a6afe2bb7ff84544ee57261af5ffeb1",
-               "tile_rows": {"q_k_v": 224, "o": 512, "gate_up": 224, "down": 224, "head": 224},
-               "dram_bytes": 102591232, "algorithmic_bytes": 102422912, "launches": 5,
-               "summary": "profiles/vbq_kernel_b1_decode_step_9b_launches.md"}
+NCU_TRAFFIC = {"kernel_source_sha256": "cdd770b25956751b1b6331940c4783b9f9124a62ac270dede7a213a7b01c81fb",
+               "tile_rows": {"q_k_v": 512, "o": 256, "gate_up": 1024, "down": 512, "head": 1024},
+               "dram_bytes": 102439424, "algorithmic_bytes": 102225376, "launches": 5}
 
 
 def kernel_source_sha256() -> str:
@@ -569,6 +568,8 @@ def run_cfg4(args):
     sampler = ClockSampler(local)
     sampler.start()
     for name, N, K in CFG4:
+        if args.matrices and name not in args.matrices.split(","):
+            continue
         m = S.cfg4((name,))[0]
         R = args.tile_rows if args.tile_rows > 0 else vbq.suggest_tile_rows(N, K, sms)
         blob, desc = vbq.vbq_pack(m.N, m.K, R, m.widths, m.scales, m.codes)
@@ -619,8 +620,8 @@ def run_cfg4(args):
         torch.cuda.empty_cache()
     clocks = sampler.stop()
     t_setup = time.perf_counter() - t_setup
-    head = [results[f"{n} {N}x{K} B=1"]["GBps"] for n, N, K in CFG4 if n in ("gate", "down")] if 1 in batches else \
-        [results[k]["GBps"] for k in results]
+    head = [results[f"{n} {N}x{K} B=1"]["GBps"] for n, N, K in CFG4
+            if n in ("gate", "down") and f"{n} {N}x{K} B=1" in results] or [results[k]["GBps"] for k in results]
     value = float(np.mean(head))
     if rank == 0:
         line = {"metric": METRIC, "value": value * world, "unit": UNIT, "n_gpus": world, "steps": 3,
@@ -777,6 +778,8 @@ def make_parser() -> argparse.ArgumentParser:
                     help="plain launches instead of programmatic dependent launch between the linears")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds for the CPU-oracle baseline (0: skip)")
     ap.add_argument("--ref-rows", type=int, default=256, help="rows per linear per step for --impl reference")
+    ap.add_argument("--matrices", default="",
+                    help="cfg4 only: comma-separated subset of q, gate, down (default: all three)")
     return ap
 
 

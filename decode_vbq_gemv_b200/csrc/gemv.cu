@@ -628,12 +628,12 @@ __device__ void finish_cta(const Params& p, int L, int H, int* cta_flags, int* e
 //    shared memory by cp.async.bulk (one copy per record plus one 128-byte copy per batch row of the column's
 //    activations), S batches ahead, each record in its own slot with its own mbarrier.
 //  - Each record gets a meta job one batch before its units run: validate it, build the width masks and item
-//    starts per 32-row word, the group sums of x (and for B <= 4 the activation and nibble tables), and note where
+//    starts per 32-row word, the group sums of x (and for B <= 2 the activation and nibble tables), and note where
 //    its buckets lie.
 //  - Per batch, the jobs are the width-bucket units of its records and the meta jobs of the next batch. Every warp
 //    computes the same job list from the meta blocks and takes the jobs whose cost midpoint falls in its share of
 //    the total, so the split is even to about one unit. A unit writes s * dot for each of its items (and batch
-//    rows) into the record's result buffer: on CUDA cores for B <= 4, through mma.sync for B = 8, 16.
+//    rows) into the record's result buffer: on CUDA cores for B <= 2, through mma.sync for B = 4, 8, 16.
 //  - One CTA barrier per batch. Then each warp adds the results of its own 32-row words to its accumulators,
 //    record by record in record order (row r takes the result of its item: the start of its bucket in its word
 //    plus the rows of the same width before it), so every row is summed in a fixed order and results are bitwise
@@ -641,9 +641,12 @@ __device__ void finish_cta(const Params& p, int L, int H, int* cta_flags, int* e
 //  - A finished tile goes to y when the CTA holds all its records, else to the CTA's partial slot; finish_cta then
 //    reduces the tiles shared with neighbouring CTAs and runs the SwiGLU epilogue.
 constexpr int kCudaCoreWarps = 16;      // warps per CTA at B = 1, 2
+// smallest batch on the tensor-core units; at batch 4 the n8 mma tile is half used, and building the operands,
+// not the mma, is the cost, so batch 4 gains from leaving its per-row CUDA-core loops
+constexpr int kTensorCoreMinBatch = 4;
 constexpr int kCtasPerSM = 1;   // CTAs per SM in its grid
 template <int B> struct KCfg {
-  static constexpr bool kTC = B >= 8;                               // tensor-core units (batch 8, 16)
+  static constexpr bool kTC = B >= kTensorCoreMinBatch;             // tensor-core units
   static constexpr int kWarps = B <= 2 ? kCudaCoreWarps : B <= 8 ? 12 : 8;
   static constexpr int kThreads = kWarps * 32;
   static constexpr int kIPU = kTC ? 32 : 32 / B;                    // items per 4-, 8-bit unit
@@ -655,7 +658,7 @@ constexpr int kDirCache = 512;   // directory entries cached in shared memory
 
 // Per-record metadata, written by the record's meta job one batch before its units run, in two blocks.
 // Table block (256-byte aligned; read only by the units, so two sets serve alternate batches). The tables exist
-// for B <= 4 only, and each is built only when the record has rows of the widths that read it:
+// for B <= 2 only, and each is built only when the record has rows of the widths that read it:
 //  t1 [B][16][16] f32: 1-bit nibble tables; entry n of position p is the sum of x[4p + i] over the set bits i of n
 //  t2 [B][32][16] f32: 2-bit nibble tables; entry n of position p is (n & 3) x[2p] + (n >> 2) x[2p + 1]
 //  xt [2][B][64] f32:  x, and x * 2^-shift for the magic-number expansion of 4-bit codes
@@ -670,7 +673,7 @@ struct MetaOff {
   int t1, t2, xt, sg, fl, size;      // table block
   int mk, pf, wc, kind, row_size;    // row block
   __host__ __device__ explicit MetaOff(int B) {
-    const int tb = B >= 8 ? 0 : B;   // the tensor-core path (batch 8, 16) needs no activation tables
+    const int tb = B >= kTensorCoreMinBatch ? 0 : B;   // the tensor-core path needs no activation tables
     t1 = 0;
     t2 = 1024 * tb;
     xt = t2 + 2048 * tb;
@@ -804,7 +807,7 @@ __device__ __forceinline__ void unit_range(int n, int lo, int hi, int lane, uint
   }
 }
 
-// Tensor-core A fragments (batch 8, 16). Lane (g, t) = (lane / 4, lane % 4) of an mma.sync m16n8k16 holds, for
+// Tensor-core A fragments (batch 4, 8, 16). Lane (g, t) = (lane / 4, lane % 4) of an mma.sync m16n8k16 holds, for
 // each k-step ks, two bf16 pairs of A row g: logical columns 16 ks + 2t + {0, 1} and + {8, 9}. Logical columns
 // map to codes so that lane t reads one contiguous run of its item's codes: 16t .. 16t + 15, as 8 bf16 pairs
 // a[0..7], a[2 ks] and a[2 ks + 1] feeding k-step ks. The activations take the same map (tc_x_frags), so any
@@ -861,10 +864,15 @@ __device__ __forceinline__ void tc_a_frag(uint32_t addr, bool ok, uint32_t tab, 
 // b = 8 nt + g, k-step ks: bfr[ks][nt][0] pairs with a[2 ks], bfr[ks][nt][1] with a[2 ks + 1]. xb: the staged
 // bf16 activations [B][64] of the record's group. perm4: the 4-bit map, else adjacent pairs.
 template <int B>
-__device__ __forceinline__ void tc_x_frags(uint32_t xb, int lane, bool perm4, uint32_t (&bfr)[4][B / 8][2]) {
+__device__ __forceinline__ void tc_x_frags(uint32_t xb, int lane, bool perm4, uint32_t (&bfr)[4][(B + 7) / 8][2]) {
   const int g = lane >> 2, t = lane & 3;
 #pragma unroll
-  for (int nt = 0; nt < B / 8; ++nt) {
+  for (int nt = 0; nt < (B + 7) / 8; ++nt) {
+    if (nt * 8 + g >= B) {   // batch 4: columns 4..7 of the n8 tile are zero
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks) bfr[ks][nt][0] = bfr[ks][nt][1] = 0u;
+      continue;
+    }
     const uint32_t row = xb + 128 * (nt * 8 + g) + 32 * t;
 #pragma unroll
     for (int ks = 0; ks < 4; ++ks) {
@@ -882,14 +890,14 @@ __device__ __forceinline__ void tc_x_frags(uint32_t xb, int lane, bool perm4, ui
   }
 }
 
-// Tensor-core units [lo, hi) of one width bucket, 32 items each (B = 8, 16): per 16-item m-tile, lane (g, t) builds
+// Tensor-core units [lo, hi) of one width bucket, 32 items each (B = 4, 8, 16): per 16-item m-tile, lane (g, t) builds
 // the fragments of items 16 mt + g and + 8 from their codes, mma.sync m16n8k16 (bf16 in, fp32 accumulate, seeded
 // with the grid-offset term init[nt]) against the activations bfr, and writes s times each result to res[item][b].
 template <int B, int KB>
 __device__ __forceinline__ void unit_range_tc(int n, int lo, int hi, int lane, uint32_t codes, uint32_t scales,
-                                              uint32_t res, uint32_t tab, const float2 (&init)[B / 8],
-                                              const uint32_t (&bfr)[4][B / 8][2]) {
-  constexpr int NTL = B / 8;
+                                              uint32_t res, uint32_t tab, const float2 (&init)[(B + 7) / 8],
+                                              const uint32_t (&bfr)[4][(B + 7) / 8][2]) {
+  constexpr int NTL = (B + 7) / 8;
   const int g = lane >> 2, t = lane & 3;
   for (int u = lo; u < hi; ++u) {
 #pragma unroll
@@ -921,6 +929,7 @@ __device__ __forceinline__ void unit_range_tc(int n, int lo, int hi, int lane, u
 #pragma unroll
       for (int nt = 0; nt < NTL; ++nt) {
         const int b = nt * 8 + 2 * t;
+        if (B % 8 != 0 && b >= B) continue;   // batch 4: only lanes t < 2 hold real columns
         if (ok0) sts64f(res + 4 * (i0 * B + b), s0 * c4[nt][0], s0 * c4[nt][1]);
         if (ok1) sts64f(res + 4 * (i1 * B + b), s1 * c4[nt][2], s1 * c4[nt][3]);
       }
@@ -1244,7 +1253,7 @@ __global__ void __launch_bounds__(KCfg<B>::kThreads, 1) vbq_kernel(const __grid_
     int loaded = -1;
     const bool grid_sym = pick(p.sym, mat_of_tile(p, cur.t)) != 0;
     const float corr = grid_sym ? 1.f : 0.5f;
-    uint32_t bfr[4][C::kTC ? B / 8 : 1][2];   // tensor-core path: the record's activations as mma B fragments
+    uint32_t bfr[4][C::kTC ? (B + 7) / 8 : 1][2];   // tensor-core path: the record's activations as B fragments
     while (todo) {
       const int sgi = __ffs(todo) - 1;
       todo &= todo - 1;
@@ -1271,12 +1280,13 @@ __global__ void __launch_bounds__(KCfg<B>::kThreads, 1) vbq_kernel(const __grid_
           loaded = kind;
         }
         // accumulator seed: (2^(k-1) - c) sum x for 4 and 8 bits (1/2 on the default grid, 1 on the symmetric)
-        float2 init[B / 8];
+        float2 init[(B + 7) / 8];
         const float* sgv = reinterpret_cast<const float*>(mb + mo.sg);
         const float f = k < 2 ? 0.f : corr;
 #pragma unroll
-        for (int nt = 0; nt < B / 8; ++nt) {
-          const float2 sg2 = *reinterpret_cast<const float2*>(sgv + nt * 8 + 2 * (lane & 3));
+        for (int nt = 0; nt < (B + 7) / 8; ++nt) {
+          const int b = nt * 8 + 2 * (lane & 3);
+          const float2 sg2 = b < B ? *reinterpret_cast<const float2*>(sgv + b) : make_float2(0.f, 0.f);
           init[nt] = make_float2(f * sg2.x, f * sg2.y);
         }
         const uint32_t tb = smem_u32(tc_tab);
@@ -1644,10 +1654,10 @@ int launch(const Problem& pr, const void* const* blobs, const void* x, float* co
   // job costs (about the instructions a warp spends): units of 1-, 2-, 4-, 8-bit groups; a meta job
   // job costs, in scheduler cycles of one lane (integer and packed fp32 instructions take two, fp32 one):
   // 1- and 2-bit units (nibble tables, all batch rows), 4- and 8-bit units (magic-number expansion), a meta job
-  // batch 8, 16: tensor-core units of 32 items (fragment building dominates; mma.sync adds 8 B / 8 per unit)
-  if (B <= 4) {
+  // tensor-core batches: units of 32 items (fragment building dominates; mma.sync adds little per unit)
+  if (!KCfg<B>::kTC) {
     p.cost[0] = 60 + 20 * B;
-    p.cost[1] = 100 + 35 * B;
+    p.cost[1] = 150 + 35 * B;
     p.cost[2] = 285;
     p.cost[3] = 275;
     p.cost[4] = 400 + 100 * B;
