@@ -622,8 +622,8 @@ __device__ void finish_cta(const Params& p, int L, int H, int* cta_flags, int* e
 }
 
 // ===================================================================================== record-batch kernel
-// Every batch B in {1, 2, 4, 8, 16}. One CTA per SM whose warps (16 at B = 1, 2; 12 at B = 4, 8; 8 at B = 16:
-// as many as the registers of each batch size allow) work on the CTA's records together:
+// Every batch B in {1, 2, 4, 8, 16}. One CTA per SM whose warps (16 at B = 1, 2; 12 at B = 4, 8, 16: as many as
+// the registers of each batch size allow) work on the CTA's records together:
 //  - The CTA's record range is cut into batches of up to NB records of one row tile. Records stream HBM ->
 //    shared memory by cp.async.bulk (one copy per record plus one 128-byte copy per batch row of the column's
 //    activations), S batches ahead, each record in its own slot with its own mbarrier.
@@ -644,10 +644,13 @@ constexpr int kCudaCoreWarps = 16;      // warps per CTA at B = 1, 2
 // smallest batch on the tensor-core units; at batch 4 the n8 mma tile is half used, and building the operands,
 // not the mma, is the cost, so batch 4 gains from leaving its per-row CUDA-core loops
 constexpr int kTensorCoreMinBatch = 4;
+// floats per item in a record's result buffer: B, padded by 4 at B >= 8 so that the row pass's 16-byte loads of
+// consecutive items (and the units' 8-byte stores) fall in distinct shared-memory banks
+__host__ __device__ constexpr int res_stride(int B) { return B >= 8 ? B + 4 : B; }
 constexpr int kCtasPerSM = 1;   // CTAs per SM in its grid
 template <int B> struct KCfg {
   static constexpr bool kTC = B >= kTensorCoreMinBatch;             // tensor-core units
-  static constexpr int kWarps = B <= 2 ? kCudaCoreWarps : B <= 8 ? 12 : 8;
+  static constexpr int kWarps = B <= 2 ? kCudaCoreWarps : 12;
   static constexpr int kThreads = kWarps * 32;
   static constexpr int kIPU = kTC ? 32 : 32 / B;                    // items per 4-, 8-bit unit
   static constexpr int kWordsPerWarp = (32 + kWarps - 1) / kWarps;  // row-pass words per warp (R <= 1024)
@@ -930,8 +933,8 @@ __device__ __forceinline__ void unit_range_tc(int n, int lo, int hi, int lane, u
       for (int nt = 0; nt < NTL; ++nt) {
         const int b = nt * 8 + 2 * t;
         if (B % 8 != 0 && b >= B) continue;   // batch 4: only lanes t < 2 hold real columns
-        if (ok0) sts64f(res + 4 * (i0 * B + b), s0 * c4[nt][0], s0 * c4[nt][1]);
-        if (ok1) sts64f(res + 4 * (i1 * B + b), s1 * c4[nt][2], s1 * c4[nt][3]);
+        if (ok0) sts64f(res + 4 * (i0 * res_stride(B) + b), s0 * c4[nt][0], s0 * c4[nt][1]);
+        if (ok1) sts64f(res + 4 * (i1 * res_stride(B) + b), s1 * c4[nt][2], s1 * c4[nt][3]);
       }
     }
   }
@@ -1271,7 +1274,7 @@ __global__ void __launch_bounds__(KCfg<B>::kThreads, 1) vbq_kernel(const __grid_
       unsigned parity;
       cur.slot_of(pos, slot, parity);
       const uint32_t sa = smem_u32(slot_ptr(slot));
-      const uint32_t res = res_addr(rp, pos) + 4 * B * ib;
+      const uint32_t res = res_addr(rp, pos) + 4 * res_stride(B) * ib;
       const uint32_t sca = sa + sc + 2 * ib;
       if constexpr (C::kTC) {
         const int kind = pos * 2 + (k == 2 ? 1 : 0);   // the 4-bit code map differs from the others'
@@ -1377,7 +1380,7 @@ __global__ void __launch_bounds__(KCfg<B>::kThreads, 1) vbq_kernel(const __grid_
 #pragma unroll
       for (int pos = 0; pos < kMaxNB; ++pos)
         if (item[pos] >= 0) {
-          const uint32_t res = res_addr(rp_, pos) + 4 * (item[pos] * B);
+          const uint32_t res = res_addr(rp_, pos) + 4 * (item[pos] * res_stride(B));
           if constexpr (B >= 4) {
 #pragma unroll
             for (int b = 0; b < B; b += 4) {
@@ -1545,7 +1548,7 @@ inline bool make_plan_b(const Problem& pr, int sms, Plan& pl) {
   const int R = pr.R;
   pl.stage_bytes = align128i(int(pr.max_record_bytes));
   pl.stage_size = pl.stage_bytes + align128i(128 * B);
-  pl.res_rec = align128i(R * B * 4);
+  pl.res_rec = align128i(R * res_stride(B) * 4);
   pl.meta_rec = MetaOff(B).size;
   const int dir_bytes = 8 * kDirCache;
   // units per record at the paper's allocation: 1-bit units of 32 items, the others of 32 / B; bucket tails
