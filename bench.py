@@ -528,6 +528,16 @@ def run_vbq(args):
             and kernel_source_sha256() == NCU_TRAFFIC["kernel_source_sha256"]):
         traffic = launch_bytes * NCU_TRAFFIC["dram_bytes"] / NCU_TRAFFIC["algorithmic_bytes"]
 
+    # Batch sweep (outside the timed step): the 14336x4096 gate linear alone at batch 1-16, streaming from HBM, so
+    # that the step's JSON line also carries the skinny-GEMM batch sizes.
+    sweep = None
+    if not args.no_batch_sweep:
+        speak, _ = peaks()
+        res, _ = rotation_sweep(args, dev, stream, sms, speak, "gate", (1, 2, 4, 8, 16))
+        sweep = {"workload": "gate 14336x4096 alone at each batch size, >= 4x L2 of distinct copies in rotation, "
+                             "best of 3 graph replays",
+                 "results": {k: {"us": round(v["us"], 2), "GBps": round(v["GBps"], 1), "frac": round(v["frac"], 4),
+                                 "status": v["status"]} for k, v in res.items()}}
     if rank == 0:
         peak, peak_kind = peaks()
         cpu = cpu_baseline(B, args.cpu_budget) if (world == 1 and args.cpu_budget > 0) else None
@@ -537,6 +547,7 @@ def run_vbq(args):
                         t_setup=t_setup, launch_bytes=launch_bytes, launch_ms=launch_ms, traffic=traffic,
                         per_shape=per_shape, e2e_val=e2e_val, h2d=h2d, d2h=d2h, fp16=fp16, n_launches=n_launches,
                         clocks=clocks, cpu=cpu, peak=peak, peak_kind=peak_kind)
+        line["batch_sweep"] = sweep
         print(json.dumps(line), flush=True)
     del graph, graph_e2e
     if world > 1:
@@ -547,6 +558,66 @@ def run_vbq(args):
 
 # ------------------------------------------------------------------------------------------- config 4
 CFG4 = (("q", 4096, 4096), ("gate", 14336, 4096), ("down", 4096, 14336))
+
+
+def rotation_sweep(args, dev, stream, sms, peak, name, batches):
+    """One config-4 matrix timed alone at each batch size: M distinct device copies of the packed matrix, together
+    at least 4x the L2, launched round-robin in one CUDA graph (chained by programmatic dependent launch), so every
+    launch streams its weights from HBM; time per launch = replay time / M, the best of three replays after
+    warm-up. Returns ({"name NxK B=b": {...}}, launches)."""
+    import torch
+    from decode_vbq_gemv_b200 import vbq
+    N, K = dict((n, (a, b)) for n, a, b in CFG4)[name]
+    m = S.cfg4((name,))[0]
+    R = args.tile_rows if args.tile_rows > 0 else vbq.suggest_tile_rows(N, K, sms)
+    blob, desc = vbq.vbq_pack(m.N, m.K, R, m.widths, m.scales, m.codes)
+    stride = (blob.size + 255) // 256 * 256
+    M = max(2, int(np.ceil(4 * L2_BYTES / stride)))
+    copies = torch.empty(M * stride, dtype=torch.uint8, device=dev)
+    first = torch.from_numpy(blob).to(dev)
+    for c in range(M):
+        copies[c * stride:c * stride + blob.size].copy_(first)
+    del first
+    results, n_launches = {}, 0
+    for B in batches:
+        ws_bytes = vbq.vbq_workspace_size(desc, B)
+        ws = torch.zeros(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+        x = torch.from_numpy(S.make_x(4, name, B, K).astype(np.int16)).view(torch.bfloat16).to(dev)
+        y = torch.empty((B, N), dtype=torch.float32, device=dev)
+        flags = 0 if args.no_overlap else vbq.VBQ_LAUNCH_OVERLAP
+        with torch.cuda.stream(stream):
+            def run_all():
+                for c in range(M):
+                    vbq.vbq_gemm_skinny_ex(desc, copies[c * stride:c * stride + blob.size], x, B, y, ws, flags,
+                                           stream)
+            run_all()
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                run_all()
+            for _ in range(args.warmup):
+                g.replay()
+            torch.cuda.synchronize()
+            best = None
+            for _ in range(3):
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                g.replay()
+                e1.record(stream)
+                torch.cuda.synchronize()
+                t = e0.elapsed_time(e1) / M
+                best = t if best is None else min(best, t)
+            n_launches += 3 * M   # the timed replays
+        status = int(ws[ws_bytes - 4:ws_bytes].cpu().numpy().view(np.uint32)[0]) if ws_bytes >= 4 else 0
+        nbytes = blob.size + B * K * 2 + B * N * 4
+        gbps = nbytes / (best / 1e3) / 1e9
+        results[f"{name} {N}x{K} B={B}"] = {"us": best * 1e3, "GBps": gbps, "frac": gbps / peak, "tile_rows": R,
+                                            "copies": M, "status": status}
+        del g, ws
+    del copies
+    torch.cuda.empty_cache()
+    return results, n_launches
 
 
 def run_cfg4(args):
@@ -570,54 +641,9 @@ def run_cfg4(args):
     for name, N, K in CFG4:
         if args.matrices and name not in args.matrices.split(","):
             continue
-        m = S.cfg4((name,))[0]
-        R = args.tile_rows if args.tile_rows > 0 else vbq.suggest_tile_rows(N, K, sms)
-        blob, desc = vbq.vbq_pack(m.N, m.K, R, m.widths, m.scales, m.codes)
-        stride = (blob.size + 255) // 256 * 256
-        M = max(2, int(np.ceil(4 * L2_BYTES / stride)))
-        copies = torch.empty(M * stride, dtype=torch.uint8, device=dev)
-        first = torch.from_numpy(blob).to(dev)
-        for c in range(M):
-            copies[c * stride:c * stride + blob.size].copy_(first)
-        del first
-        for B in batches:
-            ws_bytes = vbq.vbq_workspace_size(desc, B)
-            ws = torch.zeros(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
-            x = torch.from_numpy(S.make_x(4, name, B, K).astype(np.int16)).view(torch.bfloat16).to(dev)
-            y = torch.empty((B, N), dtype=torch.float32, device=dev)
-            flags = 0 if args.no_overlap else vbq.VBQ_LAUNCH_OVERLAP
-            with torch.cuda.stream(stream):
-                def run_all():
-                    for c in range(M):
-                        vbq.vbq_gemm_skinny_ex(desc, copies[c * stride:c * stride + blob.size], x, B, y, ws, flags,
-                                               stream)
-                run_all()
-                torch.cuda.synchronize()
-                g = torch.cuda.CUDAGraph()
-                with torch.cuda.graph(g, stream=stream):
-                    run_all()
-                for _ in range(args.warmup):
-                    g.replay()
-                torch.cuda.synchronize()
-                best = None
-                for _ in range(3):
-                    e0 = torch.cuda.Event(enable_timing=True)
-                    e1 = torch.cuda.Event(enable_timing=True)
-                    e0.record(stream)
-                    g.replay()
-                    e1.record(stream)
-                    torch.cuda.synchronize()
-                    t = e0.elapsed_time(e1) / M
-                    best = t if best is None else min(best, t)
-                n_launches += M * (args.warmup + 3)
-            status = int(ws[ws_bytes - 4:ws_bytes].cpu().numpy().view(np.uint32)[0]) if ws_bytes >= 4 else 0
-            nbytes = blob.size + B * K * 2 + B * N * 4
-            gbps = nbytes / (best / 1e3) / 1e9
-            results[f"{name} {N}x{K} B={B}"] = {"us": best * 1e3, "GBps": gbps, "frac": gbps / peak, "tile_rows": R,
-                                                "copies": M, "status": status}
-            del g, ws
-        del copies
-        torch.cuda.empty_cache()
+        res, nl = rotation_sweep(args, dev, stream, sms, peak, name, batches)
+        results.update(res)
+        n_launches += nl
     clocks = sampler.stop()
     t_setup = time.perf_counter() - t_setup
     head = [results[f"{n} {N}x{K} B=1"]["GBps"] for n, N, K in CFG4
@@ -722,7 +748,7 @@ def run_pad512(args):
                     torch.cuda.synchronize()
                     t = e0.elapsed_time(e1) / M
                     best = t if best is None else min(best, t)
-                n_launches += 2 * M * (args.warmup + 3)
+                n_launches += 2 * 3 * M   # the timed replays
             logical_bytes = sum(vbq.vbq_packed_size(m.N, m.K, r, m.widths) for m, r in ((gm, R), (um, R), (dm, Rd)))
             nbytes = logical_bytes + B * H * 2 + 2 * B * I * 4 + B * I * 2 + B * I * 2 + B * H * 4
             gbps = nbytes / (best / 1e3) / 1e9
@@ -778,6 +804,8 @@ def make_parser() -> argparse.ArgumentParser:
                     help="plain launches instead of programmatic dependent launch between the linears")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds for the CPU-oracle baseline (0: skip)")
     ap.add_argument("--ref-rows", type=int, default=256, help="rows per linear per step for --impl reference")
+    ap.add_argument("--no-batch-sweep", action="store_true",
+                    help="step workloads: skip the batch 1-16 sweep of the 14336x4096 linear after the timed step")
     ap.add_argument("--matrices", default="",
                     help="cfg4 only: comma-separated subset of q, gate, down (default: all three)")
     return ap
