@@ -1537,9 +1537,10 @@ inline void plan_workspace(const Problem& pr, int B, Plan& pl) {
   pl.status_off = pl.ws_bytes - 4;
 }
 
-// Records per batch NB and batches in flight S. Above batch 2, NB aims at about three jobs per warp
-// per batch (from an estimate of the units per record at the paper's allocation); S = 3 when it fits (the meta
-// jobs of a batch read records issued two batches earlier), else 2. Fewer records per batch before fewer sets.
+// Records per batch NB, batches in flight S and result sets RS: as many records per batch as fit (fewer batches
+// cut the per-batch bookkeeping and barriers; measured faster at every batch size), then S = 3 when it fits (the
+// meta jobs of a batch read records issued two batches earlier), else 2; at B >= 8 one result set (with a barrier
+// after each row pass) before fewer records per batch.
 template <int B>
 inline bool make_plan_b(const Problem& pr, int sms, Plan& pl) {
   using C = KCfg<B>;
@@ -1551,20 +1552,17 @@ inline bool make_plan_b(const Problem& pr, int sms, Plan& pl) {
   pl.res_rec = align128i(R * res_stride(B) * 4);
   pl.meta_rec = MetaOff(B).size;
   const int dir_bytes = 8 * kDirCache;
-  // units per record at the paper's allocation: 1-bit units of 32 items, the others of 32 / B; bucket tails
-  const int upr = (7 * R / 10 + 31) / 32 + (16 * R / 100 + 31) / 32 + (15 * R / 100 + C::kIPU - 1) / C::kIPU + 2;
-  // batch 1 and 2: as many records per batch as fit (fewer batches, less per-batch bookkeeping: measured faster)
-  const int nb_want = B <= 2 ? kMaxNB : std::min(kMaxNB, std::max(1, (5 * C::kWarps + upr - 1) / upr));
+  const int nb_want = kMaxNB;
   const MetaOff mo(B);
   auto need = [&](int NB, int S, int RS) {
     return (long long)S * NB * pl.stage_size + (long long)RS * NB * pl.res_rec + 256 + 2ll * NB * pl.meta_rec +
            3ll * NB * mo.row_size + dir_bytes;
   };
-  // two result sets let the next batch's units start before every warp has finished this batch's row pass; one
-  // set (with a barrier after each row pass) is the last resort for large records at batch 16
+  // two result sets let the next batch's units start before every warp has finished this batch's row pass; at
+  // B >= 8 (results of 48 or 80 bytes per row) a larger batch with one set measured faster than a smaller with two
   pl.NB = 0;
-  for (int RS = 2; RS >= (B < 8 ? 2 : 1) && pl.NB == 0; --RS)
-    for (int NB = nb_want; NB >= 1 && pl.NB == 0; --NB)
+  for (int NB = nb_want; NB >= 1 && pl.NB == 0; --NB)
+    for (int RS = 2; RS >= (B < 8 ? 2 : 1) && pl.NB == 0; --RS)
       for (int S = 3; S >= 2; --S)
         if (need(NB, S, RS) <= kSmemBudget) {
           pl.NB = NB;
