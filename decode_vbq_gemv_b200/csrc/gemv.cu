@@ -4,24 +4,22 @@
 // "Fused kernels over packed weights"): y[b][r] = sum_g s[r][g] * sum_i (q[r][64g+i] - (2^k-1)/2) * x[b][64g+i].
 // The low-bit codes are expanded in registers. The dense matrix never exists in memory.
 //
-// Kernel structure (B200, sm_100a), one CTA per SM:
+// Kernel structure (B200, sm_100a), one CTA per SM (details at the record-batch kernel below):
 //  - The blob is one record per (row tile, group column), stored tile-major. Inside a record, the tile's groups
-//    sit in four width buckets (1, 2, 4, 8 bits), each in ascending row order. CTA c owns the c-th equal share
-//    of the records (by count, computed without reading memory).
-//  - The CTA's warps form independent teams (one warp each when the CTA has many records, several warps each
-//    when it has few). A team owns a contiguous run of the CTA's records, streams them into its own ring of
-//    shared-memory stages with cp.async.bulk (the TMA engine, no multicast) and waits on mbarrier transaction
-//    counts, bounded by a timer; nothing waits on another team or another CTA.
-//  - Inside a team, warps take units of items of one bucket, so every warp instruction runs a single width.
-//    Batch 1, 2, 4 (CUDA cores): each lane owns one 64-weight group and one batch row (32/B groups per unit) and
-//    holds that row's activations in registers. 1-bit groups add the activations whose bit is set (predicated
-//    adds); 2/4-bit groups expand codes with a magic-number bit-to-float trick against pre-scaled activations;
-//    8-bit groups use byte permutes. Results land in item order, and a row pass adds them to the tile's rows.
-//    Batch 8/16: mma.sync bf16 tensor cores on the exact integers 2(q - c), units of 32 groups.
-//  - Row tiles that several owners share are reduced without floating-point atomics: teams of one CTA that
-//    share a tile are summed in shared memory in team order; CTAs that share a tile write partial sums to the
-//    workspace and count themselves in, and the last to arrive adds all partials in CTA order. Results are
-//    bitwise deterministic, and no CTA ever waits for another.
+//    sit in four width buckets (1, 2, 4, 8 bits), each in ascending row order. CTA c owns the c-th share of the
+//    records: equal counts in closed form, or equal estimated cost found in the directory when record sizes
+//    differ much.
+//  - The CTA streams its records in batches of up to seven records of one row tile into shared memory with
+//    cp.async.bulk (the TMA engine, no multicast), waiting on mbarrier transaction counts bounded by a timer. A
+//    meta job per record validates it and prepares its masks and activation side one batch ahead.
+//  - All warps of the CTA split each batch's width-bucket units by estimated cost, so every unit runs a single
+//    width. Batch 1, 2 (CUDA cores): 1- and 2-bit codes index nibble tables of partial sums of x, 4-bit codes go
+//    through a magic-number bit-to-float expansion, 8-bit codes through byte permutes. Batch 4, 8, 16: mma.sync
+//    bf16 tensor cores on exact small integers built from the codes in registers. Results land in item order,
+//    and a row pass adds each record's results to the tile's rows in record order.
+//  - Row tiles that several CTAs share are reduced without floating-point atomics: each CTA writes its partial
+//    sums to the workspace and counts itself in, and the last to arrive adds every element over the owners in
+//    CTA order. Results are bitwise deterministic, and no CTA ever waits for another.
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>

@@ -177,8 +177,9 @@ int vbq_gemv(const vbq_desc* d, const void* blob_dev, const void* x_bf16, float*
  * applied to several activation rows at once; the paper decodes at batch 1, the small batches are this library's
  * extension.
  * x_bf16: B*K bf16 values, row-major (row b is activation b), 16-byte aligned. y: B*N fp32, row-major.
- * B <= 4 runs on CUDA cores; B = 8 and 16 run the dequantized groups through tensor cores (bf16 operands
- * that hold the exact integers 2(q - c), fp32 accumulation, the group scale applied in fp32).
+ * B <= 2 runs on CUDA cores; B = 4, 8 and 16 run the dequantized groups through tensor cores (bf16 operands
+ * that hold exact small integers or half-integers: q - c, q - 8 or q - 128, fp32 accumulation seeded with the
+ * leftover grid offset times the group's activation sum, the group scale applied in fp32).
  * Other arguments and guarantees as in vbq_gemv. Errors: NULL, BATCH, ALIGN, WORKSPACE, FORMAT, CUDA. */
 int vbq_gemm_skinny(const vbq_desc* d, const void* blob_dev, const void* x_bf16, int B, float* y,
                     void* workspace, uint64_t workspace_bytes, void* stream);

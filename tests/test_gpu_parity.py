@@ -404,7 +404,7 @@ def sym_matrix(seed, N, K, p):
 @pytest.mark.parametrize("B", vbq.BATCHES)
 def test_symmetric_grid_all_batches(B):
     """Blobs flagged with Eq. 1's symmetric grid (VBQ_FLAG_GRID_SYMMETRIC) through every batch path (CUDA cores
-    at B <= 4, tensor cores at B = 8, 16) against the oracle's flag-aware matvec; and one fused launch mixing a
+    at B <= 2, tensor cores at B = 4, 8, 16) against the oracle's flag-aware matvec; and one fused launch mixing a
     flagged and an unflagged matrix."""
     sym = vbq.VBQ_FLAG_GRID_SYMMETRIC
     for (N, K, R, dist) in ((1030, 256, 64, "flat"), (777, 2048, 256, "base"), (300, 512, 1024, "all8")):
