@@ -30,10 +30,10 @@ def suggest_tile_rows(rows: int, K: int, sms: int = 148) -> int:
     SMs: the largest of 1024, 512 and 256 that still gives every SM at least 7 records (tile, group column).
 
     Larger tiles fill the width-bucket units better and cut per-record work; too few records per SM leave the
-    CTAs' batches short. From graph-timed launch groups of the 9B-shaped decode step on B200 at batch 1, this
-    picks the fastest of the three sizes for each: fused q/k/v 512 rows (21.8 us; 1024: 22.2), the lone 4096x4096
-    projection 256 (12.8 us; 512: 15.3), fused gate/up 1024 (34.1 us; 512: 40.3), down 512 (25.4 us; 1024:
-    27.7) and the LM head 1024 (33.3 us; 512: 40.3)."""
+    CTAs' batches short. Graph-timed at batch 1 on B200, this picks the fastest size for each 9B-shaped launch:
+    the lone 4096x4096 projection 256 rows (13.5 us; 128: 17.9, 512: 16.9), gate 14336x4096 512 (21.5 us; 256:
+    26.3, 1024: 22.9), down 4096x14336 512 (23.7 us; 256: 26.1, 1024: 30.2), the LM head 1024 (30.0 us; 512:
+    33.6) and fused gate/up 1024 (35.2 us; 512: 36.1)."""
     G = max(K // 64, 1)
     for R in (1024, 512, 256):
         if -(-rows // R) * G >= 7 * sms:
