@@ -1526,6 +1526,15 @@ inline int make_problem(int nmat, const vbq_desc* const* d, Problem& pr) {
   return VBQ_OK;
 }
 
+// CTAs split the records by estimated cost when record sizes differ much: the largest record over 1.3 times the
+// mean (an LM head whose frequent rows are wider, a small last tile); otherwise by count, which needs no directory
+// search.
+inline bool cost_split(const Problem& pr) {
+  uint64_t units = 0;
+  for (int m = 0; m < pr.nmat; ++m) units += (pr.d[m]->total_bytes - pr.d[m]->rec_offset) / 16;
+  return double(pr.max_record_bytes) > 1.3 * 16.0 * double(units) / double(pr.nrec);
+}
+
 // Workspace: partial slots [nCTA + T][B][R] f32 of the row tiles that CTAs share, then an arrival counter and a
 // SwiGLU pair counter per tile, then the status word.
 inline void plan_workspace(const Problem& pr, int B, Plan& pl) {
@@ -1622,9 +1631,7 @@ int launch(const Problem& pr, const void* const* blobs, const void* x, float* co
   }
   p.tile_start[kMaxMats] = tiles;
   p.rec_start[kMaxMats] = recs;
-  // Split by cost when record sizes differ much (the largest record over 1.3 times the mean, as in an LM head
-  // whose frequent rows are wider); otherwise by count, which needs no directory search.
-  p.balanced = (double(pr.max_record_bytes) > 1.3 * 16.0 * double(total16) / double(recs)) ? 1 : 0;
+  p.balanced = cost_split(pr) ? 1 : 0;
   // the fixed part of a record's cost, measured on LM heads: four mean records at batch 1 (the per-record work
   // dominates), two at larger batches (the units' share grows with B)
   p.rec_w16 = std::max<unsigned long long>(1, (B == 1 ? 4ull : 2ull) * total16 / unsigned(recs));
@@ -1711,6 +1718,25 @@ int vbq_workspace_size_multi(int nmat, const vbq_desc* const* d, int B, uint64_t
   vbq::Plan pl;
   if (!vbq::make_plan(pr, B, vbq::num_sms(), pl)) return VBQ_ERR_FORMAT;
   *out_bytes = pl.ws_bytes;
+  return VBQ_OK;
+}
+
+int vbq_plan_info_get(int nmat, const vbq_desc* const* d, int B, int sm_count, vbq_plan_info* out) {
+  if (!d || !out) return VBQ_ERR_NULL;
+  if (!vbq::batch_ok(B)) return VBQ_ERR_BATCH;
+  if (sm_count < 1 || sm_count > 4096) return VBQ_ERR_SHAPE;
+  vbq::Problem pr;
+  if (int st = vbq::make_problem(nmat, d, pr)) return st;
+  vbq::Plan pl;
+  if (!vbq::make_plan(pr, B, sm_count, pl)) return VBQ_ERR_FORMAT;
+  out->grid = pl.grid;
+  out->threads = pl.threads;
+  out->records_per_batch = pl.NB;
+  out->batches_in_flight = pl.S;
+  out->result_sets = pl.RS;
+  out->cost_split = vbq::cost_split(pr) ? 1 : 0;
+  out->smem_bytes = uint32_t(pl.smem);
+  out->workspace_bytes = pl.ws_bytes;
   return VBQ_OK;
 }
 

@@ -54,6 +54,12 @@ class vbq_desc(ctypes.Structure):
                 ("total_bytes", ctypes.c_uint64), ("max_record_bytes", ctypes.c_uint64)]
 
 
+class vbq_plan_info(ctypes.Structure):
+    _fields_ = [("grid", ctypes.c_int32), ("threads", ctypes.c_int32), ("records_per_batch", ctypes.c_int32),
+                ("batches_in_flight", ctypes.c_int32), ("result_sets", ctypes.c_int32), ("cost_split", ctypes.c_int32),
+                ("smem_bytes", ctypes.c_uint32), ("workspace_bytes", ctypes.c_uint64)]
+
+
 _lib = None
 
 
@@ -83,6 +89,7 @@ def lib() -> ctypes.CDLL:
             "vbq_describe": (i32, [vp, u64, dp]),
             "vbq_unpack": (i32, [vp, u64, vp, vp, vp]),
             "vbq_workspace_size": (i32, [dp, i32, ctypes.POINTER(u64)]),
+            "vbq_plan_info_get": (i32, [i32, vp, i32, i32, ctypes.POINTER(vbq_plan_info)]),
             "vbq_workspace_init": (i32, [vp, u64, vp]),
             "vbq_gemv": (i32, [dp, vp, vp, vp, vp, u64, vp]),
             "vbq_gemm_skinny": (i32, [dp, vp, vp, i32, vp, vp, u64, vp]),
@@ -240,6 +247,15 @@ def vbq_unpack(blob: np.ndarray):
     st, out = vbq_unpack_status(blob)
     _check(st, "vbq_unpack")
     return out
+
+
+def vbq_plan_info_get(descs, B: int, sm_count: int = 148) -> dict:
+    """The launch plan of a device call over the given descriptors (one, or the matrices of one fused launch) at
+    batch B on a GPU with sm_count SMs (vbq_plan_info_get; host only, no GPU needed)."""
+    ds = [descs] if isinstance(descs, vbq_desc) else list(descs)
+    out = vbq_plan_info()
+    _check(lib().vbq_plan_info_get(len(ds), _desc_array(ds), B, sm_count, ctypes.byref(out)), "vbq_plan_info_get")
+    return {f: getattr(out, f) for f, _ in vbq_plan_info._fields_}
 
 
 def vbq_workspace_size(desc: vbq_desc, B: int) -> int:

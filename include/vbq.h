@@ -154,6 +154,24 @@ int vbq_unpack(const void* blob_host, uint64_t blob_bytes, uint8_t* widths, uint
  * Errors: NULL, BATCH, FORMAT (desc inconsistent). */
 int vbq_workspace_size(const vbq_desc* d, int B, uint64_t* out_bytes);
 
+/* The launch plan of a device call (no passage of the VBQ paper: it describes this library's kernels), computed
+ * on the host without any CUDA call, for sm_count SMs: nmat descriptors as in vbq_gemm_skinny_multi (1 for
+ * vbq_gemm_skinny), batch B.
+ *   grid, threads:       CTAs (one per SM) and threads per CTA;
+ *   records_per_batch:   records of one row tile handled between two CTA barriers (1..7);
+ *   batches_in_flight:   record batches streamed ahead of the compute (2 or 3);
+ *   result_sets:         item-result buffers (2: alternate batches; 1: a barrier after each row pass);
+ *   cost_split:          1 when CTAs split the records by estimated cost (record sizes differ much), 0 by count;
+ *   smem_bytes:          dynamic shared memory per CTA;
+ *   workspace_bytes:     what vbq_workspace_size[_multi] returns on a GPU with sm_count SMs.
+ * Errors: NULL, BATCH, SHAPE (nmat or sm_count out of range), TILE, FORMAT (no plan fits). Pure, thread-safe. */
+typedef struct vbq_plan_info {
+  int32_t grid, threads, records_per_batch, batches_in_flight, result_sets, cost_split;
+  uint32_t smem_bytes;
+  uint64_t workspace_bytes;
+} vbq_plan_info;
+int vbq_plan_info_get(int nmat, const vbq_desc* const* d, int B, int sm_count, vbq_plan_info* out);
+
 /* Zero a workspace before its first use (cudaMemsetAsync on `stream`). Every kernel call leaves the arrival
  * counters at zero again, so one zeroing per workspace is enough. Errors: NULL, CUDA. */
 int vbq_workspace_init(void* workspace, uint64_t workspace_bytes, void* stream);

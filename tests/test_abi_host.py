@@ -339,3 +339,65 @@ def test_padded_pack_refuses_shrinking_or_unaligned_padding():
     for N_pad, K_pad in ((9, 128), (10, 64), (10, 200), (0, 128)):
         st, blob, _ = vbq.vbq_pack_padded_status(10, 128, 16, w, s, c, N_pad, K_pad)
         assert st == vbq.VBQ_ERR_SHAPE and blob is None
+
+
+def plan(descs, B, sms=148):
+    return vbq.vbq_plan_info_get(descs, B, sms)
+
+
+@pytest.mark.parametrize("B", [1, 2, 4, 8, 16])
+def test_launch_plans_of_the_9b_linears_fit_the_sm(B):
+    """Host-side launch plans (vbq_plan_info_get, no GPU): for every 9B-shaped linear at its suggested tile rows,
+    a plan exists within 227 KB of shared memory per CTA, one CTA per SM, 16 warps at batch 1-2 and 12 at 4-16,
+    1-7 records per batch, 2-3 batches in flight, two result sets below batch 8; records of similar size are
+    split by count; the workspace holds one partial slot per CTA and tile plus two counters per tile and the
+    status word."""
+    for m in S.cfg4(("q", "gate", "down")):
+        R = vbq.suggest_tile_rows(m.N, m.K, 148)
+        _, d = vbq.vbq_pack(m.N, m.K, R, m.widths, m.scales, m.codes)
+        p = plan(d, B)
+        assert p["grid"] == 148 and p["threads"] == (512 if B <= 2 else 384)
+        assert 0 < p["smem_bytes"] <= 227 * 1024
+        assert 1 <= p["records_per_batch"] <= 7 and p["batches_in_flight"] in (2, 3)
+        assert p["result_sets"] == 2 if B < 8 else p["result_sets"] in (1, 2)
+        assert p["cost_split"] == 0
+        ws = ((148 + d.T) * R * B * 4 + d.T * 8 + 4 + 15) // 16 * 16
+        assert p["workspace_bytes"] == ws
+        assert plan(d, B, 74)["workspace_bytes"] < ws and plan(d, B, 74)["grid"] == 74
+
+
+def test_cost_split_is_chosen_for_uneven_records_only():
+    """The launch splits records by estimated cost exactly when the largest record exceeds 1.3 times the mean:
+    the LM head (frequent rows wider) and a matrix whose first rows are 8-bit, not the base-mix linears, alone or
+    fused."""
+    head = S.cfg5_head()
+    _, dh = vbq.vbq_pack(head.N, head.K, 1024, head.widths, head.scales, head.codes)
+    assert plan(dh, 1)["cost_split"] == 1
+    w = np.ones((3000, 8), np.uint8)
+    w[:300] = 8
+    g = np.random.default_rng(1)
+    _, du = vbq.vbq_pack(3000, 512, 64, w, S.scales_uniform(3000, 8, g), S.codes_uniform(w, g))
+    assert plan(du, 4)["cost_split"] == 1
+    gate, up = S.cfg4(("gate", "up"))
+    dg = vbq.vbq_pack(gate.N, gate.K, 1024, gate.widths, gate.scales, gate.codes)[1]
+    du2 = vbq.vbq_pack(up.N, up.K, 1024, up.widths, up.scales, up.codes)[1]
+    assert plan(dg, 1)["cost_split"] == 0 and plan([dg, du2], 1)["cost_split"] == 0
+
+
+def test_plan_of_the_largest_records_and_argument_errors():
+    """All-8-bit 1024-row records (the largest a record gets) still plan at batch 16; bad batch sizes, SM counts,
+    matrix counts and mismatched fused shapes are refused with the documented codes."""
+    N, K = 2048, 512
+    w = np.full((N, K // 64), 8, np.uint8)
+    g = np.random.default_rng(2)
+    _, d = vbq.vbq_pack(N, K, 1024, w, S.scales_uniform(N, K // 64, g), S.codes_uniform(w, g))
+    p = plan(d, 16)
+    assert p["records_per_batch"] >= 1 and p["smem_bytes"] <= 227 * 1024
+    out = vbq.vbq_plan_info()
+    L = vbq.lib()
+    assert L.vbq_plan_info_get(1, vbq._desc_array([d]), 3, 148, ctypes.byref(out)) == vbq.VBQ_ERR_BATCH
+    assert L.vbq_plan_info_get(1, vbq._desc_array([d]), 1, 0, ctypes.byref(out)) == vbq.VBQ_ERR_SHAPE
+    assert L.vbq_plan_info_get(5, vbq._desc_array([d] * 5), 1, 148, ctypes.byref(out)) == vbq.VBQ_ERR_SHAPE
+    _, d2 = vbq.vbq_pack(N, 256, 1024, w[:, :4], S.scales_uniform(N, 4, g), S.codes_uniform(w[:, :4], g))
+    assert L.vbq_plan_info_get(2, vbq._desc_array([d, d2]), 1, 148, ctypes.byref(out)) == vbq.VBQ_ERR_SHAPE
+    assert L.vbq_plan_info_get(1, None, 1, 148, ctypes.byref(out)) == vbq.VBQ_ERR_NULL
