@@ -78,8 +78,9 @@ def test_replica_timing_is_the_slowest_rank_over_gloo():
 
 
 def test_kernel_source_hash_ignores_comments_only():
-    """The bench keys its ncu traffic capture to the kernel source's code: comment and blank-line edits keep the
-    key, any code edit changes it."""
+    """The bench keys its ncu traffic capture to the device code of the kernel source (the part before the
+    host-side launch-plan section): comment, blank-line and host-only edits keep the key, any device-code edit
+    changes it."""
     import hashlib
     import re
     sys.path.insert(0, ROOT)
@@ -92,7 +93,11 @@ def test_kernel_source_hash_ignores_comments_only():
 
     with open(os.path.join(ROOT, "decode_vbq_gemv_b200", "csrc", "gemv.cu")) as f:
         src = f.read()
-    assert bench.kernel_source_sha256() == key(src)
+    marker = "// " + "-" * 90 + " launch plan"
+    assert src.count(marker) == 1
+    device = src[:src.index(marker)]
+    assert "__global__" in device and "__global__" not in src[src.index(marker):]
+    assert bench.kernel_source_sha256() == key(device)
     assert key("// note\nint a;\n\n/* block\n comment */ int b;  // tail\n") == key("int a;\n int b;\n")
     assert key("int a = 1;\n") != key("int a = 2;\n")
 
